@@ -1,0 +1,191 @@
+"""Seeded synthetic inputs for the MLA latent-cache path.
+
+This module holds no part of the attention arithmetic: it only draws
+numbers. Both the CUDA path's tests/bench and the CPU oracle consume what it
+returns, so the two sides see bit-identical inputs.
+
+Generator (counter based, so any element can be drawn on its own):
+  * SplitMix64 (Steele, Lea & Flood, "Fast splittable pseudorandom number
+    generators", OOPSLA 2014): state_n = key + (n + 1) * 0x9E3779B97F4A7C15,
+    output = mix64(state_n) with the published finaliser constants.
+  * key(seed, tensor_id) = mix64((seed << 32) + tensor_id), one independent
+    stream per tensor.
+  * uniform(n) = (u64(n) >> 11) * 2^-53 in [0, 1).
+  * normal(i) by Box-Muller on the pair of uniforms (2i, 2i+1):
+    sqrt(-2 ln(1 - a)) * cos(2 pi b), in float64, then scaled by std.
+  * Rounding to the input dtype: float64 -> float32 (round to nearest even),
+    then for bf16 float32 -> bf16 (round to nearest even). Values are
+    returned as float32 arrays that hold the rounded values exactly.
+
+Workload recipes follow the DeepSeek-V3 model hyper-parameters (the notes
+"【论文解读】DeepSeek-V3", section 三(二)1 "model hyper-parameters": d = 7168,
+n_h = 128, d_h = 128, d_c = 512, d_c' = 1536, d_h^R = 64) and the decode /
+prefill shapes listed in WORKLOADS below.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+# Tensor ids: one stream per named input.
+TID_H, TID_WDQ, TID_WUQ, TID_WQR, TID_WDKV, TID_WKR, TID_WUK, TID_WUV, TID_WO = range(9)
+TID_CACHE_C, TID_CACHE_KR, TID_LENGTHS = 9, 10, 11
+TID_POSITIONS, TID_SLOTS = 12, 13
+
+_CHUNK = 1 << 22
+
+
+def _mix64(z: np.ndarray) -> np.ndarray:
+    z = (z ^ (z >> np.uint64(30))) * _M1
+    z = (z ^ (z >> np.uint64(27))) * _M2
+    return z ^ (z >> np.uint64(31))
+
+
+def stream_key(seed: int, tensor_id: int) -> np.uint64:
+    with np.errstate(over="ignore"):
+        base = np.array([(int(seed) << 32) + int(tensor_id)], dtype=np.uint64)
+        return _mix64(base + _GAMMA)[0]
+
+
+def u64(seed: int, tensor_id: int, counters: np.ndarray) -> np.ndarray:
+    """Raw 64-bit draws for the given counters of stream (seed, tensor_id)."""
+    key = stream_key(seed, tensor_id)
+    c = np.asarray(counters, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        return _mix64(key + (c + np.uint64(1)) * _GAMMA)
+
+
+def _uniform(seed, tensor_id, counters):
+    return (u64(seed, tensor_id, counters) >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+
+
+def normal_f64(seed: int, tensor_id: int, n: int, start: int = 0) -> np.ndarray:
+    """N(0,1) draws for element indices [start, start+n), float64."""
+    out = np.empty(n, dtype=np.float64)
+    for lo in range(0, n, _CHUNK):
+        hi = min(n, lo + _CHUNK)
+        idx = np.arange(start + lo, start + hi, dtype=np.uint64)
+        a = _uniform(seed, tensor_id, idx * np.uint64(2))
+        b = _uniform(seed, tensor_id, idx * np.uint64(2) + np.uint64(1))
+        out[lo:hi] = np.sqrt(-2.0 * np.log1p(-a)) * np.cos(2.0 * np.pi * b)
+    return out
+
+
+def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round float64 values to 'fp32' or 'bf16'; returns float32 holding them."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    if dtype == "fp32":
+        return f
+    if dtype != "bf16":
+        raise ValueError(f"unknown dtype {dtype!r}")
+    bits = f.view(np.uint32).astype(np.uint64)
+    rounded = (bits + np.uint64(0x7FFF) + ((bits >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    return (rounded.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def normal(seed: int, tensor_id: int, shape, std: float = 1.0, dtype: str = "bf16") -> np.ndarray:
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.float32)
+    for lo in range(0, n, _CHUNK):
+        hi = min(n, lo + _CHUNK)
+        out[lo:hi] = round_to(normal_f64(seed, tensor_id, hi - lo, start=lo) * std, dtype)
+    return out.reshape(shape)
+
+
+@dataclass(frozen=True)
+class Dims:
+    """MLA dimensions in the notes' symbols: d, n_h, d_h, d_c, d_c' (d_cq), d_h^R (d_r)."""
+    d: int
+    n_h: int
+    d_h: int
+    d_c: int
+    d_cq: int
+    d_r: int
+    rope_base: float = 10000.0
+
+    @property
+    def row(self) -> int:
+        """Elements per latent-cache row: [c^KV (d_c) | k^R (d_r)]."""
+        return self.d_c + self.d_r
+
+
+TINY = Dims(d=256, n_h=4, d_h=32, d_c=64, d_cq=96, d_r=16)
+V3 = Dims(d=7168, n_h=128, d_h=128, d_c=512, d_cq=1536, d_r=64)
+
+# Weight name -> (tensor id, shape(dims) [out, in]); std = 1/sqrt(fan_in) with fan_in = in.
+WEIGHT_SPECS = {
+    "w_dq": (TID_WDQ, lambda m: (m.d_cq, m.d)),
+    "w_uq": (TID_WUQ, lambda m: (m.n_h * m.d_h, m.d_cq)),
+    "w_qr": (TID_WQR, lambda m: (m.n_h * m.d_r, m.d_cq)),
+    "w_dkv": (TID_WDKV, lambda m: (m.d_c, m.d)),
+    "w_kr": (TID_WKR, lambda m: (m.d_r, m.d)),
+    "w_uk": (TID_WUK, lambda m: (m.n_h * m.d_h, m.d_c)),
+    "w_uv": (TID_WUV, lambda m: (m.n_h * m.d_h, m.d_c)),
+    "w_o": (TID_WO, lambda m: (m.d, m.n_h * m.d_h)),
+}
+
+
+def weights(dims: Dims, seed: int = 0, dtype: str = "bf16", names=None) -> dict:
+    out = {}
+    for name, (tid, shape_fn) in WEIGHT_SPECS.items():
+        if names is not None and name not in names:
+            continue
+        shape = shape_fn(dims)
+        out[name] = normal(seed, tid, shape, std=1.0 / np.sqrt(shape[1]), dtype=dtype)
+    return out
+
+
+def hidden(dims: Dims, tokens: int, seed: int = 0, dtype: str = "bf16") -> np.ndarray:
+    return normal(seed, TID_H, (tokens, dims.d), dtype=dtype)
+
+
+def latent_cache(dims: Dims, rows: int, seed: int = 0, dtype: str = "bf16") -> np.ndarray:
+    """Synthetic latent cache rows [rows, d_c + d_r]: c^KV ~ N(0,1) then k^R ~ N(0,1)."""
+    c = normal(seed, TID_CACHE_C, (rows, dims.d_c), dtype=dtype)
+    kr = normal(seed, TID_CACHE_KR, (rows, dims.d_r), dtype=dtype)
+    return np.concatenate([c, kr], axis=1)
+
+
+def ragged_lengths(batch: int, lo: int, hi: int, seed: int = 0) -> np.ndarray:
+    """Lengths uniform on [lo, hi] (inclusive) from the seed's length stream."""
+    span = np.uint64(hi - lo + 1)
+    draws = u64(seed, TID_LENGTHS, np.arange(batch, dtype=np.uint64))
+    return (draws % span).astype(np.int64) + lo
+
+
+def cu_seqlens(lengths) -> np.ndarray:
+    lengths = np.asarray(lengths, dtype=np.int64)
+    return np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str            # "prefill" or "decode"
+    dims: Dims
+    dtype: str
+    batch: int
+    tq: int = 1          # query tokens per sequence (decode)
+    length: int = 0      # fixed cache/sequence length
+    ragged: tuple = field(default=())  # (lo, hi) for ragged lengths
+
+    def lengths(self, seed: int = 0) -> np.ndarray:
+        if self.ragged:
+            return ragged_lengths(self.batch, self.ragged[0], self.ragged[1], seed)
+        return np.full(self.batch, self.length, dtype=np.int64)
+
+
+WORKLOADS = {
+    "tiny_prefill_fp32": Workload("tiny_prefill_fp32", "prefill", TINY, "fp32", batch=1, length=64),
+    "decode_b16_l4096": Workload("decode_b16_l4096", "decode", V3, "bf16", batch=16, tq=1, length=4096),
+    "decode_mtp_b64_ragged": Workload("decode_mtp_b64_ragged", "decode", V3, "bf16", batch=64, tq=2,
+                                      ragged=(1024, 32768)),
+    "prefill_l32768": Workload("prefill_l32768", "prefill", V3, "bf16", batch=1, length=32768),
+    "decode_long_b4_l131072": Workload("decode_long_b4_l131072", "decode", V3, "bf16", batch=4, tq=1,
+                                       length=131072),
+}

@@ -1,0 +1,323 @@
+"""CPU float64 oracle for DeepSeek-V3 Multi-head Latent Attention (MLA) over the latent KV cache.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import or call this
+module: only the tests, the package's smoke check and the benchmark's CPU
+baseline leg use it. It shares no code with the CUDA path and imports nothing
+from the package; callers hand it plain numpy arrays.
+
+Source. The definitions follow the notes "【论文解读】DeepSeek-V3"
+(wkq9411.github.io/2026-01-01/Paper-DeepSeek-V3.html), section 一(一)
+"多头潜在注意力MLA" (multi-head latent attention):
+  * 1 "回顾多头注意力MHA"      - multi-head attention, causal softmax over j <= t, W^O last;
+  * 2 "低秩KV联合压缩"         - c^KV = W^DKV h, k^C = W^UK c^KV, v^C = W^UV c^KV,
+                                 c^Q = W^DQ h, q^C = W^UQ c^Q, and the 【思考】 block
+                                 on absorbing W^UK into the query and W^UV into W^O;
+  * 3 "解耦RoPE"               - block-diagonal 2x2 RoPE, decoupled q^R = RoPE(W^QR c^Q)
+                                 per head, shared k^R = RoPE(W^KR h), score scale
+                                 1/sqrt(d_h + d_h^R), and the ten-step computation
+                                 (1)-(10) that this file spells out.
+Decode semantics (cache the keys/values of past tokens, compute only the new
+query, attend over every cached position) follow the explainer at
+mlqm.cn/news/135256, paragraph "KV Cache的核心原理".
+
+Readings where the pages leave a step open (each is also listed in the design doc):
+  R1 RoPE pairs are the interleaved pairs (2m, 2m+1) of the block-diagonal
+     form, rotated by [[cos, -sin], [sin, cos]] with angle pos * base^(-2m/d_R).
+  R2 Positions are 0-based within a sequence; packing does not shift them.
+  R3 The scale is 1/sqrt(d_h + d_h^R) in both the absorbed and unabsorbed forms.
+  R4 No RMSNorm on c^Q / c^KV (no equation of the section has one) and no YaRN.
+  R5 Decode: a sequence's cache length includes its Tq new tokens (appended
+     first); query k sits at position len - Tq + k and sees rows j <= position.
+  R6 A synthetic decode cache holds c^KV and an already-rotated k^R.
+  R7 lse is the natural log of sum_j exp(s_j) over the scaled scores s_j.
+
+Arithmetic is float64 throughout; inputs are the rounded (bf16 or fp32)
+values widened to float64. Library matmuls serve only as the sums that the
+equations write out; there is no blocking, fusion or reordering beyond that.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# RoPE (section 3, the R_m block-diagonal rotation; reading R1)
+# ---------------------------------------------------------------------------
+def rope_angles(pos, d_r: int, base: float) -> np.ndarray:
+    """Angles pos * theta_m with theta_m = base^(-2m/d_r), m = 0..d_r/2-1; shape pos.shape + (d_r/2,)."""
+    m = np.arange(d_r // 2, dtype=np.float64)
+    theta = base ** (-2.0 * m / d_r)
+    return f64(pos)[..., None] * theta
+
+
+def rope(x, pos, base: float) -> np.ndarray:
+    """Rotate each pair (x_2m, x_2m+1) of the last axis by the angle of position pos.
+
+    pos must broadcast against x.shape[:-1].
+    """
+    x = f64(x)
+    ang = rope_angles(pos, x.shape[-1], base)
+    c, s = np.cos(ang), np.sin(ang)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    a = x0 * c - x1 * s
+    b = x0 * s + x1 * c
+    return np.stack([a, b], axis=-1).reshape(a.shape[:-1] + (2 * a.shape[-1],))
+
+
+# ---------------------------------------------------------------------------
+# Projections (section 2 and section 3, steps (1)-(3), (5)-(7), (9))
+# ---------------------------------------------------------------------------
+def query_projections(h, W, dims, pos):
+    """Steps (1)-(3): c^Q = W^DQ h; q^C = W^UQ c^Q split by heads; q^R = RoPE(W^QR c^Q) per head.
+
+    h [T, d], pos [T] -> c_q [T, d_cq], q_c [T, n_h, d_h], q_r [T, n_h, d_r].
+    """
+    h = f64(h)
+    T = h.shape[0]
+    c_q = h @ f64(W["w_dq"]).T
+    q_c = (c_q @ f64(W["w_uq"]).T).reshape(T, dims.n_h, dims.d_h)
+    q_r_hat = (c_q @ f64(W["w_qr"]).T).reshape(T, dims.n_h, dims.d_r)
+    q_r = rope(q_r_hat, f64(pos)[:, None], dims.rope_base)
+    return c_q, q_c, q_r
+
+
+def kv_compression(h, W, dims, pos):
+    """Steps (5) and (7): c^KV = W^DKV h and k^R = RoPE(W^KR h). Returns c_kv [T, d_c], k_r [T, d_r]."""
+    h = f64(h)
+    c_kv = h @ f64(W["w_dkv"]).T
+    k_r = rope(h @ f64(W["w_kr"]).T, pos, dims.rope_base)
+    return c_kv, k_r
+
+
+def cache_rows(c_kv, k_r) -> np.ndarray:
+    """One latent-cache row per token: [c^KV | k^R], (d_c + d_h^R) elements (section 3, cache size)."""
+    return np.concatenate([f64(c_kv), f64(k_r)], axis=1)
+
+
+def up_project_head(c_kv, W, dims, i):
+    """Steps (6) and (9) for head i: k^C_i = W_i^UK c^KV and v^C_i = W_i^UV c^KV.
+
+    W_i^UK are rows [i d_h, (i+1) d_h) of W^UK (head-major split of section 2's 【思考】).
+    c_kv [L, d_c] -> k_c_i [L, d_h], v_c_i [L, d_h].
+    """
+    rows = slice(i * dims.d_h, (i + 1) * dims.d_h)
+    c_kv = f64(c_kv)
+    return c_kv @ f64(W["w_uk"])[rows].T, c_kv @ f64(W["w_uv"])[rows].T
+
+
+# ---------------------------------------------------------------------------
+# Attention (step (4), (8), (10))
+# ---------------------------------------------------------------------------
+def causal_softmax_attend(q, k, v, lat, qpos, scale):
+    """One head: s_j = q.k_j * scale for j <= qpos, p = softmax(s), returns (sum p v, sum p lat, lse, p).
+
+    q [Tq, e], k [L, e], v [L, dv], lat [L, d_c] or None, qpos [Tq] (reading R5: key j is
+    visible to a query at position qpos iff j <= qpos; masked keys are left out of the sum).
+    """
+    q, k, v = f64(q), f64(k), f64(v)
+    Tq, L = q.shape[0], k.shape[0]
+    s = (q @ k.T) * scale
+    visible = np.arange(L)[None, :] <= np.asarray(qpos)[:, None]
+    s_masked = np.where(visible, s, -np.inf)
+    m = s_masked.max(axis=1, keepdims=True)
+    e = np.where(visible, np.exp(s_masked - m), 0.0)
+    z = e.sum(axis=1, keepdims=True)
+    p = e / z
+    o = p @ v
+    o_lat = None if lat is None else p @ f64(lat)
+    lse = (m + np.log(z))[:, 0]
+    return o, o_lat, lse, p
+
+
+def attend_unabsorbed(q_c, q_r, c_kv, k_r, W, dims, qpos, heads=None):
+    """Steps (4), (6), (8), (9), (10) for one sequence, keys/values up-projected explicitly.
+
+    q_c [Tq, n_h, d_h], q_r [Tq, n_h, d_r], c_kv [L, d_c], k_r [L, d_r] (shared by all heads).
+    Returns o [Tq, H, d_h], o_lat [Tq, H, d_c] (= sum_j p_j c_j, the factor that section 2's
+    【思考】 moves W_i^UV out of), lse [Tq, H] for the heads asked for (default all).
+    """
+    heads = range(dims.n_h) if heads is None else list(heads)
+    scale = 1.0 / np.sqrt(dims.d_h + dims.d_r)
+    Tq = q_c.shape[0]
+    H = len(heads)
+    o = np.empty((Tq, H, dims.d_h))
+    o_lat = np.empty((Tq, H, dims.d_c))
+    lse = np.empty((Tq, H))
+    k_r = f64(k_r)
+    for hi, i in enumerate(heads):
+        k_c_i, v_c_i = up_project_head(c_kv, W, dims, i)           # steps (6), (9)
+        q_i = np.concatenate([f64(q_c[:, i]), f64(q_r[:, i])], axis=1)   # step (4)
+        k_i = np.concatenate([k_c_i, k_r], axis=1)                  # step (8)
+        o[:, hi], o_lat[:, hi], lse[:, hi], _ = causal_softmax_attend(q_i, k_i, v_c_i, c_kv, qpos, scale)
+    return o, o_lat, lse
+
+
+def output_projection(o, W) -> np.ndarray:
+    """Step (10), second equation: u_t = W^O [o_t,1; ...; o_t,n_h]. o [T, n_h, d_h] -> u [T, d]."""
+    o = f64(o)
+    return o.reshape(o.shape[0], -1) @ f64(W["w_o"]).T
+
+
+# ---------------------------------------------------------------------------
+# Whole calls
+# ---------------------------------------------------------------------------
+def cache_append(h, positions, W, dims) -> np.ndarray:
+    """Rows [c^KV | RoPE(W^KR h)] for tokens h [T, d] at the given positions (steps (5), (7))."""
+    c_kv, k_r = kv_compression(h, W, dims, positions)
+    return cache_rows(c_kv, k_r)
+
+
+def decode_positions(cu_seqlens, tq):
+    """Reading R5: query k of sequence b sits at position len_b - Tq + k."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    lens = cu[1:] - cu[:-1]
+    return np.concatenate([np.arange(L - tq, L) for L in lens]).astype(np.int64)
+
+
+def mla_decode(h_q, cache, cu_seqlens, tq, W, dims, seqs=None, heads=None):
+    """Decode step over a latent cache, unabsorbed (steps (1)-(10) with cached c^KV, k^R).
+
+    h_q [B*Tq, d] (sequence-major), cache [rows, d_c + d_r] holding every sequence's rows
+    (including its Tq new tokens) packed by cu_seqlens. Returns a dict for the sequences
+    asked for (default all): rows (token indices), o_lat, lse, o and, when all heads are
+    computed, u.
+    """
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    B = len(cu) - 1
+    seqs = range(B) if seqs is None else list(seqs)
+    pos_all = decode_positions(cu, tq)
+    cache = f64(cache)
+    rows, o_l, lat_l, lse_l = [], [], [], []
+    for b in seqs:
+        r = np.arange(b * tq, (b + 1) * tq)
+        _, q_c, q_r = query_projections(f64(h_q)[r], W, dims, pos_all[r])
+        seq = cache[cu[b]:cu[b + 1]]
+        o, o_lat, lse = attend_unabsorbed(q_c, q_r, seq[:, :dims.d_c], seq[:, dims.d_c:], W, dims,
+                                          pos_all[r], heads)
+        rows.append(r); o_l.append(o); lat_l.append(o_lat); lse_l.append(lse)
+    out = {"rows": np.concatenate(rows), "o": np.concatenate(o_l), "o_lat": np.concatenate(lat_l),
+           "lse": np.concatenate(lse_l)}
+    if heads is None:
+        out["u"] = output_projection(out["o"], W)
+    return out
+
+
+def mla_prefill(h, cu_seqlens, W, dims, query_rows=None, heads=None):
+    """Causal prefill from hidden states, steps (1)-(10) for every sequence packed by cu_seqlens.
+
+    Every token's cache row is computed; attention, o and u only for query_rows (global token
+    indices, default all). Returns dict with cache [T, d_c + d_r], rows, o, o_lat, lse, u.
+    """
+    h = f64(h)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    T = h.shape[0]
+    pos = np.concatenate([np.arange(cu[b + 1] - cu[b]) for b in range(len(cu) - 1)]).astype(np.int64)
+    c_kv, k_r = kv_compression(h, W, dims, pos)
+    rows_all = np.arange(T) if query_rows is None else np.sort(np.asarray(query_rows, dtype=np.int64))
+    rows, o_l, lat_l, lse_l = [], [], [], []
+    for b in range(len(cu) - 1):
+        r = rows_all[(rows_all >= cu[b]) & (rows_all < cu[b + 1])]
+        if len(r) == 0:
+            continue
+        _, q_c, q_r = query_projections(h[r], W, dims, pos[r])
+        o, o_lat, lse = attend_unabsorbed(q_c, q_r, c_kv[cu[b]:cu[b + 1]], k_r[cu[b]:cu[b + 1]], W, dims,
+                                          pos[r], heads)
+        rows.append(r); o_l.append(o); lat_l.append(o_lat); lse_l.append(lse)
+    out = {"cache": cache_rows(c_kv, k_r), "rows": np.concatenate(rows), "o": np.concatenate(o_l),
+           "o_lat": np.concatenate(lat_l), "lse": np.concatenate(lse_l)}
+    if heads is None:
+        out["u"] = output_projection(out["o"], W)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# The latent-attention core by its own definition (absorbed score, section 2 【思考】 + section 3)
+# ---------------------------------------------------------------------------
+def absorb_query(q_c, W, dims) -> np.ndarray:
+    """q~_t,i = W_i^UK^T q^C_t,i in R^{d_c} (section 2 【思考】: W^UK folded into the query)."""
+    q_c = f64(q_c)
+    w_uk = f64(W["w_uk"]).reshape(dims.n_h, dims.d_h, dims.d_c)
+    return np.einsum("thk,hkc->thc", q_c, w_uk)
+
+
+def attn_decode_latent(q_abs, q_rope, cache, cu_seqlens, tq, dims, seqs=None, heads=None):
+    """Core over the latent cache: s_j = (q~.c_j + q^R.k^R_j)/sqrt(d_h + d_h^R), j <= pos,
+    o^lat = sum_j p_j c_j and lse (section 3's split of the score into a position-free
+    latent term and a RoPE term). q_abs [B*Tq, n_h, d_c], q_rope [B*Tq, n_h, d_r].
+    """
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    B = len(cu) - 1
+    seqs = range(B) if seqs is None else list(seqs)
+    heads = range(dims.n_h) if heads is None else list(heads)
+    pos_all = decode_positions(cu, tq)
+    scale = 1.0 / np.sqrt(dims.d_h + dims.d_r)
+    cache = f64(cache)
+    lat_l, lse_l = [], []
+    for b in seqs:
+        r = np.arange(b * tq, (b + 1) * tq)
+        seq = cache[cu[b]:cu[b + 1]]
+        lat = np.empty((tq, len(heads), dims.d_c))
+        lse = np.empty((tq, len(heads)))
+        for hi, i in enumerate(heads):
+            q = np.concatenate([f64(q_abs)[r, i], f64(q_rope)[r, i]], axis=1)
+            lat[:, hi], _, lse[:, hi], _ = causal_softmax_attend(q, seq, seq[:, :dims.d_c], None,
+                                                                   pos_all[r], scale)
+        lat_l.append(lat); lse_l.append(lse)
+    return np.concatenate(lat_l), np.concatenate(lse_l)
+
+
+def value_up_projection(o_lat, W, dims) -> np.ndarray:
+    """o_t,i = W_i^UV o^lat_t,i (section 2 【思考】: the value path moved after attention)."""
+    w_uv = f64(W["w_uv"]).reshape(dims.n_h, dims.d_h, dims.d_c)
+    return np.einsum("thc,hdc->thd", f64(o_lat), w_uv)
+
+
+def mla_decode_absorbed(h_q, cache, cu_seqlens, tq, W, dims):
+    """The absorbed form end to end: W^UK folded into the query, W^UV after attention.
+
+    Used only to check the unabsorbed oracle against the exact identity of section 2 【思考】.
+    """
+    pos = decode_positions(cu_seqlens, tq)
+    _, q_c, q_r = query_projections(h_q, W, dims, pos)
+    q_abs = absorb_query(q_c, W, dims)
+    o_lat, lse = attn_decode_latent(q_abs, q_r, cache, cu_seqlens, tq, dims)
+    o = value_up_projection(o_lat, W, dims)
+    return {"o_lat": o_lat, "lse": lse, "o": o, "u": output_projection(o, W), "q_abs": q_abs, "q_r": q_r}
+
+
+def output_absorbed(o_lat, W, dims) -> np.ndarray:
+    """u_t = sum_i W_i^O' o^lat_t,i with W_i^O' = W_i^O W_i^UV (section 2 【思考】, second absorption)."""
+    w_o = f64(W["w_o"]).reshape(-1, dims.n_h, dims.d_h)          # [d, n_h, d_h]
+    w_uv = f64(W["w_uv"]).reshape(dims.n_h, dims.d_h, dims.d_c)  # [n_h, d_h, d_c]
+    w_o_prime = np.einsum("xhd,hdc->xhc", w_o, w_uv)              # [d, n_h, d_c]
+    return np.einsum("thc,xhc->tx", f64(o_lat), w_o_prime)
+
+
+# ---------------------------------------------------------------------------
+# Split-KV combine (exact identity of the softmax; used by the tests' combine pin)
+# ---------------------------------------------------------------------------
+def lse_combine(parts):
+    """Merge (o_s, lse_s) partial results over disjoint key sets: lse = log sum_s e^{lse_s},
+    o = sum_s e^{lse_s - lse} o_s."""
+    lses = np.stack([f64(l) for _, l in parts])
+    top = lses.max(axis=0)
+    lse = top + np.log(np.exp(lses - top).sum(axis=0))
+    o = sum(np.exp(f64(l) - lse)[..., None] * f64(x) for x, l in parts)
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Cache-size bookkeeping (section 1 MHA cache, section 3 decoupled-key cache)
+# ---------------------------------------------------------------------------
+def mha_cache_elements_per_token(dims, layers: int) -> int:
+    """2 n_h d_h l elements per token for multi-head attention."""
+    return 2 * dims.n_h * dims.d_h * layers
+
+
+def mla_cache_elements_per_token(dims, layers: int) -> int:
+    """(d_c + d_h^R) l elements per token for MLA with the decoupled RoPE key."""
+    return (dims.d_c + dims.d_r) * layers
