@@ -1,0 +1,182 @@
+/*
+ * mla.h - C ABI of libmla.so: DeepSeek-V3 Multi-head Latent Attention (MLA) over the
+ * latent KV cache, hand-written CUDA for B200 (sm_100a).
+ *
+ * Source of the operations: the notes "【论文解读】DeepSeek-V3"
+ * (wkq9411.github.io/2026-01-01/Paper-DeepSeek-V3.html), section 一(一) "多头潜在注意力MLA":
+ *   2 "低秩KV联合压缩"  c^KV = W^DKV h, k^C = W^UK c^KV, v^C = W^UV c^KV, c^Q = W^DQ h, q^C = W^UQ c^Q;
+ *                       the 【思考】 block folds W_i^UK into the query and moves W_i^UV after attention;
+ *   3 "解耦RoPE"        q^R = RoPE(W^QR c^Q) per head, shared k^R = RoPE(W^KR h), the score
+ *                       q^C_i.k^C_j,i + q^R_i.k^R_j scaled by 1/sqrt(d_h + d_h^R), causal softmax,
+ *                       o_i = sum_j p_j v^C_j,i, u = W^O [o_1; ...; o_nh]; only c^KV and k^R are
+ *                       cached, (d_c + d_h^R) elements per token and layer.
+ *
+ * Conventions for every call
+ *   - Tensors are caller-owned device memory, borrowed for the duration of the call (weights:
+ *     until the handle is destroyed or given new weights). Nothing is copied to the host.
+ *   - Row-major. Weights are [out, in]: W^DQ [d_cq, d], W^UQ [n_h d_h, d_cq], W^QR [n_h d_r, d_cq],
+ *     W^DKV [d_c, d], W^KR [d_r, d], W^UK [n_h d_h, d_c], W^UV [n_h d_h, d_c], W^O [d, n_h d_h].
+ *     Multi-head vectors are head-major concatenations [x_1; ...; x_nh], so W_i^UK is rows
+ *     [i d_h, (i+1) d_h) of W^UK.
+ *   - The latent cache is [capacity, d_c + d_r] in the handle's dtype: c^KV in columns [0, d_c),
+ *     the rotated k^R in columns [d_c, d_c + d_r). At the V3 sizes a row is 1152 bytes in bf16.
+ *   - Sequences are packed and addressed by cu_seqlens: device int64 [B + 1], cu[0] = 0,
+ *     non-decreasing; sequence b owns cache rows [cu[b], cu[b+1]). Positions are 0-based
+ *     within a sequence. RoPE rotates interleaved pairs (2m, 2m+1) by pos * base^(-2m/d_r).
+ *   - Every call is asynchronous on the given stream and returns a status; it never throws.
+ *     Host-side validation (null pointers, sizes, alignment, workspace) runs before any launch:
+ *     on failure nothing is launched and nothing is written. Device-side checks (cu_seqlens
+ *     order, lengths, slots, positions) set a sticky error word in the handle and skip the
+ *     offending rows; mla_sync_status() reports it.
+ *   - Device pointers must be 16-byte aligned (MLA_ERR_ALIGNMENT otherwise).
+ *   - A handle may be used from several streams for different calls as long as calls that
+ *     share a workspace or output buffer are ordered by the caller.
+ */
+#ifndef MLA_H
+#define MLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; callers need no CUDA header. NULL is the legacy default stream. */
+typedef struct CUstream_st *mla_stream_t;
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, Tq outside {1, 2}, bad op        */
+  MLA_ERR_ALIGNMENT = 2,     /* a device pointer is not 16-byte aligned                         */
+  MLA_ERR_UNSUPPORTED = 3,   /* dims/dtype combination this build has no kernel for              */
+  MLA_ERR_WORKSPACE = 4,     /* ws_bytes below mla_workspace_size()                              */
+  MLA_ERR_CUDA = 5,          /* a CUDA runtime call failed (the CUDA error is not cleared)       */
+  MLA_ERR_TIMEOUT = 6,       /* a device-side bounded wait gave up (kernel returned early)       */
+  MLA_ERR_DEVICE_CHECK = 7,  /* a device-side argument check failed (see mla_device_error_bits)  */
+  MLA_ERR_NO_WEIGHTS = 8     /* mla_set_weights() was not called                                  */
+} mla_status_t;
+
+typedef enum { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype_t;
+
+/* Notation of section 一(一): d, n_h, d_h, d_c, d_c' (d_cq), d_h^R (d_r); RoPE base (10000). */
+typedef struct {
+  int32_t d, n_h, d_h, d_c, d_cq, d_r;
+  double rope_base;
+} mla_dims_t;
+
+/* Device pointers in the handle's dtype, row-major [out, in]; borrowed, not copied. */
+typedef struct {
+  const void *w_dq, *w_uq, *w_qr, *w_dkv, *w_kr, *w_uk, *w_uv, *w_o;
+} mla_weights_t;
+
+typedef enum {
+  MLA_OP_CACHE_APPEND = 0,
+  MLA_OP_DECODE = 1,
+  MLA_OP_PREFILL = 2,
+  MLA_OP_ATTN_DECODE_LATENT = 3
+} mla_op_t;
+
+/* Named workspace regions, readable after a call for step-level inspection. */
+typedef enum {
+  MLA_BUF_CQ = 0,      /* c^Q   [T, d_cq]          handle dtype (decode, prefill)               */
+  MLA_BUF_QC = 1,      /* q^C   [T, n_h, d_h]      handle dtype (decode, prefill)               */
+  MLA_BUF_QR = 2,      /* q^R   [T, n_h, d_r]      handle dtype, rotated (decode, prefill)      */
+  MLA_BUF_QABS = 3,    /* q~    [T, n_h, d_c]      handle dtype, W^UK folded in (decode)        */
+  MLA_BUF_OLAT = 4,    /* o^lat [T, n_h, d_c]      handle dtype, sum_j p_j c_j (decode)         */
+  MLA_BUF_O = 5,       /* o     [T, n_h, d_h]      handle dtype (decode, prefill)               */
+  MLA_BUF_KC = 6,      /* k^C   [T, n_h, d_h]      handle dtype (prefill)                       */
+  MLA_BUF_VC = 7,      /* v^C   [T, n_h, d_h]      handle dtype (prefill)                       */
+  MLA_BUF_LSE = 8      /* lse   [T, n_h]           fp32 (decode)                                */
+} mla_buffer_t;
+
+typedef struct mla_handle mla_handle_t;
+
+/* Creates a handle for one device. Host-only: no CUDA call is made here.
+ * dims must describe an MLA layer (all sizes > 0, d_r even); *out receives the handle. */
+mla_status_t mla_create(const mla_dims_t *dims, mla_dtype_t dtype, int device, mla_handle_t **out);
+
+/* Borrows the eight weight matrices (section 一(一)2 and 3). The first call on a device also
+ * allocates the handle's 4-byte device error word. */
+mla_status_t mla_set_weights(mla_handle_t *h, const mla_weights_t *w);
+
+/* Workspace bytes for one call of `op` on num_seqs sequences with tq query tokens each
+ * (decode, attention core) or total_tokens packed tokens (prefill, cache append).
+ * Host-only arithmetic. */
+mla_status_t mla_workspace_size(const mla_handle_t *h, mla_op_t op, int64_t num_seqs, int32_t tq,
+                                int64_t total_tokens, size_t *bytes);
+
+/* Byte offset of a named region inside that workspace (same arguments as mla_workspace_size).
+ * MLA_ERR_INVALID_ARG if the op has no such region. Host-only arithmetic. */
+mla_status_t mla_workspace_offset(const mla_handle_t *h, mla_op_t op, int64_t num_seqs, int32_t tq,
+                                  int64_t total_tokens, mla_buffer_t which, size_t *offset);
+
+/* Steps (5), (7) and the cache write of section 一(一)3: for each of the T tokens,
+ * c^KV = W^DKV h_t and k^R = RoPE_pos(W^KR h_t), stored as one row at cache[slots[t]].
+ *   h          [T, d]            handle dtype
+ *   positions  [T] device int64  position of each token within its sequence (>= 0)
+ *   slots      [T] device int64  destination row, 0 <= slot < capacity (else skipped + flagged)
+ *   cache      [capacity, d_c + d_r]
+ * No workspace is needed (ws may be NULL when ws_bytes is 0). */
+mla_status_t mla_cache_append(mla_handle_t *h, const void *hidden, const int64_t *positions,
+                              const int64_t *slots, int64_t T, void *cache, int64_t capacity,
+                              void *ws, size_t ws_bytes, mla_stream_t stream);
+
+/* Decode step, absorbed form (section 一(一)2 【思考】 with the decoupled RoPE of section 3):
+ * c^Q = W^DQ h; q^C = W^UQ c^Q; q^R = RoPE(W^QR c^Q); q~_i = W_i^UK^T q^C_i;
+ * split-KV latent attention s_j = (q~_i.c_j + q^R_i.k^R_j)/sqrt(d_h + d_r) over j <= pos with an
+ * exact log-sum-exp merge of the splits; o_i = W_i^UV o^lat_i; u = W^O [o_1; ...; o_nh].
+ *   h_q        [B*Tq, d]          query tokens, sequence-major (token k of sequence b at b*Tq + k)
+ *   cu_seqlens [B + 1] device     cache lengths INCLUDING the Tq query tokens (append first);
+ *                                 query k of sequence b is at position len_b - Tq + k and sees
+ *                                 cache rows cu[b] .. cu[b] + its position. len_b >= Tq.
+ *   cache      [capacity, d_c + d_r]
+ *   u_out      [B*Tq, d]          handle dtype
+ * Tq is 1 or 2. */
+mla_status_t mla_decode(mla_handle_t *h, const void *h_q, int64_t B, int32_t Tq,
+                        const int64_t *cu_seqlens, const void *cache, int64_t capacity, void *u_out,
+                        void *ws, size_t ws_bytes, mla_stream_t stream);
+
+/* Causal prefill from hidden states, unabsorbed form (section 一(一)3 steps (1)-(10)):
+ * writes every token's latent row to cache[cu[b] + t], up-projects k^C, v^C from those rows,
+ * runs causal attention per head (keys [k^C_i; k^R], values v^C_i) and applies W^O.
+ *   hidden     [total_tokens, d]  packed by cu_seqlens (cu[B] == total_tokens)
+ *   max_seqlen upper bound on any sequence length (sizes the launch; longer rows are skipped
+ *              and flagged)
+ *   cache      [capacity, d_c + d_r], capacity >= total_tokens
+ *   u_out      [total_tokens, d]  handle dtype */
+mla_status_t mla_prefill(mla_handle_t *h, const void *hidden, int64_t B, const int64_t *cu_seqlens,
+                         int64_t total_tokens, int64_t max_seqlen, void *cache, int64_t capacity,
+                         void *u_out, void *ws, size_t ws_bytes, mla_stream_t stream);
+
+/* The latent attention core alone (decode semantics as mla_decode):
+ *   q_abs  [B*Tq, n_h, d_c]  handle dtype (q~ = W_i^UK^T q^C_i)
+ *   q_rope [B*Tq, n_h, d_r]  handle dtype (rotated q^R)
+ *   o_lat  [B*Tq, n_h, d_c]  fp32, sum_j p_j c_j
+ *   lse    [B*Tq, n_h]       fp32, natural log of sum_j exp(s_j) */
+mla_status_t mla_attn_decode_latent(mla_handle_t *h, const void *q_abs, const void *q_rope, int64_t B,
+                                    int32_t Tq, const int64_t *cu_seqlens, const void *cache,
+                                    int64_t capacity, float *o_lat, float *lse, void *ws,
+                                    size_t ws_bytes, mla_stream_t stream);
+
+/* Synchronizes the stream, then reports (and clears) the handle's device error word:
+ * MLA_ERR_TIMEOUT, MLA_ERR_DEVICE_CHECK or MLA_OK. */
+mla_status_t mla_sync_status(mla_handle_t *h, mla_stream_t stream);
+
+/* Bits of the last error word read by mla_sync_status (see MLA_DEVERR_* in the source). */
+uint32_t mla_device_error_bits(const mla_handle_t *h);
+
+/* Which kernel family a call of `op` takes with this handle: 1 = tcgen05/TMA (BF16 at the V3
+ * sizes), 0 = generic CUDA-core kernels (FP32, or other sizes). Host-only. */
+int mla_uses_tensor_cores(const mla_handle_t *h, mla_op_t op);
+
+const char *mla_status_string(mla_status_t s);
+
+/* Frees the handle's own device memory (its error word). Borrowed tensors are untouched. */
+void mla_destroy(mla_handle_t *h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H */

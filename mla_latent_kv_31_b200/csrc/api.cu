@@ -1,0 +1,456 @@
+// C ABI of libmla.so (declared in include/mla.h): validation, workspace layout, dispatch.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "mla.h"
+#include "common.cuh"
+#include "simt.cuh"
+#include "tc.cuh"
+
+struct mla_handle {
+  mla_dims_t dims;
+  mla_dtype_t dtype;
+  int device;
+  mla_weights_t w;
+  bool has_weights;
+  uint32_t* d_err;         // device error word (sticky until mla_sync_status)
+  uint32_t last_err_bits;  // last word read by mla_sync_status
+  int num_sms;
+};
+
+namespace {
+
+using mla::SimtAttnArgs;
+using mla::SimtGemmArgs;
+
+constexpr size_t kAlign = 1024;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t elem_size(const mla_handle* h) { return h->dtype == MLA_BF16 ? 2 : 4; }
+
+// True when the tcgen05/TMA kernels cover this handle: BF16 at the DeepSeek-V3 sizes.
+bool tc_dims(const mla_handle* h) {
+  const mla_dims_t& d = h->dims;
+  return h->dtype == MLA_BF16 && d.n_h == 128 && d.d_h == 128 && d.d_c == 512 && d.d_r == 64 &&
+         d.d_cq % 64 == 0 && d.d % 64 == 0;
+}
+
+struct Layout {
+  size_t off[9];
+  bool has[9];
+  size_t pos_off;     // int64 positions [T]
+  size_t tc_off;      // tensor-core attention scratch
+  size_t total;
+};
+
+// Workspace layout of one call; every region starts on a 1024-byte boundary.
+Layout layout(const mla_handle* h, mla_op_t op, int64_t B, int32_t tq, int64_t total_tokens) {
+  Layout L;
+  memset(&L, 0, sizeof(L));
+  const mla_dims_t& d = h->dims;
+  const size_t es = elem_size(h);
+  const int64_t T = (op == MLA_OP_DECODE || op == MLA_OP_ATTN_DECODE_LATENT) ? B * tq : total_tokens;
+  size_t cur = 0;
+  auto take = [&](int which, size_t bytes) {
+    L.off[which] = cur;
+    L.has[which] = true;
+    cur = align_up(cur + bytes);
+  };
+  if (op == MLA_OP_DECODE || op == MLA_OP_PREFILL) {
+    take(MLA_BUF_CQ, (size_t)T * d.d_cq * es);
+    take(MLA_BUF_QC, (size_t)T * d.n_h * d.d_h * es);
+    take(MLA_BUF_QR, (size_t)T * d.n_h * d.d_r * es);
+    take(MLA_BUF_O, (size_t)T * d.n_h * d.d_h * es);
+  }
+  if (op == MLA_OP_DECODE) {
+    take(MLA_BUF_QABS, (size_t)T * d.n_h * d.d_c * es);
+    take(MLA_BUF_OLAT, (size_t)T * d.n_h * d.d_c * es);
+    take(MLA_BUF_LSE, (size_t)T * d.n_h * sizeof(float));
+  }
+  if (op == MLA_OP_PREFILL) {
+    take(MLA_BUF_KC, (size_t)T * d.n_h * d.d_h * es);
+    take(MLA_BUF_VC, (size_t)T * d.n_h * d.d_h * es);
+  }
+  if (op != MLA_OP_CACHE_APPEND) {
+    L.pos_off = cur;
+    cur = align_up(cur + (size_t)(T > 0 ? T : 1) * sizeof(int64_t));
+  }
+  if ((op == MLA_OP_DECODE || op == MLA_OP_ATTN_DECODE_LATENT) && tc_dims(h)) {
+    L.tc_off = cur;
+    cur = align_up(cur + mla::tc_decode_scratch_bytes(B, tq));
+  }
+  L.total = cur;
+  return L;
+}
+
+mla_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+#define MLA_TRY(expr)                              \
+  do {                                             \
+    cudaError_t _e = (expr);                       \
+    if (_e != cudaSuccess) return MLA_ERR_CUDA;    \
+  } while (0)
+
+mla_status_t ensure_device(mla_handle* h) {
+  MLA_TRY(cudaSetDevice(h->device));
+  if (!h->d_err) {
+    MLA_TRY(cudaMalloc(&h->d_err, sizeof(uint32_t)));
+    MLA_TRY(cudaMemset(h->d_err, 0, sizeof(uint32_t)));
+    int sms = 0;
+    MLA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device));
+    h->num_sms = sms;
+  }
+  return MLA_OK;
+}
+
+mla_status_t check_ready(mla_handle* h) {
+  if (!h) return MLA_ERR_INVALID_ARG;
+  if (!h->has_weights) return MLA_ERR_NO_WEIGHTS;
+  return ensure_device(h);
+}
+
+// --- generic (CUDA-core) building blocks ----------------------------------------------------
+SimtGemmArgs gemm_args() {
+  SimtGemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.batch = 1;
+  return a;
+}
+
+// C[M, N] = A[M, K] . W[N, K]^T with dense row-major A (row stride lda) and W.
+SimtGemmArgs dense_nt(const void* A, int64_t lda, const void* W, void* C, int64_t ldc, int64_t M, int64_t N,
+                      int64_t K) {
+  SimtGemmArgs a = gemm_args();
+  a.A = A; a.sam = lda; a.sak = 1;
+  a.B = W; a.sbn = K; a.sbk = 1;
+  a.C = C; a.scm = ldc; a.scn = 1;
+  a.M = M; a.N = N; a.K = K;
+  return a;
+}
+
+mla_status_t run_simt_gemm(const mla_handle* h, SimtGemmArgs a, cudaStream_t st, bool out_bf16) {
+  a.err = h->d_err;
+  return cuda_status(mla::simt_gemm(a, h->dtype == MLA_BF16, out_bf16, st));
+}
+
+// Steps (5), (7) + cache write: rows [c^KV | RoPE(W^KR h)] scattered to cache[rowmap[t]].
+mla_status_t simt_cache_rows(const mla_handle* h, const void* hidden, const int64_t* pos, const int64_t* rowmap,
+                             int64_t T, void* cache, int64_t capacity, cudaStream_t st) {
+  const mla_dims_t& d = h->dims;
+  const size_t es = elem_size(h);
+  const bool bf = h->dtype == MLA_BF16;
+  const int64_t R = d.d_c + d.d_r;
+  SimtGemmArgs a = dense_nt(hidden, d.d, h->w.w_dkv, cache, R, T, d.d_c, d.d);
+  a.rowmap = rowmap; a.rowmap_limit = capacity;
+  mla_status_t s = run_simt_gemm(h, a, st, bf);
+  if (s != MLA_OK) return s;
+  SimtGemmArgs b = dense_nt(hidden, d.d, h->w.w_kr, (char*)cache + (size_t)d.d_c * es, R, T, d.d_r, d.d);
+  b.rowmap = rowmap; b.rowmap_limit = capacity;
+  b.pos = pos; b.rope_col0 = 0; b.d_r = d.d_r; b.rope_base = d.rope_base;
+  return run_simt_gemm(h, b, st, bf);
+}
+
+// Steps (1)-(3): c^Q, q^C and the rotated q^R of T tokens at positions pos.
+mla_status_t simt_queries(const mla_handle* h, const void* hidden, const int64_t* pos, int64_t T, void* cq,
+                          void* qc, void* qr, cudaStream_t st) {
+  const mla_dims_t& d = h->dims;
+  const bool bf = h->dtype == MLA_BF16;
+  mla_status_t s = run_simt_gemm(h, dense_nt(hidden, d.d, h->w.w_dq, cq, d.d_cq, T, d.d_cq, d.d), st, bf);
+  if (s != MLA_OK) return s;
+  s = run_simt_gemm(h, dense_nt(cq, d.d_cq, h->w.w_uq, qc, (int64_t)d.n_h * d.d_h, T, (int64_t)d.n_h * d.d_h,
+                                d.d_cq), st, bf);
+  if (s != MLA_OK) return s;
+  SimtGemmArgs a = dense_nt(cq, d.d_cq, h->w.w_qr, qr, (int64_t)d.n_h * d.d_r, T, (int64_t)d.n_h * d.d_r, d.d_cq);
+  a.pos = pos; a.rope_col0 = 0; a.d_r = d.d_r; a.rope_base = d.rope_base;
+  return run_simt_gemm(h, a, st, bf);
+}
+
+// Step (10), second equation: u = W^O [o_1; ...; o_nh].
+mla_status_t simt_output(const mla_handle* h, const void* o, int64_t T, void* u, cudaStream_t st) {
+  const mla_dims_t& d = h->dims;
+  const int64_t HD = (int64_t)d.n_h * d.d_h;
+  return run_simt_gemm(h, dense_nt(o, HD, h->w.w_o, u, d.d, T, d.d, HD), st, h->dtype == MLA_BF16);
+}
+
+// Latent attention core by CUDA cores: q~ [T, n_h, d_c], q^R [T, n_h, d_r] over the cache.
+mla_status_t simt_latent_core(const mla_handle* h, const void* q_abs, const void* q_rope, int64_t B, int32_t tq,
+                              const int64_t* cu, const void* cache, int64_t capacity, void* o_lat, bool o_f32,
+                              float* lse, cudaStream_t st) {
+  const mla_dims_t& d = h->dims;
+  const size_t es = elem_size(h);
+  const int64_t R = d.d_c + d.d_r;
+  SimtAttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q1 = q_abs; a.sq1t = (int64_t)d.n_h * d.d_c; a.sq1h = d.d_c; a.d1 = d.d_c;
+  a.q2 = q_rope; a.sq2t = (int64_t)d.n_h * d.d_r; a.sq2h = d.d_r; a.d2 = d.d_r;
+  a.k1 = cache; a.sk1 = R; a.sk1h = 0;
+  a.k2 = (const char*)cache + (size_t)d.d_c * es; a.sk2 = R;
+  a.v = cache; a.sv = R; a.svh = 0; a.dv = d.d_c;
+  a.o = o_lat; a.sot = (int64_t)d.n_h * d.d_c; a.soh = d.d_c;
+  a.lse = lse;
+  a.cu = cu; a.B = B; a.tq = tq; a.T = B * tq; a.n_h = d.n_h; a.capacity = capacity;
+  a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
+  a.err = h->d_err;
+  return cuda_status(mla::simt_attention(a, h->dtype == MLA_BF16, o_f32, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status_t s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG: null pointer, bad size or bad enum";
+    case MLA_ERR_ALIGNMENT: return "MLA_ERR_ALIGNMENT: device pointer not 16-byte aligned";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: no kernel for these dims/dtype";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE: workspace smaller than mla_workspace_size()";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA runtime call failed";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT: a bounded device-side wait gave up";
+    case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK: device-side argument check failed";
+    case MLA_ERR_NO_WEIGHTS: return "MLA_ERR_NO_WEIGHTS: mla_set_weights() not called";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+mla_status_t mla_create(const mla_dims_t* dims, mla_dtype_t dtype, int device, mla_handle_t** out) {
+  if (!dims || !out) return MLA_ERR_INVALID_ARG;
+  *out = nullptr;
+  const mla_dims_t& d = *dims;
+  if (d.d <= 0 || d.n_h <= 0 || d.d_h <= 0 || d.d_c <= 0 || d.d_cq <= 0 || d.d_r <= 0 || (d.d_r & 1) ||
+      !(d.rope_base > 1.0) || device < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (dtype != MLA_BF16 && dtype != MLA_FP32) return MLA_ERR_INVALID_ARG;
+  // Generic kernels hold one latent row of q in shared memory and up to 512 value columns.
+  if (d.d_c > 512 || d.d_h > 512 || d.d_c + d.d_r > 1024 || d.d_h + d.d_r > 1024) return MLA_ERR_UNSUPPORTED;
+  mla_handle* h = new (std::nothrow) mla_handle;
+  if (!h) return MLA_ERR_INVALID_ARG;
+  memset(h, 0, sizeof(*h));
+  h->dims = d;
+  h->dtype = dtype;
+  h->device = device;
+  *out = h;
+  return MLA_OK;
+}
+
+mla_status_t mla_set_weights(mla_handle_t* h, const mla_weights_t* w) {
+  if (!h || !w) return MLA_ERR_INVALID_ARG;
+  const void* ps[8] = {w->w_dq, w->w_uq, w->w_qr, w->w_dkv, w->w_kr, w->w_uk, w->w_uv, w->w_o};
+  for (const void* p : ps) {
+    if (!p) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(p)) return MLA_ERR_ALIGNMENT;
+  }
+  mla_status_t s = ensure_device(h);
+  if (s != MLA_OK) return s;
+  h->w = *w;
+  h->has_weights = true;
+  return MLA_OK;
+}
+
+mla_status_t mla_workspace_size(const mla_handle_t* h, mla_op_t op, int64_t num_seqs, int32_t tq,
+                                int64_t total_tokens, size_t* bytes) {
+  if (!h || !bytes) return MLA_ERR_INVALID_ARG;
+  if (op < MLA_OP_CACHE_APPEND || op > MLA_OP_ATTN_DECODE_LATENT) return MLA_ERR_INVALID_ARG;
+  if (op == MLA_OP_DECODE || op == MLA_OP_ATTN_DECODE_LATENT) {
+    if (num_seqs <= 0 || (tq != 1 && tq != 2)) return MLA_ERR_INVALID_ARG;
+  } else if (total_tokens <= 0) {
+    return MLA_ERR_INVALID_ARG;
+  }
+  *bytes = op == MLA_OP_CACHE_APPEND ? 0 : layout(h, op, num_seqs, tq, total_tokens).total;
+  return MLA_OK;
+}
+
+mla_status_t mla_workspace_offset(const mla_handle_t* h, mla_op_t op, int64_t num_seqs, int32_t tq,
+                                  int64_t total_tokens, mla_buffer_t which, size_t* offset) {
+  size_t total = 0;
+  mla_status_t s = mla_workspace_size(h, op, num_seqs, tq, total_tokens, &total);
+  if (s != MLA_OK) return s;
+  if (!offset || which < MLA_BUF_CQ || which > MLA_BUF_LSE) return MLA_ERR_INVALID_ARG;
+  Layout L = layout(h, op, num_seqs, tq, total_tokens);
+  if (!L.has[which]) return MLA_ERR_INVALID_ARG;
+  *offset = L.off[which];
+  return MLA_OK;
+}
+
+int mla_uses_tensor_cores(const mla_handle_t* h, mla_op_t op) {
+  if (!h) return 0;
+  return tc_dims(h) && mla::tc_available(op) ? 1 : 0;
+}
+
+mla_status_t mla_cache_append(mla_handle_t* h, const void* hidden, const int64_t* positions, const int64_t* slots,
+                              int64_t T, void* cache, int64_t capacity, void* ws, size_t ws_bytes,
+                              mla_stream_t stream) {
+  (void)ws; (void)ws_bytes;
+  if (!h || !hidden || !positions || !slots || !cache || T <= 0 || capacity <= 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(cache) || !aligned16(positions) || !aligned16(slots))
+    return MLA_ERR_ALIGNMENT;
+  mla_status_t s = check_ready(h);
+  if (s != MLA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (tc_dims(h) && mla::tc_available(MLA_OP_CACHE_APPEND))
+    return cuda_status(mla::tc_cache_append(h->dims, h->w, hidden, positions, slots, T, cache, capacity,
+                                            h->d_err, st));
+  return simt_cache_rows(h, hidden, positions, slots, T, cache, capacity, st);
+}
+
+mla_status_t mla_attn_decode_latent(mla_handle_t* h, const void* q_abs, const void* q_rope, int64_t B, int32_t Tq,
+                                    const int64_t* cu_seqlens, const void* cache, int64_t capacity, float* o_lat,
+                                    float* lse, void* ws, size_t ws_bytes, mla_stream_t stream) {
+  if (!h || !q_abs || !q_rope || !cu_seqlens || !cache || !o_lat || !lse || B <= 0 || capacity <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (Tq != 1 && Tq != 2) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_abs) || !aligned16(q_rope) || !aligned16(cache) || !aligned16(o_lat) || !aligned16(lse) ||
+      !aligned16(cu_seqlens) || (ws && !aligned16(ws)))
+    return MLA_ERR_ALIGNMENT;
+  Layout L = layout(h, MLA_OP_ATTN_DECODE_LATENT, B, Tq, 0);
+  if (ws_bytes < L.total || (L.total > 0 && !ws)) return MLA_ERR_WORKSPACE;
+  mla_status_t s = ensure_device(h);  // the core needs no weights
+  if (s != MLA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* w = (char*)ws;
+  MLA_TRY(mla::check_and_positions(cu_seqlens, B, Tq, B * Tq, capacity, 0, (int64_t*)(w + L.pos_off), h->d_err,
+                                   st));
+  if (tc_dims(h) && mla::tc_available(MLA_OP_ATTN_DECODE_LATENT))
+    return cuda_status(mla::tc_latent_core(h->dims, q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, true,
+                                           lse, w + L.tc_off, h->num_sms, h->d_err, st));
+  return simt_latent_core(h, q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, true, lse, st);
+}
+
+mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq, const int64_t* cu_seqlens,
+                        const void* cache, int64_t capacity, void* u_out, void* ws, size_t ws_bytes,
+                        mla_stream_t stream) {
+  if (!h || !h_q || !cu_seqlens || !cache || !u_out || !ws || B <= 0 || capacity <= 0) return MLA_ERR_INVALID_ARG;
+  if (Tq != 1 && Tq != 2) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h_q) || !aligned16(cache) || !aligned16(u_out) || !aligned16(ws) || !aligned16(cu_seqlens))
+    return MLA_ERR_ALIGNMENT;
+  Layout L = layout(h, MLA_OP_DECODE, B, Tq, 0);
+  if (ws_bytes < L.total) return MLA_ERR_WORKSPACE;
+  mla_status_t s = check_ready(h);
+  if (s != MLA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const mla_dims_t& d = h->dims;
+  char* w = (char*)ws;
+  const int64_t T = B * Tq;
+  int64_t* pos = (int64_t*)(w + L.pos_off);
+  void* cq = w + L.off[MLA_BUF_CQ];
+  void* qc = w + L.off[MLA_BUF_QC];
+  void* qr = w + L.off[MLA_BUF_QR];
+  void* qabs = w + L.off[MLA_BUF_QABS];
+  void* olat = w + L.off[MLA_BUF_OLAT];
+  void* o = w + L.off[MLA_BUF_O];
+  float* lse = (float*)(w + L.off[MLA_BUF_LSE]);
+  MLA_TRY(mla::check_and_positions(cu_seqlens, B, Tq, T, capacity, 0, pos, h->d_err, st));
+  if (tc_dims(h) && mla::tc_available(MLA_OP_DECODE))
+    return cuda_status(mla::tc_decode(d, h->w, h_q, B, Tq, cu_seqlens, pos, cache, capacity, u_out, cq, qc, qr,
+                                      qabs, olat, o, lse, w + L.tc_off, h->num_sms, h->d_err, st));
+  // Steps (1)-(3)
+  s = simt_queries(h, h_q, pos, T, cq, qc, qr, st);
+  if (s != MLA_OK) return s;
+  // q~_i = W_i^UK^T q^C_i (batched over heads): A(t, k) = q^C[t, i d_h + k], B(c, k) = W^UK[i d_h + k, c]
+  SimtGemmArgs a = gemm_args();
+  a.A = qc; a.sam = (int64_t)d.n_h * d.d_h; a.sak = 1; a.sab = d.d_h;
+  a.B = h->w.w_uk; a.sbn = 1; a.sbk = d.d_c; a.sbb = (int64_t)d.d_h * d.d_c;
+  a.C = qabs; a.scm = (int64_t)d.n_h * d.d_c; a.scn = 1; a.scb = d.d_c;
+  a.M = T; a.N = d.d_c; a.K = d.d_h; a.batch = d.n_h;
+  s = run_simt_gemm(h, a, st, h->dtype == MLA_BF16);
+  if (s != MLA_OK) return s;
+  s = simt_latent_core(h, qabs, qr, B, Tq, cu_seqlens, cache, capacity, olat, h->dtype == MLA_FP32, lse, st);
+  if (s != MLA_OK) return s;
+  // o_i = W_i^UV o^lat_i: A(t, c) = o^lat[t, i, c], B(k, c) = W^UV[i d_h + k, c]
+  SimtGemmArgs v = gemm_args();
+  v.A = olat; v.sam = (int64_t)d.n_h * d.d_c; v.sak = 1; v.sab = d.d_c;
+  v.B = h->w.w_uv; v.sbn = d.d_c; v.sbk = 1; v.sbb = (int64_t)d.d_h * d.d_c;
+  v.C = o; v.scm = (int64_t)d.n_h * d.d_h; v.scn = 1; v.scb = d.d_h;
+  v.M = T; v.N = d.d_h; v.K = d.d_c; v.batch = d.n_h;
+  s = run_simt_gemm(h, v, st, h->dtype == MLA_BF16);
+  if (s != MLA_OK) return s;
+  return simt_output(h, o, T, u_out, st);
+}
+
+mla_status_t mla_prefill(mla_handle_t* h, const void* hidden, int64_t B, const int64_t* cu_seqlens,
+                         int64_t total_tokens, int64_t max_seqlen, void* cache, int64_t capacity, void* u_out,
+                         void* ws, size_t ws_bytes, mla_stream_t stream) {
+  if (!h || !hidden || !cu_seqlens || !cache || !u_out || !ws || B <= 0 || total_tokens <= 0 || max_seqlen <= 0 ||
+      capacity < total_tokens)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(cache) || !aligned16(u_out) || !aligned16(ws) || !aligned16(cu_seqlens))
+    return MLA_ERR_ALIGNMENT;
+  Layout L = layout(h, MLA_OP_PREFILL, B, 0, total_tokens);
+  if (ws_bytes < L.total) return MLA_ERR_WORKSPACE;
+  mla_status_t s = check_ready(h);
+  if (s != MLA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const mla_dims_t& d = h->dims;
+  const size_t es = elem_size(h);
+  const int64_t T = total_tokens, R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
+  char* w = (char*)ws;
+  int64_t* pos = (int64_t*)(w + L.pos_off);
+  void* cq = w + L.off[MLA_BUF_CQ];
+  void* qc = w + L.off[MLA_BUF_QC];
+  void* qr = w + L.off[MLA_BUF_QR];
+  void* o = w + L.off[MLA_BUF_O];
+  void* kc = w + L.off[MLA_BUF_KC];
+  void* vc = w + L.off[MLA_BUF_VC];
+  MLA_TRY(mla::check_and_positions(cu_seqlens, B, 0, T, capacity, max_seqlen, pos, h->d_err, st));
+  if (tc_dims(h) && mla::tc_available(MLA_OP_PREFILL))
+    return cuda_status(mla::tc_prefill(d, h->w, hidden, B, cu_seqlens, T, max_seqlen, pos, cache, capacity, u_out,
+                                       cq, qc, qr, kc, vc, o, h->d_err, st));
+  // Steps (5), (7): cache rows of every token at row t (= cu[b] + position)
+  s = simt_cache_rows(h, hidden, pos, nullptr, T, cache, capacity, st);
+  if (s != MLA_OK) return s;
+  s = simt_queries(h, hidden, pos, T, cq, qc, qr, st);
+  if (s != MLA_OK) return s;
+  // Steps (6), (9): k^C = W^UK c^KV, v^C = W^UV c^KV from the cache rows just written
+  s = run_simt_gemm(h, dense_nt(cache, R, h->w.w_uk, kc, HD, T, HD, d.d_c), st, h->dtype == MLA_BF16);
+  if (s != MLA_OK) return s;
+  s = run_simt_gemm(h, dense_nt(cache, R, h->w.w_uv, vc, HD, T, HD, d.d_c), st, h->dtype == MLA_BF16);
+  if (s != MLA_OK) return s;
+  // Steps (4), (8), (10): causal attention per head with keys [k^C_i; k^R], values v^C_i
+  SimtAttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q1 = qc; a.sq1t = HD; a.sq1h = d.d_h; a.d1 = d.d_h;
+  a.q2 = qr; a.sq2t = (int64_t)d.n_h * d.d_r; a.sq2h = d.d_r; a.d2 = d.d_r;
+  a.k1 = kc; a.sk1 = HD; a.sk1h = d.d_h;
+  a.k2 = (const char*)cache + (size_t)d.d_c * es; a.sk2 = R;
+  a.v = vc; a.sv = HD; a.svh = d.d_h; a.dv = d.d_h;
+  a.o = o; a.sot = HD; a.soh = d.d_h;
+  a.lse = nullptr;
+  a.cu = cu_seqlens; a.B = B; a.tq = 0; a.T = T; a.n_h = d.n_h; a.capacity = capacity;
+  a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
+  a.err = h->d_err;
+  MLA_TRY(mla::simt_attention(a, h->dtype == MLA_BF16, h->dtype == MLA_FP32, st));
+  return simt_output(h, o, T, u_out, st);
+}
+
+mla_status_t mla_sync_status(mla_handle_t* h, mla_stream_t stream) {
+  if (!h) return MLA_ERR_INVALID_ARG;
+  if (!h->d_err) return MLA_OK;
+  MLA_TRY(cudaSetDevice(h->device));
+  MLA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+  uint32_t bits = 0;
+  MLA_TRY(cudaMemcpy(&bits, h->d_err, sizeof(bits), cudaMemcpyDeviceToHost));
+  MLA_TRY(cudaMemset(h->d_err, 0, sizeof(uint32_t)));
+  h->last_err_bits = bits;
+  if (bits & mla::DEVERR_TIMEOUT) return MLA_ERR_TIMEOUT;
+  if (bits) return MLA_ERR_DEVICE_CHECK;
+  return MLA_OK;
+}
+
+uint32_t mla_device_error_bits(const mla_handle_t* h) { return h ? h->last_err_bits : 0u; }
+
+void mla_destroy(mla_handle_t* h) {
+  if (!h) return;
+  if (h->d_err) {
+    cudaSetDevice(h->device);
+    cudaFree(h->d_err);
+  }
+  delete h;
+}
+
+}  // extern "C"

@@ -1,0 +1,35 @@
+// Tensor-core (tcgen05 / TMEM / TMA) kernels for BF16 at the DeepSeek-V3 MLA sizes
+// (n_h = 128, d_h = 128, d_c = 512, d_h^R = 64; d and d_c' multiples of 64).
+#pragma once
+
+#include <stdint.h>
+
+#include "mla.h"
+
+namespace mla {
+
+// Whether this build routes `op` through the tensor-core kernels.
+bool tc_available(mla_op_t op);
+
+// Scratch bytes of the split-KV latent core for B sequences of tq query tokens.
+size_t tc_decode_scratch_bytes(int64_t B, int32_t tq);
+
+cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const void* hidden,
+                            const int64_t* positions, const int64_t* slots, int64_t T, void* cache,
+                            int64_t capacity, uint32_t* err, cudaStream_t st);
+
+cudaError_t tc_latent_core(const mla_dims_t& d, const void* q_abs, const void* q_rope, int64_t B, int32_t tq,
+                           const int64_t* cu, const void* cache, int64_t capacity, void* o_lat, bool o_f32,
+                           float* lse, void* scratch, int num_sms, uint32_t* err, cudaStream_t st);
+
+cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const void* h_q, int64_t B, int32_t tq,
+                      const int64_t* cu, const int64_t* pos, const void* cache, int64_t capacity, void* u_out,
+                      void* cq, void* qc, void* qr, void* qabs, void* olat, void* o, float* lse, void* scratch,
+                      int num_sms, uint32_t* err, cudaStream_t st);
+
+cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, int64_t B,
+                       const int64_t* cu, int64_t T, int64_t max_seqlen, const int64_t* pos, void* cache,
+                       int64_t capacity, void* u_out, void* cq, void* qc, void* qr, void* kc, void* vc, void* o,
+                       uint32_t* err, cudaStream_t st);
+
+}  // namespace mla

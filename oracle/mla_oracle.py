@@ -190,12 +190,11 @@ def mla_decode(h_q, cache, cu_seqlens, tq, W, dims, seqs=None, heads=None):
     B = len(cu) - 1
     seqs = range(B) if seqs is None else list(seqs)
     pos_all = decode_positions(cu, tq)
-    cache = f64(cache)
     rows, o_l, lat_l, lse_l = [], [], [], []
     for b in seqs:
         r = np.arange(b * tq, (b + 1) * tq)
-        _, q_c, q_r = query_projections(f64(h_q)[r], W, dims, pos_all[r])
-        seq = cache[cu[b]:cu[b + 1]]
+        _, q_c, q_r = query_projections(f64(np.asarray(h_q)[r]), W, dims, pos_all[r])
+        seq = f64(cache[cu[b]:cu[b + 1]])
         o, o_lat, lse = attend_unabsorbed(q_c, q_r, seq[:, :dims.d_c], seq[:, dims.d_c:], W, dims,
                                           pos_all[r], heads)
         rows.append(r); o_l.append(o); lat_l.append(o_lat); lse_l.append(lse)
@@ -255,15 +254,14 @@ def attn_decode_latent(q_abs, q_rope, cache, cu_seqlens, tq, dims, seqs=None, he
     heads = range(dims.n_h) if heads is None else list(heads)
     pos_all = decode_positions(cu, tq)
     scale = 1.0 / np.sqrt(dims.d_h + dims.d_r)
-    cache = f64(cache)
     lat_l, lse_l = [], []
     for b in seqs:
         r = np.arange(b * tq, (b + 1) * tq)
-        seq = cache[cu[b]:cu[b + 1]]
+        seq = f64(cache[cu[b]:cu[b + 1]])
         lat = np.empty((tq, len(heads), dims.d_c))
         lse = np.empty((tq, len(heads)))
         for hi, i in enumerate(heads):
-            q = np.concatenate([f64(q_abs)[r, i], f64(q_rope)[r, i]], axis=1)
+            q = np.concatenate([f64(np.asarray(q_abs)[r, i]), f64(np.asarray(q_rope)[r, i])], axis=1)
             lat[:, hi], _, lse[:, hi], _ = causal_softmax_attend(q, seq, seq[:, :dims.d_c], None,
                                                                    pos_all[r], scale)
         lat_l.append(lat); lse_l.append(lse)
@@ -276,17 +274,26 @@ def value_up_projection(o_lat, W, dims) -> np.ndarray:
     return np.einsum("thc,hdc->thd", f64(o_lat), w_uv)
 
 
-def mla_decode_absorbed(h_q, cache, cu_seqlens, tq, W, dims):
+def mla_decode_absorbed(h_q, cache, cu_seqlens, tq, W, dims, seqs=None):
     """The absorbed form end to end: W^UK folded into the query, W^UV after attention.
 
-    Used only to check the unabsorbed oracle against the exact identity of section 2 【思考】.
+    An exact rewrite of the unabsorbed definition (section 2 【思考】; the tests pin the two
+    together to 1e-12). It costs O(d_c) instead of O(n_h d_h d_c) per cached row, which is what
+    lets the full-size tests check u over 128K-row caches. Rows are those of `seqs` (default all).
     """
-    pos = decode_positions(cu_seqlens, tq)
-    _, q_c, q_r = query_projections(h_q, W, dims, pos)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    seqs = range(len(cu) - 1) if seqs is None else list(seqs)
+    rows = np.concatenate([np.arange(b * tq, (b + 1) * tq) for b in seqs])
+    pos = decode_positions(cu, tq)[rows]
+    _, q_c, q_r = query_projections(np.asarray(h_q)[rows], W, dims, pos)
     q_abs = absorb_query(q_c, W, dims)
-    o_lat, lse = attn_decode_latent(q_abs, q_r, cache, cu_seqlens, tq, dims)
+    # re-index the chosen sequences as a packed batch of their own
+    sub_cache = np.concatenate([np.asarray(cache)[cu[b]:cu[b + 1]] for b in seqs])
+    sub_cu = np.concatenate([[0], np.cumsum([cu[b + 1] - cu[b] for b in seqs])]).astype(np.int64)
+    o_lat, lse = attn_decode_latent(q_abs, q_r, sub_cache, sub_cu, tq, dims)
     o = value_up_projection(o_lat, W, dims)
-    return {"o_lat": o_lat, "lse": lse, "o": o, "u": output_projection(o, W), "q_abs": q_abs, "q_r": q_r}
+    return {"rows": rows, "o_lat": o_lat, "lse": lse, "o": o, "u": output_projection(o, W), "q_abs": q_abs,
+            "q_r": q_r, "q_c": q_c}
 
 
 def output_absorbed(o_lat, W, dims) -> np.ndarray:

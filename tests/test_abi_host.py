@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared symbol, and rejects
+bad arguments before any CUDA call (so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mla_latent_kv_31_b200 import build as mla_build
+from mla_latent_kv_31_b200 import mla, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    mla_build.build()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "mla.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 12
+    L = ctypes.CDLL(mla._LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    for i, name in enumerate(mla.STATUS_NAMES):
+        assert mla.mla_status_string(i).startswith(name)
+
+
+def test_create_validates_dims():
+    with pytest.raises(mla.MLAError) as e:
+        mla.mla_create(synth.Dims(d=0, n_h=1, d_h=1, d_c=1, d_cq=1, d_r=2))
+    assert e.value.status == 1
+    with pytest.raises(mla.MLAError):
+        mla.mla_create(synth.Dims(d=8, n_h=1, d_h=4, d_c=4, d_cq=4, d_r=3))  # odd d_r
+    with pytest.raises(mla.MLAError) as e:
+        mla.mla_create(synth.Dims(d=8, n_h=1, d_h=4, d_c=1024, d_cq=4, d_r=2))
+    assert e.value.status == 3
+    h = mla.mla_create(synth.V3)
+    assert h
+    mla.mla_destroy(h)
+
+
+def test_workspace_sizes_and_offsets():
+    h = mla.mla_create(synth.V3, mla.MLA_BF16)
+    try:
+        n = mla.mla_workspace_size(h, mla.OP_DECODE, 16, 1, 0)
+        T = 16
+        d = synth.V3
+        # c^Q, q^C, q^R, o, q~, o^lat, lse, positions at least
+        floor = T * (d.d_cq + 2 * d.n_h * d.d_h + d.n_h * d.d_r + 2 * d.n_h * d.d_c) * 2 + T * d.n_h * 4
+        assert n >= floor
+        offs = [mla.mla_workspace_offset(h, mla.OP_DECODE, b, 16, 1, 0)
+                for b in (mla.BUF_CQ, mla.BUF_QC, mla.BUF_QR, mla.BUF_O, mla.BUF_QABS, mla.BUF_OLAT, mla.BUF_LSE)]
+        assert offs == sorted(offs) and len(set(offs)) == len(offs)
+        assert all(o % 1024 == 0 and o < n for o in offs)
+        with pytest.raises(mla.MLAError):
+            mla.mla_workspace_offset(h, mla.OP_DECODE, mla.BUF_KC, 16, 1, 0)  # prefill-only region
+        assert mla.mla_workspace_size(h, mla.OP_CACHE_APPEND, 0, 1, 10) == 0
+        p = mla.mla_workspace_size(h, mla.OP_PREFILL, 1, 1, 4096)
+        assert p > 4096 * d.n_h * d.d_h * 2 * 3
+        with pytest.raises(mla.MLAError):
+            mla.mla_workspace_size(h, mla.OP_DECODE, 4, 3, 0)   # Tq must be 1 or 2
+        with pytest.raises(mla.MLAError):
+            mla.mla_workspace_size(h, 7, 4, 1, 0)
+    finally:
+        mla.mla_destroy(h)
+
+
+def test_calls_reject_bad_arguments_before_any_launch():
+    h = mla.mla_create(synth.TINY, mla.MLA_FP32)
+    A = 0x10000  # aligned fake device address: never dereferenced, validation fails first
+    try:
+        with pytest.raises(mla.MLAError) as e:   # null h_q
+            mla.mla_decode(h, None, 2, 1, A, A, 10, A, A, 1 << 20, stream=0)
+        assert e.value.status == 1
+        with pytest.raises(mla.MLAError) as e:   # Tq = 3
+            mla.mla_decode(h, A, 2, 3, A, A, 10, A, A, 1 << 20, stream=0)
+        assert e.value.status == 1
+        with pytest.raises(mla.MLAError) as e:   # misaligned cache
+            mla.mla_decode(h, A, 2, 1, A, A + 2, 10, A, A, 1 << 20, stream=0)
+        assert e.value.status == 2
+        with pytest.raises(mla.MLAError) as e:   # workspace too small
+            mla.mla_decode(h, A, 2, 1, A, A, 10, A, A, 16, stream=0)
+        assert e.value.status == 4
+        with pytest.raises(mla.MLAError) as e:   # no weights given yet
+            mla.mla_decode(h, A, 2, 1, A, A, 10, A, A, 1 << 30, stream=0)
+        assert e.value.status == 8
+        with pytest.raises(mla.MLAError) as e:   # prefill: capacity below the token count
+            mla.mla_prefill(h, A, 1, A, 64, 64, A, 32, A, A, 1 << 30, stream=0)
+        assert e.value.status == 1
+        with pytest.raises(mla.MLAError) as e:   # cache append: misaligned slots
+            mla.mla_cache_append(h, A, A, A + 8, 4, A, 10, stream=0)
+        assert e.value.status == 2
+        with pytest.raises(mla.MLAError) as e:   # core: workspace too small
+            mla.mla_attn_decode_latent(h, A, A, 2, 1, A, A, 10, A, A, A, 0, stream=0)
+        assert e.value.status in (1, 4)
+        with pytest.raises(mla.MLAError) as e:   # weights: misaligned pointer
+            mla.mla_set_weights(h, {n: A + (2 if n == "w_o" else 0) for n in mla.WEIGHT_NAMES})
+        assert e.value.status == 2
+    finally:
+        mla.mla_destroy(h)
+
+
+def test_tensor_core_routing_is_declared():
+    bf = mla.mla_create(synth.V3, mla.MLA_BF16)
+    f32 = mla.mla_create(synth.TINY, mla.MLA_FP32)
+    try:
+        for op in range(4):
+            assert mla.mla_uses_tensor_cores(f32, op) is False
+            assert isinstance(mla.mla_uses_tensor_cores(bf, op), bool)
+    finally:
+        mla.mla_destroy(bf)
+        mla.mla_destroy(f32)

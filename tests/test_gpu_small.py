@@ -1,0 +1,199 @@
+"""GPU parity on small cases that span several key tiles and ragged tails: every call of the
+C ABI against the float64 oracle on the same seeded inputs (max-normalised error, see
+mla_testlib.rel; bound 1e-2 for bf16 inputs with fp32 accumulation, 1e-5 for fp32)."""
+import numpy as np
+import pytest
+
+from mla_testlib import TOL, dev, dev_i64, host, make_module, mla, orc, rel, synth
+
+pytestmark = pytest.mark.gpu
+
+V3_SMALL_SEED = 7
+
+
+@pytest.fixture(scope="module")
+def v3_weights():
+    return synth.weights(synth.V3, seed=V3_SMALL_SEED, dtype="bf16")
+
+
+@pytest.fixture(scope="module")
+def v3_module(v3_weights):
+    m = make_module(synth.V3, v3_weights, "bf16")
+    yield m
+    m.close()
+
+
+def _status_ok(m):
+    s = m.sync_status()
+    assert s == 0, (mla.mla_status_string(s), hex(mla.mla_device_error_bits(m.handle)))
+
+
+# ---------------------------------------------------------------------------
+# FP32 tiny configuration: L = 64, d = 256, n_h = 4, d_h = 32, d_c = 64, d_c' = 96, d_R = 16
+# ---------------------------------------------------------------------------
+def test_tiny_prefill_fp32_unabsorbed_and_absorbed():
+    dims = synth.TINY
+    W = synth.weights(dims, seed=0, dtype="fp32")
+    h = synth.hidden(dims, 64, seed=0, dtype="fp32")
+    cu = synth.cu_seqlens([64])
+    ref = orc.mla_prefill(h, cu, W, dims)
+    m = make_module(dims, W, "fp32")
+    cache = dev(np.zeros((64, dims.row)), "fp32")
+    u = m.prefill(dev(h, "fp32"), 1, dev_i64(cu), 64, cache)
+    _status_ok(m)
+    assert rel(host(u), ref["u"]) <= TOL["fp32"]
+    assert rel(host(cache), ref["cache"]) <= TOL["fp32"]
+    o = m.region(mla.OP_PREFILL, mla.BUF_O, (64, dims.n_h, dims.d_h), m.torch.float32, 1, 1, 64)
+    assert rel(host(o), ref["o"]) <= TOL["fp32"]
+    # absorbed form over the same cache: every token as a one-query decode of its prefix is
+    # the same computation; use the last two tokens (Tq = 2) of the sequence.
+    u_dec = m.decode(dev(h[62:64], "fp32"), 1, 2, dev_i64(cu), cache)
+    _status_ok(m)
+    assert rel(host(u_dec), ref["u"][62:64]) <= TOL["fp32"]
+    m.close()
+
+
+@pytest.mark.parametrize("tq", [1, 2])
+def test_tiny_decode_fp32_ragged(tq):
+    dims = synth.TINY
+    W = synth.weights(dims, seed=1, dtype="fp32")
+    lens = np.array([tq, 5, 64, 65, 130, 257])
+    cu = synth.cu_seqlens(lens)
+    cache = synth.latent_cache(dims, int(cu[-1]), seed=2, dtype="fp32")
+    h_q = synth.hidden(dims, len(lens) * tq, seed=3, dtype="fp32")
+    ref = orc.mla_decode(h_q, cache, cu, tq, W, dims)
+    m = make_module(dims, W, "fp32")
+    u = m.decode(dev(h_q, "fp32"), len(lens), tq, dev_i64(cu), dev(cache, "fp32"))
+    _status_ok(m)
+    assert rel(host(u), ref["u"]) <= TOL["fp32"]
+    T = len(lens) * tq
+    olat = m.region(mla.OP_DECODE, mla.BUF_OLAT, (T, dims.n_h, dims.d_c), m.torch.float32, len(lens), tq)
+    assert rel(host(olat), ref["o_lat"]) <= TOL["fp32"]
+    lse = m.region(mla.OP_DECODE, mla.BUF_LSE, (T, dims.n_h), m.torch.float32, len(lens), tq)
+    assert rel(host(lse), ref["lse"]) <= TOL["fp32"]
+    m.close()
+
+
+def test_tiny_cache_append_fp32_scattered_slots():
+    dims = synth.TINY
+    W = synth.weights(dims, seed=4, dtype="fp32")
+    T, cap = 37, 100
+    h = synth.hidden(dims, T, seed=5, dtype="fp32")
+    pos = np.arange(T) * 3 + 11
+    slots = np.random.default_rng(0).permutation(cap)[:T]
+    ref = orc.cache_append(h, pos, W, dims)
+    m = make_module(dims, W, "fp32")
+    cache = dev(np.full((cap, dims.row), 7.0), "fp32")
+    m.cache_append(dev(h, "fp32"), dev_i64(pos), dev_i64(slots), cache)
+    _status_ok(m)
+    got = host(cache)
+    assert rel(got[slots], ref) <= TOL["fp32"]
+    untouched = np.setdiff1d(np.arange(cap), slots)
+    assert np.all(got[untouched] == 7.0)
+    m.close()
+
+
+# ---------------------------------------------------------------------------
+# BF16 at the DeepSeek-V3 sizes, small batches with ragged tails
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("tq", [1, 2])
+def test_v3_attn_core_bf16_ragged(v3_module, tq):
+    dims = synth.V3
+    lens = np.array([tq, 63, 64, 65, 129, 1000, 4097])
+    cu = synth.cu_seqlens(lens)
+    B, T = len(lens), len(lens) * tq
+    cache = synth.latent_cache(dims, int(cu[-1]), seed=10 + tq, dtype="bf16")
+    q_abs = synth.normal(11, 20, (T, dims.n_h, dims.d_c), std=0.5, dtype="bf16")
+    q_rope = synth.normal(11, 21, (T, dims.n_h, dims.d_r), std=1.0, dtype="bf16")
+    lat_ref, lse_ref = orc.attn_decode_latent(q_abs, q_rope, cache, cu, tq, dims)
+    o_lat, lse = v3_module.attn_decode_latent(dev(q_abs, "bf16"), dev(q_rope, "bf16"), B, tq, dev_i64(cu),
+                                              dev(cache, "bf16"))
+    _status_ok(v3_module)
+    assert rel(host(o_lat), lat_ref) <= TOL["bf16"]
+    assert rel(host(lse), lse_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("tq", [1, 2])
+def test_v3_decode_bf16_steps(v3_module, v3_weights, tq):
+    dims = synth.V3
+    lens = np.array([tq, 64, 65, 300])
+    cu = synth.cu_seqlens(lens)
+    B, T = len(lens), len(lens) * tq
+    cache = synth.latent_cache(dims, int(cu[-1]), seed=20 + tq, dtype="bf16")
+    h_q = synth.hidden(dims, T, seed=22, dtype="bf16")
+    ref = orc.mla_decode_absorbed(h_q, cache, cu, tq, v3_weights, dims)
+    u = v3_module.decode(dev(h_q, "bf16"), B, tq, dev_i64(cu), dev(cache, "bf16"))
+    _status_ok(v3_module)
+    bf = v3_module.torch.bfloat16
+    reg = lambda which, shape, dt=bf: host(v3_module.region(mla.OP_DECODE, which, shape, dt, B, tq))  # noqa: E731
+    assert rel(reg(mla.BUF_QC, (T, dims.n_h, dims.d_h)), ref["q_c"]) <= TOL["bf16"]
+    assert rel(reg(mla.BUF_QR, (T, dims.n_h, dims.d_r)), ref["q_r"]) <= TOL["bf16"]
+    assert rel(reg(mla.BUF_QABS, (T, dims.n_h, dims.d_c)), ref["q_abs"]) <= TOL["bf16"]
+    assert rel(reg(mla.BUF_OLAT, (T, dims.n_h, dims.d_c)), ref["o_lat"]) <= TOL["bf16"]
+    assert rel(reg(mla.BUF_LSE, (T, dims.n_h), v3_module.torch.float32), ref["lse"]) <= TOL["bf16"]
+    assert rel(reg(mla.BUF_O, (T, dims.n_h, dims.d_h)), ref["o"]) <= TOL["bf16"]
+    assert rel(host(u), ref["u"]) <= TOL["bf16"]
+    # the unabsorbed oracle on one sequence (explicit per-head up-projection)
+    un = orc.mla_decode(h_q, cache, cu, tq, v3_weights, dims, seqs=[2])
+    assert rel(host(u)[un["rows"]], un["u"]) <= TOL["bf16"]
+
+
+def test_v3_cache_append_bf16(v3_module, v3_weights):
+    dims = synth.V3
+    T, cap = 45, 300
+    h = synth.hidden(dims, T, seed=30, dtype="bf16")
+    pos = np.array([0, 1, 4095, 131071] + list(range(100, 141)))
+    slots = np.random.default_rng(1).permutation(cap)[:T]
+    ref = orc.cache_append(h, pos, v3_weights, dims)
+    cache = dev(np.zeros((cap, dims.row)), "bf16")
+    v3_module.cache_append(dev(h, "bf16"), dev_i64(pos), dev_i64(slots), cache)
+    _status_ok(v3_module)
+    assert rel(host(cache)[slots], ref) <= TOL["bf16"]
+
+
+def test_v3_prefill_bf16_two_sequences(v3_module, v3_weights):
+    dims = synth.V3
+    lens = [200, 37]
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    h = synth.hidden(dims, T, seed=40, dtype="bf16")
+    ref = orc.mla_prefill(h, cu, v3_weights, dims)
+    cache = dev(np.zeros((T + 5, dims.row)), "bf16")
+    u = v3_module.prefill(dev(h, "bf16"), 2, dev_i64(cu), max(lens), cache)
+    _status_ok(v3_module)
+    assert rel(host(cache)[:T], ref["cache"]) <= TOL["bf16"]
+    o = v3_module.region(mla.OP_PREFILL, mla.BUF_O, (T, dims.n_h, dims.d_h), v3_module.torch.bfloat16, 2, 1, T)
+    assert rel(host(o), ref["o"]) <= TOL["bf16"]
+    assert rel(host(u), ref["u"]) <= TOL["bf16"]
+
+
+# ---------------------------------------------------------------------------
+# Device-side checks and determinism
+# ---------------------------------------------------------------------------
+def test_device_checks_flag_bad_cu_seqlens_and_slots(v3_module):
+    dims = synth.V3
+    cache = dev(np.zeros((64, dims.row)), "bf16")
+    q = dev(np.zeros((2, dims.n_h, dims.d_c)), "bf16")
+    qr = dev(np.zeros((2, dims.n_h, dims.d_r)), "bf16")
+    bad_cu = dev_i64([0, 10, 5])          # decreasing
+    v3_module.attn_decode_latent(q, qr, 2, 1, bad_cu, cache)
+    s = v3_module.sync_status()
+    assert mla.STATUS_NAMES[s] == "MLA_ERR_DEVICE_CHECK"
+    assert mla.mla_device_error_bits(v3_module.handle) & 1
+    assert v3_module.sync_status() == 0    # the word is cleared once read
+    h = dev(np.zeros((2, dims.d)), "bf16")
+    v3_module.cache_append(h, dev_i64([0, 1]), dev_i64([3, 64]), cache)   # slot 64 == capacity
+    assert mla.STATUS_NAMES[v3_module.sync_status()] == "MLA_ERR_DEVICE_CHECK"
+    assert mla.mla_device_error_bits(v3_module.handle) & 4
+
+
+def test_decode_is_deterministic(v3_module):
+    dims = synth.V3
+    lens = np.array([700, 3000])
+    cu = synth.cu_seqlens(lens)
+    cache = dev(synth.latent_cache(dims, int(cu[-1]), seed=50, dtype="bf16"), "bf16")
+    h_q = dev(synth.hidden(dims, 2, seed=51, dtype="bf16"), "bf16")
+    a = v3_module.decode(h_q, 2, 1, dev_i64(cu), cache).clone()
+    b = v3_module.decode(h_q, 2, 1, dev_i64(cu), cache).clone()
+    _status_ok(v3_module)
+    assert bool((a == b).all())

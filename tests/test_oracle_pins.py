@@ -51,6 +51,9 @@ def test_absorbed_equals_unabsorbed_decode(dims, tq):
     assert _rel(ab["u"], un["u"]) < 1e-12
     # second absorption: W^O' = W^O W^UV applied to the latent outputs
     assert _rel(orc.output_absorbed(un["o_lat"], W, dims), un["u"]) < 1e-12
+    # a subset of sequences, re-packed on their own, gives the same rows
+    sub = orc.mla_decode_absorbed(h_q, cache, cu, tq, W, dims, seqs=[1, 3])
+    assert _rel(sub["u"], un["u"][sub["rows"]]) < 1e-12
 
 
 def test_absorbed_core_matches_unabsorbed_prefill():
