@@ -117,7 +117,8 @@ mla_status_t mla_workspace_offset(const mla_handle_t *h, mla_op_t op, int64_t nu
  *   positions  [T] device int64  position of each token within its sequence (>= 0)
  *   slots      [T] device int64  destination row, 0 <= slot < capacity (else skipped + flagged)
  *   cache      [capacity, d_c + d_r]
- * No workspace is needed (ws may be NULL when ws_bytes is 0). */
+ * ws: mla_workspace_size(MLA_OP_CACHE_APPEND, total_tokens = T) bytes (split-K partials of the
+ * projection at small T; may be 0, in which case ws may be NULL). */
 mla_status_t mla_cache_append(mla_handle_t *h, const void *hidden, const int64_t *positions,
                               const int64_t *slots, int64_t T, void *cache, int64_t capacity,
                               void *ws, size_t ws_bytes, mla_stream_t stream);

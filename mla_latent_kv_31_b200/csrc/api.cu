@@ -81,9 +81,11 @@ Layout layout(const mla_handle* h, mla_op_t op, int64_t B, int32_t tq, int64_t t
     L.pos_off = cur;
     cur = align_up(cur + (size_t)(T > 0 ? T : 1) * sizeof(int64_t));
   }
-  if ((op == MLA_OP_DECODE || op == MLA_OP_ATTN_DECODE_LATENT) && tc_dims(h)) {
+  if (tc_dims(h)) {
     L.tc_off = cur;
-    cur = align_up(cur + mla::tc_decode_scratch_bytes(B, tq));
+    if (op == MLA_OP_DECODE) cur = align_up(cur + mla::tc_decode_scratch_bytes(d, B, tq));
+    if (op == MLA_OP_ATTN_DECODE_LATENT) cur = align_up(cur + mla::tc_core_scratch_bytes(d, B, tq));
+    if (op == MLA_OP_CACHE_APPEND) cur = align_up(cur + mla::tc_append_scratch_bytes(d, total_tokens));
   }
   L.total = cur;
   return L;
@@ -262,7 +264,7 @@ mla_status_t mla_workspace_size(const mla_handle_t* h, mla_op_t op, int64_t num_
   } else if (total_tokens <= 0) {
     return MLA_ERR_INVALID_ARG;
   }
-  *bytes = op == MLA_OP_CACHE_APPEND ? 0 : layout(h, op, num_seqs, tq, total_tokens).total;
+  *bytes = layout(h, op, num_seqs, tq, total_tokens).total;
   return MLA_OK;
 }
 
@@ -286,16 +288,18 @@ int mla_uses_tensor_cores(const mla_handle_t* h, mla_op_t op) {
 mla_status_t mla_cache_append(mla_handle_t* h, const void* hidden, const int64_t* positions, const int64_t* slots,
                               int64_t T, void* cache, int64_t capacity, void* ws, size_t ws_bytes,
                               mla_stream_t stream) {
-  (void)ws; (void)ws_bytes;
   if (!h || !hidden || !positions || !slots || !cache || T <= 0 || capacity <= 0) return MLA_ERR_INVALID_ARG;
-  if (!aligned16(hidden) || !aligned16(cache) || !aligned16(positions) || !aligned16(slots))
+  if (!aligned16(hidden) || !aligned16(cache) || !aligned16(positions) || !aligned16(slots) ||
+      (ws && !aligned16(ws)))
     return MLA_ERR_ALIGNMENT;
+  Layout L = layout(h, MLA_OP_CACHE_APPEND, 0, 1, T);
+  if (ws_bytes < L.total || (L.total > 0 && !ws)) return MLA_ERR_WORKSPACE;
   mla_status_t s = check_ready(h);
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   if (tc_dims(h) && mla::tc_available(MLA_OP_CACHE_APPEND))
     return cuda_status(mla::tc_cache_append(h->dims, h->w, hidden, positions, slots, T, cache, capacity,
-                                            h->d_err, st));
+                                            (char*)ws + L.tc_off, L.total - L.tc_off, h->d_err, st));
   return simt_cache_rows(h, hidden, positions, slots, T, cache, capacity, st);
 }
 

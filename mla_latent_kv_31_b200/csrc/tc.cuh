@@ -11,12 +11,18 @@ namespace mla {
 // Whether this build routes `op` through the tensor-core kernels.
 bool tc_available(mla_op_t op);
 
-// Scratch bytes of the split-KV latent core for B sequences of tq query tokens.
-size_t tc_decode_scratch_bytes(int64_t B, int32_t tq);
+// Scratch bytes of the tensor-core decode path (split-K partials of the projections and the
+// split-KV partials of the latent core) for B sequences of tq query tokens.
+size_t tc_decode_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq);
+// Scratch bytes of the latent core alone.
+size_t tc_core_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq);
+// Scratch bytes of mla_cache_append for T tokens (split-K partials when T is small).
+size_t tc_append_scratch_bytes(const mla_dims_t& d, int64_t T);
 
 cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const void* hidden,
                             const int64_t* positions, const int64_t* slots, int64_t T, void* cache,
-                            int64_t capacity, uint32_t* err, cudaStream_t st);
+                            int64_t capacity, void* scratch, size_t scratch_bytes, uint32_t* err,
+                            cudaStream_t st);
 
 cudaError_t tc_latent_core(const mla_dims_t& d, const void* q_abs, const void* q_rope, int64_t B, int32_t tq,
                            const int64_t* cu, const void* cache, int64_t capacity, void* o_lat, bool o_f32,

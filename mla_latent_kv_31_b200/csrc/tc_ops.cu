@@ -1,0 +1,220 @@
+// Tensor-core op sequences (BF16, DeepSeek-V3 sizes): the projection GEMMs on tcgen05, the
+// latent attention core, the output projection. Steps follow section 一(一) of the DeepSeek-V3
+// notes: (1)-(3) queries, (5)/(7) cache rows, the absorbed core, then W^UV and W^O.
+#include <string.h>
+
+#include "simt.cuh"
+#include "tc.cuh"
+#include "tc_gemm.cuh"
+
+namespace mla {
+namespace {
+
+constexpr size_t kAlign = 1024;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+TcMatrix mat(const void* p, int64_t rows, int64_t cols, int64_t ld) {
+  TcMatrix m;
+  m.ptr = p; m.rows = rows; m.cols = cols; m.ld = ld;
+  return m;
+}
+
+TcEpiSeg epi(void* out, int64_t so_t, int64_t so_f, int64_t f_rows) {
+  TcEpiSeg e;
+  memset(&e, 0, sizeof(e));
+  e.out = out; e.so_t = so_t; e.so_f = so_f; e.f_rows = f_rows;
+  return e;
+}
+
+TcGemmDesc desc(const TcMatrix& x, int64_t T, int64_t K, uint32_t* err) {
+  TcGemmDesc g;
+  memset(&g, 0, sizeof(g));
+  g.x = x; g.T = T; g.K = K; g.batch = 1; g.err = err;
+  return g;
+}
+
+int64_t tiles128(int64_t n) { return (n + 127) / 128; }
+
+size_t decode_gemm_partials(const mla_dims_t& d, int64_t T) {
+  const size_t a = tc_gemm_partial_bytes(T, tiles128(d.d_cq), d.d_cq, d.d, 1);                      // W^DQ
+  const size_t b = tc_gemm_partial_bytes(T, tiles128(d.d), d.d, (int64_t)d.n_h * d.d_h, 1);         // W^O
+  return align_up(a > b ? a : b);
+}
+
+// Steps (5) and (7) with the cache write: rows [c^KV | RoPE(W^KR h)] -> cache[rowmap[t]].
+cudaError_t cache_rows(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, const int64_t* pos,
+                       const int64_t* rowmap, int64_t T, void* cache, int64_t capacity, void* scratch,
+                       size_t scratch_bytes, uint32_t* err, cudaStream_t st) {
+  const int64_t R = d.d_c + d.d_r;
+  TcGemmDesc g = desc(mat(hidden, T, d.d, d.d), T, d.d, err);
+  g.nseg = 2;
+  g.seg[0].w = mat(w.w_dkv, d.d_c, d.d, d.d);
+  g.seg[0].epi = epi(cache, R, 1, d.d_c);
+  g.seg[1].w = mat(w.w_kr, d.d_r, d.d, d.d);
+  g.seg[1].epi = epi((char*)cache + (size_t)d.d_c * 2, R, 1, d.d_r);
+  g.seg[1].epi.rope = 1;
+  for (int s = 0; s < 2; ++s) {
+    g.seg[s].epi.rowmap = rowmap;
+    g.seg[s].epi.rowmap_limit = capacity;
+  }
+  g.pos = pos; g.d_r = d.d_r; g.rope_base = d.rope_base;
+  g.partial = (float*)scratch; g.partial_bytes = scratch_bytes;
+  return tc_gemm(g, st);
+}
+
+// Steps (1)-(3): c^Q = W^DQ h; q^C = W^UQ c^Q; q^R = RoPE(W^QR c^Q).
+cudaError_t queries(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, const int64_t* pos, int64_t T,
+                    void* cq, void* qc, void* qr, void* scratch, size_t scratch_bytes, uint32_t* err,
+                    cudaStream_t st) {
+  const int64_t HD = (int64_t)d.n_h * d.d_h, HR = (int64_t)d.n_h * d.d_r;
+  TcGemmDesc a = desc(mat(hidden, T, d.d, d.d), T, d.d, err);
+  a.nseg = 1;
+  a.seg[0].w = mat(w.w_dq, d.d_cq, d.d, d.d);
+  a.seg[0].epi = epi(cq, d.d_cq, 1, d.d_cq);
+  a.partial = (float*)scratch; a.partial_bytes = scratch_bytes;
+  cudaError_t e = tc_gemm(a, st);
+  if (e != cudaSuccess) return e;
+  TcGemmDesc b = desc(mat(cq, T, d.d_cq, d.d_cq), T, d.d_cq, err);
+  b.nseg = 2;
+  b.seg[0].w = mat(w.w_uq, HD, d.d_cq, d.d_cq);
+  b.seg[0].epi = epi(qc, HD, 1, HD);
+  b.seg[1].w = mat(w.w_qr, HR, d.d_cq, d.d_cq);
+  b.seg[1].epi = epi(qr, HR, 1, HR);
+  b.seg[1].epi.rope = 1;
+  b.pos = pos; b.d_r = d.d_r; b.rope_base = d.rope_base;
+  b.partial = (float*)scratch; b.partial_bytes = scratch_bytes;
+  return tc_gemm(b, st);
+}
+
+// Step (10), second equation: u = W^O [o_1; ...; o_nh].
+cudaError_t output(const mla_dims_t& d, const mla_weights_t& w, const void* o, int64_t T, void* u, void* scratch,
+                   size_t scratch_bytes, uint32_t* err, cudaStream_t st) {
+  const int64_t HD = (int64_t)d.n_h * d.d_h;
+  TcGemmDesc g = desc(mat(o, T, HD, HD), T, HD, err);
+  g.nseg = 1;
+  g.seg[0].w = mat(w.w_o, d.d, HD, HD);
+  g.seg[0].epi = epi(u, d.d, 1, d.d);
+  g.partial = (float*)scratch; g.partial_bytes = scratch_bytes;
+  return tc_gemm(g, st);
+}
+
+cudaError_t simt_core(const mla_dims_t& d, const void* q_abs, const void* q_rope, int64_t B, int32_t tq,
+                      const int64_t* cu, const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse,
+                      uint32_t* err, cudaStream_t st) {
+  const int64_t R = d.d_c + d.d_r;
+  SimtAttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q1 = q_abs; a.sq1t = (int64_t)d.n_h * d.d_c; a.sq1h = d.d_c; a.d1 = d.d_c;
+  a.q2 = q_rope; a.sq2t = (int64_t)d.n_h * d.d_r; a.sq2h = d.d_r; a.d2 = d.d_r;
+  a.k1 = cache; a.sk1 = R; a.sk1h = 0;
+  a.k2 = (const char*)cache + (size_t)d.d_c * 2; a.sk2 = R;
+  a.v = cache; a.sv = R; a.svh = 0; a.dv = d.d_c;
+  a.o = o_lat; a.sot = (int64_t)d.n_h * d.d_c; a.soh = d.d_c;
+  a.lse = lse;
+  a.cu = cu; a.B = B; a.tq = tq; a.T = B * tq; a.n_h = d.n_h; a.capacity = capacity;
+  a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
+  a.err = err;
+  return simt_attention(a, true, o_f32, st);
+}
+
+}  // namespace
+
+bool tc_available(mla_op_t op) { return op != MLA_OP_ATTN_DECODE_LATENT; }
+
+size_t tc_core_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq) {
+  (void)d; (void)B; (void)tq;
+  return 0;
+}
+
+size_t tc_decode_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq) {
+  return decode_gemm_partials(d, B * tq) + align_up(tc_core_scratch_bytes(d, B, tq));
+}
+
+size_t tc_append_scratch_bytes(const mla_dims_t& d, int64_t T) {
+  return align_up(tc_gemm_partial_bytes(T, tiles128(d.d_c) + tiles128(d.d_r), d.d_c + d.d_r, d.d, 1));
+}
+
+cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const void* hidden,
+                            const int64_t* positions, const int64_t* slots, int64_t T, void* cache,
+                            int64_t capacity, void* scratch, size_t scratch_bytes, uint32_t* err,
+                            cudaStream_t st) {
+  return cache_rows(d, w, hidden, positions, slots, T, cache, capacity, scratch, scratch_bytes, err, st);
+}
+
+cudaError_t tc_latent_core(const mla_dims_t& d, const void* q_abs, const void* q_rope, int64_t B, int32_t tq,
+                           const int64_t* cu, const void* cache, int64_t capacity, void* o_lat, bool o_f32,
+                           float* lse, void* scratch, int num_sms, uint32_t* err, cudaStream_t st) {
+  (void)scratch; (void)num_sms;
+  return simt_core(d, q_abs, q_rope, B, tq, cu, cache, capacity, o_lat, o_f32, lse, err, st);
+}
+
+cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const void* h_q, int64_t B, int32_t tq,
+                      const int64_t* cu, const int64_t* pos, const void* cache, int64_t capacity, void* u_out,
+                      void* cq, void* qc, void* qr, void* qabs, void* olat, void* o, float* lse, void* scratch,
+                      int num_sms, uint32_t* err, cudaStream_t st) {
+  const int64_t T = B * tq, HD = (int64_t)d.n_h * d.d_h;
+  const size_t part_bytes = decode_gemm_partials(d, T);
+  void* core_scratch = (char*)scratch + part_bytes;
+  cudaError_t e = queries(d, w, h_q, pos, T, cq, qc, qr, scratch, part_bytes, err, st);
+  if (e != cudaSuccess) return e;
+  // q~_i = W_i^UK^T q^C_i for every head i: the weight operand is W^UK read MN-major.
+  TcGemmDesc a = desc(mat(qc, T, HD, HD), T, d.d_h, err);
+  a.nseg = 1;
+  a.w_mn = true;
+  a.seg[0].w = mat(w.w_uk, HD, d.d_c, d.d_c);
+  a.seg[0].epi = epi(qabs, (int64_t)d.n_h * d.d_c, 1, d.d_c);
+  a.seg[0].epi.so_z = d.d_c;
+  a.batch = d.n_h; a.w_row_z = d.d_h; a.x_col_z = d.d_h;
+  e = tc_gemm(a, st);
+  if (e != cudaSuccess) return e;
+  e = tc_latent_core(d, qabs, qr, B, tq, cu, cache, capacity, olat, false, lse, core_scratch, num_sms, err, st);
+  if (e != cudaSuccess) return e;
+  // o_i = W_i^UV o^lat_i for every head i.
+  TcGemmDesc v = desc(mat(olat, T, (int64_t)d.n_h * d.d_c, (int64_t)d.n_h * d.d_c), T, d.d_c, err);
+  v.nseg = 1;
+  v.seg[0].w = mat(w.w_uv, HD, d.d_c, d.d_c);
+  v.seg[0].epi = epi(o, HD, 1, d.d_h);
+  v.seg[0].epi.so_z = d.d_h;
+  v.batch = d.n_h; v.w_row_z = d.d_h; v.x_col_z = d.d_c;
+  e = tc_gemm(v, st);
+  if (e != cudaSuccess) return e;
+  return output(d, w, o, T, u_out, scratch, part_bytes, err, st);
+}
+
+cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, int64_t B,
+                       const int64_t* cu, int64_t T, int64_t max_seqlen, const int64_t* pos, void* cache,
+                       int64_t capacity, void* u_out, void* cq, void* qc, void* qr, void* kc, void* vc, void* o,
+                       uint32_t* err, cudaStream_t st) {
+  (void)max_seqlen;
+  const int64_t R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
+  cudaError_t e = cache_rows(d, w, hidden, pos, nullptr, T, cache, capacity, nullptr, 0, err, st);
+  if (e != cudaSuccess) return e;
+  e = queries(d, w, hidden, pos, T, cq, qc, qr, nullptr, 0, err, st);
+  if (e != cudaSuccess) return e;
+  // Steps (6), (9): [k^C; v^C] = [W^UK; W^UV] c^KV from the cache rows just written.
+  TcGemmDesc p3 = desc(mat(cache, T, d.d_c, R), T, d.d_c, err);
+  p3.nseg = 2;
+  p3.seg[0].w = mat(w.w_uk, HD, d.d_c, d.d_c);
+  p3.seg[0].epi = epi(kc, HD, 1, HD);
+  p3.seg[1].w = mat(w.w_uv, HD, d.d_c, d.d_c);
+  p3.seg[1].epi = epi(vc, HD, 1, HD);
+  e = tc_gemm(p3, st);
+  if (e != cudaSuccess) return e;
+  // Steps (4), (8), (10): causal attention per head, keys [k^C_i; k^R], values v^C_i.
+  SimtAttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q1 = qc; a.sq1t = HD; a.sq1h = d.d_h; a.d1 = d.d_h;
+  a.q2 = qr; a.sq2t = (int64_t)d.n_h * d.d_r; a.sq2h = d.d_r; a.d2 = d.d_r;
+  a.k1 = kc; a.sk1 = HD; a.sk1h = d.d_h;
+  a.k2 = (const char*)cache + (size_t)d.d_c * 2; a.sk2 = R;
+  a.v = vc; a.sv = HD; a.svh = d.d_h; a.dv = d.d_h;
+  a.o = o; a.sot = HD; a.soh = d.d_h;
+  a.cu = cu; a.B = B; a.tq = 0; a.T = T; a.n_h = d.n_h; a.capacity = capacity;
+  a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
+  a.err = err;
+  e = simt_attention(a, true, false, st);
+  if (e != cudaSuccess) return e;
+  return output(d, w, o, T, u_out, nullptr, 0, err, st);
+}
+
+}  // namespace mla

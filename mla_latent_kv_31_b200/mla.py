@@ -206,7 +206,10 @@ class MLA:
         return self._ws[off:off + n * es].view(dtype).view(*shape)
 
     def cache_append(self, hidden, positions, slots, cache):
-        mla_cache_append(self.handle, hidden, positions, slots, hidden.shape[0], cache, cache.shape[0],
+        T = hidden.shape[0]
+        n = mla_workspace_size(self.handle, OP_CACHE_APPEND, 0, 1, T)
+        ws = self.workspace(n) if n else None
+        mla_cache_append(self.handle, hidden, positions, slots, T, cache, cache.shape[0], ws, n if n else 0,
                          device=self.device)
 
     def decode(self, h_q, B, Tq, cu_seqlens, cache, u_out=None):

@@ -65,7 +65,10 @@ def test_workspace_sizes_and_offsets():
         assert all(o % 1024 == 0 and o < n for o in offs)
         with pytest.raises(mla.MLAError):
             mla.mla_workspace_offset(h, mla.OP_DECODE, mla.BUF_KC, 16, 1, 0)  # prefill-only region
-        assert mla.mla_workspace_size(h, mla.OP_CACHE_APPEND, 0, 1, 10) == 0
+        # cache append: split-K partials of the [W^DKV; W^KR] projection at small T only
+        small = mla.mla_workspace_size(h, mla.OP_CACHE_APPEND, 0, 1, 10)
+        assert small >= 2 * 10 * (d.d_c + d.d_r) * 4 and small % 1024 == 0
+        assert mla.mla_workspace_size(h, mla.OP_CACHE_APPEND, 0, 1, 4096) == 0
         p = mla.mla_workspace_size(h, mla.OP_PREFILL, 1, 1, 4096)
         assert p > 4096 * d.n_h * d.d_h * 2 * 3
         with pytest.raises(mla.MLAError):
