@@ -28,6 +28,11 @@ cudaError_t tc_latent_core(const mla_dims_t& d, const void* q_abs, const void* q
                            const int64_t* cu, const void* cache, int64_t capacity, void* o_lat, bool o_f32,
                            float* lse, void* scratch, int num_sms, uint32_t* err, cudaStream_t st);
 
+// The split-KV tcgen05 latent core (q~, q^R -> o^lat, lse); scratch of tc_core_scratch_bytes().
+cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
+                                const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse,
+                                void* scratch, int num_sms, uint32_t* err, cudaStream_t st);
+
 cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const void* h_q, int64_t B, int32_t tq,
                       const int64_t* cu, const int64_t* pos, const void* cache, int64_t capacity, void* u_out,
                       void* cq, void* qc, void* qr, void* qabs, void* olat, void* o, float* lse, void* scratch,

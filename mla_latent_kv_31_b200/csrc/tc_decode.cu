@@ -1,0 +1,570 @@
+// Split-KV latent attention core for decode at the DeepSeek-V3 sizes (n_h = 128, d_c = 512,
+// d_h^R = 64), bf16 inputs, fp32 accumulation, tcgen05 + TMA on sm_100a.
+//
+// It computes, for every query token t of sequence b and head i, the absorbed score of the
+// DeepSeek-V3 notes (section 一(一)2 【思考】 and 3 "解耦RoPE"):
+//   s_j = (q~_t,i . c_j + q^R_t,i . k^R_j) / sqrt(d_h + d_h^R),  j <= pos_t,
+//   o^lat_t,i = sum_j softmax(s)_j c_j,   lse_t,i = log sum_j exp(s_j).
+//
+// Work split. Each sequence's cache rows form tiles of 32 keys; all tiles of all sequences are
+// cut into equal contiguous ranges, one per CTA pair (a 2-CTA cluster); a pair whose range
+// crosses a sequence boundary emits one partial result per sequence piece, and a final pass
+// merges the pieces of a sequence exactly (log-sum-exp). Within a pair, CTA r owns latent
+// columns [256 r, 256 r + 256): it streams only that half of every cache row (CTA 0 also the
+// 64 k^R columns), computes the partial score over its columns, swaps the 128 x 32 fp32
+// partial with its peer through distributed shared memory, and then both run the same
+// softmax and accumulate P . c into their own 256 TMEM columns of O. The 128 heads form the
+// MMA M dimension; one TMA-loaded cache tile is read K-major by QK^T and MN-major by P.V.
+//
+// Roles per CTA (192 threads): warps 0-3 softmax/epilogue (thread i = head i = TMEM lane i),
+// warp 4 TMA producer, warp 5 TMEM owner + MMA issuer. Every wait is bounded.
+#include <cuda_bf16.h>
+#include <string.h>
+
+#include "sm100.cuh"
+#include "tc.cuh"
+#include "tc_gemm.cuh"
+
+namespace mla {
+namespace {
+
+using namespace sm100;
+
+constexpr int H = 128, DC = 512, DR = 64, ROW = DC + DR;
+constexpr int NK = 32;                       // keys per tile
+constexpr int STAGES = 4;
+constexpr int kThreads = 192;
+constexpr int kMaxPairs = 74;
+constexpr float kRescaleLog2 = 8.f;          // lazy rescale: keep the running max until it grows by 2^8
+
+constexpr uint32_t Q_CHUNK = H * 128;        // [128 rows x 64 cols] bf16, SW128: 16 KB
+constexpr uint32_t KV_BOX = NK * 128;        // [32 keys x 64 cols] bf16, SW128: 4 KB
+constexpr uint32_t STAGE_BYTES = 5 * KV_BOX; // 4 latent boxes + (CTA 0) the k^R box
+constexpr uint32_t P_BYTES = H * NK * 2;     // [128 x 32] bf16, SW64: 8 KB
+constexpr uint32_t X_BYTES = H * NK * 4;     // [128 x 32] fp32 partial scores: 16 KB
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_KV = OFF_Q + 5 * Q_CHUNK;
+constexpr uint32_t OFF_P = OFF_KV + STAGES * STAGE_BYTES;
+constexpr uint32_t OFF_X = OFF_P + 2 * P_BYTES;
+constexpr uint32_t OFF_BAR = OFF_X + 2 * X_BYTES;
+constexpr int NBAR = 2 * STAGES + 15;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
+constexpr uint32_t TMEM_COLS = 512;          // O half: [0, 256); S buffers: 256 + 32 b
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// barrier indices
+constexpr int B_FULL = 0, B_EMPTY = STAGES, B_SFULL = 2 * STAGES, B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2,
+              B_PVDONE = B_PFULL + 2, B_XFULL = B_PVDONE + 2, B_XFREE = B_XFULL + 2, B_QFULL = B_XFREE + 2,
+              B_QEMPTY = B_QFULL + 1, B_OFREE = B_QEMPTY + 1;
+static_assert(B_OFREE + 1 <= NBAR, "barrier count");
+
+struct CoreParams {
+  CUtensorMap qmap;   // q~ as [T*H, DC], box {64, 128}
+  CUtensorMap rmap;   // q^R as [T*H, DR], box {64, 128}
+  CUtensorMap cmap;   // cache as [capacity, ROW], box {64, 32}
+  const int64_t* cu;
+  const int32_t* tile_start;  // [B+1]: first global tile of each sequence
+  const int32_t* slot_base;   // [B+1]: first partial slot of each sequence
+  int32_t B, tq, pairs, s_max;
+  float* part_o;     // [tq][s_max][H][DC]
+  float* part_lse;   // [tq][s_max][H]
+  void* o_lat;       // [T][H][DC] (fp32 or bf16)
+  float* lse;        // [T][H]
+  float scale_log2;  // log2(e) / sqrt(d_h + d_h^R)
+  uint32_t* err;
+};
+
+__device__ __forceinline__ int32_t range_start(int64_t p, int64_t NT, int64_t P) { return (int32_t)(p * NT / P); }
+
+// The last sequence b in [0, B) with tile_start[b] <= x.
+__device__ __forceinline__ int find_seq(const int32_t* ts, int B, int32_t x) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ts[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Iterates the sequence pieces of a tile range [x, end): b, [x, seg_end).
+struct SegWalk {
+  const int32_t* ts;
+  int B;
+  int32_t x, end;
+  int b;
+  __device__ void init(const int32_t* ts_, int B_, int32_t x0, int32_t x1) {
+    ts = ts_; B = B_; x = x0; end = x1;
+    b = x < end ? find_seq(ts, B, x) : 0;
+  }
+  __device__ bool valid() const { return x < end; }
+  __device__ int32_t seg_end() const { return min(end, ts[b + 1]); }
+  __device__ void next() {
+    x = seg_end();
+    ++b;
+    while (b < B && ts[b + 1] <= x) ++b;
+  }
+};
+
+template <bool OUT_F32>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    latent_core_kernel(const __grid_constant__ CoreParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
+  const uint32_t sbase = smem_addr(smem);
+  auto bar = [&](int i) { return smem_addr(&bars[i]); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t r = cluster_rank();
+  const uint32_t peer = r ^ 1u;
+  const int k = blockIdx.y;                          // query token within the sequence window
+  const int pair = blockIdx.x >> 1;
+  const int64_t NT = p.tile_start[p.B];
+  // Active pairs: never more than tiles, so that every active range holds at least one tile.
+  const int64_t npairs = NT < p.pairs ? NT : p.pairs;
+  const int32_t t_begin = pair < npairs ? range_start(pair, NT, npairs) : 0;
+  const int32_t t_end = pair < npairs ? range_start(pair + 1, NT, npairs) : 0;
+  const int nkc = r == 0 ? 5 : 4;                    // 64-column K chunks of this CTA's score half
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBAR; ++i) {
+      uint32_t cnt = 1;
+      if (i == B_SEMPTY || i == B_SEMPTY + 1 || i == B_PFULL || i == B_PFULL + 1 || i == B_XFULL ||
+          i == B_XFULL + 1 || i == B_XFREE || i == B_XFREE + 1 || i == B_OFREE)
+        cnt = 128;
+      mbar_init(bar(i), cnt);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&p.qmap);
+    prefetch_tmap(&p.rmap);
+    prefetch_tmap(&p.cmap);
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  SegWalk w;
+  w.init(p.tile_start, p.B, t_begin, t_end);
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int j = 0, g = 0, issued = 0;
+      bool ok = true;
+      for (; ok && w.valid(); w.next(), ++g) {
+        const int b = w.b;
+        if (!mbar_wait(bar(B_QEMPTY), (g & 1) ^ 1)) { ok = false; break; }
+        mbar_expect_tx(bar(B_QFULL), nkc * Q_CHUNK);
+        const int32_t qrow = (b * p.tq + k) * H;
+        for (int c = 0; c < 4; ++c)
+          tma_load_2d(sbase + OFF_Q + c * Q_CHUNK, &p.qmap, 256 * (int)r + 64 * c, qrow, bar(B_QFULL));
+        if (r == 0) tma_load_2d(sbase + OFF_Q + 4 * Q_CHUNK, &p.rmap, 0, qrow, bar(B_QFULL));
+        const int32_t ts_b = p.tile_start[b];
+        const int32_t row_base = (int32_t)p.cu[b];
+        for (int32_t xt = w.x; xt < w.seg_end(); ++xt, ++j) {
+          const int st = j % STAGES;
+          if (!mbar_wait(bar(B_EMPTY + st), ((j / STAGES) & 1) ^ 1)) { ok = false; break; }
+          mbar_expect_tx(bar(B_FULL + st), nkc * KV_BOX);
+          const int32_t row0 = row_base + (xt - ts_b) * NK;
+          const uint32_t dst = sbase + OFF_KV + st * STAGE_BYTES;
+          for (int c = 0; c < 4; ++c)
+            tma_load_2d(dst + c * KV_BOX, &p.cmap, 256 * (int)r + 64 * c, row0, bar(B_FULL + st));
+          if (r == 0) tma_load_2d(dst + 4 * KV_BOX, &p.cmap, DC, row0, bar(B_FULL + st));
+          issued = j + 1;
+        }
+      }
+      if (!ok) {
+        flag_error(p.err, DEVERR_TIMEOUT);
+        for (int i = max(0, issued - STAGES); i < issued; ++i) mbar_wait(bar(B_FULL + i % STAGES), (i / STAGES) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(128, NK, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
+      int j = 0, g = 0;
+      bool ok = true;
+      auto issue_pv = [&](int jj, bool first) -> bool {
+        const int pb = jj & 1;
+        if (!mbar_wait(bar(B_PFULL + pb), (jj >> 1) & 1)) return false;
+        if (first && !mbar_wait(bar(B_OFREE), (g & 1) ^ 1)) return false;
+        tc_fence_after();
+        const int st = jj % STAGES;
+        const uint32_t pa = sbase + OFF_P + pb * P_BYTES;
+        const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < NK / 16; ++kk)
+          mma_bf16_ss(tmem, sw64_desc(pa + kk * 32, 512), sw128_desc(kv + kk * 2048, KV_BOX, 1024), idesc_pv,
+                      (first && kk == 0) ? 0u : 1u);
+        mma_commit(bar(B_PVDONE + pb));
+        mma_commit(bar(B_EMPTY + st));
+        return true;
+      };
+      for (; ok && w.valid(); w.next(), ++g) {
+        if (!mbar_wait(bar(B_QFULL), g & 1)) { ok = false; break; }
+        const int jfirst = j;
+        const int32_t send = w.seg_end();
+        for (int32_t xt = w.x; xt < send; ++xt, ++j) {
+          const int st = j % STAGES, sb = j & 1;
+          if (!mbar_wait(bar(B_FULL + st), (j / STAGES) & 1) ||
+              !mbar_wait(bar(B_SEMPTY + sb), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
+          for (int kc = 0; kc < nkc; ++kc)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(tmem + 256 + 32 * sb, sw128_desc(sbase + OFF_Q + kc * Q_CHUNK + kk * 32, 0, 1024),
+                          sw128_desc(kv + kc * KV_BOX + kk * 32, 0, 1024), idesc_qk, (kc | kk) ? 1u : 0u);
+          mma_commit(bar(B_SFULL + sb));
+          if (xt == send - 1) mma_commit(bar(B_QEMPTY));
+          if (j > jfirst && !issue_pv(j - 1, j - 1 == jfirst)) { ok = false; break; }
+        }
+        if (!ok || !issue_pv(j - 1, j - 1 == jfirst)) { ok = false; break; }
+      }
+      if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int i = threadIdx.x;                       // head
+    const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+    const uint32_t xpeer = map_peer(sbase + OFF_X, peer) + i * 128;
+    const uint32_t xfull_peer = map_peer(bar(B_XFULL), peer);
+    const uint32_t xfree_peer = map_peer(bar(B_XFREE), peer);
+    int j = 0;
+    bool ok = true;
+    for (; ok && w.valid(); w.next()) {
+      const int b = w.b;
+      const int64_t len = p.cu[b + 1] - p.cu[b];
+      const int64_t vis = len - p.tq + k + 1;        // keys visible to this query token
+      const int32_t ts_b = p.tile_start[b];
+      const int32_t send = w.seg_end();
+      float m_ref = -INFINITY, l = 0.f;
+      const int jfirst = j;
+      for (int32_t xt = w.x; xt < send; ++xt, ++j) {
+        const int sb = j & 1, n = j >> 1;
+        uint32_t own[32];
+        float s[32];
+        // 1. this CTA's partial scores
+        if (!mbar_wait(bar(B_SFULL + sb), n & 1)) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld32(trow + 256 + 32 * sb, own);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_SEMPTY + sb));
+        // 2. send them to the peer, 3. receive the peer's
+        if (!mbar_wait_cluster(bar(B_XFREE + sb), (n & 1) ^ 1)) { ok = false; break; }
+        const uint32_t xdst = xpeer + sb * X_BYTES;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) st_peer_v4(xdst + 16 * c, own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
+        mbar_arrive_peer(xfull_peer + 8 * sb);
+        if (!mbar_wait_cluster(bar(B_XFULL + sb), n & 1)) { ok = false; break; }
+        const float4* xr = reinterpret_cast<const float4*>(smem + OFF_X + sb * X_BYTES + i * 128);
+        const int64_t key0 = (int64_t)(xt - ts_b) * NK;
+        const int nvis = (int)max((int64_t)0, min((int64_t)NK, vis - key0));
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 q = xr[c];
+          s[4 * c + 0] = __uint_as_float(own[4 * c + 0]) + q.x;
+          s[4 * c + 1] = __uint_as_float(own[4 * c + 1]) + q.y;
+          s[4 * c + 2] = __uint_as_float(own[4 * c + 2]) + q.z;
+          s[4 * c + 3] = __uint_as_float(own[4 * c + 3]) + q.w;
+        }
+        mbar_arrive_peer(xfree_peer + 8 * sb);
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          s[c] = c < nvis ? s[c] * p.scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, s[c]);
+        }
+        // rows of this stage past the sequence end: zero the latent half before P.V reads it
+        const int nrows = (int)max((int64_t)0, min((int64_t)NK, len - key0));
+        if (nrows < NK) {
+          uint8_t* kvs = smem + OFF_KV + (j % STAGES) * STAGE_BYTES;
+          const int chunks = (NK - nrows) * 4 * 8;   // 16-byte chunks over 4 boxes
+          for (int q = i; q < chunks; q += 128) {
+            const int row = nrows + q / 32, box = (q / 8) & 3, c16 = q & 7;
+            *reinterpret_cast<uint4*>(kvs + box * KV_BOX + row * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+        // 4. lazy rescale of the running max (identical decision in both CTAs)
+        if (tmax > -INFINITY && (m_ref == -INFINITY || tmax > m_ref + kRescaleLog2)) {
+          const float alpha = exp2f(m_ref - tmax);
+          if (j > jfirst) {
+            const int jp = j - 1;
+            if (!mbar_wait(bar(B_PVDONE + (jp & 1)), (jp >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 256; c += 32) {
+              uint32_t v[32];
+              tmem_ld32(trow + c, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+              tmem_st32(trow + c, v);
+            }
+            tmem_wait_st();
+          }
+          l *= alpha;
+          m_ref = tmax;
+        }
+        // 5. P = exp2(s - m_ref) in bf16 into the SW64 K-major A tile; its buffer was last read by PV(j-2)
+        if (!mbar_wait(bar(B_PVDONE + sb), (n & 1) ^ 1)) { ok = false; break; }
+        uint32_t pk[16];
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float e0 = s[2 * c] == -INFINITY ? 0.f : exp2f(s[2 * c] - m_ref);
+          const float e1 = s[2 * c + 1] == -INFINITY ? 0.f : exp2f(s[2 * c + 1] - m_ref);
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+          lsum += __low2float(h2) + __high2float(h2);
+          pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        l += lsum;
+        uint8_t* prow = smem + OFF_P + sb * P_BYTES + i * 64;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ ((i >> 1) & 3)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL + sb));
+      }
+      if (!ok) break;
+      // segment epilogue: O / l for this CTA's 256 columns (+ lse from CTA 0)
+      const int jl = j - 1;
+      if (!mbar_wait(bar(B_PVDONE + (jl & 1)), (jl >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const int64_t t = (int64_t)b * p.tq + k;
+      const int32_t nseg = p.slot_base[b + 1] - p.slot_base[b];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float lse_v = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      float* po = nullptr;
+      if (nseg > 1) {
+        const int64_t slot = (int64_t)p.slot_base[b] + (pair - (int)(((int64_t)(ts_b + 1) * npairs - 1) / NT));
+        const int64_t row = ((int64_t)k * p.s_max + slot) * H + i;
+        po = p.part_o + row * DC + 256 * r;
+        if (r == 0) p.part_lse[row] = lse_v;
+      } else if (r == 0) {
+        p.lse[t * H + i] = lse_v;
+      }
+#pragma unroll 1
+      for (int c = 0; c < 256; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + c, v);
+        tmem_wait_ld();
+        if (po) {
+          float4* dst = reinterpret_cast<float4*>(po + c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
+                                 __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
+        } else if (OUT_F32) {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o_lat) + (t * H + i) * DC + 256 * r + c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
+                                 __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o_lat) + (t * H + i) * DC +
+                                                256 * r + c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pack_bf16(__uint_as_float(v[8 * e]) * inv, __uint_as_float(v[8 * e + 1]) * inv),
+                                pack_bf16(__uint_as_float(v[8 * e + 2]) * inv, __uint_as_float(v[8 * e + 3]) * inv),
+                                pack_bf16(__uint_as_float(v[8 * e + 4]) * inv, __uint_as_float(v[8 * e + 5]) * inv),
+                                pack_bf16(__uint_as_float(v[8 * e + 6]) * inv, __uint_as_float(v[8 * e + 7]) * inv));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_OFREE));
+    }
+    if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
+  }
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Tile prefix and partial-slot bases of every sequence (one block). Tiles per sequence are
+// counted on the cache length len_b (the last query token sees all of them). A sequence gets
+// one slot per active pair whose tile range meets it.
+__global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B, int32_t pairs, int32_t* ts,
+                                                   int32_t* sb) {
+  __shared__ int32_t part[256];
+  const int tid = threadIdx.x;
+  const int per = (B + 255) / 256;
+  const int lo = min(B, tid * per), hi = min(B, lo + per);
+  auto ntiles = [&](int b) -> int32_t {
+    const int64_t len = cu[b + 1] - cu[b];
+    return len > 0 ? (int32_t)((len + NK - 1) / NK) : 0;
+  };
+  // pass 1: tile prefix
+  int32_t acc = 0;
+  for (int b = lo; b < hi; ++b) acc += ntiles(b);
+  part[tid] = acc;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t run = 0;
+    for (int q = 0; q < 256; ++q) { const int32_t v = part[q]; part[q] = run; run += v; }
+    ts[B] = run;
+  }
+  __syncthreads();
+  acc = part[tid];
+  for (int b = lo; b < hi; ++b) { ts[b] = acc; acc += ntiles(b); }
+  __syncthreads();
+  // pass 2: pieces per sequence (pairs whose range meets it) and slot prefix
+  const int64_t NT = ts[B];
+  const int64_t npairs = NT < pairs ? NT : pairs;   // every active pair holds >= 1 tile
+  auto pair_of = [&](int64_t x) -> int64_t { return ((x + 1) * npairs - 1) / NT; };
+  auto nseg = [&](int b) -> int32_t {
+    const int32_t a = ts[b], e = ts[b + 1];
+    return e > a ? (int32_t)(pair_of(e - 1) - pair_of(a) + 1) : 0;
+  };
+  acc = 0;
+  for (int b = lo; b < hi; ++b) acc += nseg(b);
+  __syncthreads();
+  part[tid] = acc;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t run = 0;
+    for (int q = 0; q < 256; ++q) { const int32_t v = part[q]; part[q] = run; run += v; }
+    sb[B] = run;
+  }
+  __syncthreads();
+  acc = part[tid];
+  for (int b = lo; b < hi; ++b) { sb[b] = acc; acc += nseg(b); }
+}
+
+// Exact merge of a sequence's pieces: lse = log sum_s e^{lse_s}, o = sum_s e^{lse_s - lse} o_s.
+// One block of 128 threads per (token, head); sequences in a single piece were written directly.
+template <bool OUT_F32>
+__global__ void __launch_bounds__(128) combine_kernel(const int32_t* sb, int32_t tq, int32_t s_max,
+                                                      const float* part_o, const float* part_lse, void* o_lat,
+                                                      float* lse) {
+  const int64_t t = blockIdx.x;
+  const int h = blockIdx.y;
+  const int b = (int)(t / tq), k = (int)(t % tq);
+  const int32_t s0 = sb[b], ns = sb[b + 1] - s0;
+  if (ns == 1) return;
+  float mx = -INFINITY;
+  for (int s = 0; s < ns; ++s) mx = fmaxf(mx, part_lse[((int64_t)k * s_max + s0 + s) * H + h]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
+  if (mx > -INFINITY) {
+    for (int s = 0; s < ns; ++s) {
+      const int64_t row = ((int64_t)k * s_max + s0 + s) * H + h;
+      const float wgt = __expf(part_lse[row] - mx);
+      wsum += wgt;
+      const float4 v = reinterpret_cast<const float4*>(part_o + row * DC)[threadIdx.x];
+      acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+  if (OUT_F32) {
+    reinterpret_cast<float4*>(reinterpret_cast<float*>(o_lat) + (t * H + h) * DC)[threadIdx.x] = acc;
+  } else {
+    uint2 v2 = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+    reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(o_lat) + (t * H + h) * DC)[threadIdx.x] = v2;
+  }
+  if (threadIdx.x == 0) lse[t * H + h] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+}
+
+size_t align1k(size_t x) { return (x + 1023) / 1024 * 1024; }
+
+struct CoreScratch {
+  int32_t* ts;
+  int32_t* sb;
+  float* part_lse;
+  float* part_o;
+  int32_t s_max;
+};
+
+CoreScratch carve(void* scratch, int64_t B, int32_t tq) {
+  CoreScratch c;
+  char* p = (char*)scratch;
+  c.s_max = (int32_t)(kMaxPairs + B);
+  c.ts = (int32_t*)p;
+  p += align1k((B + 1) * 4);
+  c.sb = (int32_t*)p;
+  p += align1k((B + 1) * 4);
+  c.part_lse = (float*)p;
+  p += align1k((size_t)tq * c.s_max * H * 4);
+  c.part_o = (float*)p;
+  return c;
+}
+
+template <bool OUT_F32>
+cudaError_t launch_core(const CoreParams& p, dim3 grid, cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(latent_core_kernel<OUT_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  latent_core_kernel<OUT_F32><<<grid, kThreads, SMEM_BYTES, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t tc_core_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq) {
+  (void)d;
+  const int64_t s_max = kMaxPairs + B;
+  return 2 * align1k((B + 1) * 4) + align1k((size_t)tq * s_max * H * 4) + (size_t)tq * s_max * H * DC * 4;
+}
+
+cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
+                                const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse,
+                                void* scratch, int num_sms, uint32_t* err, cudaStream_t st) {
+  if (B <= 0) return cudaSuccess;
+  if (B > (int64_t)1 << 20 || capacity > INT32_MAX || B * tq * H > INT32_MAX) return cudaErrorInvalidValue;
+  const int64_t T = B * tq;
+  CoreScratch c = carve(scratch, B, tq);
+  int pairs = num_sms / (2 * tq);
+  pairs = pairs < kMaxPairs ? pairs : kMaxPairs;
+  pairs = pairs < 1 ? 1 : pairs;
+  plan_kernel<<<1, 256, 0, st>>>(cu, (int32_t)B, pairs, c.ts, c.sb);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CoreParams p;
+  memset(&p, 0, sizeof(p));
+  if ((e = make_tmap_bf16(&p.qmap, q_abs, DC, T * H, DC, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&p.rmap, q_rope, DR, T * H, DR, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&p.cmap, cache, ROW, capacity, ROW, 64, NK)) != cudaSuccess) return e;
+  p.cu = cu;
+  p.tile_start = c.ts;
+  p.slot_base = c.sb;
+  p.B = (int32_t)B;
+  p.tq = tq;
+  p.pairs = pairs;
+  p.s_max = c.s_max;
+  p.part_o = c.part_o;
+  p.part_lse = c.part_lse;
+  p.o_lat = o_lat;
+  p.lse = lse;
+  p.scale_log2 = (float)(1.4426950408889634 / sqrt(128.0 + 64.0));
+  p.err = err;
+  dim3 grid((unsigned)(2 * pairs), (unsigned)tq);
+  e = o_f32 ? launch_core<true>(p, grid, st) : launch_core<false>(p, grid, st);
+  if (e != cudaSuccess) return e;
+  dim3 cg((unsigned)T, (unsigned)H);
+  if (o_f32) combine_kernel<true><<<cg, 128, 0, st>>>(c.sb, tq, c.s_max, c.part_o, c.part_lse, o_lat, lse);
+  else combine_kernel<false><<<cg, 128, 0, st>>>(c.sb, tq, c.s_max, c.part_o, c.part_lse, o_lat, lse);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -98,32 +98,11 @@ cudaError_t output(const mla_dims_t& d, const mla_weights_t& w, const void* o, i
   return tc_gemm(g, st);
 }
 
-cudaError_t simt_core(const mla_dims_t& d, const void* q_abs, const void* q_rope, int64_t B, int32_t tq,
-                      const int64_t* cu, const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse,
-                      uint32_t* err, cudaStream_t st) {
-  const int64_t R = d.d_c + d.d_r;
-  SimtAttnArgs a;
-  memset(&a, 0, sizeof(a));
-  a.q1 = q_abs; a.sq1t = (int64_t)d.n_h * d.d_c; a.sq1h = d.d_c; a.d1 = d.d_c;
-  a.q2 = q_rope; a.sq2t = (int64_t)d.n_h * d.d_r; a.sq2h = d.d_r; a.d2 = d.d_r;
-  a.k1 = cache; a.sk1 = R; a.sk1h = 0;
-  a.k2 = (const char*)cache + (size_t)d.d_c * 2; a.sk2 = R;
-  a.v = cache; a.sv = R; a.svh = 0; a.dv = d.d_c;
-  a.o = o_lat; a.sot = (int64_t)d.n_h * d.d_c; a.soh = d.d_c;
-  a.lse = lse;
-  a.cu = cu; a.B = B; a.tq = tq; a.T = B * tq; a.n_h = d.n_h; a.capacity = capacity;
-  a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
-  a.err = err;
-  return simt_attention(a, true, o_f32, st);
-}
-
 }  // namespace
 
-bool tc_available(mla_op_t op) { return op != MLA_OP_ATTN_DECODE_LATENT; }
-
-size_t tc_core_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq) {
-  (void)d; (void)B; (void)tq;
-  return 0;
+bool tc_available(mla_op_t op) {
+  (void)op;
+  return true;
 }
 
 size_t tc_decode_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq) {
@@ -144,8 +123,9 @@ cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const v
 cudaError_t tc_latent_core(const mla_dims_t& d, const void* q_abs, const void* q_rope, int64_t B, int32_t tq,
                            const int64_t* cu, const void* cache, int64_t capacity, void* o_lat, bool o_f32,
                            float* lse, void* scratch, int num_sms, uint32_t* err, cudaStream_t st) {
-  (void)scratch; (void)num_sms;
-  return simt_core(d, q_abs, q_rope, B, tq, cu, cache, capacity, o_lat, o_f32, lse, err, st);
+  (void)d;
+  return tc_latent_core_impl(q_abs, q_rope, B, tq, cu, cache, capacity, o_lat, o_f32, lse, scratch, num_sms, err,
+                             st);
 }
 
 cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const void* h_q, int64_t B, int32_t tq,

@@ -96,10 +96,12 @@ def test_tiny_cache_append_fp32_scattered_slots():
 # ---------------------------------------------------------------------------
 # BF16 at the DeepSeek-V3 sizes, small batches with ragged tails
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("tq", [1, 2])
-def test_v3_attn_core_bf16_ragged(v3_module, tq):
+@pytest.mark.parametrize("tq,lens", [(1, [1, 63, 64, 65, 129, 1000, 4097]), (2, [2, 63, 64, 65, 129, 1000, 4097]),
+                                     (1, [1, 40, 100]), (2, [33, 2, 97])])
+def test_v3_attn_core_bf16_ragged(v3_module, tq, lens):
+    # the last two cases hold fewer key tiles than there are CTA pairs
     dims = synth.V3
-    lens = np.array([tq, 63, 64, 65, 129, 1000, 4097])
+    lens = np.array(lens)
     cu = synth.cu_seqlens(lens)
     B, T = len(lens), len(lens) * tq
     cache = synth.latent_cache(dims, int(cu[-1]), seed=10 + tq, dtype="bf16")
@@ -111,6 +113,28 @@ def test_v3_attn_core_bf16_ragged(v3_module, tq):
     _status_ok(v3_module)
     assert rel(host(o_lat), lat_ref) <= TOL["bf16"]
     assert rel(host(lse), lse_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("tq", [1, 2])
+def test_v3_attn_core_many_short_sequences(v3_module, tq):
+    # more sequences than CTA pairs: one pair walks many sequence pieces; lengths from Tq up
+    dims = synth.V3
+    lens = synth.ragged_lengths(300, tq, 70, seed=tq)
+    lens[:3] = tq
+    cu = synth.cu_seqlens(lens)
+    B, T = len(lens), len(lens) * tq
+    cache = synth.latent_cache(dims, int(cu[-1]), seed=30 + tq, dtype="bf16")
+    q_abs = synth.normal(31, 20, (T, dims.n_h, dims.d_c), std=0.5, dtype="bf16")
+    q_rope = synth.normal(31, 21, (T, dims.n_h, dims.d_r), std=1.0, dtype="bf16")
+    seqs = [0, 1, 2, 57, 150, 299]
+    lat_ref, lse_ref = orc.attn_decode_latent(q_abs, q_rope, cache, cu, tq, dims, seqs=seqs)
+    o_lat, lse = v3_module.attn_decode_latent(dev(q_abs, "bf16"), dev(q_rope, "bf16"), B, tq, dev_i64(cu),
+                                              dev(cache, "bf16"))
+    _status_ok(v3_module)
+    rows = np.concatenate([np.arange(b * tq, (b + 1) * tq) for b in seqs])
+    assert rel(host(o_lat)[rows], lat_ref) <= TOL["bf16"]
+    assert rel(host(lse)[rows], lse_ref) <= TOL["bf16"]
+    assert np.all(np.isfinite(host(o_lat)))
 
 
 @pytest.mark.parametrize("tq", [1, 2])
