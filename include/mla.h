@@ -167,6 +167,9 @@ mla_status_t mla_sync_status(mla_handle_t *h, mla_stream_t stream);
 /* Bits of the last error word read by mla_sync_status (see MLA_DEVERR_* in the source). */
 uint32_t mla_device_error_bits(const mla_handle_t *h);
 
+/* Number of kernels this library has launched in this process (all handles, all devices). */
+uint64_t mla_kernel_launches(void);
+
 /* Which kernel family a call of `op` takes with this handle: 1 = tcgen05/TMA (BF16 at the V3
  * sizes), 0 = generic CUDA-core kernels (FP32, or other sizes). Host-only. */
 int mla_uses_tensor_cores(const mla_handle_t *h, mla_op_t op);

@@ -5,6 +5,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <new>
 
 #include "mla.h"
@@ -22,6 +23,11 @@ struct mla_handle {
   uint32_t last_err_bits;  // last word read by mla_sync_status
   int num_sms;
 };
+
+namespace mla {
+static std::atomic<unsigned long long> g_launches{0};
+void note_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace mla
 
 namespace {
 
@@ -447,6 +453,8 @@ mla_status_t mla_sync_status(mla_handle_t* h, mla_stream_t stream) {
 }
 
 uint32_t mla_device_error_bits(const mla_handle_t* h) { return h ? h->last_err_bits : 0u; }
+
+uint64_t mla_kernel_launches(void) { return mla::g_launches.load(std::memory_order_relaxed); }
 
 void mla_destroy(mla_handle_t* h) {
   if (!h) return;

@@ -18,6 +18,9 @@ enum : uint32_t {
   DEVERR_TIMEOUT = 1u << 6,       // a bounded mbarrier wait gave up
 };
 
+// Host-side count of kernels this library has launched (mla_kernel_launches()).
+void note_launch(unsigned n = 1);
+
 __device__ __forceinline__ void flag_error(uint32_t* err, uint32_t bits) {
   if (err) atomicOr(err, bits);
 }

@@ -193,6 +193,7 @@ cudaError_t simt_gemm(const SimtGemmArgs& a, bool in_bf16, bool out_bf16, cudaSt
   else if (in_bf16) simt_gemm_kernel<__nv_bfloat16, float><<<grid, 256, 0, st>>>(a);
   else if (out_bf16) simt_gemm_kernel<float, __nv_bfloat16><<<grid, 256, 0, st>>>(a);
   else simt_gemm_kernel<float, float><<<grid, 256, 0, st>>>(a);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -203,6 +204,7 @@ cudaError_t simt_attention(const SimtAttnArgs& a, bool in_bf16, bool out_f32, cu
   if (in_bf16 && out_f32) simt_attention_kernel<__nv_bfloat16, float><<<grid, ATT_THREADS, 0, st>>>(a);
   else if (in_bf16) simt_attention_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, ATT_THREADS, 0, st>>>(a);
   else simt_attention_kernel<float, float><<<grid, ATT_THREADS, 0, st>>>(a);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -210,6 +212,7 @@ cudaError_t check_and_positions(const int64_t* cu, int64_t B, int32_t tq, int64_
                                 int64_t capacity, int64_t max_seqlen, int64_t* pos_out, uint32_t* err,
                                 cudaStream_t st) {
   check_positions_kernel<<<1, 512, 0, st>>>(cu, B, tq, total_tokens, capacity, max_seqlen, pos_out, err);
+  note_launch();
   return cudaGetLastError();
 }
 

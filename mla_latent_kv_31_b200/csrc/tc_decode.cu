@@ -31,37 +31,37 @@ namespace {
 using namespace sm100;
 
 constexpr int H = 128, DC = 512, DR = 64, ROW = DC + DR;
-constexpr int NK = 32;                       // keys per tile
+constexpr int NK = 64;                       // keys per tile (the N of QK^T, the K of P.V)
 constexpr int STAGES = 4;
 constexpr int kThreads = 192;
 constexpr int kMaxPairs = 74;
 constexpr float kRescaleLog2 = 8.f;          // lazy rescale: keep the running max until it grows by 2^8
 
-constexpr uint32_t Q_CHUNK = H * 128;        // [128 rows x 64 cols] bf16, SW128: 16 KB
-constexpr uint32_t KV_BOX = NK * 128;        // [32 keys x 64 cols] bf16, SW128: 4 KB
+constexpr uint32_t KV_BOX = NK * 128;        // [64 keys x 64 cols] bf16, SW128: 8 KB
 constexpr uint32_t STAGE_BYTES = 5 * KV_BOX; // 4 latent boxes + (CTA 0) the k^R box
-constexpr uint32_t P_BYTES = H * NK * 2;     // [128 x 32] bf16, SW64: 8 KB
-constexpr uint32_t X_BYTES = H * NK * 4;     // [128 x 32] fp32 partial scores: 16 KB
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_KV = OFF_Q + 5 * Q_CHUNK;
-constexpr uint32_t OFF_P = OFF_KV + STAGES * STAGE_BYTES;
-constexpr uint32_t OFF_X = OFF_P + 2 * P_BYTES;
+constexpr uint32_t X_BYTES = H * NK * 4;     // [128 x 64] fp32 partial scores from the peer: 32 KB
+constexpr uint32_t OFF_KV = 0;
+constexpr uint32_t OFF_X = OFF_KV + STAGES * STAGE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_X + 2 * X_BYTES;
-constexpr int NBAR = 2 * STAGES + 15;
+constexpr int NBAR = 2 * STAGES + 12;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
-constexpr uint32_t TMEM_COLS = 512;          // O half: [0, 256); S buffers: 256 + 32 b
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// TMEM columns: O half [0, 256); q~ half + (CTA 0) q^R [256, 416) as bf16 pairs (the A operand of
+// QK^T); S [416, 480); P [480, 512) as bf16 pairs (the A operand of P.V).
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t T_Q = 256, T_S = 416, T_P = T_S + NK;
+static_assert(T_P + NK / 2 <= TMEM_COLS, "TMEM budget");
 
 // barrier indices
-constexpr int B_FULL = 0, B_EMPTY = STAGES, B_SFULL = 2 * STAGES, B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2,
-              B_PVDONE = B_PFULL + 2, B_XFULL = B_PVDONE + 2, B_XFREE = B_XFULL + 2, B_QFULL = B_XFREE + 2,
+constexpr int B_FULL = 0, B_EMPTY = STAGES, B_SFULL = 2 * STAGES, B_SEMPTY = B_SFULL + 1, B_PFULL = B_SEMPTY + 1,
+              B_PVDONE = B_PFULL + 1, B_XFULL = B_PVDONE + 1, B_XFREE = B_XFULL + 2, B_QFULL = B_XFREE + 2,
               B_QEMPTY = B_QFULL + 1, B_OFREE = B_QEMPTY + 1;
 static_assert(B_OFREE + 1 <= NBAR, "barrier count");
 
 struct CoreParams {
-  CUtensorMap qmap;   // q~ as [T*H, DC], box {64, 128}
-  CUtensorMap rmap;   // q^R as [T*H, DR], box {64, 128}
-  CUtensorMap cmap;   // cache as [capacity, ROW], box {64, 32}
+  CUtensorMap cmap;   // cache as [capacity, ROW], box {64, NK}
+  const __nv_bfloat16* q_abs;   // [T][H][DC]
+  const __nv_bfloat16* q_rope;  // [T][H][DR]
   const int64_t* cu;
   const int32_t* tile_start;  // [B+1]: first global tile of each sequence
   const int32_t* slot_base;   // [B+1]: first partial slot of each sequence
@@ -105,6 +105,30 @@ struct SegWalk {
   }
 };
 
+// Walks the tiles of a range one by one: j (tile count), g (piece count), first/last of a piece.
+struct TileCursor {
+  SegWalk w;
+  int32_t xt;
+  int j, g;
+  __device__ void init(const int32_t* ts, int B, int32_t x0, int32_t x1) {
+    w.init(ts, B, x0, x1);
+    xt = w.x;
+    j = 0;
+    g = 0;
+  }
+  __device__ bool valid() const { return w.valid(); }
+  __device__ bool first() const { return xt == w.x; }
+  __device__ bool last() const { return xt == w.seg_end() - 1; }
+  __device__ void advance() {
+    ++j;
+    if (++xt >= w.seg_end()) {
+      w.next();
+      ++g;
+      xt = w.x;
+    }
+  }
+};
+
 template <bool OUT_F32>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     latent_core_kernel(const __grid_constant__ CoreParams p) {
@@ -129,23 +153,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
-      uint32_t cnt = 1;
-      if (i == B_SEMPTY || i == B_SEMPTY + 1 || i == B_PFULL || i == B_PFULL + 1 || i == B_XFULL ||
-          i == B_XFULL + 1 || i == B_XFREE || i == B_XFREE + 1 || i == B_OFREE)
-        cnt = 128;
-      mbar_init(bar(i), cnt);
+      const bool many = i == B_SEMPTY || i == B_PFULL || i == B_XFREE || i == B_XFREE + 1 || i == B_OFREE ||
+                        i == B_QFULL;
+      mbar_init(bar(i), many ? 128 : 1);
     }
+    // the exchange buffers' first phase: one arrival plus the bytes the peer's st.async will bring
+    mbar_expect_tx(bar(B_XFULL), X_BYTES);
+    mbar_expect_tx(bar(B_XFULL + 1), X_BYTES);
     fence_mbar_init();
   }
   if (warp == 5) {
     tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&p.qmap);
-    prefetch_tmap(&p.rmap);
-    prefetch_tmap(&p.cmap);
-  }
+  if (threadIdx.x == 0) prefetch_tmap(&p.cmap);
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
@@ -157,16 +178,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 4) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int j = 0, g = 0, issued = 0;
+      int j = 0, issued = 0;
       bool ok = true;
-      for (; ok && w.valid(); w.next(), ++g) {
+      for (; ok && w.valid(); w.next()) {
         const int b = w.b;
-        if (!mbar_wait(bar(B_QEMPTY), (g & 1) ^ 1)) { ok = false; break; }
-        mbar_expect_tx(bar(B_QFULL), nkc * Q_CHUNK);
-        const int32_t qrow = (b * p.tq + k) * H;
-        for (int c = 0; c < 4; ++c)
-          tma_load_2d(sbase + OFF_Q + c * Q_CHUNK, &p.qmap, 256 * (int)r + 64 * c, qrow, bar(B_QFULL));
-        if (r == 0) tma_load_2d(sbase + OFF_Q + 4 * Q_CHUNK, &p.rmap, 0, qrow, bar(B_QFULL));
         const int32_t ts_b = p.tile_start[b];
         const int32_t row_base = (int32_t)p.cu[b];
         for (int32_t xt = w.x; xt < w.seg_end(); ++xt, ++j) {
@@ -188,47 +203,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
+    // Greedy: P.V for the oldest tile whose P is ready, else QK^T of the next tile once its cache
+    // tile has landed and the softmax has taken the previous scores out of TMEM.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, NK, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
-      int j = 0, g = 0;
+      TileCursor cq, cp;
+      cq.init(p.tile_start, p.B, t_begin, t_end);
+      cp.init(p.tile_start, p.B, t_begin, t_end);
+      uint64_t stall_since = 0;
       bool ok = true;
-      auto issue_pv = [&](int jj, bool first) -> bool {
-        const int pb = jj & 1;
-        if (!mbar_wait(bar(B_PFULL + pb), (jj >> 1) & 1)) return false;
-        if (first && !mbar_wait(bar(B_OFREE), (g & 1) ^ 1)) return false;
-        tc_fence_after();
-        const int st = jj % STAGES;
-        const uint32_t pa = sbase + OFF_P + pb * P_BYTES;
-        const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < NK / 16; ++kk)
-          mma_bf16_ss(tmem, sw64_desc(pa + kk * 32, 512), sw128_desc(kv + kk * 2048, KV_BOX, 1024), idesc_pv,
-                      (first && kk == 0) ? 0u : 1u);
-        mma_commit(bar(B_PVDONE + pb));
-        mma_commit(bar(B_EMPTY + st));
-        return true;
-      };
-      for (; ok && w.valid(); w.next(), ++g) {
-        if (!mbar_wait(bar(B_QFULL), g & 1)) { ok = false; break; }
-        const int jfirst = j;
-        const int32_t send = w.seg_end();
-        for (int32_t xt = w.x; xt < send; ++xt, ++j) {
-          const int st = j % STAGES, sb = j & 1;
-          if (!mbar_wait(bar(B_FULL + st), (j / STAGES) & 1) ||
-              !mbar_wait(bar(B_SEMPTY + sb), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+      while (cp.valid()) {
+        bool did = false;
+        if (cp.j < cq.j && mbar_test(bar(B_PFULL), cp.j & 1) &&
+            (!cp.first() || mbar_test(bar(B_OFREE), (cp.g & 1) ^ 1))) {
           tc_fence_after();
+          const int st = cp.j % STAGES;
           const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
-          for (int kc = 0; kc < nkc; ++kc)
+          const bool first = cp.first();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(tmem + 256 + 32 * sb, sw128_desc(sbase + OFF_Q + kc * Q_CHUNK + kk * 32, 0, 1024),
-                          sw128_desc(kv + kc * KV_BOX + kk * 32, 0, 1024), idesc_qk, (kc | kk) ? 1u : 0u);
-          mma_commit(bar(B_SFULL + sb));
-          if (xt == send - 1) mma_commit(bar(B_QEMPTY));
-          if (j > jfirst && !issue_pv(j - 1, j - 1 == jfirst)) { ok = false; break; }
+          for (int kk = 0; kk < NK / 16; ++kk)
+            mma_bf16_ts(tmem, tmem + T_P + 8 * kk, sw128_desc(kv + kk * 2048, KV_BOX, 1024), idesc_pv,
+                        (first && kk == 0) ? 0u : 1u);
+          mma_commit(bar(B_PVDONE));
+          mma_commit(bar(B_EMPTY + st));
+          cp.advance();
+          did = true;
         }
-        if (!ok || !issue_pv(j - 1, j - 1 == jfirst)) { ok = false; break; }
+        if (!did && cq.valid()) {
+          const int st = cq.j % STAGES;
+          if (mbar_test(bar(B_FULL + st), (cq.j / STAGES) & 1) && mbar_test(bar(B_SEMPTY), (cq.j & 1) ^ 1) &&
+              (!cq.first() || mbar_test(bar(B_QFULL), cq.g & 1))) {
+            tc_fence_after();
+            const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
+            for (int kc = 0; kc < nkc; ++kc)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(tmem + T_S, tmem + T_Q + 32 * kc + 8 * kk, sw128_desc(kv + kc * KV_BOX + kk * 32, 0, 1024),
+                            idesc_qk, (kc | kk) ? 1u : 0u);
+            mma_commit(bar(B_SFULL));
+            if (cq.last()) mma_commit(bar(B_QEMPTY));
+            cq.advance();
+            did = true;
+          }
+        }
+        if (did) {
+          stall_since = 0;
+        } else if (stall_since == 0) {
+          stall_since = globaltimer();
+        } else if (globaltimer() - stall_since > kWaitTimeoutNs) {
+          ok = false;
+          break;
+        }
       }
       if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
     }
@@ -236,10 +262,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ softmax + epilogue
     const int i = threadIdx.x;                       // head
     const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
-    const uint32_t xpeer = map_peer(sbase + OFF_X, peer) + i * 128;
+    const uint32_t xpeer = map_peer(sbase + OFF_X, peer) + i * 16;
     const uint32_t xfull_peer = map_peer(bar(B_XFULL), peer);
     const uint32_t xfree_peer = map_peer(bar(B_XFREE), peer);
-    int j = 0;
+    const float c2 = p.scale_log2;                   // raw score -> log2 units
+    const float thr_raw = kRescaleLog2 / c2;
+    // This CTA's partial scores of tile jj: TMEM -> registers; then sent to the peer with st.async
+    // (chunk-major layout: element c of head i at ((c / 4) * 128 + i) * 16 + (c % 4) * 4), each store
+    // counting its bytes on the peer's x_full barrier.
+    auto fetch_send = [&](int jj, uint32_t(&own)[NK]) -> bool {
+      if (!mbar_wait(bar(B_SFULL), jj & 1)) return false;
+      tc_fence_after();
+      tmem_ld32(trow + T_S, own);
+      tmem_ld32(trow + T_S + 32, own + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_SEMPTY));
+      const int xb = jj & 1;
+      if (!mbar_wait_cluster(bar(B_XFREE + xb), ((jj >> 1) & 1) ^ 1)) return false;
+      const uint32_t dst = xpeer + xb * X_BYTES, xbar = xfull_peer + 8 * xb;
+#pragma unroll
+      for (int c = 0; c < NK / 4; ++c)
+        st_async_peer_v4(dst + c * 2048, own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3], xbar);
+      return true;
+    };
+    int gq = 0, j = 0;
     bool ok = true;
     for (; ok && w.valid(); w.next()) {
       const int b = w.b;
@@ -247,44 +294,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int64_t vis = len - p.tq + k + 1;        // keys visible to this query token
       const int32_t ts_b = p.tile_start[b];
       const int32_t send = w.seg_end();
-      float m_ref = -INFINITY, l = 0.f;
+      float m_ref = -INFINITY, l = 0.f;              // running max in raw score units
       const int jfirst = j;
-      for (int32_t xt = w.x; xt < send; ++xt, ++j) {
-        const int sb = j & 1, n = j >> 1;
-        uint32_t own[32];
-        float s[32];
-        // 1. this CTA's partial scores
-        if (!mbar_wait(bar(B_SFULL + sb), n & 1)) { ok = false; break; }
+      // q~ half (and q^R on CTA 0) of this token and head -> TMEM, once the last piece's QK^T is done
+      {
+        const int64_t t = (int64_t)b * p.tq + k;
+        if (!mbar_wait(bar(B_QEMPTY), (gq & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        tmem_ld32(trow + 256 + 32 * sb, own);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(B_SEMPTY + sb));
-        // 2. send them to the peer, 3. receive the peer's
-        if (!mbar_wait_cluster(bar(B_XFREE + sb), (n & 1) ^ 1)) { ok = false; break; }
-        const uint32_t xdst = xpeer + sb * X_BYTES;
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (t * H + i) * DC + 256 * r);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) st_peer_v4(xdst + 16 * c, own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
-        mbar_arrive_peer(xfull_peer + 8 * sb);
-        if (!mbar_wait_cluster(bar(B_XFULL + sb), n & 1)) { ok = false; break; }
-        const float4* xr = reinterpret_cast<const float4*>(smem + OFF_X + sb * X_BYTES + i * 128);
+          for (int e = 0; e < 8; ++e) {
+            const uint4 u = __ldg(src + 8 * c + e);
+            v[4 * e] = u.x; v[4 * e + 1] = u.y; v[4 * e + 2] = u.z; v[4 * e + 3] = u.w;
+          }
+          tmem_st32(trow + T_Q + 32 * c, v);
+        }
+        if (r == 0) {
+          const uint4* rsrc = reinterpret_cast<const uint4*>(p.q_rope + (t * H + i) * DR);
+          uint32_t v[32];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint4 u = __ldg(rsrc + e);
+            v[4 * e] = u.x; v[4 * e + 1] = u.y; v[4 * e + 2] = u.z; v[4 * e + 3] = u.w;
+          }
+          tmem_st32(trow + T_Q + 128, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_QFULL));
+        ++gq;
+      }
+      // One tile: cur holds this CTA's partial scores of tile j; the next tile's go to nxt.
+      auto tile = [&](int32_t xt, uint32_t(&cur)[NK], uint32_t(&nxt)[NK]) -> bool {
+        const bool more = xt + 1 < send;
+        if (more && !fetch_send(j + 1, nxt)) return false;
+        const int xb = j & 1;
+        if (!mbar_wait_cluster(bar(B_XFULL + xb), (j >> 1) & 1)) return false;
+        const float4* xr = reinterpret_cast<const float4*>(smem + OFF_X + xb * X_BYTES) + i;
+        float s[NK];
+#pragma unroll
+        for (int c = 0; c < NK / 4; ++c) {
+          const float4 q = xr[c * 128];
+          f2_unpack(f2_add(f2_pack(__uint_as_float(cur[4 * c]), __uint_as_float(cur[4 * c + 1])), f2_pack(q.x, q.y)),
+                    s[4 * c], s[4 * c + 1]);
+          f2_unpack(f2_add(f2_pack(__uint_as_float(cur[4 * c + 2]), __uint_as_float(cur[4 * c + 3])), f2_pack(q.z, q.w)),
+                    s[4 * c + 2], s[4 * c + 3]);
+        }
+        // re-arm this buffer's next phase (one arrival + the bytes), then tell the peer it is free
+        if (i == 0) mbar_expect_tx(bar(B_XFULL + xb), X_BYTES);
+        mbar_arrive_peer_relaxed(xfree_peer + 8 * xb);
         const int64_t key0 = (int64_t)(xt - ts_b) * NK;
         const int nvis = (int)max((int64_t)0, min((int64_t)NK, vis - key0));
+        if (nvis < NK) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float4 q = xr[c];
-          s[4 * c + 0] = __uint_as_float(own[4 * c + 0]) + q.x;
-          s[4 * c + 1] = __uint_as_float(own[4 * c + 1]) + q.y;
-          s[4 * c + 2] = __uint_as_float(own[4 * c + 2]) + q.z;
-          s[4 * c + 3] = __uint_as_float(own[4 * c + 3]) + q.w;
+          for (int c = 0; c < NK; ++c) s[c] = c < nvis ? s[c] : -INFINITY;
         }
-        mbar_arrive_peer(xfree_peer + 8 * sb);
-        float tmax = -INFINITY;
+        float mx[NK / 2];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          s[c] = c < nvis ? s[c] * p.scale_log2 : -INFINITY;
-          tmax = fmaxf(tmax, s[c]);
-        }
+        for (int c = 0; c < NK / 2; ++c) mx[c] = fmaxf(s[2 * c], s[2 * c + 1]);
+#pragma unroll
+        for (int w2 = NK / 4; w2 > 0; w2 >>= 1)
+#pragma unroll
+          for (int c = 0; c < w2; ++c) mx[c] = fmaxf(mx[c], mx[c + w2]);
+        const float tmax = mx[0];
         // rows of this stage past the sequence end: zero the latent half before P.V reads it
         const int nrows = (int)max((int64_t)0, min((int64_t)NK, len - key0));
         if (nrows < NK) {
@@ -294,13 +369,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int row = nrows + q / 32, box = (q / 8) & 3, c16 = q & 7;
             *reinterpret_cast<uint4*>(kvs + box * KV_BOX + row * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
           }
+          fence_proxy_async_smem();
         }
-        // 4. lazy rescale of the running max (identical decision in both CTAs)
-        if (tmax > -INFINITY && (m_ref == -INFINITY || tmax > m_ref + kRescaleLog2)) {
-          const float alpha = exp2f(m_ref - tmax);
+        // P.V of the previous tile must be done before P is overwritten or O rescaled
+        if (!mbar_wait(bar(B_PVDONE), (j & 1) ^ 1)) return false;
+        // lazy rescale of the running max (identical decision in both CTAs)
+        if (tmax > -INFINITY && (m_ref == -INFINITY || tmax > m_ref + thr_raw)) {
+          const float alpha = ex2_approx((m_ref - tmax) * c2);
           if (j > jfirst) {
-            const int jp = j - 1;
-            if (!mbar_wait(bar(B_PVDONE + (jp & 1)), (jp >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < 256; c += 32) {
@@ -316,37 +392,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           l *= alpha;
           m_ref = tmax;
         }
-        // 5. P = exp2(s - m_ref) in bf16 into the SW64 K-major A tile; its buffer was last read by PV(j-2)
-        if (!mbar_wait(bar(B_PVDONE + sb), (n & 1) ^ 1)) { ok = false; break; }
-        uint32_t pk[16];
-        float lsum = 0.f;
+        // P = 2^((s - m_ref) c2) in bf16 into TMEM (the A operand of P.V)
+        uint32_t pk[NK / 2];
+        if (m_ref > -INFINITY) {
+          const uint64_t cc = f2_pack(c2, c2), off = f2_pack(-m_ref * c2, -m_ref * c2);
+          uint64_t acc2[8];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float e0 = s[2 * c] == -INFINITY ? 0.f : exp2f(s[2 * c] - m_ref);
-          const float e1 = s[2 * c + 1] == -INFINITY ? 0.f : exp2f(s[2 * c + 1] - m_ref);
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-          lsum += __low2float(h2) + __high2float(h2);
-          pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
+          for (int c = 0; c < NK / 2; ++c) {
+            float a0, a1;
+            f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), cc, off), a0, a1);
+            const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+            pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
+            if (c < 8) acc2[c] = f2_pack(e0, e1);
+            else acc2[c & 7] = f2_add(acc2[c & 7], f2_pack(e0, e1));
+          }
+#pragma unroll
+          for (int w2 = 4; w2 > 0; w2 >>= 1)
+#pragma unroll
+            for (int c = 0; c < w2; ++c) acc2[c] = f2_add(acc2[c], acc2[c + w2]);
+          float l0, l1;
+          f2_unpack(acc2[0], l0, l1);
+          l += l0 + l1;
+        } else {
+#pragma unroll
+          for (int c = 0; c < NK / 2; ++c) pk[c] = 0u;
         }
-        l += lsum;
-        uint8_t* prow = smem + OFF_P + sb * P_BYTES + i * 64;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ ((i >> 1) & 3)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        fence_proxy_async_smem();
+        tmem_st32(trow + T_P, pk);
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_PFULL + sb));
+        mbar_arrive(bar(B_PFULL));
+        ++j;
+        return true;
+      };
+      uint32_t bufA[NK], bufB[NK];
+      if (!fetch_send(j, bufA)) { ok = false; break; }
+      for (int32_t xt = w.x; xt < send; xt += 2) {
+        if (!tile(xt, bufA, bufB)) { ok = false; break; }
+        if (xt + 1 < send && !tile(xt + 1, bufB, bufA)) { ok = false; break; }
       }
       if (!ok) break;
       // segment epilogue: O / l for this CTA's 256 columns (+ lse from CTA 0)
       const int jl = j - 1;
-      if (!mbar_wait(bar(B_PVDONE + (jl & 1)), (jl >> 1) & 1)) { ok = false; break; }
+      const float m_log2 = m_ref * c2;
+      if (!mbar_wait(bar(B_PVDONE), jl & 1)) { ok = false; break; }
       tc_fence_after();
       const int64_t t = (int64_t)b * p.tq + k;
       const int32_t nseg = p.slot_base[b + 1] - p.slot_base[b];
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float lse_v = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const float lse_v = l > 0.f ? (m_log2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
       float* po = nullptr;
       if (nseg > 1) {
         const int64_t slot = (int64_t)p.slot_base[b] + (pair - (int)(((int64_t)(ts_b + 1) * npairs - 1) / NT));
@@ -400,9 +494,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // Tile prefix and partial-slot bases of every sequence (one block). Tiles per sequence are
 // counted on the cache length len_b (the last query token sees all of them). A sequence gets
 // one slot per active pair whose tile range meets it.
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_tot, int32_t* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int32_t t = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < (int)(blockDim.x >> 5)) warp_tot[lane] = t;   // inclusive warp prefix
+    if (lane == (int)(blockDim.x >> 5) - 1) *total = t;
+  }
+  __syncthreads();
+  const int32_t r = x - v + (wid > 0 ? warp_tot[wid - 1] : 0);
+  __syncthreads();
+  return r;
+}
+
 __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B, int32_t pairs, int32_t* ts,
                                                    int32_t* sb) {
-  __shared__ int32_t part[256];
+  __shared__ int32_t warp_tot[8];
+  __shared__ int32_t total;
   const int tid = threadIdx.x;
   const int per = (B + 255) / 256;
   const int lo = min(B, tid * per), hi = min(B, lo + per);
@@ -410,22 +531,13 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
     const int64_t len = cu[b + 1] - cu[b];
     return len > 0 ? (int32_t)((len + NK - 1) / NK) : 0;
   };
-  // pass 1: tile prefix
   int32_t acc = 0;
   for (int b = lo; b < hi; ++b) acc += ntiles(b);
-  part[tid] = acc;
-  __syncthreads();
-  if (tid == 0) {
-    int32_t run = 0;
-    for (int q = 0; q < 256; ++q) { const int32_t v = part[q]; part[q] = run; run += v; }
-    ts[B] = run;
-  }
-  __syncthreads();
-  acc = part[tid];
+  acc = block_exclusive_scan(acc, warp_tot, &total);
   for (int b = lo; b < hi; ++b) { ts[b] = acc; acc += ntiles(b); }
+  if (tid == 0) ts[B] = total;
   __syncthreads();
-  // pass 2: pieces per sequence (pairs whose range meets it) and slot prefix
-  const int64_t NT = ts[B];
+  const int64_t NT = total;
   const int64_t npairs = NT < pairs ? NT : pairs;   // every active pair holds >= 1 tile
   auto pair_of = [&](int64_t x) -> int64_t { return ((x + 1) * npairs - 1) / NT; };
   auto nseg = [&](int b) -> int32_t {
@@ -434,17 +546,9 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
   };
   acc = 0;
   for (int b = lo; b < hi; ++b) acc += nseg(b);
-  __syncthreads();
-  part[tid] = acc;
-  __syncthreads();
-  if (tid == 0) {
-    int32_t run = 0;
-    for (int q = 0; q < 256; ++q) { const int32_t v = part[q]; part[q] = run; run += v; }
-    sb[B] = run;
-  }
-  __syncthreads();
-  acc = part[tid];
+  acc = block_exclusive_scan(acc, warp_tot, &total);
   for (int b = lo; b < hi; ++b) { sb[b] = acc; acc += nseg(b); }
+  if (tid == 0) sb[B] = total;
 }
 
 // Exact merge of a sequence's pieces: lse = log sum_s e^{lse_s}, o = sum_s e^{lse_s - lse} o_s.
@@ -453,23 +557,34 @@ template <bool OUT_F32>
 __global__ void __launch_bounds__(128) combine_kernel(const int32_t* sb, int32_t tq, int32_t s_max,
                                                       const float* part_o, const float* part_lse, void* o_lat,
                                                       float* lse) {
+  __shared__ float wts[kMaxPairs + 64];
+  __shared__ float red[32];
   const int64_t t = blockIdx.x;
   const int h = blockIdx.y;
   const int b = (int)(t / tq), k = (int)(t % tq);
-  const int32_t s0 = sb[b], ns = sb[b + 1] - s0;
+  const int32_t s0 = sb[b], ns = min(sb[b + 1] - s0, kMaxPairs + 64);
   if (ns == 1) return;
-  float mx = -INFINITY;
-  for (int s = 0; s < ns; ++s) mx = fmaxf(mx, part_lse[((int64_t)k * s_max + s0 + s) * H + h]);
+  const int64_t row0 = ((int64_t)k * s_max + s0) * H + h;
+  float lmax = -INFINITY;
+  for (int s = threadIdx.x; s < ns; s += 128) {
+    const float v = part_lse[row0 + (int64_t)s * H];
+    wts[s] = v;
+    lmax = fmaxf(lmax, v);
+  }
+  const float mx = block_max(lmax, red);
+  float wpart = 0.f;
+  for (int s = threadIdx.x; s < ns; s += 128) {
+    const float wv = mx > -INFINITY ? __expf(wts[s] - mx) : 0.f;
+    wts[s] = wv;
+    wpart += wv;
+  }
+  const float wsum = block_sum(wpart, red);   // includes a __syncthreads: wts[] is complete
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float wsum = 0.f;
-  if (mx > -INFINITY) {
-    for (int s = 0; s < ns; ++s) {
-      const int64_t row = ((int64_t)k * s_max + s0 + s) * H + h;
-      const float wgt = __expf(part_lse[row] - mx);
-      wsum += wgt;
-      const float4 v = reinterpret_cast<const float4*>(part_o + row * DC)[threadIdx.x];
-      acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
-    }
+#pragma unroll 4
+  for (int s = 0; s < ns; ++s) {
+    const float wgt = wts[s];
+    const float4 v = reinterpret_cast<const float4*>(part_o + (row0 + (int64_t)s * H) * DC)[threadIdx.x];
+    acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
@@ -516,6 +631,7 @@ cudaError_t launch_core(const CoreParams& p, dim3 grid, cudaStream_t st) {
     configured = true;
   }
   latent_core_kernel<OUT_F32><<<grid, kThreads, SMEM_BYTES, st>>>(p);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -538,12 +654,13 @@ cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B
   pairs = pairs < kMaxPairs ? pairs : kMaxPairs;
   pairs = pairs < 1 ? 1 : pairs;
   plan_kernel<<<1, 256, 0, st>>>(cu, (int32_t)B, pairs, c.ts, c.sb);
+  note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CoreParams p;
   memset(&p, 0, sizeof(p));
-  if ((e = make_tmap_bf16(&p.qmap, q_abs, DC, T * H, DC, 64, 128)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16(&p.rmap, q_rope, DR, T * H, DR, 64, 128)) != cudaSuccess) return e;
+  p.q_abs = reinterpret_cast<const __nv_bfloat16*>(q_abs);
+  p.q_rope = reinterpret_cast<const __nv_bfloat16*>(q_rope);
   if ((e = make_tmap_bf16(&p.cmap, cache, ROW, capacity, ROW, 64, NK)) != cudaSuccess) return e;
   p.cu = cu;
   p.tile_start = c.ts;
@@ -564,6 +681,7 @@ cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B
   dim3 cg((unsigned)T, (unsigned)H);
   if (o_f32) combine_kernel<true><<<cg, 128, 0, st>>>(c.sb, tq, c.s_max, c.part_o, c.part_lse, o_lat, lse);
   else combine_kernel<false><<<cg, 128, 0, st>>>(c.sb, tq, c.s_max, c.part_o, c.part_lse, o_lat, lse);
+  note_launch();
   return cudaGetLastError();
 }
 

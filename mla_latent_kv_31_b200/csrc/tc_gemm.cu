@@ -1,6 +1,11 @@
-// tcgen05 GEMM kernel (TMA -> shared memory ring -> tcgen05.mma into TMEM -> epilogue), the
+// tcgen05 GEMM kernel (TMA -> shared-memory ring -> tcgen05.mma into TMEM -> epilogue), the
 // split-K reduce pass, and the host launcher that encodes the TMA tensor maps.
+//
+// The kernel is persistent: each CTA walks output tiles blockIdx.x, +gridDim.x, ... The TMA
+// producer streams k-blocks of consecutive tiles through one ring; the MMA issuer alternates
+// between two TMEM accumulators so the epilogue of one tile overlaps the MMAs of the next.
 #include <cuda_bf16.h>
+#include <math.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -15,6 +20,7 @@ using namespace sm100;
 constexpr int BK = 64;           // k-block: one 128-byte swizzle row of bf16
 constexpr int kThreads = 192;    // warp 0: TMA producer, warp 1: TMEM owner + MMA issuer, warps 2-5: epilogue
 constexpr int kMaxSplits = 64;
+constexpr int kMaxRopePairs = 64;
 
 struct GemmParams {
   CUtensorMap wmap[2];
@@ -22,11 +28,12 @@ struct GemmParams {
   TcEpiSeg seg[2];
   int32_t nseg;
   int32_t splits, kb_total, kb_per_split;
+  int32_t wtiles, ttiles, tiles;   // weight tiles (all segments), token tiles, total tiles
   int64_t T;
   int32_t w_row_z, w_col_z, x_col_z;
   const int64_t* pos;
   int32_t d_r;
-  double rope_base;
+  double theta[kMaxRopePairs];     // RoPE frequencies base^(-2m/d_r)
   float* partial;
   int64_t f_total;
   uint32_t* err;
@@ -47,21 +54,24 @@ __device__ __forceinline__ void store_out(const TcEpiSeg& E, uint32_t* err, int 
   else reinterpret_cast<__nv_bfloat16*>(E.out)[idx] = __float2bfloat16_rn(v);
 }
 
-// RoPE of one element of the pair (2m, 2m+1) holding feature f (segment-local): `own` is x_f,
-// `partner` is x_{f^1}.
+// RoPE of one element of the pair (2m, 2m+1) that holds feature f (segment-local): `own` is x_f,
+// `partner` is x_{f^1}. The angle pos * theta_m is reduced modulo 2 pi in double, then sincosf.
 __device__ __forceinline__ float rope_one(int64_t f, int64_t pos, float own, float partner, int d_r,
-                                          double base) {
-  float c, s;
-  rope_cos_sin(pos, (int)((f % d_r) >> 1), d_r, base, &c, &s);
+                                          const double* theta) {
+  const double a = (double)pos * theta[(f % d_r) >> 1];
+  const double red = a - 6.283185307179586 * rint(a * 0.15915494309189535);
+  float s, c;
+  sincosf((float)red, &s, &c);
   return (f & 1) ? (partner * s + own * c) : (own * c - partner * s);
 }
 
 template <int BN, bool SWAP, bool W_MN, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr uint32_t A_BYTES = 128 * 128;
   constexpr uint32_t B_BYTES = BN * 128;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  constexpr uint32_t TMEM_COLS = BN <= 32 ? 32 : BN;
+  constexpr uint32_t ACC_COLS = BN < 32 ? 32 : BN;     // one accumulator
+  constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;          // double-buffered
   constexpr int W_TILE = SWAP ? 128 : BN;
   constexpr int X_TILE = SWAP ? BN : 128;
   constexpr int CH = BN < 32 ? BN : 32;
@@ -70,24 +80,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);  // full[S], empty[S], done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  // barriers: full[S], empty[S], acc_full[2], acc_empty[2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  auto bar = [&](int i) { return smem_addr(&bars[i]); };
+  const int B_FULL = 0, B_EMPTY = STAGES, B_ACCF = 2 * STAGES, B_ACCE = 2 * STAGES + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int wt = blockIdx.x, s = 0;
-  if (p.nseg > 1 && wt >= p.seg[0].tiles) {
-    s = 1;
-    wt -= p.seg[0].tiles;
-  }
-  const TcEpiSeg& E = p.seg[s];
-  const int z = blockIdx.z / p.splits, split = blockIdx.z % p.splits;
-  const int kb0 = split * p.kb_per_split;
-  const int nkb = min(p.kb_total, kb0 + p.kb_per_split) - kb0;
-  const int64_t f0 = (int64_t)wt * W_TILE;
-  const int64_t t0 = (int64_t)blockIdx.y * X_TILE;
-
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2 * STAGES + 1; ++i) mbar_init(smem_addr(&bars[i]), 1);
+    for (int i = 0; i < 2 * STAGES + 2; ++i) mbar_init(bar(i), 1);
+    mbar_init(bar(B_ACCE), 128);
+    mbar_init(bar(B_ACCE + 1), 128);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -95,117 +98,150 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
-    prefetch_tmap(&p.wmap[s]);
+    prefetch_tmap(&p.wmap[0]);
+    if (p.nseg > 1) prefetch_tmap(&p.wmap[1]);
     prefetch_tmap(&p.xmap);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t done_bar = smem_addr(&bars[2 * STAGES]);
+
+  // tile index -> (segment, weight tile within it, token tile, batch z, split)
+  struct Tile {
+    int s, wt, tt, z, split, kb0, nkb;
+  };
+  auto decode_tile = [&](int idx) {
+    Tile d;
+    d.tt = idx % p.ttiles;
+    int rest = idx / p.ttiles;
+    int wt = rest % p.wtiles;
+    rest /= p.wtiles;
+    d.z = rest / p.splits;
+    d.split = rest % p.splits;
+    d.s = 0;
+    if (p.nseg > 1 && wt >= p.seg[0].tiles) {
+      d.s = 1;
+      wt -= p.seg[0].tiles;
+    }
+    d.wt = wt;
+    d.kb0 = d.split * p.kb_per_split;
+    d.nkb = min(p.kb_total, d.kb0 + p.kb_per_split) - d.kb0;
+    return d;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
-      const CUtensorMap* wm = &p.wmap[s];
-      const CUtensorMap* xm = &p.xmap;
-      int issued = 0;
+      int it = 0, issued = 0;
       bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
-        const int st = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        if (!mbar_wait(smem_addr(&bars[STAGES + st]), ph ^ 1)) {
-          ok = false;
-          break;
-        }
-        const uint32_t full = smem_addr(&bars[st]);
-        mbar_expect_tx(full, STAGE_BYTES);
-        const int k0 = (kb0 + i) * BK;
-        const uint32_t a_dst = smem_addr(sA + st * A_BYTES), b_dst = smem_addr(sB + st * B_BYTES);
-        const uint32_t w_dst = SWAP ? a_dst : b_dst, x_dst = SWAP ? b_dst : a_dst;
-        if (W_MN) {
+      for (int idx = blockIdx.x; ok && idx < p.tiles; idx += gridDim.x) {
+        const Tile d = decode_tile(idx);
+        const CUtensorMap* wm = &p.wmap[d.s];
+        const int64_t f0 = (int64_t)d.wt * W_TILE, t0 = (int64_t)d.tt * X_TILE;
+        for (int i = 0; i < d.nkb; ++i, ++it) {
+          const int st = it % STAGES;
+          if (!mbar_wait(bar(B_EMPTY + st), ((it / STAGES) & 1) ^ 1)) { ok = false; break; }
+          const uint32_t full = bar(B_FULL + st);
+          mbar_expect_tx(full, STAGE_BYTES);
+          const int k0 = (d.kb0 + i) * BK;
+          const uint32_t a_dst = smem_addr(sA + st * A_BYTES), b_dst = smem_addr(sB + st * B_BYTES);
+          const uint32_t w_dst = SWAP ? a_dst : b_dst, x_dst = SWAP ? b_dst : a_dst;
+          if (W_MN) {
 #pragma unroll
-          for (int j = 0; j < W_TILE / 64; ++j)
-            tma_load_2d(w_dst + j * 8192, wm, (int)(f0 + 64 * j) + z * p.w_col_z, k0 + z * p.w_row_z, full);
-        } else {
-          tma_load_2d(w_dst, wm, k0 + z * p.w_col_z, (int)f0 + z * p.w_row_z, full);
+            for (int jb = 0; jb < W_TILE / 64; ++jb)
+              tma_load_2d(w_dst + jb * 8192, wm, (int)(f0 + 64 * jb) + d.z * p.w_col_z, k0 + d.z * p.w_row_z, full);
+          } else {
+            tma_load_2d(w_dst, wm, k0 + d.z * p.w_col_z, (int)f0 + d.z * p.w_row_z, full);
+          }
+          tma_load_2d(x_dst, &p.xmap, k0 + d.z * p.x_col_z, (int)t0, full);
+          issued = it + 1;
         }
-        tma_load_2d(x_dst, xm, k0 + z * p.x_col_z, (int)t0, full);
-        issued = i + 1;
       }
       if (!ok) {
         flag_error(p.err, DEVERR_TIMEOUT);
-        // let the loads already issued land before the CTA can exit
-        for (int i = max(0, issued - STAGES); i < issued; ++i)
-          mbar_wait(smem_addr(&bars[i % STAGES]), (i / STAGES) & 1);
+        for (int i = max(0, issued - STAGES); i < issued; ++i) mbar_wait(bar(B_FULL + i % STAGES), (i / STAGES) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, BN, (SWAP && W_MN) ? 1 : 0, (!SWAP && W_MN) ? 1 : 0);
+      int it = 0, n = 0;
       bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
-        const int st = i % STAGES;
-        if (!mbar_wait(smem_addr(&bars[st]), (i / STAGES) & 1)) {
-          ok = false;
-          break;
-        }
+      for (int idx = blockIdx.x; ok && idx < p.tiles; idx += gridDim.x, ++n) {
+        const Tile d = decode_tile(idx);
+        const int acc = n & 1;
+        if (!mbar_wait(bar(B_ACCE + acc), ((n >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a_base = smem_addr(sA + st * A_BYTES), b_base = smem_addr(sB + st * B_BYTES);
+        const uint32_t dt = tmem + acc * ACC_COLS;
+        for (int i = 0; i < d.nkb; ++i, ++it) {
+          const int st = it % STAGES;
+          if (!mbar_wait(bar(B_FULL + st), (it / STAGES) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_addr(sA + st * A_BYTES), b_base = smem_addr(sB + st * B_BYTES);
 #pragma unroll
-        for (int j = 0; j < BK / 16; ++j) {
-          const uint64_t ad = (SWAP && W_MN) ? sw128_desc(a_base + j * 2048, 8192, 1024)
-                                             : sw128_desc(a_base + j * 32, 0, 1024);
-          const uint64_t bd = (!SWAP && W_MN) ? sw128_desc(b_base + j * 2048, 8192, 1024)
-                                              : sw128_desc(b_base + j * 32, 0, 1024);
-          mma_bf16_ss(tmem, ad, bd, idesc, (i > 0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < BK / 16; ++j) {
+            const uint64_t ad = (SWAP && W_MN) ? sw128_desc(a_base + j * 2048, 8192, 1024)
+                                               : sw128_desc(a_base + j * 32, 0, 1024);
+            const uint64_t bd = (!SWAP && W_MN) ? sw128_desc(b_base + j * 2048, 8192, 1024)
+                                                : sw128_desc(b_base + j * 32, 0, 1024);
+            mma_bf16_ss(dt, ad, bd, idesc, (i > 0 || j > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(B_EMPTY + st));
         }
-        mma_commit(smem_addr(&bars[STAGES + st]));
+        if (!ok) break;
+        mma_commit(bar(B_ACCF + acc));
       }
-      if (ok) {
-        mma_commit(done_bar);
-      } else {
-        flag_error(p.err, DEVERR_TIMEOUT);
-        mbar_arrive(done_bar);
-      }
+      if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
     }
   } else {
     const int q = warp & 3;
     const int r = q * 32 + lane;  // accumulator row = TMEM lane
-    if (!mbar_wait(done_bar, 0)) flag_error(p.err, DEVERR_TIMEOUT);
-    tc_fence_after();
-    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+    int n = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; ok && idx < p.tiles; idx += gridDim.x, ++n) {
+      const Tile d = decode_tile(idx);
+      const TcEpiSeg& E = p.seg[d.s];
+      const int acc = n & 1;
+      if (!mbar_wait(bar(B_ACCF + acc), (n >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t trow = tmem + acc * ACC_COLS + ((uint32_t)(q * 32) << 16);
+      const int64_t f0 = (int64_t)d.wt * W_TILE, t0 = (int64_t)d.tt * X_TILE;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += CH) {
-      uint32_t v[32];
-      if (CH == 32) tmem_ld32(trow + c, v);
-      else tmem_ld16(trow + c, v);
-      tmem_wait_ld();
+      for (int c = 0; c < BN; c += CH) {
+        uint32_t v[32];
+        if (CH == 32) tmem_ld32(trow + c, v);
+        else tmem_ld16(trow + c, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < CH; ++j) {
-        const float x = __uint_as_float(v[j]);
-        int64_t f, t;
-        if (SWAP) { f = f0 + r; t = t0 + c + j; }
-        else { f = f0 + c + j; t = t0 + r; }
-        float partner = 0.f;
-        if (SWAP) partner = __shfl_xor_sync(0xffffffffu, x, 1);
-        else partner = __uint_as_float(v[j ^ 1]);
-        if (f >= E.f_rows || t >= p.T) continue;
-        if (p.splits > 1) {
-          p.partial[((int64_t)split * p.T + t) * p.f_total + E.f_base + f] = x;
-          continue;
-        }
-        float y = x;
-        if (E.rope) {
-          const int64_t ps = p.pos[t];
-          if (ps < 0) {
-            flag_error(p.err, DEVERR_POSITION);
+        for (int j = 0; j < CH; ++j) {
+          const float x = __uint_as_float(v[j]);
+          int64_t f, t;
+          if (SWAP) { f = f0 + r; t = t0 + c + j; }
+          else { f = f0 + c + j; t = t0 + r; }
+          float partner;
+          if (SWAP) partner = __shfl_xor_sync(0xffffffffu, x, 1);
+          else partner = __uint_as_float(v[j ^ 1]);
+          if (f >= E.f_rows || t >= p.T) continue;
+          if (p.splits > 1) {
+            p.partial[((int64_t)d.split * p.T + t) * p.f_total + E.f_base + f] = x;
             continue;
           }
-          y = rope_one(f, ps, x, partner, p.d_r, p.rope_base);
+          float y = x;
+          if (E.rope) {
+            const int64_t ps = p.pos[t];
+            if (ps < 0) {
+              flag_error(p.err, DEVERR_POSITION);
+              continue;
+            }
+            y = rope_one(f, ps, x, partner, p.d_r, p.theta);
+          }
+          store_out(E, p.err, d.z, f, t, y);
         }
-        store_out(E, p.err, z, f, t, y);
       }
+      tc_fence_before();
+      mbar_arrive(bar(B_ACCE + acc));
     }
+    if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
   }
   tc_fence_before();
   __syncthreads();
@@ -222,32 +258,42 @@ struct ReduceParams {
   const float* partial;
   const int64_t* pos;
   int32_t d_r;
-  double rope_base;
+  double theta[kMaxRopePairs];
   uint32_t* err;
 };
 
 // Sums the split-K partials of feature pairs (f, f+1) in split order, then applies the epilogue.
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const ReduceParams p) {
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constant__ ReduceParams p) {
   const int64_t f = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
   const int64_t t = blockIdx.y;
   if (f >= p.f_total) return;
   const int s = (p.nseg > 1 && f >= p.seg[1].f_base) ? 1 : 0;
   const TcEpiSeg& E = p.seg[s];
   const int64_t fl = f - E.f_base;
-  float a = 0.f, b = 0.f;
-  for (int k = 0; k < p.splits; ++k) {
-    const float* src = p.partial + ((int64_t)k * p.T + t) * p.f_total + f;
-    a += src[0];
-    if (fl + 1 < E.f_rows) b += src[1];
+  // eight independent partial sums (loads in flight together), combined in a fixed order
+  float pa[8] = {}, pb[8] = {};
+  const float* src = p.partial + t * p.f_total + f;
+  const int64_t kstride = p.T * p.f_total;
+  for (int k0 = 0; k0 < p.splits; k0 += 8) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (k0 + u < p.splits) {
+        const float2 v = *reinterpret_cast<const float2*>(src + (int64_t)(k0 + u) * kstride);
+        pa[u] += v.x;
+        pb[u] += v.y;
+      }
+    }
   }
+  float a = ((pa[0] + pa[1]) + (pa[2] + pa[3])) + ((pa[4] + pa[5]) + (pa[6] + pa[7]));
+  float b = ((pb[0] + pb[1]) + (pb[2] + pb[3])) + ((pb[4] + pb[5]) + (pb[6] + pb[7]));
   if (E.rope) {
     const int64_t ps = p.pos[t];
     if (ps < 0) {
       flag_error(p.err, DEVERR_POSITION);
       return;
     }
-    const float a2 = rope_one(fl, ps, a, b, p.d_r, p.rope_base);
-    const float b2 = rope_one(fl + 1, ps, b, a, p.d_r, p.rope_base);
+    const float a2 = rope_one(fl, ps, a, b, p.d_r, p.theta);
+    const float b2 = rope_one(fl + 1, ps, b, a, p.d_r, p.theta);
     a = a2;
     b = b2;
   }
@@ -274,8 +320,6 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-// 2-D bf16 tensor map over a row-major [outer, inner] matrix with row stride ld (elements),
-// box {box_inner, box_outer}, 128-byte swizzle, zero fill out of bounds.
 cudaError_t make_tmap_bf16(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, int64_t ld, int box_inner,
                            int box_outer) {
   EncodeTiledFn fn = encode_fn();
@@ -292,8 +336,20 @@ cudaError_t make_tmap_bf16(CUtensorMap* m, const void* ptr, int64_t inner, int64
 
 namespace {
 
+int g_num_sms = 0;
+
+int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_num_sms = n > 0 ? n : 148;
+  }
+  return g_num_sms;
+}
+
 template <int BN, bool SWAP, bool W_MN, int STAGES>
-cudaError_t launch_gemm(const GemmParams& p, dim3 grid, cudaStream_t st) {
+cudaError_t launch_gemm(const GemmParams& p, int ctas_per_sm, cudaStream_t st) {
   constexpr size_t smem = (size_t)STAGES * (128 * 128 + BN * 128) + 1024 + 256;
   static bool configured = false;
   auto kern = gemm_kernel<BN, SWAP, W_MN, STAGES>;
@@ -302,19 +358,25 @@ cudaError_t launch_gemm(const GemmParams& p, dim3 grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
+  int grid = num_sms() * ctas_per_sm;
+  if (grid > p.tiles) grid = p.tiles;
   kern<<<grid, kThreads, smem, st>>>(p);
+  note_launch();
   return cudaGetLastError();
 }
 
 int swap_bn(int64_t T) { return T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128; }
 
-}  // namespace
+// CTA slots of a weight-streaming launch on a 148-SM B200 (two CTAs per SM up to BN = 64). The
+// split decision uses this fixed count so that workspace sizing and launches always agree.
+int swap_slots(int BN) { return BN <= 64 ? 2 * 148 : 148; }
 
-// Split-K factor for a swap-orientation launch of `ctas` CTAs over kb_total k-blocks: enough
-// splits to cover the 148 SMs once; returns (splits, k-blocks per split).
-static void choose_splits(int64_t ctas, int kb_total, int* splits_out, int* kbps_out) {
-  int splits = (int)((148 + ctas - 1) / ctas);
-  splits = splits < kb_total ? splits : kb_total;
+// Split-K factor for a swap-orientation launch of `ctas` output tiles over kb_total k-blocks:
+// as many splits as fit the CTA slots in one wave; returns (splits, k-blocks per split).
+void choose_splits(int64_t ctas, int kb_total, int slots, int* splits_out, int* kbps_out) {
+  int splits = (int)(slots / ctas);
+  const int max_splits = kb_total / 4;   // at least four k-blocks (256 of K) per split
+  splits = splits < max_splits ? splits : max_splits;
   splits = splits < kMaxSplits ? splits : kMaxSplits;
   splits = splits < 1 ? 1 : splits;
   const int kbps = (kb_total + splits - 1) / splits;
@@ -322,18 +384,21 @@ static void choose_splits(int64_t ctas, int kb_total, int* splits_out, int* kbps
   *kbps_out = kbps;
 }
 
+}  // namespace
+
 size_t tc_gemm_partial_bytes(int64_t T, int64_t f_tiles, int64_t f_total, int64_t K, int32_t batch) {
   if (T <= 0 || T > 256 || batch != 1) return 0;
   const int64_t ctas = f_tiles * ((T + swap_bn(T) - 1) / swap_bn(T));
-  if (ctas >= 120) return 0;
+  const int slots = swap_slots(swap_bn(T));
+  if (2 * ctas > slots) return 0;
   int splits, kbps;
-  choose_splits(ctas, (int)(K / BK), &splits, &kbps);
+  choose_splits(ctas, (int)(K / BK), slots, &splits, &kbps);
   return splits > 1 ? (size_t)splits * T * f_total * sizeof(float) : 0;
 }
 
 cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st) {
   if (g.T <= 0) return cudaSuccess;
-  if (g.K % BK != 0 || g.nseg < 1 || g.nseg > 2) return cudaErrorInvalidValue;
+  if (g.K % BK != 0 || g.nseg < 1 || g.nseg > 2 || g.d_r > 2 * kMaxRopePairs) return cudaErrorInvalidValue;
   const bool swap = g.T <= 256;
   if (g.w_mn && !swap) return cudaErrorInvalidValue;
   const int BN = swap ? swap_bn(g.T) : 256;
@@ -361,39 +426,42 @@ cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st) {
   p.splits = 1;
   p.kb_per_split = p.kb_total;
   const int64_t ctas = (int64_t)wtiles * ttiles * g.batch;
-  if (swap && g.batch == 1 && ctas < 120 && g.partial) {
+  if (swap && g.batch == 1 && 2 * ctas <= swap_slots(BN) && g.partial) {
     int splits, kbps;
-    choose_splits(ctas, p.kb_total, &splits, &kbps);
+    choose_splits(ctas, p.kb_total, swap_slots(BN), &splits, &kbps);
     if ((size_t)splits * g.T * f_total * sizeof(float) <= g.partial_bytes && splits > 1) {
       p.splits = splits;
       p.kb_per_split = kbps;
     }
   }
+  p.wtiles = wtiles;
+  p.ttiles = ttiles;
+  p.tiles = wtiles * ttiles * g.batch * p.splits;
   p.T = g.T;
   p.w_row_z = (int32_t)g.w_row_z;
   p.w_col_z = (int32_t)g.w_col_z;
   p.x_col_z = (int32_t)g.x_col_z;
   p.pos = g.pos;
   p.d_r = g.d_r;
-  p.rope_base = g.rope_base;
+  for (int m = 0; m < g.d_r / 2; ++m) p.theta[m] = pow(g.rope_base, -2.0 * m / g.d_r);
   p.partial = g.partial;
   p.f_total = f_total;
   p.err = g.err;
-  dim3 grid((unsigned)wtiles, (unsigned)ttiles, (unsigned)(g.batch * p.splits));
-  if (!swap) e = launch_gemm<256, false, false, 4>(p, grid, st);
+  // weight streaming (swap): 4 stages, two CTAs per SM; large token counts: 128x256 tiles, 4 stages
+  if (!swap) e = launch_gemm<256, false, false, 4>(p, 1, st);
   else if (g.w_mn) {
     switch (BN) {
-      case 16: e = launch_gemm<16, true, true, 8>(p, grid, st); break;
-      case 32: e = launch_gemm<32, true, true, 8>(p, grid, st); break;
-      case 64: e = launch_gemm<64, true, true, 8>(p, grid, st); break;
-      default: e = launch_gemm<128, true, true, 6>(p, grid, st); break;
+      case 16: e = launch_gemm<16, true, true, 4>(p, 2, st); break;
+      case 32: e = launch_gemm<32, true, true, 4>(p, 2, st); break;
+      case 64: e = launch_gemm<64, true, true, 4>(p, 2, st); break;
+      default: e = launch_gemm<128, true, true, 4>(p, 1, st); break;
     }
   } else {
     switch (BN) {
-      case 16: e = launch_gemm<16, true, false, 8>(p, grid, st); break;
-      case 32: e = launch_gemm<32, true, false, 8>(p, grid, st); break;
-      case 64: e = launch_gemm<64, true, false, 8>(p, grid, st); break;
-      default: e = launch_gemm<128, true, false, 6>(p, grid, st); break;
+      case 16: e = launch_gemm<16, true, false, 4>(p, 2, st); break;
+      case 32: e = launch_gemm<32, true, false, 4>(p, 2, st); break;
+      case 64: e = launch_gemm<64, true, false, 4>(p, 2, st); break;
+      default: e = launch_gemm<128, true, false, 4>(p, 1, st); break;
     }
   }
   if (e != cudaSuccess || p.splits == 1) return e;
@@ -408,10 +476,11 @@ cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st) {
   r.partial = g.partial;
   r.pos = g.pos;
   r.d_r = g.d_r;
-  r.rope_base = g.rope_base;
+  memcpy(r.theta, p.theta, sizeof(r.theta));
   r.err = g.err;
   dim3 rg((unsigned)((f_total / 2 + 255) / 256), (unsigned)g.T);
   splitk_reduce_kernel<<<rg, 256, 0, st>>>(r);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
             "mla_sync_status": (c_int, [H, c_void_p]),
             "mla_device_error_bits": (c_uint32, [H]),
             "mla_uses_tensor_cores": (c_int, [H, c_int]),
+            "mla_kernel_launches": (ctypes.c_uint64, []),
             "mla_status_string": (c_char_p, [c_int]),
             "mla_destroy": (None, [H]),
         }
@@ -154,6 +155,10 @@ def mla_device_error_bits(handle) -> int:
 
 def mla_uses_tensor_cores(handle, op: int) -> bool:
     return bool(lib().mla_uses_tensor_cores(handle, op))
+
+
+def mla_kernel_launches() -> int:
+    return lib().mla_kernel_launches()
 
 
 def mla_status_string(status: int) -> str:

@@ -106,7 +106,7 @@ def up_project_head(c_kv, W, dims, i):
     """
     rows = slice(i * dims.d_h, (i + 1) * dims.d_h)
     c_kv = f64(c_kv)
-    return c_kv @ f64(W["w_uk"])[rows].T, c_kv @ f64(W["w_uv"])[rows].T
+    return c_kv @ f64(W["w_uk"][rows]).T, c_kv @ f64(W["w_uv"][rows]).T
 
 
 # ---------------------------------------------------------------------------
