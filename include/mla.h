@@ -54,7 +54,8 @@ typedef enum {
   MLA_ERR_CUDA = 5,          /* a CUDA runtime call failed (the CUDA error is not cleared)       */
   MLA_ERR_TIMEOUT = 6,       /* a device-side bounded wait gave up (kernel returned early)       */
   MLA_ERR_DEVICE_CHECK = 7,  /* a device-side argument check failed (see mla_device_error_bits)  */
-  MLA_ERR_NO_WEIGHTS = 8     /* mla_set_weights() was not called                                  */
+  MLA_ERR_NO_WEIGHTS = 8,    /* mla_set_weights() was not called                                  */
+  MLA_ERR_SCRATCH_LIMIT = 9  /* the call needs more scratch than mla_cache_append_noalloc() holds  */
 } mla_status_t;
 
 typedef enum { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype_t;
@@ -122,6 +123,26 @@ mla_status_t mla_workspace_offset(const mla_handle_t *h, mla_op_t op, int64_t nu
 mla_status_t mla_cache_append(mla_handle_t *h, const void *hidden, const int64_t *positions,
                               const int64_t *slots, int64_t T, void *cache, int64_t capacity,
                               void *ws, size_t ws_bytes, mla_stream_t stream);
+
+/* mla_cache_append for callers that cannot allocate device memory. There is no counterpart on
+ * the pages: it is a convenience of this library. Some callers cannot call cudaMalloc or hand
+ * over a workspace: code running inside a stream capture that forbids allocation, runtimes
+ * that own a fixed memory pool, or plain C callers that have no allocator of their own. This
+ * call takes no workspace and allocates nothing; the split-K scratch it needs lives in one
+ * fixed 4 MiB device array inside the library, which every GPU that loads the library holds
+ * until the process exits.
+ *   Same arguments, layouts and results as mla_cache_append, minus the workspace.
+ *   Returns MLA_ERR_SCRATCH_LIMIT, before any launch, when the call would need more than
+ *   4 MiB of scratch (at the DeepSeek-V3 sizes in bf16: 65 <= T <= 256 tokens; smaller and
+ *   larger T need 4 MiB or less). MLA_ERR_NO_WEIGHTS if mla_set_weights() was not called.
+ *   The first call on a device looks up the device address of the array (no allocation); make
+ *   that first call outside any stream capture.
+ *   All calls share the one array and it keeps the last call's contents; nothing in it needs
+ *   to start at zero, but calls that overlap on the GPU (different streams, no ordering)
+ *   race on it. */
+mla_status_t mla_cache_append_noalloc(mla_handle_t *h, const void *hidden, const int64_t *positions,
+                                      const int64_t *slots, int64_t T, void *cache, int64_t capacity,
+                                      mla_stream_t stream);
 
 /* Decode step, absorbed form (section 一(一)2 【思考】 with the decoupled RoPE of section 3):
  * c^Q = W^DQ h; q^C = W^UQ c^Q; q^R = RoPE(W^QR c^Q); q~_i = W_i^UK^T q^C_i;

@@ -223,6 +223,8 @@ const char* mla_status_string(mla_status_t s) {
     case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT: a bounded device-side wait gave up";
     case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK: device-side argument check failed";
     case MLA_ERR_NO_WEIGHTS: return "MLA_ERR_NO_WEIGHTS: mla_set_weights() not called";
+    case MLA_ERR_SCRATCH_LIMIT:
+      return "MLA_ERR_SCRATCH_LIMIT: the call needs more than the 4 MiB fixed scratch of mla_cache_append_noalloc";
   }
   return "MLA_ERR_UNKNOWN";
 }
@@ -466,3 +468,55 @@ void mla_destroy(mla_handle_t* h) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// mla_cache_append_noalloc: the cache append for callers that cannot allocate. Its split-K
+// scratch is this fixed device array; host code never touches the array's name as an address
+// but asks the runtime for the device address once per device.
+// ---------------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on `device` (which must be current), looked up once.
+mla_status_t noalloc_scratch(int device, void** out) {
+  if (device < 0 || device >= kMaxDevices) return MLA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[device]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MLA_ERR_CUDA;
+    g_noalloc_addr[device] = p;
+  }
+  *out = g_noalloc_addr[device];
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" mla_status_t mla_cache_append_noalloc(mla_handle_t* h, const void* hidden, const int64_t* positions,
+                                                 const int64_t* slots, int64_t T, void* cache, int64_t capacity,
+                                                 mla_stream_t stream) {
+  if (!h || !hidden || !positions || !slots || !cache || T <= 0 || capacity <= 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(cache) || !aligned16(positions) || !aligned16(slots))
+    return MLA_ERR_ALIGNMENT;
+  // mla_set_weights() already allocated the error word; this call allocates nothing itself.
+  if (!h->has_weights || !h->d_err) return MLA_ERR_NO_WEIGHTS;
+  Layout L = layout(h, MLA_OP_CACHE_APPEND, 0, 1, T);
+  if (L.total > kNoAllocScratchBytes) return MLA_ERR_SCRATCH_LIMIT;
+  MLA_TRY(cudaSetDevice(h->device));
+  void* scratch = nullptr;
+  mla_status_t s = noalloc_scratch(h->device, &scratch);
+  if (s != MLA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (tc_dims(h) && mla::tc_available(MLA_OP_CACHE_APPEND))
+    return cuda_status(mla::tc_cache_append(h->dims, h->w, hidden, positions, slots, T, cache, capacity,
+                                            (char*)scratch + L.tc_off, L.total - L.tc_off, h->d_err, st));
+  return simt_cache_rows(h, hidden, positions, slots, T, cache, capacity, st);
+}

@@ -16,7 +16,8 @@ MLA_BF16, MLA_FP32 = 0, 1
 OP_CACHE_APPEND, OP_DECODE, OP_PREFILL, OP_ATTN_DECODE_LATENT = 0, 1, 2, 3
 BUF_CQ, BUF_QC, BUF_QR, BUF_QABS, BUF_OLAT, BUF_O, BUF_KC, BUF_VC, BUF_LSE = range(9)
 STATUS_NAMES = ["MLA_OK", "MLA_ERR_INVALID_ARG", "MLA_ERR_ALIGNMENT", "MLA_ERR_UNSUPPORTED", "MLA_ERR_WORKSPACE",
-                "MLA_ERR_CUDA", "MLA_ERR_TIMEOUT", "MLA_ERR_DEVICE_CHECK", "MLA_ERR_NO_WEIGHTS"]
+                "MLA_ERR_CUDA", "MLA_ERR_TIMEOUT", "MLA_ERR_DEVICE_CHECK", "MLA_ERR_NO_WEIGHTS",
+                "MLA_ERR_SCRATCH_LIMIT"]
 WEIGHT_NAMES = ["w_dq", "w_uq", "w_qr", "w_dkv", "w_kr", "w_uk", "w_uv", "w_o"]
 
 
@@ -53,6 +54,8 @@ def lib() -> ctypes.CDLL:
             "mla_workspace_offset": (c_int, [H, c_int, c_int64, c_int32, c_int64, c_int, POINTER(c_size_t)]),
             "mla_cache_append": (c_int, [H, c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_int64, c_void_p,
                                          c_size_t, c_void_p]),
+            "mla_cache_append_noalloc": (c_int, [H, c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_int64,
+                                                 c_void_p]),
             "mla_decode": (c_int, [H, c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
                                    c_size_t, c_void_p]),
             "mla_prefill": (c_int, [H, c_void_p, c_int64, c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p,
@@ -125,6 +128,12 @@ def mla_cache_append(handle, hidden, positions, slots, T, cache, capacity, ws=No
                      device=0):
     _check(lib().mla_cache_append(handle, _ptr(hidden), _ptr(positions), _ptr(slots), T, _ptr(cache), capacity,
                                   _ptr(ws), ws_bytes, _stream(stream, device)), "mla_cache_append")
+
+
+def mla_cache_append_noalloc(handle, hidden, positions, slots, T, cache, capacity, stream=None, device=0):
+    """mla_cache_append without a workspace: its scratch is a fixed 4 MiB array in the library."""
+    _check(lib().mla_cache_append_noalloc(handle, _ptr(hidden), _ptr(positions), _ptr(slots), T, _ptr(cache),
+                                          capacity, _stream(stream, device)), "mla_cache_append_noalloc")
 
 
 def mla_decode(handle, h_q, B, Tq, cu_seqlens, cache, capacity, u_out, ws, ws_bytes, stream=None, device=0):
