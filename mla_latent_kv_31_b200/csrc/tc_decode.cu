@@ -33,6 +33,7 @@ using namespace sm100;
 constexpr int H = 128, DC = 512, DR = 64, ROW = DC + DR;
 constexpr int NK = 64;                       // keys per tile (the N of QK^T, the K of P.V)
 constexpr int STAGES = 4;
+constexpr int PREFETCH = 8;                  // tiles pulled into L2 ahead of the shared-memory ring
 constexpr int kThreads = 192;
 constexpr int kMaxPairs = 74;
 constexpr float kRescaleLog2 = 8.f;          // lazy rescale: keep the running max until it grows by 2^8
@@ -180,6 +181,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int j = 0, issued = 0;
       bool ok = true;
+      // L2 prefetch cursor, PREFETCH tiles ahead of the loads
+      TileCursor pf;
+      pf.init(p.tile_start, p.B, t_begin, t_end);
+      auto prefetch_next = [&]() {
+        if (!pf.valid()) return;
+        const int pb = pf.w.b;
+        const int32_t row0 = (int32_t)p.cu[pb] + (pf.xt - p.tile_start[pb]) * NK;
+        for (int c = 0; c < 4; ++c) tma_prefetch_l2_2d(&p.cmap, 256 * (int)r + 64 * c, row0);
+        if (r == 0) tma_prefetch_l2_2d(&p.cmap, DC, row0);
+        pf.advance();
+      };
+      for (int q = 0; q < PREFETCH; ++q) prefetch_next();
       for (; ok && w.valid(); w.next()) {
         const int b = w.b;
         const int32_t ts_b = p.tile_start[b];
@@ -194,6 +207,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tma_load_2d(dst + c * KV_BOX, &p.cmap, 256 * (int)r + 64 * c, row0, bar(B_FULL + st));
           if (r == 0) tma_load_2d(dst + 4 * KV_BOX, &p.cmap, DC, row0, bar(B_FULL + st));
           issued = j + 1;
+          prefetch_next();
         }
       }
       if (!ok) {
@@ -249,11 +263,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (did) {
           stall_since = 0;
-        } else if (stall_since == 0) {
-          stall_since = globaltimer();
-        } else if (globaltimer() - stall_since > kWaitTimeoutNs) {
-          ok = false;
-          break;
+        } else {
+          // back off so this polling warp leaves the issue slots of its sub-partition to the
+          // softmax warp that shares it
+          __nanosleep(40);
+          if (stall_since == 0) {
+            stall_since = globaltimer();
+          } else if (globaltimer() - stall_since > kWaitTimeoutNs) {
+            ok = false;
+            break;
+          }
         }
       }
       if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
@@ -267,11 +286,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t xfree_peer = map_peer(bar(B_XFREE), peer);
     const float c2 = p.scale_log2;                   // raw score -> log2 units
     const float thr_raw = kRescaleLog2 / c2;
+    // waits of the softmax warps are warp-uniform: a timeout on any lane fails the whole warp, so
+    // no lane can be left behind at a .sync.aligned tcgen05 instruction
+    auto wait_u = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(b, par)) != 0; };
+    auto wait_uc = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait_cluster(b, par)) != 0; };
     // This CTA's partial scores of tile jj: TMEM -> registers; then sent to the peer with st.async
     // (chunk-major layout: element c of head i at ((c / 4) * 128 + i) * 16 + (c % 4) * 4), each store
     // counting its bytes on the peer's x_full barrier.
     auto fetch_send = [&](int jj, uint32_t(&own)[NK]) -> bool {
-      if (!mbar_wait(bar(B_SFULL), jj & 1)) return false;
+      if (!wait_u(bar(B_SFULL), jj & 1)) return false;
       tc_fence_after();
       tmem_ld32(trow + T_S, own);
       tmem_ld32(trow + T_S + 32, own + 32);
@@ -279,7 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_SEMPTY));
       const int xb = jj & 1;
-      if (!mbar_wait_cluster(bar(B_XFREE + xb), ((jj >> 1) & 1) ^ 1)) return false;
+      if (!wait_uc(bar(B_XFREE + xb), ((jj >> 1) & 1) ^ 1)) return false;
       const uint32_t dst = xpeer + xb * X_BYTES, xbar = xfull_peer + 8 * xb;
 #pragma unroll
       for (int c = 0; c < NK / 4; ++c)
@@ -299,7 +322,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // q~ half (and q^R on CTA 0) of this token and head -> TMEM, once the last piece's QK^T is done
       {
         const int64_t t = (int64_t)b * p.tq + k;
-        if (!mbar_wait(bar(B_QEMPTY), (gq & 1) ^ 1)) { ok = false; break; }
+        if (!wait_u(bar(B_QEMPTY), (gq & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
         const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (t * H + i) * DC + 256 * r);
 #pragma unroll 1
@@ -332,7 +355,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const bool more = xt + 1 < send;
         if (more && !fetch_send(j + 1, nxt)) return false;
         const int xb = j & 1;
-        if (!mbar_wait_cluster(bar(B_XFULL + xb), (j >> 1) & 1)) return false;
+        if (!wait_uc(bar(B_XFULL + xb), (j >> 1) & 1)) return false;
         const float4* xr = reinterpret_cast<const float4*>(smem + OFF_X + xb * X_BYTES) + i;
         float s[NK];
 #pragma unroll
@@ -372,7 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
         }
         // P.V of the previous tile must be done before P is overwritten or O rescaled
-        if (!mbar_wait(bar(B_PVDONE), (j & 1) ^ 1)) return false;
+        if (!wait_u(bar(B_PVDONE), (j & 1) ^ 1)) return false;
         // lazy rescale of the running max (identical decision in both CTAs)
         if (tmax > -INFINITY && (m_ref == -INFINITY || tmax > m_ref + thr_raw)) {
           const float alpha = ex2_approx((m_ref - tmax) * c2);
@@ -435,7 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // segment epilogue: O / l for this CTA's 256 columns (+ lse from CTA 0)
       const int jl = j - 1;
       const float m_log2 = m_ref * c2;
-      if (!mbar_wait(bar(B_PVDONE), jl & 1)) { ok = false; break; }
+      if (!wait_u(bar(B_PVDONE), jl & 1)) { ok = false; break; }
       tc_fence_after();
       const int64_t t = (int64_t)b * p.tq + k;
       const int32_t nseg = p.slot_base[b + 1] - p.slot_base[b];
