@@ -6,15 +6,19 @@
 //   s_j = (q~_t,i . c_j + q^R_t,i . k^R_j) / sqrt(d_h + d_h^R),  j <= pos_t,
 //   o^lat_t,i = sum_j softmax(s)_j c_j,   lse_t,i = log sum_j exp(s_j).
 //
-// Work split. Each sequence's cache rows form tiles of 32 keys; all tiles of all sequences are
+// Work split. Each sequence's cache rows form tiles of 64 keys; all tiles of all sequences are
 // cut into equal contiguous ranges, one per CTA pair (a 2-CTA cluster); a pair whose range
 // crosses a sequence boundary emits one partial result per sequence piece, and a final pass
 // merges the pieces of a sequence exactly (log-sum-exp). Within a pair, CTA r owns latent
-// columns [256 r, 256 r + 256): it streams only that half of every cache row (CTA 0 also the
-// 64 k^R columns), computes the partial score over its columns, swaps the 128 x 32 fp32
-// partial with its peer through distributed shared memory, and then both run the same
-// softmax and accumulate P . c into their own 256 TMEM columns of O. The 128 heads form the
-// MMA M dimension; one TMA-loaded cache tile is read K-major by QK^T and MN-major by P.V.
+// columns [256 r, 256 r + 256) and k^R columns [32 r, 32 r + 32): it streams only those 288
+// columns of every cache row, computes the partial score over them, swaps the 128 x 64 fp32
+// partial with its peer through distributed shared memory, and then both run the same softmax
+// and accumulate P . c into their own 256 TMEM columns of O. The 128 heads form the MMA M
+// dimension; one TMA-loaded cache tile is read K-major by QK^T and MN-major by P.V.
+//
+// Pipelining. Scores are double-buffered in TMEM and P is double-buffered in shared memory, so
+// QK^T of tile j + 1 runs while the softmax works on tile j, and the softmax of tile j + 1 does
+// not wait for P.V of tile j (only a rescale of O does, which the lazy running max makes rare).
 //
 // Roles per CTA (192 threads): warps 0-3 softmax/epilogue (thread i = head i = TMEM lane i),
 // warp 4 TMA producer, warp 5 TMEM owner + MMA issuer. Every wait is bounded.
@@ -33,34 +37,40 @@ using namespace sm100;
 constexpr int H = 128, DC = 512, DR = 64, ROW = DC + DR;
 constexpr int NK = 64;                       // keys per tile (the N of QK^T, the K of P.V)
 constexpr int STAGES = 4;
-constexpr int PREFETCH = 8;                  // tiles pulled into L2 ahead of the shared-memory ring
 constexpr int kThreads = 192;
 constexpr int kMaxPairs = 74;
 constexpr float kRescaleLog2 = 8.f;          // lazy rescale: keep the running max until it grows by 2^8
 
-constexpr uint32_t KV_BOX = NK * 128;        // [64 keys x 64 cols] bf16, SW128: 8 KB
-constexpr uint32_t STAGE_BYTES = 5 * KV_BOX; // 4 latent boxes + (CTA 0) the k^R box
+constexpr uint32_t KV_BOX = NK * 128;        // [64 keys x 64 latent cols] bf16, 128-byte swizzle: 8 KB
+constexpr uint32_t R_BOX = NK * 64;          // [64 keys x 32 k^R cols] bf16, 64-byte swizzle: 4 KB
+constexpr uint32_t STAGE_BYTES = 4 * KV_BOX + R_BOX;   // 36 KB
 constexpr uint32_t X_BYTES = H * NK * 4;     // [128 x 64] fp32 partial scores from the peer: 32 KB
+constexpr uint32_t P_BYTES = H * NK * 2;     // [128 x 64] bf16 probabilities, K-major, 128-byte swizzle
+constexpr uint32_t QR_BYTES = H * 32 * 2;    // [128 x 32] bf16 q^R half, K-major, 64-byte swizzle
 constexpr uint32_t OFF_KV = 0;
 constexpr uint32_t OFF_X = OFF_KV + STAGES * STAGE_BYTES;
-constexpr uint32_t OFF_BAR = OFF_X + 2 * X_BYTES;
-constexpr int NBAR = 2 * STAGES + 12;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-// TMEM columns: O half [0, 256); q~ half + (CTA 0) q^R [256, 416) as bf16 pairs (the A operand of
-// QK^T); S [416, 480); P [480, 512) as bf16 pairs (the A operand of P.V).
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t T_Q = 256, T_S = 416, T_P = T_S + NK;
-static_assert(T_P + NK / 2 <= TMEM_COLS, "TMEM budget");
+constexpr uint32_t OFF_P = OFF_X + X_BYTES;
+constexpr uint32_t OFF_QR = OFF_P + 2 * P_BYTES;
+constexpr uint32_t OFF_BAR = OFF_QR + QR_BYTES;
+static_assert(STAGE_BYTES % 1024 == 0 && OFF_P % 1024 == 0 && OFF_QR % 1024 == 0, "swizzle atom alignment");
 
 // barrier indices
-constexpr int B_FULL = 0, B_EMPTY = STAGES, B_SFULL = 2 * STAGES, B_SEMPTY = B_SFULL + 1, B_PFULL = B_SEMPTY + 1,
-              B_PVDONE = B_PFULL + 1, B_XFULL = B_PVDONE + 1, B_XFREE = B_XFULL + 2, B_QFULL = B_XFREE + 2,
+constexpr int B_FULL = 0, B_EMPTY = STAGES, B_SFULL = 2 * STAGES, B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2,
+              B_PVDONE = B_PFULL + 2, B_XFULL = B_PVDONE + 2, B_XFREE = B_XFULL + 1, B_QFULL = B_XFREE + 1,
               B_QEMPTY = B_QFULL + 1, B_OFREE = B_QEMPTY + 1;
-static_assert(B_OFREE + 1 <= NBAR, "barrier count");
+constexpr int NBAR = B_OFREE + 1;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// TMEM columns: O half [0, 256); q~ half as bf16 pairs [256, 384) (the A operand of QK^T);
+// two score buffers S0 [384, 448), S1 [448, 512).
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t T_Q = 256, T_S = 384;
+static_assert(T_S + 2 * NK <= TMEM_COLS, "TMEM budget");
 
 struct CoreParams {
-  CUtensorMap cmap;   // cache as [capacity, ROW], box {64, NK}
+  CUtensorMap cmap;   // cache as [capacity, ROW], box {64, NK}, 128-byte swizzle (latent columns)
+  CUtensorMap rmap;   // cache as [capacity, ROW], box {32, NK}, 64-byte swizzle (k^R columns)
   const __nv_bfloat16* q_abs;   // [T][H][DC]
   const __nv_bfloat16* q_rope;  // [T][H][DR]
   const int64_t* cu;
@@ -150,24 +160,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int64_t npairs = NT < p.pairs ? NT : p.pairs;
   const int32_t t_begin = pair < npairs ? range_start(pair, NT, npairs) : 0;
   const int32_t t_end = pair < npairs ? range_start(pair + 1, NT, npairs) : 0;
-  const int nkc = r == 0 ? 5 : 4;                    // 64-column K chunks of this CTA's score half
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
-      const bool many = i == B_SEMPTY || i == B_PFULL || i == B_XFREE || i == B_XFREE + 1 || i == B_OFREE ||
-                        i == B_QFULL;
+      const bool many = (i >= B_SEMPTY && i < B_SEMPTY + 2) || (i >= B_PFULL && i < B_PFULL + 2) || i == B_XFREE ||
+                        i == B_OFREE || i == B_QFULL;
       mbar_init(bar(i), many ? 128 : 1);
     }
-    // the exchange buffers' first phase: one arrival plus the bytes the peer's st.async will bring
+    // the exchange buffer's first phase: one arrival plus the bytes the peer's st.async will bring
     mbar_expect_tx(bar(B_XFULL), X_BYTES);
-    mbar_expect_tx(bar(B_XFULL + 1), X_BYTES);
     fence_mbar_init();
   }
   if (warp == 5) {
     tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
-  if (threadIdx.x == 0) prefetch_tmap(&p.cmap);
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&p.cmap);
+    prefetch_tmap(&p.rmap);
+  }
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
@@ -181,18 +192,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int j = 0, issued = 0;
       bool ok = true;
-      // L2 prefetch cursor, PREFETCH tiles ahead of the loads
-      TileCursor pf;
-      pf.init(p.tile_start, p.B, t_begin, t_end);
-      auto prefetch_next = [&]() {
-        if (!pf.valid()) return;
-        const int pb = pf.w.b;
-        const int32_t row0 = (int32_t)p.cu[pb] + (pf.xt - p.tile_start[pb]) * NK;
-        for (int c = 0; c < 4; ++c) tma_prefetch_l2_2d(&p.cmap, 256 * (int)r + 64 * c, row0);
-        if (r == 0) tma_prefetch_l2_2d(&p.cmap, DC, row0);
-        pf.advance();
-      };
-      for (int q = 0; q < PREFETCH; ++q) prefetch_next();
+      const int xr = DC + 32 * (int)r;               // this CTA's k^R columns
       for (; ok && w.valid(); w.next()) {
         const int b = w.b;
         const int32_t ts_b = p.tile_start[b];
@@ -200,14 +200,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int32_t xt = w.x; xt < w.seg_end(); ++xt, ++j) {
           const int st = j % STAGES;
           if (!mbar_wait(bar(B_EMPTY + st), ((j / STAGES) & 1) ^ 1)) { ok = false; break; }
-          mbar_expect_tx(bar(B_FULL + st), nkc * KV_BOX);
+          mbar_expect_tx(bar(B_FULL + st), STAGE_BYTES);
           const int32_t row0 = row_base + (xt - ts_b) * NK;
           const uint32_t dst = sbase + OFF_KV + st * STAGE_BYTES;
           for (int c = 0; c < 4; ++c)
             tma_load_2d(dst + c * KV_BOX, &p.cmap, 256 * (int)r + 64 * c, row0, bar(B_FULL + st));
-          if (r == 0) tma_load_2d(dst + 4 * KV_BOX, &p.cmap, DC, row0, bar(B_FULL + st));
+          tma_load_2d(dst + 4 * KV_BOX, &p.rmap, xr, row0, bar(B_FULL + st));
           issued = j + 1;
-          prefetch_next();
         }
       }
       if (!ok) {
@@ -218,46 +217,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
     // Greedy: P.V for the oldest tile whose P is ready, else QK^T of the next tile once its cache
-    // tile has landed and the softmax has taken the previous scores out of TMEM.
+    // tile has landed and its score buffer has been read out by the softmax. QK^T goes out in two
+    // halves of 9 MMAs, so that a P.V that becomes ready meanwhile does not wait for all of it.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, NK, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
+      const uint32_t qr = sbase + OFF_QR;
       TileCursor cq, cp;
       cq.init(p.tile_start, p.B, t_begin, t_end);
       cp.init(p.tile_start, p.B, t_begin, t_end);
       uint64_t stall_since = 0;
       bool ok = true;
+      int qk_half = 0;                               // halves of QK^T(cq.j) issued so far
       while (cp.valid()) {
         bool did = false;
-        if (cp.j < cq.j && mbar_test(bar(B_PFULL), cp.j & 1) &&
+        if (cp.j < cq.j && mbar_test(bar(B_PFULL + (cp.j & 1)), (cp.j >> 1) & 1) &&
             (!cp.first() || mbar_test(bar(B_OFREE), (cp.g & 1) ^ 1))) {
           tc_fence_after();
-          const int st = cp.j % STAGES;
+          const int st = cp.j % STAGES, pb = cp.j & 1;
           const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
+          const uint32_t pa = sbase + OFF_P + pb * P_BYTES;
           const bool first = cp.first();
 #pragma unroll
           for (int kk = 0; kk < NK / 16; ++kk)
-            mma_bf16_ts(tmem, tmem + T_P + 8 * kk, sw128_desc(kv + kk * 2048, KV_BOX, 1024), idesc_pv,
+            mma_bf16_ss(tmem, sw128_desc(pa + kk * 32, 0, 1024), sw128_desc(kv + kk * 2048, KV_BOX, 1024), idesc_pv,
                         (first && kk == 0) ? 0u : 1u);
-          mma_commit(bar(B_PVDONE));
+          mma_commit(bar(B_PVDONE + pb));
           mma_commit(bar(B_EMPTY + st));
           cp.advance();
           did = true;
         }
         if (!did && cq.valid()) {
-          const int st = cq.j % STAGES;
-          if (mbar_test(bar(B_FULL + st), (cq.j / STAGES) & 1) && mbar_test(bar(B_SEMPTY), (cq.j & 1) ^ 1) &&
-              (!cq.first() || mbar_test(bar(B_QFULL), cq.g & 1))) {
-            tc_fence_after();
+          const int st = cq.j % STAGES, sb = cq.j & 1;
+          if (qk_half == 1 ||
+              (mbar_test(bar(B_FULL + st), (cq.j / STAGES) & 1) && mbar_test(bar(B_SEMPTY + sb), ((cq.j >> 1) & 1) ^ 1) &&
+               (!cq.first() || mbar_test(bar(B_QFULL), cq.g & 1)))) {
+            if (qk_half == 0) tc_fence_after();
             const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
-            for (int kc = 0; kc < nkc; ++kc)
+            const uint32_t d = tmem + T_S + NK * sb;
+            // MMA m < 16: latent chunk m / 4, K step m % 4 (A from TMEM); m = 16, 17: the k^R half
+            // (A from shared memory)
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(tmem + T_S, tmem + T_Q + 32 * kc + 8 * kk, sw128_desc(kv + kc * KV_BOX + kk * 32, 0, 1024),
-                            idesc_qk, (kc | kk) ? 1u : 0u);
-            mma_commit(bar(B_SFULL));
-            if (cq.last()) mma_commit(bar(B_QEMPTY));
-            cq.advance();
+            for (int mm = 0; mm < 9; ++mm) {
+              const int m = 9 * qk_half + mm;
+              if (m < 16)
+                mma_bf16_ts(d, tmem + T_Q + 8 * m, sw128_desc(kv + (m >> 2) * KV_BOX + (m & 3) * 32, 0, 1024), idesc_qk,
+                            m ? 1u : 0u);
+              else
+                mma_bf16_ss(d, sw64_desc(qr + (m - 16) * 32, 512), sw64_desc(kv + 4 * KV_BOX + (m - 16) * 32, 512),
+                            idesc_qk, 1u);
+            }
+            if (qk_half == 1) {
+              mma_commit(bar(B_SFULL + sb));
+              if (cq.last()) mma_commit(bar(B_QEMPTY));
+              cq.advance();
+            }
+            qk_half ^= 1;
             did = true;
           }
         }
@@ -290,27 +305,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // no lane can be left behind at a .sync.aligned tcgen05 instruction
     auto wait_u = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(b, par)) != 0; };
     auto wait_uc = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait_cluster(b, par)) != 0; };
-    // This CTA's partial scores of tile jj: TMEM -> registers; then sent to the peer with st.async
+    int gq = 0, j = 0;
+    // q~ half -> TMEM and q^R half -> shared memory (64-byte swizzle) for the piece of sequence bq,
+    // once the previous piece's last QK^T is done with them.
+    auto load_q = [&](int bq) -> bool {
+      const int64_t t = (int64_t)bq * p.tq + k;
+      if (!wait_u(bar(B_QEMPTY), (gq & 1) ^ 1)) return false;
+      tc_fence_after();
+      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (t * H + i) * DC + 256 * r);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint4 u = __ldg(src + 8 * c + e);
+          v[4 * e] = u.x; v[4 * e + 1] = u.y; v[4 * e + 2] = u.z; v[4 * e + 3] = u.w;
+        }
+        tmem_st32(trow + T_Q + 32 * c, v);
+      }
+      const uint4* rsrc = reinterpret_cast<const uint4*>(p.q_rope + (t * H + i) * DR + 32 * r);
+      uint8_t* qrow = smem + OFF_QR + i * 64;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(qrow + ((c ^ ((i >> 1) & 3)) << 4)) = __ldg(rsrc + c);
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(B_QFULL));
+      ++gq;
+      return true;
+    };
+    // This CTA's partial scores of tile jj: TMEM -> registers, then sent to the peer with st.async
     // (chunk-major layout: element c of head i at ((c / 4) * 128 + i) * 16 + (c % 4) * 4), each store
     // counting its bytes on the peer's x_full barrier.
     auto fetch_send = [&](int jj, uint32_t(&own)[NK]) -> bool {
-      if (!wait_u(bar(B_SFULL), jj & 1)) return false;
+      const int sb = jj & 1;
+      if (!wait_u(bar(B_SFULL + sb), (jj >> 1) & 1)) return false;
       tc_fence_after();
-      tmem_ld32(trow + T_S, own);
-      tmem_ld32(trow + T_S + 32, own + 32);
+      tmem_ld32(trow + T_S + NK * sb, own);
+      tmem_ld32(trow + T_S + NK * sb + 32, own + 32);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(B_SEMPTY));
-      const int xb = jj & 1;
-      if (!wait_uc(bar(B_XFREE + xb), ((jj >> 1) & 1) ^ 1)) return false;
-      const uint32_t dst = xpeer + xb * X_BYTES, xbar = xfull_peer + 8 * xb;
+      mbar_arrive(bar(B_SEMPTY + sb));
+      // the peer has read the previous tile out of its exchange buffer
+      if (!wait_uc(bar(B_XFREE), (jj & 1) ^ 1)) return false;
 #pragma unroll
       for (int c = 0; c < NK / 4; ++c)
-        st_async_peer_v4(dst + c * 2048, own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3], xbar);
+        st_async_peer_v4(xpeer + c * 2048, own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3], xfull_peer);
       return true;
     };
-    int gq = 0, j = 0;
-    bool ok = true;
+    uint32_t cur[NK];
+    bool ok = !w.valid() || load_q(w.b);
     for (; ok && w.valid(); w.next()) {
       const int b = w.b;
       const int64_t len = p.cu[b + 1] - p.cu[b];
@@ -319,56 +363,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int32_t send = w.seg_end();
       float m_ref = -INFINITY, l = 0.f;              // running max in raw score units
       const int jfirst = j;
-      // q~ half (and q^R on CTA 0) of this token and head -> TMEM, once the last piece's QK^T is done
-      {
-        const int64_t t = (int64_t)b * p.tq + k;
-        if (!wait_u(bar(B_QEMPTY), (gq & 1) ^ 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (t * H + i) * DC + 256 * r);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint4 u = __ldg(src + 8 * c + e);
-            v[4 * e] = u.x; v[4 * e + 1] = u.y; v[4 * e + 2] = u.z; v[4 * e + 3] = u.w;
-          }
-          tmem_st32(trow + T_Q + 32 * c, v);
-        }
-        if (r == 0) {
-          const uint4* rsrc = reinterpret_cast<const uint4*>(p.q_rope + (t * H + i) * DR);
-          uint32_t v[32];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint4 u = __ldg(rsrc + e);
-            v[4 * e] = u.x; v[4 * e + 1] = u.y; v[4 * e + 2] = u.z; v[4 * e + 3] = u.w;
-          }
-          tmem_st32(trow + T_Q + 128, v);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(B_QFULL));
-        ++gq;
-      }
-      // One tile: cur holds this CTA's partial scores of tile j; the next tile's go to nxt.
-      auto tile = [&](int32_t xt, uint32_t(&cur)[NK], uint32_t(&nxt)[NK]) -> bool {
-        const bool more = xt + 1 < send;
-        if (more && !fetch_send(j + 1, nxt)) return false;
-        const int xb = j & 1;
-        if (!wait_uc(bar(B_XFULL + xb), (j >> 1) & 1)) return false;
-        const float4* xr = reinterpret_cast<const float4*>(smem + OFF_X + xb * X_BYTES) + i;
+      if (!fetch_send(j, cur)) { ok = false; break; }
+      for (int32_t xt = w.x; xt < send; ++xt) {
+        // full scores of tile j: this CTA's partial plus the peer's
+        if (!wait_uc(bar(B_XFULL), j & 1)) { ok = false; break; }
+        const float4* xrd = reinterpret_cast<const float4*>(smem + OFF_X) + i;
         float s[NK];
 #pragma unroll
         for (int c = 0; c < NK / 4; ++c) {
-          const float4 q = xr[c * 128];
+          const float4 q = xrd[c * 128];
           f2_unpack(f2_add(f2_pack(__uint_as_float(cur[4 * c]), __uint_as_float(cur[4 * c + 1])), f2_pack(q.x, q.y)),
                     s[4 * c], s[4 * c + 1]);
           f2_unpack(f2_add(f2_pack(__uint_as_float(cur[4 * c + 2]), __uint_as_float(cur[4 * c + 3])), f2_pack(q.z, q.w)),
                     s[4 * c + 2], s[4 * c + 3]);
         }
-        // re-arm this buffer's next phase (one arrival + the bytes), then tell the peer it is free
-        if (i == 0) mbar_expect_tx(bar(B_XFULL + xb), X_BYTES);
-        mbar_arrive_peer_relaxed(xfree_peer + 8 * xb);
+        // re-arm the buffer's next phase (one arrival + the bytes), then tell the peer it is free
+        if (i == 0) mbar_expect_tx(bar(B_XFULL), X_BYTES);
+        mbar_arrive_peer(xfree_peer);
+        // the next tile's partial goes out now if its scores are ready, so that the exchange overlaps
+        // this tile's softmax; otherwise after P of this tile is out, so the softmax does not wait
+        const bool more = xt + 1 < send;
+        bool sent = false;
+        if (more && __all_sync(0xffffffffu, mbar_test(bar(B_SFULL + ((j + 1) & 1)), ((j + 1) >> 1) & 1))) {
+          if (!fetch_send(j + 1, cur)) { ok = false; break; }
+          sent = true;
+        }
         const int64_t key0 = (int64_t)(xt - ts_b) * NK;
         const int nvis = (int)max((int64_t)0, min((int64_t)NK, vis - key0));
         if (nvis < NK) {
@@ -392,14 +411,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int row = nrows + q / 32, box = (q / 8) & 3, c16 = q & 7;
             *reinterpret_cast<uint4*>(kvs + box * KV_BOX + row * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
           }
-          fence_proxy_async_smem();
         }
-        // P.V of the previous tile must be done before P is overwritten or O rescaled
-        if (!wait_u(bar(B_PVDONE), (j & 1) ^ 1)) return false;
-        // lazy rescale of the running max (identical decision in both CTAs)
+        // lazy rescale of the running max (identical decision in both CTAs); O must be at rest,
+        // so P.V of the previous tile has to be done first
         if (tmax > -INFINITY && (m_ref == -INFINITY || tmax > m_ref + thr_raw)) {
           const float alpha = ex2_approx((m_ref - tmax) * c2);
           if (j > jfirst) {
+            if (!wait_u(bar(B_PVDONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < 256; c += 32) {
@@ -411,11 +429,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               tmem_st32(trow + c, v);
             }
             tmem_wait_st();
+            tc_fence_before();
           }
           l *= alpha;
           m_ref = tmax;
         }
-        // P = 2^((s - m_ref) c2) in bf16 into TMEM (the A operand of P.V)
+        // P = 2^((s - m_ref) c2) in bf16, row i of the K-major P tile (128-byte swizzle)
         uint32_t pk[NK / 2];
         if (m_ref > -INFINITY) {
           const uint64_t cc = f2_pack(c2, c2), off = f2_pack(-m_ref * c2, -m_ref * c2);
@@ -425,8 +444,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             float a0, a1;
             f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), cc, off), a0, a1);
             const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-            pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
+            pk[c] = pack_bf16(e0, e1);
             if (c < 8) acc2[c] = f2_pack(e0, e1);
             else acc2[c & 7] = f2_add(acc2[c & 7], f2_pack(e0, e1));
           }
@@ -441,24 +459,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < NK / 2; ++c) pk[c] = 0u;
         }
-        tmem_st32(trow + T_P, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(B_PFULL));
+        // this P buffer was last read by P.V of tile j - 2
+        const int pb = j & 1;
+        if (!wait_u(bar(B_PVDONE + pb), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+        uint8_t* prow = smem + OFF_P + pb * P_BYTES + i * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ (i & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        mbar_arrive(bar(B_PFULL + pb));
+        if (more && !sent && !fetch_send(j + 1, cur)) { ok = false; break; }
         ++j;
-        return true;
-      };
-      uint32_t bufA[NK], bufB[NK];
-      if (!fetch_send(j, bufA)) { ok = false; break; }
-      for (int32_t xt = w.x; xt < send; xt += 2) {
-        if (!tile(xt, bufA, bufB)) { ok = false; break; }
-        if (xt + 1 < send && !tile(xt + 1, bufB, bufA)) { ok = false; break; }
       }
       if (!ok) break;
-      // segment epilogue: O / l for this CTA's 256 columns (+ lse from CTA 0)
+      // the next piece's query goes in now, so that its first QK^T overlaps this epilogue
+      {
+        SegWalk nx = w;
+        nx.next();
+        if (nx.valid() && !load_q(nx.b)) { ok = false; break; }
+      }
+      // piece epilogue: O / l for this CTA's 256 columns (+ lse from CTA 0)
       const int jl = j - 1;
       const float m_log2 = m_ref * c2;
-      if (!wait_u(bar(B_PVDONE), jl & 1)) { ok = false; break; }
+      if (!wait_u(bar(B_PVDONE + (jl & 1)), (jl >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const int64_t t = (int64_t)b * p.tq + k;
       const int32_t nseg = p.slot_base[b + 1] - p.slot_base[b];
@@ -513,6 +537,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, TMEM_COLS);
   }
 }
+
 
 // Tile prefix and partial-slot bases of every sequence (one block). Tiles per sequence are
 // counted on the cache length len_b (the last query token sees all of them). A sequence gets
@@ -685,6 +710,7 @@ cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B
   p.q_abs = reinterpret_cast<const __nv_bfloat16*>(q_abs);
   p.q_rope = reinterpret_cast<const __nv_bfloat16*>(q_rope);
   if ((e = make_tmap_bf16(&p.cmap, cache, ROW, capacity, ROW, 64, NK)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&p.rmap, cache, ROW, capacity, ROW, 32, NK, 64)) != cudaSuccess) return e;
   p.cu = cu;
   p.tile_start = c.ts;
   p.slot_base = c.sb;

@@ -58,9 +58,10 @@ struct TcGemmDesc {
 size_t tc_gemm_partial_bytes(int64_t T, int64_t f_tiles, int64_t f_total, int64_t K, int32_t batch);
 
 // 2-D bf16 TMA map over a row-major [outer, inner] matrix (row stride ld elements), box
-// {box_inner, box_outer}, 128-byte swizzle, zero fill out of bounds.
+// {box_inner, box_outer}, 128-byte swizzle (64-byte with swizzle_bytes = 64, for boxes of
+// 32 bf16 columns), zero fill out of bounds.
 cudaError_t make_tmap_bf16(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, int64_t ld, int box_inner,
-                           int box_outer);
+                           int box_outer, int swizzle_bytes = 128);
 
 cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st);
 
