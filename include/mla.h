@@ -181,6 +181,22 @@ mla_status_t mla_attn_decode_latent(mla_handle_t *h, const void *q_abs, const vo
                                     int64_t capacity, float *o_lat, float *lse, void *ws,
                                     size_t ws_bytes, mla_stream_t stream);
 
+/* The causal prefill attention core alone: step (10) of section 一(一)3 in the unabsorbed form, as
+ * inside mla_prefill. For head i and packed token t at position p of its sequence,
+ *   o[t, i] = sum_{j <= p} softmax_j([q^C; q^R][t, i] . [k^C[j, i]; k^R[j]] / sqrt(d_h + d_r)) v^C[j, i]
+ * over the tokens j of the same sequence.
+ *   q_c    [total_tokens, n_h, d_h]  handle dtype (q^C)
+ *   q_rope [total_tokens, n_h, d_r]  handle dtype (rotated q^R)
+ *   k_c    [total_tokens, n_h, d_h]  handle dtype (k^C = W^UK c^KV)
+ *   v_c    [total_tokens, n_h, d_h]  handle dtype (v^C = W^UV c^KV)
+ *   cache  [capacity, d_c + d_r]     k^R of packed token t in row t, columns [d_c, d_c + d_r)
+ *   o      [total_tokens, n_h, d_h]  handle dtype
+ * cu_seqlens, total_tokens and max_seqlen as for mla_prefill. No workspace, no weights. */
+mla_status_t mla_attn_prefill(mla_handle_t *h, const void *q_c, const void *q_rope, const void *k_c,
+                              const void *v_c, int64_t B, const int64_t *cu_seqlens, int64_t total_tokens,
+                              int64_t max_seqlen, const void *cache, int64_t capacity, void *o,
+                              mla_stream_t stream);
+
 /* Synchronizes the stream, then reports (and clears) the handle's device error word:
  * MLA_ERR_TIMEOUT, MLA_ERR_DEVICE_CHECK or MLA_OK. */
 mla_status_t mla_sync_status(mla_handle_t *h, mla_stream_t stream);

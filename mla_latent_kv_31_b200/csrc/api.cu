@@ -440,6 +440,39 @@ mla_status_t mla_prefill(mla_handle_t* h, const void* hidden, int64_t B, const i
   return simt_output(h, o, T, u_out, st);
 }
 
+mla_status_t mla_attn_prefill(mla_handle_t* h, const void* q_c, const void* q_rope, const void* k_c, const void* v_c,
+                              int64_t B, const int64_t* cu_seqlens, int64_t total_tokens, int64_t max_seqlen,
+                              const void* cache, int64_t capacity, void* o, mla_stream_t stream) {
+  if (!h || !q_c || !q_rope || !k_c || !v_c || !cu_seqlens || !cache || !o || B <= 0 || total_tokens <= 0 ||
+      max_seqlen <= 0 || capacity < total_tokens)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_c) || !aligned16(q_rope) || !aligned16(k_c) || !aligned16(v_c) || !aligned16(cache) ||
+      !aligned16(o) || !aligned16(cu_seqlens))
+    return MLA_ERR_ALIGNMENT;
+  mla_status_t s = ensure_device(h);  // the core needs no weights
+  if (s != MLA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const mla_dims_t& d = h->dims;
+  const int64_t T = total_tokens, R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
+  MLA_TRY(mla::check_and_positions(cu_seqlens, B, 0, T, capacity, max_seqlen, nullptr, h->d_err, st));
+  if (tc_dims(h) && mla::tc_available(MLA_OP_PREFILL))
+    return cuda_status(mla::tc_prefill_attention(q_c, q_rope, k_c, v_c, cache, capacity, cu_seqlens, B, T, max_seqlen,
+                                                 o, h->num_sms, h->d_err, st));
+  SimtAttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q1 = q_c; a.sq1t = HD; a.sq1h = d.d_h; a.d1 = d.d_h;
+  a.q2 = q_rope; a.sq2t = (int64_t)d.n_h * d.d_r; a.sq2h = d.d_r; a.d2 = d.d_r;
+  a.k1 = k_c; a.sk1 = HD; a.sk1h = d.d_h;
+  a.k2 = (const char*)cache + (size_t)d.d_c * elem_size(h); a.sk2 = R;
+  a.v = v_c; a.sv = HD; a.svh = d.d_h; a.dv = d.d_h;
+  a.o = o; a.sot = HD; a.soh = d.d_h;
+  a.lse = nullptr;
+  a.cu = cu_seqlens; a.B = B; a.tq = 0; a.T = T; a.n_h = d.n_h; a.capacity = capacity;
+  a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
+  a.err = h->d_err;
+  return cuda_status(mla::simt_attention(a, h->dtype == MLA_BF16, h->dtype == MLA_FP32, st));
+}
+
 mla_status_t mla_sync_status(mla_handle_t* h, mla_stream_t stream) {
   if (!h) return MLA_ERR_INVALID_ARG;
   if (!h->d_err) return MLA_OK;

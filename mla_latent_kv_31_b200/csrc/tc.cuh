@@ -38,6 +38,12 @@ cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const void* h
                       void* cq, void* qc, void* qr, void* qabs, void* olat, void* o, float* lse, void* scratch,
                       int num_sms, uint32_t* err, cudaStream_t st);
 
+// The causal prefill attention core (unabsorbed): q^C [T][H][128], q^R [T][H][64], k^C, v^C [T][H][128],
+// k^R in column 512 of the cache rows [capacity][576] (row = packed token index) -> o [T][H][128].
+cudaError_t tc_prefill_attention(const void* qc, const void* qr, const void* kc, const void* vc, const void* cache,
+                                 int64_t capacity, const int64_t* cu, int64_t B, int64_t T, int64_t max_seqlen,
+                                 void* o, int num_sms, uint32_t* err, cudaStream_t st);
+
 cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, int64_t B,
                        const int64_t* cu, int64_t T, int64_t max_seqlen, const int64_t* pos, void* cache,
                        int64_t capacity, void* u_out, void* cq, void* qc, void* qr, void* kc, void* vc, void* o,

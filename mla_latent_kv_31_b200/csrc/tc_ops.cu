@@ -165,7 +165,6 @@ cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* 
                        const int64_t* cu, int64_t T, int64_t max_seqlen, const int64_t* pos, void* cache,
                        int64_t capacity, void* u_out, void* cq, void* qc, void* qr, void* kc, void* vc, void* o,
                        uint32_t* err, cudaStream_t st) {
-  (void)max_seqlen;
   const int64_t R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
   cudaError_t e = cache_rows(d, w, hidden, pos, nullptr, T, cache, capacity, nullptr, 0, err, st);
   if (e != cudaSuccess) return e;
@@ -181,18 +180,10 @@ cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* 
   e = tc_gemm(p3, st);
   if (e != cudaSuccess) return e;
   // Steps (4), (8), (10): causal attention per head, keys [k^C_i; k^R], values v^C_i.
-  SimtAttnArgs a;
-  memset(&a, 0, sizeof(a));
-  a.q1 = qc; a.sq1t = HD; a.sq1h = d.d_h; a.d1 = d.d_h;
-  a.q2 = qr; a.sq2t = (int64_t)d.n_h * d.d_r; a.sq2h = d.d_r; a.d2 = d.d_r;
-  a.k1 = kc; a.sk1 = HD; a.sk1h = d.d_h;
-  a.k2 = (const char*)cache + (size_t)d.d_c * 2; a.sk2 = R;
-  a.v = vc; a.sv = HD; a.svh = d.d_h; a.dv = d.d_h;
-  a.o = o; a.sot = HD; a.soh = d.d_h;
-  a.cu = cu; a.B = B; a.tq = 0; a.T = T; a.n_h = d.n_h; a.capacity = capacity;
-  a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
-  a.err = err;
-  e = simt_attention(a, true, false, st);
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  e = tc_prefill_attention(qc, qr, kc, vc, cache, capacity, cu, B, T, max_seqlen, o, sms > 0 ? sms : 148, err, st);
   if (e != cudaSuccess) return e;
   return output(d, w, o, T, u_out, nullptr, 0, err, st);
 }

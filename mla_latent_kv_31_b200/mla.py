@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
                                     c_void_p, c_size_t, c_void_p]),
             "mla_attn_decode_latent": (c_int, [H, c_void_p, c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_int64,
                                                c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+            "mla_attn_prefill": (c_int, [H, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_int64,
+                                         c_int64, c_void_p, c_int64, c_void_p, c_void_p]),
             "mla_sync_status": (c_int, [H, c_void_p]),
             "mla_device_error_bits": (c_uint32, [H]),
             "mla_uses_tensor_cores": (c_int, [H, c_int]),
@@ -152,6 +154,13 @@ def mla_attn_decode_latent(handle, q_abs, q_rope, B, Tq, cu_seqlens, cache, capa
     _check(lib().mla_attn_decode_latent(handle, _ptr(q_abs), _ptr(q_rope), B, Tq, _ptr(cu_seqlens), _ptr(cache),
                                         capacity, _ptr(o_lat), _ptr(lse), _ptr(ws), ws_bytes,
                                         _stream(stream, device)), "mla_attn_decode_latent")
+
+
+def mla_attn_prefill(handle, q_c, q_rope, k_c, v_c, B, cu_seqlens, total_tokens, max_seqlen, cache, capacity, o,
+                     stream=None, device=0):
+    _check(lib().mla_attn_prefill(handle, _ptr(q_c), _ptr(q_rope), _ptr(k_c), _ptr(v_c), B, _ptr(cu_seqlens),
+                                  total_tokens, max_seqlen, _ptr(cache), capacity, _ptr(o), _stream(stream, device)),
+           "mla_attn_prefill")
 
 
 def mla_sync_status(handle, stream=None, device=0) -> int:

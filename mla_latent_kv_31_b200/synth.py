@@ -24,6 +24,8 @@ prefill shapes listed in WORKLOADS below.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -36,6 +38,7 @@ _M2 = np.uint64(0x94D049BB133111EB)
 TID_H, TID_WDQ, TID_WUQ, TID_WQR, TID_WDKV, TID_WKR, TID_WUK, TID_WUV, TID_WO = range(9)
 TID_CACHE_C, TID_CACHE_KR, TID_LENGTHS = 9, 10, 11
 TID_POSITIONS, TID_SLOTS = 12, 13
+TID_QC, TID_QR, TID_KC, TID_VC = 14, 15, 16, 17   # inputs of the prefill attention core alone
 
 _CHUNK = 1 << 22
 
@@ -89,11 +92,22 @@ def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def normal(seed: int, tensor_id: int, shape, std: float = 1.0, dtype: str = "bf16") -> np.ndarray:
+    """N(0, std^2) draws rounded to dtype. Chunks are independent (counter based), so they are drawn
+    on a thread pool; the values do not depend on the number of threads."""
     n = int(np.prod(shape))
     out = np.empty(n, dtype=np.float32)
-    for lo in range(0, n, _CHUNK):
+
+    def fill(lo):
         hi = min(n, lo + _CHUNK)
         out[lo:hi] = round_to(normal_f64(seed, tensor_id, hi - lo, start=lo) * std, dtype)
+
+    starts = range(0, n, _CHUNK)
+    if n <= _CHUNK:
+        for lo in starts:
+            fill(lo)
+    else:
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, starts))
     return out.reshape(shape)
 
 
@@ -149,6 +163,16 @@ def latent_cache(dims: Dims, rows: int, seed: int = 0, dtype: str = "bf16") -> n
     c = normal(seed, TID_CACHE_C, (rows, dims.d_c), dtype=dtype)
     kr = normal(seed, TID_CACHE_KR, (rows, dims.d_r), dtype=dtype)
     return np.concatenate([c, kr], axis=1)
+
+
+def prefill_core_inputs(dims: Dims, tokens: int, seed: int = 0, dtype: str = "bf16") -> dict:
+    """Inputs of the prefill attention core alone, all ~ N(0,1): q_c, k_c, v_c [tokens, n_h, d_h] and
+    q_r [tokens, n_h, d_r] (k^R comes from latent_cache rows)."""
+    hd = (tokens, dims.n_h, dims.d_h)
+    return {"q_c": normal(seed, TID_QC, hd, dtype=dtype),
+            "q_r": normal(seed, TID_QR, (tokens, dims.n_h, dims.d_r), dtype=dtype),
+            "k_c": normal(seed, TID_KC, hd, dtype=dtype),
+            "v_c": normal(seed, TID_VC, hd, dtype=dtype)}
 
 
 def ragged_lengths(batch: int, lo: int, hi: int, seed: int = 0) -> np.ndarray:

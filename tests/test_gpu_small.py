@@ -221,3 +221,32 @@ def test_decode_is_deterministic(v3_module):
     b = v3_module.decode(h_q, 2, 1, dev_i64(cu), cache).clone()
     _status_ok(v3_module)
     assert bool((a == b).all())
+
+
+# ---------------------------------------------------------------------------
+# The prefill attention core alone (mla_attn_prefill): 128-row query / key tiles, ragged tails,
+# a one-token sequence and a sequence that starts inside a tile of the packed layout
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("lens", [[600, 129, 1, 300], [128, 256, 127]])
+def test_v3_attn_prefill_core_ragged(v3_module, lens):
+    dims = synth.V3
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    x = synth.prefill_core_inputs(dims, T, seed=51)
+    cache_np = synth.latent_cache(dims, T + 3, seed=52)
+    d = {k: dev(v, "bf16") for k, v in x.items()}
+    cache = dev(cache_np, "bf16")
+    o = v3_module.torch.empty((T, dims.n_h, dims.d_h), device="cuda:0", dtype=v3_module.torch.bfloat16)
+    mla.mla_attn_prefill(v3_module.handle, d["q_c"], d["q_r"], d["k_c"], d["v_c"], len(lens), dev_i64(cu), T,
+                         max(lens), cache, T + 3, o, device=v3_module.device)
+    _status_ok(v3_module)
+    ref = np.empty((T, dims.n_h, dims.d_h))
+    scale = 1.0 / np.sqrt(dims.d_h + dims.d_r)
+    k_r = cache_np[:, dims.d_c:]
+    for b in range(len(lens)):
+        a, e = int(cu[b]), int(cu[b + 1])
+        for i in range(dims.n_h):
+            q = np.concatenate([x["q_c"][a:e, i], x["q_r"][a:e, i]], axis=1)
+            k = np.concatenate([x["k_c"][a:e, i], k_r[a:e]], axis=1)
+            ref[a:e, i], _, _, _ = orc.causal_softmax_attend(q, k, x["v_c"][a:e, i], None, np.arange(e - a), scale)
+    assert rel(host(o), ref) <= TOL["bf16"]
