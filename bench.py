@@ -39,6 +39,7 @@ WORKLOAD = synth.WORKLOADS["decode_b16_l4096"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CORE_FLOP_PER_ROW = 128 * 2 * (576 + 512)   # per cached row and query token: n_h * 2 * (d_c + d_R + d_c)
 ROW_BYTES = 576 * 2
+PREFILL = synth.WORKLOADS["prefill_l32768"]
 
 
 def parse():
@@ -48,6 +49,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--oracle-seconds", type=float, default=12.0, help="CPU time budget of the oracle sample")
+    ap.add_argument("--prefill-iters", type=int, default=5, help="timed prefill calls (0: no prefill leg)")
+    ap.add_argument("--prefill-seq-len", type=int, default=PREFILL.length,
+                    help="prefill sequence length (default: the 32K-token workload; smaller for profiling)")
     return ap.parse_args()
 
 
@@ -58,6 +62,22 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu record (profiles/kernel_traffic.json),
+    or None when there is none or the kernel's source has changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "kernel_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return int(rec["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def workload_config():
@@ -149,6 +169,115 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------------
 # our implementation
 # ---------------------------------------------------------------------------------------------
+def kernel_only_ms(fn, which, iters, warm, flush, world):
+    """Average duration of the library's attention-core launch inside fn() (CUDA events the library
+    records right around that launch, on its stream), each call after an L2 flush; max over ranks."""
+    import torch
+    from mla_latent_kv_31_b200 import mla
+    mla.mla_set_kernel_timing(True)
+    try:
+        for _ in range(warm):
+            flush.zero_()
+            fn()
+        tot = 0.0
+        for _ in range(iters):
+            flush.zero_()
+            fn()
+            tot += mla.mla_kernel_time_ms(which)
+    finally:
+        torch.cuda.synchronize()
+        mla.mla_set_kernel_timing(False)
+    ms = torch.tensor([tot / iters], device=flush.device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    return float(ms.item())
+
+
+def prefill_flops(dims, lens):
+    """FLOPs of one prefill: the unabsorbed attention minimum 2 (d_h + d_R + d_h) n_h per causal (q, k)
+    pair, and the projection GEMMs (W^DKV|W^KR, W^DQ, W^UQ|W^QR, W^UK|W^UV, W^O) at 2 flops per MAC."""
+    pairs = sum(L * (L + 1) // 2 for L in lens)
+    attn = pairs * dims.n_h * 2 * (dims.d_h + dims.d_r + dims.d_h)
+    T = sum(lens)
+    hd = dims.n_h * dims.d_h
+    proj = 2 * T * (dims.d * (dims.d_c + dims.d_r) + dims.d * dims.d_cq +
+                    dims.d_cq * (hd + dims.n_h * dims.d_r) + dims.d_c * 2 * hd + hd * dims.d)
+    return attn, proj
+
+
+def run_prefill(args, m, dev, rank, world, flush, timed, peaks, peak_src):
+    """Prefill of one 32K-token sequence (B = 1): the whole mla_prefill and the attention core alone
+    (mla_attn_prefill on the q^C, q^R, k^C, v^C that mla_prefill left in its workspace)."""
+    import torch
+    from mla_latent_kv_31_b200 import mla
+    L = args.prefill_seq_len
+    dims, T = PREFILL.dims, PREFILL.batch * L
+    lens = [L] * PREFILL.batch
+    h = m.handle
+    hid = torch.from_numpy(synth.hidden(dims, T, seed=rank)).to(dev, torch.bfloat16)
+    cu = torch.from_numpy(synth.cu_seqlens(lens)).to(dev)
+    cache = torch.zeros(T, dims.row, dtype=torch.bfloat16, device=dev)
+    u = torch.empty(T, dims.d, dtype=torch.bfloat16, device=dev)
+    n = mla.mla_workspace_size(h, mla.OP_PREFILL, PREFILL.batch, 1, T)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    assert mla.mla_uses_tensor_cores(h, mla.OP_PREFILL)
+    reg = lambda which: ws.data_ptr() + mla.mla_workspace_offset(h, mla.OP_PREFILL, which, PREFILL.batch, 1, T)  # noqa
+    o = torch.empty(T, dims.n_h, dims.d_h, dtype=torch.bfloat16, device=dev)
+
+    def full():
+        mla.mla_prefill(h, hid, PREFILL.batch, cu, T, L, cache, T, u, ws, n, device=dev.index)
+
+    def core():
+        mla.mla_attn_prefill(h, reg(mla.BUF_QC), reg(mla.BUF_QR), reg(mla.BUF_KC), reg(mla.BUF_VC), PREFILL.batch, cu,
+                             T, L, cache, T, o, device=dev.index)
+
+    full()
+    core()
+    torch.cuda.synchronize()
+    st = mla.mla_sync_status(h, device=dev.index)
+    if st != 0:
+        raise RuntimeError(f"device check failed in prefill: {mla.mla_status_string(st)}")
+    l0 = mla.mla_kernel_launches()
+    full()
+    launches = mla.mla_kernel_launches() - l0
+    clock = ClockSampler(dev.index)
+    clock.start()
+    ms_full = timed(full, args.prefill_iters, 3)
+    ms_core = timed(core, args.prefill_iters, 3)
+    ms_kernel = kernel_only_ms(core, mla.TIMED_PREFILL_CORE, args.prefill_iters, 1, flush, world)
+    clocks = clock.stop()
+    st = mla.mla_sync_status(h, device=dev.index)
+    if st != 0:
+        raise RuntimeError(f"device check failed after prefill timing: {mla.mla_status_string(st)}")
+    ms = torch.tensor([ms_full, ms_core], device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    ms_full, ms_core = (float(x) for x in ms.tolist())
+    attn, proj = prefill_flops(dims, lens)
+    sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    core_tf = attn / (ms_core * 1e-3) / 1e12
+    kern_tf = attn / (ms_kernel * 1e-3) / 1e12
+    full_tf = (attn + proj) / (ms_full * 1e-3) / 1e12
+    return {
+        "workload": PREFILL.name if L == PREFILL.length else f"prefill_l{L}", "batch": PREFILL.batch, "seq_len": L,
+        "call": "mla_prefill (cache append, query projections, k^C/v^C up-projection, causal attention, W^O)",
+        "ms": round(ms_full, 3), "tflops": round(world * full_tf, 1), "tokens_per_s": round(world * T / (ms_full * 1e-3), 1),
+        "flops_per_call": attn + proj, "gpu_launches_per_call": int(launches), "clocks": clocks,
+        "step_roofline": {"bound": "tensor", "achieved": round(full_tf, 1), "peak": sus, "unit": "TFLOP/s",
+                          "frac": round(full_tf / sus, 4), "peak_source": f"{peak_src} sustained"},
+        "core": {"call": "mla_attn_prefill", "ms": round(ms_core, 3), "tflops": round(core_tf, 1), "flops": attn,
+                 "kernel_ms": round(ms_kernel, 3),
+                 "roofline": {"bound": "tensor", "achieved": round(kern_tf, 1), "peak": sus, "unit": "TFLOP/s",
+                              "frac": round(kern_tf / sus, 4), "frac_of_burst_peak": round(kern_tf / burst, 4),
+                              "traffic": recorded_traffic("prefill_attn_kernel") if L == PREFILL.length else None,
+                              "kernel": "prefill_attn_kernel",
+                              "peak_source": f"{peak_src} sustained (the call runs for tens of ms)"}},
+    }
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -258,6 +387,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         u_host.copy_(u_dev, non_blocking=True)
 
     ms_e2e = timed(e2e, max(200, args.steps // 4), args.warmup)
+    del g_step, g_core
+    ms_kernel = kernel_only_ms(core, mla.TIMED_LATENT_CORE, max(200, args.steps // 4), args.warmup, flush, world)
+    peaks, peak_src = load_peaks()
+    prefill = (run_prefill(args, m, dev, rank, world, flush, timed, peaks, peak_src) if args.prefill_iters > 0
+               else {"status": "skipped (--prefill-iters 0)"})
     st = mla.mla_sync_status(h, device=local_rank)
     if st != 0:
         raise RuntimeError(f"device check failed after timing: {mla.mla_status_string(st)}")
@@ -266,14 +400,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         t = torch.tensor([ms_step, ms_core, ms_e2e], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step_max, ms_core_max, ms_e2e_max = (float(x) for x in t.tolist())
-    del g_step, g_core
     if rank != 0:
         return None
     cache_bytes = rows * ROW_BYTES
     weight_bytes = sum(v.numel() * 2 for v in W.values())
-    peaks, peak_src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     core_gbs = cache_bytes / (ms_core_max * 1e-3) / 1e9
+    kern_gbs = cache_bytes / (ms_kernel * 1e-3) / 1e9
     core_tflops = rows * tq * CORE_FLOP_PER_ROW / (ms_core_max * 1e-3) / 1e12
     step_bytes = cache_bytes + weight_bytes
     value = world * cache_bytes / (ms_step_max * 1e-3) / 1e9
@@ -291,9 +424,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                           "note": f"cache {cache_bytes} B + weights {weight_bytes} B per step, {peak_src} peak"},
         "latent_core": {"ms": round(ms_core_max, 5), "gbs": round(core_gbs, 1), "tflops": round(core_tflops, 1),
                         "call": "mla_attn_decode_latent (device check + plan + core + combine), CUDA-graph replay"},
-        "roofline": {"bound": "hbm", "achieved": round(core_gbs, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(core_gbs / hbm, 4), "traffic": None,
-                     "kernel": "latent_core_kernel (+ plan/combine in the timed call)",
+        "roofline": {"bound": "hbm", "achieved": round(kern_gbs, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(kern_gbs / hbm, 4), "traffic": recorded_traffic("latent_core_kernel"),
+                     "kernel": "latent_core_kernel", "kernel_ms": round(ms_kernel, 5),
+                     "timing": "CUDA events recorded by the library right around the kernel launch, L2 flushed",
                      "algorithmic_bytes": cache_bytes, "peak_source": peak_src},
         "e2e": {"value": round(world * cache_bytes / (ms_e2e_max * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(ms_e2e_max, 5),
@@ -303,7 +437,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "gpu_launches_per_step": int(per_step_launches),
         "clocks": clocks,
         "timed_wall_s": round(wall, 3),
-        "prefill": {"status": "not in this line: the prefill attention core on tcgen05 is not built yet"},
+        "prefill": prefill,
     }
     return out
 

@@ -211,6 +211,14 @@ uint64_t mla_kernel_launches(void);
  * sizes), 0 = generic CUDA-core kernels (FP32, or other sizes). Host-only. */
 int mla_uses_tensor_cores(const mla_handle_t *h, mla_op_t op);
 
+/* Kernel timing for measurement tools. While enabled (process-wide), the library records a CUDA event
+ * on the launching stream right before and right after every launch of its two attention cores;
+ * mla_kernel_time_ms waits for the end event of the last bracketed launch of `which`
+ * (0 = the decode latent core, 1 = the prefill attention core) and returns its elapsed ms, or
+ * MLA_ERR_INVALID_ARG if there was none. Off by default; do not enable it around stream capture. */
+mla_status_t mla_set_kernel_timing(int enabled);
+mla_status_t mla_kernel_time_ms(int which, float *ms);
+
 const char *mla_status_string(mla_status_t s);
 
 /* Frees the handle's own device memory (its error word). Borrowed tensors are untouched. */

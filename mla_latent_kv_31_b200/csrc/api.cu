@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 #include <new>
 
 #include "mla.h"
@@ -27,6 +28,30 @@ struct mla_handle {
 namespace mla {
 static std::atomic<unsigned long long> g_launches{0};
 void note_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Kernel timing: one event pair per timed kernel, created on the device of the first bracketed launch.
+static std::atomic<bool> g_timing{false};
+static cudaEvent_t g_ev[TIMED_KERNELS][2];
+static bool g_ev_made = false;
+static bool g_ev_recorded[TIMED_KERNELS] = {false, false};
+static std::mutex g_timing_mu;
+void timer_begin(TimedKernel k, cudaStream_t st) {
+  if (!g_timing.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  if (!g_ev_made) {
+    for (int i = 0; i < TIMED_KERNELS; ++i)
+      for (int j = 0; j < 2; ++j) cudaEventCreate(&g_ev[i][j]);
+    g_ev_made = true;
+  }
+  cudaEventRecord(g_ev[k][0], st);
+}
+void timer_end(TimedKernel k, cudaStream_t st) {
+  if (!g_timing.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  if (!g_ev_made) return;
+  cudaEventRecord(g_ev[k][1], st);
+  g_ev_recorded[k] = true;
+}
 }  // namespace mla
 
 namespace {
@@ -491,6 +516,20 @@ uint32_t mla_device_error_bits(const mla_handle_t* h) { return h ? h->last_err_b
 
 uint64_t mla_kernel_launches(void) { return mla::g_launches.load(std::memory_order_relaxed); }
 
+mla_status_t mla_set_kernel_timing(int enabled) {
+  mla::g_timing.store(enabled != 0, std::memory_order_relaxed);
+  return MLA_OK;
+}
+
+mla_status_t mla_kernel_time_ms(int which, float* ms) {
+  if (!ms || which < 0 || which >= mla::TIMED_KERNELS) return MLA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(mla::g_timing_mu);
+  if (!mla::g_ev_made || !mla::g_ev_recorded[which]) return MLA_ERR_INVALID_ARG;
+  MLA_TRY(cudaEventSynchronize(mla::g_ev[which][1]));
+  MLA_TRY(cudaEventElapsedTime(ms, mla::g_ev[which][0], mla::g_ev[which][1]));
+  return MLA_OK;
+}
+
 void mla_destroy(mla_handle_t* h) {
   if (!h) return;
   if (h->d_err) {
@@ -507,7 +546,6 @@ void mla_destroy(mla_handle_t* h) {
 // scratch is this fixed device array; host code never touches the array's name as an address
 // but asks the runtime for the device address once per device.
 // ---------------------------------------------------------------------------------------------
-#include <mutex>
 
 namespace {
 

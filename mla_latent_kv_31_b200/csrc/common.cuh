@@ -20,6 +20,10 @@ enum : uint32_t {
 
 // Host-side count of kernels this library has launched (mla_kernel_launches()).
 void note_launch(unsigned n = 1);
+// Optional event brackets around the attention-core launches (see mla_set_kernel_timing).
+enum TimedKernel { TIMED_LATENT_CORE = 0, TIMED_PREFILL_CORE = 1, TIMED_KERNELS = 2 };
+void timer_begin(TimedKernel k, cudaStream_t st);
+void timer_end(TimedKernel k, cudaStream_t st);
 
 __device__ __forceinline__ void flag_error(uint32_t* err, uint32_t bits) {
   if (err) atomicOr(err, bits);

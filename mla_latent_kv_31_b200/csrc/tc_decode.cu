@@ -678,7 +678,9 @@ cudaError_t launch_core(const CoreParams& p, dim3 grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
+  timer_begin(TIMED_LATENT_CORE, st);
   latent_core_kernel<OUT_F32><<<grid, kThreads, SMEM_BYTES, st>>>(p);
+  timer_end(TIMED_LATENT_CORE, st);
   note_launch();
   return cudaGetLastError();
 }

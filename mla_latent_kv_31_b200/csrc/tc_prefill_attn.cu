@@ -388,7 +388,9 @@ cudaError_t tc_prefill_attention(const void* qc, const void* qr, const void* kc,
   }
   const int64_t units = (int64_t)H * B * p.M;
   const int grid = (int)(units < num_sms ? units : num_sms);
+  timer_begin(TIMED_PREFILL_CORE, st);
   prefill_attn_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p);
+  timer_end(TIMED_PREFILL_CORE, st);
   note_launch();
   return cudaGetLastError();
 }

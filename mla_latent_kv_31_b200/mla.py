@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
             "mla_device_error_bits": (c_uint32, [H]),
             "mla_uses_tensor_cores": (c_int, [H, c_int]),
             "mla_kernel_launches": (ctypes.c_uint64, []),
+            "mla_set_kernel_timing": (c_int, [c_int]),
+            "mla_kernel_time_ms": (c_int, [c_int, POINTER(ctypes.c_float)]),
             "mla_status_string": (c_char_p, [c_int]),
             "mla_destroy": (None, [H]),
         }
@@ -173,6 +175,19 @@ def mla_device_error_bits(handle) -> int:
 
 def mla_uses_tensor_cores(handle, op: int) -> bool:
     return bool(lib().mla_uses_tensor_cores(handle, op))
+
+
+TIMED_LATENT_CORE, TIMED_PREFILL_CORE = 0, 1
+
+
+def mla_set_kernel_timing(enabled: bool):
+    _check(lib().mla_set_kernel_timing(1 if enabled else 0), "mla_set_kernel_timing")
+
+
+def mla_kernel_time_ms(which: int) -> float:
+    ms = ctypes.c_float(0.0)
+    _check(lib().mla_kernel_time_ms(which, ctypes.byref(ms)), "mla_kernel_time_ms")
+    return float(ms.value)
 
 
 def mla_kernel_launches() -> int:
