@@ -11,18 +11,24 @@
 // crosses a sequence boundary emits one partial result per sequence piece, and a final pass
 // merges the pieces of a sequence exactly (log-sum-exp). Within a pair, CTA r owns latent
 // columns [256 r, 256 r + 256) and k^R columns [32 r, 32 r + 32): it streams only those 288
-// columns of every cache row, computes the partial score over them, swaps the 128 x 64 fp32
-// partial with its peer through distributed shared memory, and then both run the same softmax
+// columns of every cache row, computes the partial score over them, swaps the 128 x 64 partial
+// (as fp16) with its peer through distributed shared memory, and then both run the same softmax
 // and accumulate P . c into their own 256 TMEM columns of O. The 128 heads form the MMA M
 // dimension; one TMA-loaded cache tile is read K-major by QK^T and MN-major by P.V.
 //
-// Pipelining. Scores are double-buffered in TMEM and P is double-buffered in shared memory, so
-// QK^T of tile j + 1 runs while the softmax works on tile j, and the softmax of tile j + 1 does
-// not wait for P.V of tile j (only a rescale of O does, which the lazy running max makes rare).
+// Pipelining. Scores are double-buffered in TMEM and the peer's partials in shared memory, so QK^T
+// of tile j + 1 and the copy of its partial run while the softmax works on tile j; P.V of tile j
+// reads P from shared memory, which the softmax of tile j + 1 rewrites once that P.V is done.
+// Sending this CTA's partial scores to the peer has warps of its own: they read a tile's partial out
+// of TMEM as soon as QK^T is done, stage it in shared memory and copy it in bulk to the peer, while
+// the softmax warps work on the tile before it; the softmax adds the peer's partial to its own.
 //
-// Roles per CTA (192 threads): warps 0-3 softmax/epilogue (thread i = head i = TMEM lane i),
-// warp 4 TMA producer, warp 5 TMEM owner + MMA issuer. Every wait is bounded.
+// Roles per CTA (448 threads): warps 0-3 and 10-13 softmax/epilogue (two warps per TMEM lane
+// quarter, thread = head = TMEM lane, one warp per half of a tile's keys), warp 4 TMA producer,
+// warp 5 TMEM owner + MMA issuer, warps 6-9 send this CTA's partial scores (warp w on TMEM lanes
+// 32 (w % 4) + [0, 32)). Every wait is bounded.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <string.h>
 
 #include "sm100.cuh"
@@ -36,29 +42,39 @@ using namespace sm100;
 
 constexpr int H = 128, DC = 512, DR = 64, ROW = DC + DR;
 constexpr int NK = 64;                       // keys per tile (the N of QK^T, the K of P.V)
+// Partial scores cross to the peer CTA as fp16; both CTAs add the same two fp16-rounded halves, so
+// they see identical scores (relative rounding 2^-11 per half, far inside the bf16 error budget).
+// Half the bytes of fp32 leave room for two receive buffers and four cache stages.
+constexpr bool kXHalf = true;
 constexpr int STAGES = 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 448;
 constexpr int kMaxPairs = 74;
 constexpr float kRescaleLog2 = 8.f;          // lazy rescale: keep the running max until it grows by 2^8
 
 constexpr uint32_t KV_BOX = NK * 128;        // [64 keys x 64 latent cols] bf16, 128-byte swizzle: 8 KB
 constexpr uint32_t R_BOX = NK * 64;          // [64 keys x 32 k^R cols] bf16, 64-byte swizzle: 4 KB
 constexpr uint32_t STAGE_BYTES = 4 * KV_BOX + R_BOX;   // 36 KB
-constexpr uint32_t X_BYTES = H * NK * 4;     // [128 x 64] fp32 partial scores from the peer: 32 KB
+constexpr uint32_t XE = kXHalf ? 2 : 4;      // bytes per exchanged score
+constexpr uint32_t X_BYTES = H * NK * XE;    // [128 x 64] partial scores: 32 KB (fp32) / 16 KB (fp16)
+constexpr int XPER = 16 / XE;                // scores per 16-byte chunk
+constexpr int XCH = NK / XPER;               // 16-byte chunks per head
 constexpr uint32_t P_BYTES = H * NK * 2;     // [128 x 64] bf16 probabilities, K-major, 128-byte swizzle
 constexpr uint32_t QR_BYTES = H * 32 * 2;    // [128 x 32] bf16 q^R half, K-major, 64-byte swizzle
 constexpr uint32_t OFF_KV = 0;
 constexpr uint32_t OFF_X = OFF_KV + STAGES * STAGE_BYTES;
-constexpr uint32_t OFF_P = OFF_X + X_BYTES;
-constexpr uint32_t OFF_QR = OFF_P + 2 * P_BYTES;
-constexpr uint32_t OFF_BAR = OFF_QR + QR_BYTES;
+constexpr uint32_t OFF_XO = OFF_X + 2 * X_BYTES;  // two receive buffers, then this CTA's staged partial
+constexpr uint32_t OFF_P = OFF_XO + X_BYTES;
+constexpr uint32_t OFF_QR = OFF_P + P_BYTES;
+constexpr uint32_t OFF_RED = OFF_QR + QR_BYTES;   // per-head maxima / sums swapped between softmax halves
+constexpr uint32_t OFF_BAR = OFF_RED + 3 * 2 * H * 4;
 static_assert(STAGE_BYTES % 1024 == 0 && OFF_P % 1024 == 0 && OFF_QR % 1024 == 0, "swizzle atom alignment");
 
 // barrier indices
 constexpr int B_FULL = 0, B_EMPTY = STAGES, B_SFULL = 2 * STAGES, B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2,
-              B_PVDONE = B_PFULL + 2, B_XFULL = B_PVDONE + 2, B_XFREE = B_XFULL + 1, B_QFULL = B_XFREE + 1,
-              B_QEMPTY = B_QFULL + 1, B_OFREE = B_QEMPTY + 1;
-constexpr int NBAR = B_OFREE + 1;
+              B_PVDONE = B_PFULL + 1, B_XFULL = B_PVDONE + 1, B_XFREE = B_XFULL + 2, B_QFULL = B_XFREE + 2,
+              B_QEMPTY = B_QFULL + 1, B_OFREE = B_QEMPTY + 1, B_XOFREE = B_OFREE + 1, B_XORDY = B_XOFREE + 1,
+              B_TMAX = B_XORDY + 1;
+constexpr int NBAR = B_TMAX + 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -163,12 +179,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
-      const bool many = (i >= B_SEMPTY && i < B_SEMPTY + 2) || (i >= B_PFULL && i < B_PFULL + 2) || i == B_XFREE ||
-                        i == B_OFREE || i == B_QFULL;
-      mbar_init(bar(i), many ? 128 : 1);
+      // counts: the 256 softmax threads (P, O, q hand-offs); SEMPTY: those plus the 128 exchange threads
+      // that also read a score buffer; XORDY: the exchange threads; XFREE: one arrival per softmax
+      // warp of the peer; TMAX: the two softmax warps of one TMEM lane quarter
+      uint32_t cnt = 1;
+      if (i == B_PFULL || i == B_OFREE || i == B_QFULL) cnt = 256;
+      else if (i >= B_SEMPTY && i < B_SEMPTY + 2) cnt = 384;
+      else if (i == B_XORDY) cnt = 128;
+      else if (i == B_XFREE || i == B_XFREE + 1) cnt = 8;
+      else if (i >= B_TMAX && i < B_TMAX + 4) cnt = 64;
+      mbar_init(bar(i), cnt);
     }
-    // the exchange buffer's first phase: one arrival plus the bytes the peer's st.async will bring
+    // the exchange buffers' first phases: one arrival plus the bytes the peer's copy will bring
     mbar_expect_tx(bar(B_XFULL), X_BYTES);
+    mbar_expect_tx(bar(B_XFULL + 1), X_BYTES);
     fence_mbar_init();
   }
   if (warp == 5) {
@@ -231,18 +255,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int qk_half = 0;                               // halves of QK^T(cq.j) issued so far
       while (cp.valid()) {
         bool did = false;
-        if (cp.j < cq.j && mbar_test(bar(B_PFULL + (cp.j & 1)), (cp.j >> 1) & 1) &&
+        if (cp.j < cq.j && mbar_test(bar(B_PFULL), cp.j & 1) &&
             (!cp.first() || mbar_test(bar(B_OFREE), (cp.g & 1) ^ 1))) {
           tc_fence_after();
-          const int st = cp.j % STAGES, pb = cp.j & 1;
+          const int st = cp.j % STAGES;
           const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
-          const uint32_t pa = sbase + OFF_P + pb * P_BYTES;
+          const uint32_t pa = sbase + OFF_P;
           const bool first = cp.first();
 #pragma unroll
           for (int kk = 0; kk < NK / 16; ++kk)
             mma_bf16_ss(tmem, sw128_desc(pa + kk * 32, 0, 1024), sw128_desc(kv + kk * 2048, KV_BOX, 1024), idesc_pv,
                         (first && kk == 0) ? 0u : 1u);
-          mma_commit(bar(B_PVDONE + pb));
+          mma_commit(bar(B_PVDONE));
           mma_commit(bar(B_EMPTY + st));
           cp.advance();
           did = true;
@@ -292,41 +316,122 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
     }
+  } else if (warp >= 6 && warp < 10) {
+    // ------------------------------------------------------------------ score exchange (send side)
+    // Per tile: this CTA's partial scores TMEM -> registers -> the local staging buffer (chunk-major:
+    // chunk c of head i at (c * 128 + i) * 16), which one thread copies in bulk into the peer's
+    // exchange buffer once the peer's softmax has read the previous tile out of it (counted on the
+    // peer's x_full barrier). The staging buffer is rewritten only once the previous copy has read it.
+    const int e = threadIdx.x - 192;                 // exchange thread 0..127
+    const int i = 32 * (warp & 3) + lane;            // head = TMEM lane
+    const bool leader = e == 0;
+    const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    const uint32_t xin_peer = map_peer(sbase + OFF_X, peer);
+    const uint32_t xfull_peer = map_peer(bar(B_XFULL), peer);
+    uint4* xo = reinterpret_cast<uint4*>(smem + OFF_XO) + i;
+    auto wait_u = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(b, par)) != 0; };
+    const int ntiles = t_end - t_begin;
+    bool ok = true;
+    for (int jj = 0; jj < ntiles; ++jj) {
+      const int sb = jj & 1;
+      const uint32_t taddr = trow + T_S + NK * sb;
+      if (leader && jj > 0) {
+        bulk_wait_read0();                           // the previous copy has read the staging buffer
+        mbar_arrive(bar(B_XOFREE));
+      }
+      if (!wait_u(bar(B_SFULL + sb), (jj >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t v[NK];
+      tmem_ld32(taddr, v);
+      tmem_ld32(taddr + 32, v + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_SEMPTY + sb));
+      if (!wait_u(bar(B_XOFREE), (jj & 1) ^ 1)) { ok = false; break; }
+#pragma unroll
+      for (int c = 0; c < XCH; ++c) {
+        uint32_t w4[4];
+        if (kXHalf) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int k2 = XPER * c + 2 * q;
+            const __half2 h2 = __floats2half2_rn(__uint_as_float(v[k2]), __uint_as_float(v[k2 + 1]));
+            w4[q] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) w4[q] = v[XPER * c + q];
+        }
+        xo[c * 128] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_XORDY));
+      if (leader) {
+        // all 128 rows staged, and the peer's softmax has read the previous tile out of its buffer
+        const int xb = jj & 1;
+        if (mbar_wait(bar(B_XORDY), jj & 1) && mbar_wait_cluster(bar(B_XFREE + xb), ((jj >> 1) & 1) ^ 1)) {
+          bulk_copy_to_peer(xin_peer + xb * X_BYTES, sbase + OFF_XO, X_BYTES, xfull_peer + 8 * xb);
+          bulk_commit();
+        } else {
+          ok = false;
+        }
+      }
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+    }
+    if (leader) bulk_wait_read0();
+    if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int i = threadIdx.x;                       // head
-    const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
-    const uint32_t xpeer = map_peer(sbase + OFF_X, peer) + i * 16;
-    const uint32_t xfull_peer = map_peer(bar(B_XFULL), peer);
+    // Two warps per TMEM lane quarter: half 0 (warps 0-3) takes keys [0, 32) of every tile, half 1
+    // (warps 10-13) keys [32, 64), for the same 32 heads; they agree on each tile's max through
+    // shared memory and a per-quarter barrier. O columns (rescale, epilogue) and the query load are
+    // split between the halves the same way.
+    const int quarter = warp & 3, half = warp >= 10 ? 1 : 0;
+    const int i = 32 * quarter + lane;               // head
+    const int tid = 128 * half + i;                  // 0..255 over both halves
+    const int kc0 = 32 * half;                       // first key of this half within a tile
+    const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
     const uint32_t xfree_peer = map_peer(bar(B_XFREE), peer);
+    const uint32_t tmax_bar = bar(B_TMAX + quarter);
+    float* redbuf = reinterpret_cast<float*>(smem + OFF_RED);   // [2 parity][2 half][128] maxima, then [2][128] sums
     const float c2 = p.scale_log2;                   // raw score -> log2 units
     const float thr_raw = kRescaleLog2 / c2;
     // waits of the softmax warps are warp-uniform: a timeout on any lane fails the whole warp, so
     // no lane can be left behind at a .sync.aligned tcgen05 instruction
     auto wait_u = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(b, par)) != 0; };
     auto wait_uc = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait_cluster(b, par)) != 0; };
-    int gq = 0, j = 0;
-    // q~ half -> TMEM and q^R half -> shared memory (64-byte swizzle) for the piece of sequence bq,
-    // once the previous piece's last QK^T is done with them.
+    int gq = 0, j = 0, tph = 0;
+    // one exchange of a value per head with the other half of this quarter: returns the partner's
+    auto swap_half = [&](float x, int slot) -> float {
+      redbuf[(slot * 2 + half) * 128 + i] = x;
+      mbar_arrive(tmax_bar);
+      const bool okw = wait_u(tmax_bar, tph & 1);
+      ++tph;
+      const float y = redbuf[(slot * 2 + (half ^ 1)) * 128 + i];
+      return okw ? y : NAN;
+    };
+    // q~ half -> TMEM (this half's 64 columns) and q^R half -> shared memory (64-byte swizzle, this
+    // half's two chunks) for the piece of sequence bq, once the previous piece's last QK^T is done.
     auto load_q = [&](int bq) -> bool {
       const int64_t t = (int64_t)bq * p.tq + k;
       if (!wait_u(bar(B_QEMPTY), (gq & 1) ^ 1)) return false;
       tc_fence_after();
-      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (t * H + i) * DC + 256 * r);
+      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (t * H + i) * DC + 256 * r + 128 * half);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const uint4 u = __ldg(src + 8 * c + e);
           v[4 * e] = u.x; v[4 * e + 1] = u.y; v[4 * e + 2] = u.z; v[4 * e + 3] = u.w;
         }
-        tmem_st32(trow + T_Q + 32 * c, v);
+        tmem_st32(trow + T_Q + 64 * half + 32 * c, v);
       }
       const uint4* rsrc = reinterpret_cast<const uint4*>(p.q_rope + (t * H + i) * DR + 32 * r);
       uint8_t* qrow = smem + OFF_QR + i * 64;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(qrow + ((c ^ ((i >> 1) & 3)) << 4)) = __ldg(rsrc + c);
+      for (int c = 2 * half; c < 2 * half + 2; ++c)
+        *reinterpret_cast<uint4*>(qrow + ((c ^ ((i >> 1) & 3)) << 4)) = __ldg(rsrc + c);
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
@@ -334,26 +439,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ++gq;
       return true;
     };
-    // This CTA's partial scores of tile jj: TMEM -> registers, then sent to the peer with st.async
-    // (chunk-major layout: element c of head i at ((c / 4) * 128 + i) * 16 + (c % 4) * 4), each store
-    // counting its bytes on the peer's x_full barrier.
-    auto fetch_send = [&](int jj, uint32_t(&own)[NK]) -> bool {
-      const int sb = jj & 1;
-      if (!wait_u(bar(B_SFULL + sb), (jj >> 1) & 1)) return false;
-      tc_fence_after();
-      tmem_ld32(trow + T_S + NK * sb, own);
-      tmem_ld32(trow + T_S + NK * sb + 32, own + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_SEMPTY + sb));
-      // the peer has read the previous tile out of its exchange buffer
-      if (!wait_uc(bar(B_XFREE), (jj & 1) ^ 1)) return false;
-#pragma unroll
-      for (int c = 0; c < NK / 4; ++c)
-        st_async_peer_v4(xpeer + c * 2048, own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3], xfull_peer);
-      return true;
-    };
-    uint32_t cur[NK];
     bool ok = !w.valid() || load_q(w.b);
     for (; ok && w.valid(); w.next()) {
       const int b = w.b;
@@ -361,66 +446,74 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int64_t vis = len - p.tq + k + 1;        // keys visible to this query token
       const int32_t ts_b = p.tile_start[b];
       const int32_t send = w.seg_end();
-      float m_ref = -INFINITY, l = 0.f;              // running max in raw score units
+      float m_ref = -INFINITY, l = 0.f;              // running max (raw score units); this half's sum
       const int jfirst = j;
-      if (!fetch_send(j, cur)) { ok = false; break; }
       for (int32_t xt = w.x; xt < send; ++xt) {
-        // full scores of tile j: this CTA's partial plus the peer's
-        if (!wait_uc(bar(B_XFULL), j & 1)) { ok = false; break; }
-        const float4* xrd = reinterpret_cast<const float4*>(smem + OFF_X) + i;
-        float s[NK];
+        // scores of this half's 32 keys: this CTA's partial (TMEM) plus the peer's (exchange buffer)
+        const int sb = j & 1, xb = j & 1;
+        if (!wait_u(bar(B_SFULL + sb), (j >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        float s[32];
+        tmem_ld32(trow + T_S + NK * sb + kc0, reinterpret_cast<uint32_t*>(s));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_SEMPTY + sb));
+        if (!wait_uc(bar(B_XFULL + xb), (j >> 1) & 1)) { ok = false; break; }
+        {
+          const uint4* xi = reinterpret_cast<const uint4*>(smem + OFF_X + xb * X_BYTES) + i;
 #pragma unroll
-        for (int c = 0; c < NK / 4; ++c) {
-          const float4 q = xrd[c * 128];
-          f2_unpack(f2_add(f2_pack(__uint_as_float(cur[4 * c]), __uint_as_float(cur[4 * c + 1])), f2_pack(q.x, q.y)),
-                    s[4 * c], s[4 * c + 1]);
-          f2_unpack(f2_add(f2_pack(__uint_as_float(cur[4 * c + 2]), __uint_as_float(cur[4 * c + 3])), f2_pack(q.z, q.w)),
-                    s[4 * c + 2], s[4 * c + 3]);
+          for (int c = 0; c < 4; ++c) {
+            const uint4 q = xi[(4 * half + c) * 128];
+            const uint32_t q4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              // both CTAs add the two fp16-rounded partials, so they see the same scores
+              const int k2 = 8 * c + 2 * u;
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&q4[u]));
+              const float2 o = __half22float2(__floats2half2_rn(s[k2], s[k2 + 1]));
+              s[k2] = o.x + f.x;
+              s[k2 + 1] = o.y + f.y;
+            }
+          }
         }
         // re-arm the buffer's next phase (one arrival + the bytes), then tell the peer it is free
-        if (i == 0) mbar_expect_tx(bar(B_XFULL), X_BYTES);
-        mbar_arrive_peer(xfree_peer);
-        // the next tile's partial goes out now if its scores are ready, so that the exchange overlaps
-        // this tile's softmax; otherwise after P of this tile is out, so the softmax does not wait
-        const bool more = xt + 1 < send;
-        bool sent = false;
-        if (more && __all_sync(0xffffffffu, mbar_test(bar(B_SFULL + ((j + 1) & 1)), ((j + 1) >> 1) & 1))) {
-          if (!fetch_send(j + 1, cur)) { ok = false; break; }
-          sent = true;
-        }
+        if (tid == 0) mbar_expect_tx(bar(B_XFULL + xb), X_BYTES);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_peer(xfree_peer + 8 * xb);
         const int64_t key0 = (int64_t)(xt - ts_b) * NK;
-        const int nvis = (int)max((int64_t)0, min((int64_t)NK, vis - key0));
-        if (nvis < NK) {
+        const int nvis = (int)max((int64_t)0, min((int64_t)NK, vis - key0)) - kc0;
+        if (nvis < 32) {
 #pragma unroll
-          for (int c = 0; c < NK; ++c) s[c] = c < nvis ? s[c] : -INFINITY;
+          for (int c = 0; c < 32; ++c) s[c] = c < nvis ? s[c] : -INFINITY;
         }
-        float mx[NK / 2];
+        float mx[16];
 #pragma unroll
-        for (int c = 0; c < NK / 2; ++c) mx[c] = fmaxf(s[2 * c], s[2 * c + 1]);
+        for (int c = 0; c < 16; ++c) mx[c] = fmaxf(s[2 * c], s[2 * c + 1]);
 #pragma unroll
-        for (int w2 = NK / 4; w2 > 0; w2 >>= 1)
+        for (int w2 = 8; w2 > 0; w2 >>= 1)
 #pragma unroll
           for (int c = 0; c < w2; ++c) mx[c] = fmaxf(mx[c], mx[c + w2]);
-        const float tmax = mx[0];
+        const float tmax = fmaxf(mx[0], swap_half(mx[0], j & 1));
+        if (tmax != tmax) { ok = false; break; }      // the partner half gave up (timeout)
         // rows of this stage past the sequence end: zero the latent half before P.V reads it
         const int nrows = (int)max((int64_t)0, min((int64_t)NK, len - key0));
         if (nrows < NK) {
           uint8_t* kvs = smem + OFF_KV + (j % STAGES) * STAGE_BYTES;
           const int chunks = (NK - nrows) * 4 * 8;   // 16-byte chunks over 4 boxes
-          for (int q = i; q < chunks; q += 128) {
+          for (int q = tid; q < chunks; q += 256) {
             const int row = nrows + q / 32, box = (q / 8) & 3, c16 = q & 7;
             *reinterpret_cast<uint4*>(kvs + box * KV_BOX + row * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
           }
         }
-        // lazy rescale of the running max (identical decision in both CTAs); O must be at rest,
-        // so P.V of the previous tile has to be done first
+        // lazy rescale of the running max (identical decision in both halves and both CTAs); O must
+        // be at rest, so P.V of the previous tile has to be done first
         if (tmax > -INFINITY && (m_ref == -INFINITY || tmax > m_ref + thr_raw)) {
           const float alpha = ex2_approx((m_ref - tmax) * c2);
           if (j > jfirst) {
-            if (!wait_u(bar(B_PVDONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) { ok = false; break; }
+            if (!wait_u(bar(B_PVDONE), (j - 1) & 1)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < 256; c += 32) {
+            for (int c = 128 * half; c < 128 * half + 128; c += 32) {
               uint32_t v[32];
               tmem_ld32(trow + c, v);
               tmem_wait_ld();
@@ -434,13 +527,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           l *= alpha;
           m_ref = tmax;
         }
-        // P = 2^((s - m_ref) c2) in bf16, row i of the K-major P tile (128-byte swizzle)
-        uint32_t pk[NK / 2];
+        // P = 2^((s - m_ref) c2) in bf16: this half's 4 chunks of row i of the K-major P tile
+        uint32_t pk[16];
         if (m_ref > -INFINITY) {
           const uint64_t cc = f2_pack(c2, c2), off = f2_pack(-m_ref * c2, -m_ref * c2);
           uint64_t acc2[8];
 #pragma unroll
-          for (int c = 0; c < NK / 2; ++c) {
+          for (int c = 0; c < 16; ++c) {
             float a0, a1;
             f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), cc, off), a0, a1);
             const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
@@ -457,19 +550,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           l += l0 + l1;
         } else {
 #pragma unroll
-          for (int c = 0; c < NK / 2; ++c) pk[c] = 0u;
+          for (int c = 0; c < 16; ++c) pk[c] = 0u;
         }
-        // this P buffer was last read by P.V of tile j - 2
-        const int pb = j & 1;
-        if (!wait_u(bar(B_PVDONE + pb), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
-        uint8_t* prow = smem + OFF_P + pb * P_BYTES + i * 128;
+        // the P tile was last read by P.V of tile j - 1
+        if (!wait_u(bar(B_PVDONE), (j - 1) & 1)) { ok = false; break; }
+        uint8_t* prow = smem + OFF_P + i * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (i & 7)) << 4)) =
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (i & 7)) << 4)) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         fence_proxy_async_smem();
-        mbar_arrive(bar(B_PFULL + pb));
-        if (more && !sent && !fetch_send(j + 1, cur)) { ok = false; break; }
+        mbar_arrive(bar(B_PFULL));
         ++j;
       }
       if (!ok) break;
@@ -479,26 +570,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         nx.next();
         if (nx.valid() && !load_q(nx.b)) { ok = false; break; }
       }
-      // piece epilogue: O / l for this CTA's 256 columns (+ lse from CTA 0)
+      // piece epilogue: O / l for this half's 128 of this CTA's 256 columns (+ lse from CTA 0)
+      const float lt = l + swap_half(l, 2);          // both halves' sums
+      if (lt != lt) { ok = false; break; }
       const int jl = j - 1;
       const float m_log2 = m_ref * c2;
-      if (!wait_u(bar(B_PVDONE + (jl & 1)), (jl >> 1) & 1)) { ok = false; break; }
+      if (!wait_u(bar(B_PVDONE), jl & 1)) { ok = false; break; }
       tc_fence_after();
       const int64_t t = (int64_t)b * p.tq + k;
       const int32_t nseg = p.slot_base[b + 1] - p.slot_base[b];
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float lse_v = l > 0.f ? (m_log2 + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float lse_v = lt > 0.f ? (m_log2 + log2f(lt)) * 0.69314718055994531f : -INFINITY;
       float* po = nullptr;
       if (nseg > 1) {
         const int64_t slot = (int64_t)p.slot_base[b] + (pair - (int)(((int64_t)(ts_b + 1) * npairs - 1) / NT));
         const int64_t row = ((int64_t)k * p.s_max + slot) * H + i;
         po = p.part_o + row * DC + 256 * r;
-        if (r == 0) p.part_lse[row] = lse_v;
-      } else if (r == 0) {
+        if (r == 0 && half == 0) p.part_lse[row] = lse_v;
+      } else if (r == 0 && half == 0) {
         p.lse[t * H + i] = lse_v;
       }
 #pragma unroll 1
-      for (int c = 0; c < 256; c += 32) {
+      for (int c = 128 * half; c < 128 * half + 128; c += 32) {
         uint32_t v[32];
         tmem_ld32(trow + c, v);
         tmem_wait_ld();

@@ -262,30 +262,36 @@ struct ReduceParams {
   uint32_t* err;
 };
 
-// Sums the split-K partials of feature pairs (f, f+1) in split order, then applies the epilogue.
+// Sums the split-K partials of feature pairs (f, f+1), then applies the epilogue. One group of L lanes
+// (L a power of two >= splits, at most 32) per (token, feature pair): lane l adds partials l, l + L, ...
+// in order, then the group adds its lanes by a fixed xor tree, so the result does not depend on timing.
+template <int L>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constant__ ReduceParams p) {
-  const int64_t f = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
-  const int64_t t = blockIdx.y;
-  if (f >= p.f_total) return;
+  const int64_t npairs = p.f_total / 2;
+  const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / L;
+  const int l = threadIdx.x & (L - 1);
+  const bool active = gid < npairs * p.T;
+  const int64_t t = active ? gid / npairs : 0;
+  const int64_t f = active ? 2 * (gid % npairs) : 0;
+  float a = 0.f, b = 0.f;
+  if (active) {
+    const float* src = p.partial + t * p.f_total + f;
+    const int64_t kstride = p.T * p.f_total;
+    for (int k = l; k < p.splits; k += L) {
+      const float2 v = *reinterpret_cast<const float2*>(src + (int64_t)k * kstride);
+      a += v.x;
+      b += v.y;
+    }
+  }
+#pragma unroll
+  for (int o = L / 2; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  if (!active || l != 0) return;
   const int s = (p.nseg > 1 && f >= p.seg[1].f_base) ? 1 : 0;
   const TcEpiSeg& E = p.seg[s];
   const int64_t fl = f - E.f_base;
-  // eight independent partial sums (loads in flight together), combined in a fixed order
-  float pa[8] = {}, pb[8] = {};
-  const float* src = p.partial + t * p.f_total + f;
-  const int64_t kstride = p.T * p.f_total;
-  for (int k0 = 0; k0 < p.splits; k0 += 8) {
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (k0 + u < p.splits) {
-        const float2 v = *reinterpret_cast<const float2*>(src + (int64_t)(k0 + u) * kstride);
-        pa[u] += v.x;
-        pb[u] += v.y;
-      }
-    }
-  }
-  float a = ((pa[0] + pa[1]) + (pa[2] + pa[3])) + ((pa[4] + pa[5]) + (pa[6] + pa[7]));
-  float b = ((pb[0] + pb[1]) + (pb[2] + pb[3])) + ((pb[4] + pb[5]) + (pb[6] + pb[7]));
   if (E.rope) {
     const int64_t ps = p.pos[t];
     if (ps < 0) {
@@ -374,15 +380,26 @@ int swap_bn(int64_t T) { return T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128
 // split decision uses this fixed count so that workspace sizing and launches always agree.
 int swap_slots(int BN) { return BN <= 64 ? 2 * 148 : 148; }
 
-// Split-K factor for a swap-orientation launch of `ctas` output tiles over kb_total k-blocks:
-// as many splits as fit the CTA slots in one wave; returns (splits, k-blocks per split).
+// Split-K factor for a swap-orientation launch of `ctas` output tiles over kb_total k-blocks on
+// `slots` resident CTAs: going up from 1, a factor is taken when it cuts the k-blocks the busiest
+// CTA streams (ceil(items / slots) * ceil(kb_total / splits)) by at least 10% against the best so
+// far (more splits also mean more fp32 partials to write and sum), with at least four k-blocks
+// (256 of K) per split. Returns (splits, k-blocks per split).
 void choose_splits(int64_t ctas, int kb_total, int slots, int* splits_out, int* kbps_out) {
-  int splits = (int)(slots / ctas);
-  const int max_splits = kb_total / 4;   // at least four k-blocks (256 of K) per split
-  splits = splits < max_splits ? splits : max_splits;
-  splits = splits < kMaxSplits ? splits : kMaxSplits;
-  splits = splits < 1 ? 1 : splits;
-  const int kbps = (kb_total + splits - 1) / splits;
+  int max_splits = kb_total / 4;
+  max_splits = max_splits < kMaxSplits ? max_splits : kMaxSplits;
+  int best = 1;
+  int64_t best_load = ((ctas + slots - 1) / slots) * (int64_t)kb_total;
+  for (int sp = 2; sp <= max_splits; ++sp) {
+    const int kbps = (kb_total + sp - 1) / sp;
+    const int real = (kb_total + kbps - 1) / kbps;
+    const int64_t load = ((ctas * real + slots - 1) / slots) * (int64_t)kbps;
+    if (load * 10 < best_load * 9) {
+      best_load = load;
+      best = real;
+    }
+  }
+  const int kbps = (kb_total + best - 1) / best;
   *splits_out = (kb_total + kbps - 1) / kbps;
   *kbps_out = kbps;
 }
@@ -393,7 +410,6 @@ size_t tc_gemm_partial_bytes(int64_t T, int64_t f_tiles, int64_t f_total, int64_
   if (T <= 0 || T > 256 || batch != 1) return 0;
   const int64_t ctas = f_tiles * ((T + swap_bn(T) - 1) / swap_bn(T));
   const int slots = swap_slots(swap_bn(T));
-  if (2 * ctas > slots) return 0;
   int splits, kbps;
   choose_splits(ctas, (int)(K / BK), slots, &splits, &kbps);
   return splits > 1 ? (size_t)splits * T * f_total * sizeof(float) : 0;
@@ -429,7 +445,7 @@ cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st) {
   p.splits = 1;
   p.kb_per_split = p.kb_total;
   const int64_t ctas = (int64_t)wtiles * ttiles * g.batch;
-  if (swap && g.batch == 1 && 2 * ctas <= swap_slots(BN) && g.partial) {
+  if (swap && g.batch == 1 && g.partial) {
     int splits, kbps;
     choose_splits(ctas, p.kb_total, swap_slots(BN), &splits, &kbps);
     if ((size_t)splits * g.T * f_total * sizeof(float) <= g.partial_bytes && splits > 1) {
@@ -481,8 +497,17 @@ cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st) {
   r.d_r = g.d_r;
   memcpy(r.theta, p.theta, sizeof(r.theta));
   r.err = g.err;
-  dim3 rg((unsigned)((f_total / 2 + 255) / 256), (unsigned)g.T);
-  splitk_reduce_kernel<<<rg, 256, 0, st>>>(r);
+  int L = 2;
+  while (L < p.splits && L < 32) L <<= 1;
+  const int64_t threads = (f_total / 2) * g.T * L;
+  const unsigned rg = (unsigned)((threads + 255) / 256);
+  switch (L) {
+    case 2: splitk_reduce_kernel<2><<<rg, 256, 0, st>>>(r); break;
+    case 4: splitk_reduce_kernel<4><<<rg, 256, 0, st>>>(r); break;
+    case 8: splitk_reduce_kernel<8><<<rg, 256, 0, st>>>(r); break;
+    case 16: splitk_reduce_kernel<16><<<rg, 256, 0, st>>>(r); break;
+    default: splitk_reduce_kernel<32><<<rg, 256, 0, st>>>(r); break;
+  }
   note_launch();
   return cudaGetLastError();
 }

@@ -36,9 +36,12 @@ TcGemmDesc desc(const TcMatrix& x, int64_t T, int64_t K, uint32_t* err) {
 int64_t tiles128(int64_t n) { return (n + 127) / 128; }
 
 size_t decode_gemm_partials(const mla_dims_t& d, int64_t T) {
+  const int64_t HD = (int64_t)d.n_h * d.d_h, HR = (int64_t)d.n_h * d.d_r;
   const size_t a = tc_gemm_partial_bytes(T, tiles128(d.d_cq), d.d_cq, d.d, 1);                      // W^DQ
-  const size_t b = tc_gemm_partial_bytes(T, tiles128(d.d), d.d, (int64_t)d.n_h * d.d_h, 1);         // W^O
-  return align_up(a > b ? a : b);
+  const size_t b = tc_gemm_partial_bytes(T, tiles128(HD) + tiles128(HR), HD + HR, d.d_cq, 1);       // [W^UQ; W^QR]
+  const size_t c = tc_gemm_partial_bytes(T, tiles128(d.d), d.d, HD, 1);                             // W^O
+  const size_t ab = a > b ? a : b;
+  return align_up(ab > c ? ab : c);
 }
 
 // Steps (5) and (7) with the cache write: rows [c^KV | RoPE(W^KR h)] -> cache[rowmap[t]].
