@@ -21,6 +21,7 @@ constexpr int BK = 64;           // k-block: one 128-byte swizzle row of bf16
 constexpr int kThreads = 192;    // warp 0: TMA producer, warp 1: TMEM owner + MMA issuer, warps 2-5: epilogue
 constexpr int kMaxSplits = 64;
 constexpr int kMaxRopePairs = 64;
+constexpr int kRasterW = 8;      // weight tiles per raster group (large token counts)
 
 struct GemmParams {
   CUtensorMap wmap[2];
@@ -113,10 +114,22 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
   };
   auto decode_tile = [&](int idx) {
     Tile d;
-    d.tt = idx % p.ttiles;
-    int rest = idx / p.ttiles;
-    int wt = rest % p.wtiles;
-    rest /= p.wtiles;
+    int wt, rest;
+    if (!SWAP) {
+      // large token counts: groups of kRasterW weight tiles x all token tiles, weight tile fastest,
+      // so the CTAs running at the same time share a few weight tiles and a few token tiles in L2
+      // (one batch, one split on this path)
+      const int group = idx / (kRasterW * p.ttiles), local = idx % (kRasterW * p.ttiles);
+      const int gw = min(kRasterW, p.wtiles - group * kRasterW);
+      wt = group * kRasterW + local % gw;
+      d.tt = local / gw;
+      rest = 0;
+    } else {
+      d.tt = idx % p.ttiles;
+      rest = idx / p.ttiles;
+      wt = rest % p.wtiles;
+      rest /= p.wtiles;
+    }
     d.z = rest / p.splits;
     d.split = rest % p.splits;
     d.s = 0;
@@ -212,6 +225,37 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
         if (CH == 32) tmem_ld32(trow + c, v);
         else tmem_ld16(trow + c, v);
         tmem_wait_ld();
+        if (!SWAP && CH == 32) {
+          // a token row's 32 consecutive features: bf16, 16-byte stores, when the layout allows
+          const int64_t t = t0 + r, f = f0 + c;
+          if (p.splits == 1 && !E.rowmap && !E.out_f32 && E.so_f == 1 && d.z == 0 && f + 32 <= E.f_rows &&
+              t < p.T && ((t * E.so_t + f) & 7) == 0 && (reinterpret_cast<uintptr_t>(E.out) & 15) == 0) {
+            int64_t ps = 0;
+            if (E.rope) {
+              ps = p.pos[t];
+              if (ps < 0) {
+                flag_error(p.err, DEVERR_POSITION);
+                continue;
+              }
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float a = __uint_as_float(v[j]), b2 = __uint_as_float(v[j + 1]);
+              if (E.rope) {
+                const float a2 = rope_one(f + j, ps, a, b2, p.d_r, p.theta);
+                const float b3 = rope_one(f + j + 1, ps, b2, a, p.d_r, p.theta);
+                a = a2;
+                b2 = b3;
+              }
+              pk[j / 2] = pack_bf16(a, b2);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(E.out) + t * E.so_t + f);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            continue;
+          }
+        }
 #pragma unroll
         for (int j = 0; j < CH; ++j) {
           const float x = __uint_as_float(v[j]);
