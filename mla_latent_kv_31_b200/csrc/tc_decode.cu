@@ -401,14 +401,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto wait_u = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(b, par)) != 0; };
     auto wait_uc = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait_cluster(b, par)) != 0; };
     int gq = 0, j = 0, tph = 0;
-    // one exchange of a value per head with the other half of this quarter: returns the partner's
-    auto swap_half = [&](float x, int slot) -> float {
+    // one exchange of a value per head with the other half of this quarter: the partner's value in
+    // y; false if the wait gave up
+    auto swap_half = [&](float x, int slot, float& y) -> bool {
       redbuf[(slot * 2 + half) * 128 + i] = x;
       mbar_arrive(tmax_bar);
       const bool okw = wait_u(tmax_bar, tph & 1);
       ++tph;
-      const float y = redbuf[(slot * 2 + (half ^ 1)) * 128 + i];
-      return okw ? y : NAN;
+      y = redbuf[(slot * 2 + (half ^ 1)) * 128 + i];
+      return okw;
     };
     // q~ half -> TMEM (this half's 64 columns) and q^R half -> shared memory (64-byte swizzle, this
     // half's two chunks) for the piece of sequence bq, once the previous piece's last QK^T is done.
@@ -493,8 +494,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int w2 = 8; w2 > 0; w2 >>= 1)
 #pragma unroll
           for (int c = 0; c < w2; ++c) mx[c] = fmaxf(mx[c], mx[c + w2]);
-        const float tmax = fmaxf(mx[0], swap_half(mx[0], j & 1));
-        if (tmax != tmax) { ok = false; break; }      // the partner half gave up (timeout)
+        float pmax;
+        if (!swap_half(mx[0], j & 1, pmax)) { ok = false; break; }
+        const float tmax = fmaxf(mx[0], pmax);
         // rows of this stage past the sequence end: zero the latent half before P.V reads it
         const int nrows = (int)max((int64_t)0, min((int64_t)NK, len - key0));
         if (nrows < NK) {
@@ -571,8 +573,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (nx.valid() && !load_q(nx.b)) { ok = false; break; }
       }
       // piece epilogue: O / l for this half's 128 of this CTA's 256 columns (+ lse from CTA 0)
-      const float lt = l + swap_half(l, 2);          // both halves' sums
-      if (lt != lt) { ok = false; break; }
+      float lp;
+      if (!swap_half(l, 2, lp)) { ok = false; break; }
+      const float lt = l + lp;                       // both halves' sums
       const int jl = j - 1;
       const float m_log2 = m_ref * c2;
       if (!wait_u(bar(B_PVDONE), jl & 1)) { ok = false; break; }
