@@ -103,6 +103,11 @@ struct CoreParams {
 
 __device__ __forceinline__ int32_t range_start(int64_t p, int64_t NT, int64_t P) { return (int32_t)(p * NT / P); }
 
+template <int V>
+struct IC {
+  static constexpr int value = V;
+};
+
 // The last sequence b in [0, B) with tile_start[b] <= x.
 __device__ __forceinline__ int find_seq(const int32_t* ts, int B, int32_t x) {
   int lo = 0, hi = B - 1;
@@ -260,12 +265,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const int st = cp.j % STAGES;
           const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
-          const uint32_t pa = sbase + OFF_P;
           const bool first = cp.first();
+          // descriptors advance by adding (byte offset >> 4) to the start-address field (bits 0-13,
+          // shared-memory addresses stay below 2^18): one add per MMA instead of a full encode
+          const uint64_t ap = sw128_desc(sbase + OFF_P, 0, 1024), bp = sw128_desc(kv, KV_BOX, 1024);
 #pragma unroll
           for (int kk = 0; kk < NK / 16; ++kk)
-            mma_bf16_ss(tmem, sw128_desc(pa + kk * 32, 0, 1024), sw128_desc(kv + kk * 2048, KV_BOX, 1024), idesc_pv,
-                        (first && kk == 0) ? 0u : 1u);
+            mma_bf16_ss(tmem, ap + (kk * 32 >> 4), bp + (kk * 2048 >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
           mma_commit(bar(B_PVDONE));
           mma_commit(bar(B_EMPTY + st));
           cp.advance();
@@ -280,16 +286,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
             const uint32_t d = tmem + T_S + NK * sb;
             // MMA m < 16: latent chunk m / 4, K step m % 4 (A from TMEM); m = 16, 17: the k^R half
-            // (A from shared memory)
-#pragma unroll
-            for (int mm = 0; mm < 9; ++mm) {
-              const int m = 9 * qk_half + mm;
+            // (A from shared memory). Descriptors: base + (byte offset >> 4), as for P.V.
+            const uint64_t bq = sw128_desc(kv, 0, 1024);
+            auto issue = [&](auto m_c) {
+              constexpr int m = decltype(m_c)::value;
               if (m < 16)
-                mma_bf16_ts(d, tmem + T_Q + 8 * m, sw128_desc(kv + (m >> 2) * KV_BOX + (m & 3) * 32, 0, 1024), idesc_qk,
+                mma_bf16_ts(d, tmem + T_Q + 8 * m, bq + (((m >> 2) * KV_BOX + (m & 3) * 32) >> 4), idesc_qk,
                             m ? 1u : 0u);
               else
-                mma_bf16_ss(d, sw64_desc(qr + (m - 16) * 32, 512), sw64_desc(kv + 4 * KV_BOX + (m - 16) * 32, 512),
-                            idesc_qk, 1u);
+                mma_bf16_ss(d, sw64_desc(qr, 512) + (((m - 16) * 32) >> 4),
+                            sw64_desc(kv + 4 * KV_BOX, 512) + (((m - 16) * 32) >> 4), idesc_qk, 1u);
+            };
+            if (qk_half == 0) {
+              issue(IC<0>{}); issue(IC<1>{}); issue(IC<2>{}); issue(IC<3>{}); issue(IC<4>{});
+              issue(IC<5>{}); issue(IC<6>{}); issue(IC<7>{}); issue(IC<8>{});
+            } else {
+              issue(IC<9>{}); issue(IC<10>{}); issue(IC<11>{}); issue(IC<12>{}); issue(IC<13>{});
+              issue(IC<14>{}); issue(IC<15>{}); issue(IC<16>{}); issue(IC<17>{});
             }
             if (qk_half == 1) {
               mma_commit(bar(B_SFULL + sb));

@@ -191,14 +191,13 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
           if (!mbar_wait(bar(B_FULL + st), (it / STAGES) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_addr(sA + st * A_BYTES), b_base = smem_addr(sB + st * B_BYTES);
+          // base descriptors, advanced by (byte offset >> 4) in the start-address field per K step
+          const uint64_t ad0 = (SWAP && W_MN) ? sw128_desc(a_base, 8192, 1024) : sw128_desc(a_base, 0, 1024);
+          const uint64_t bd0 = (!SWAP && W_MN) ? sw128_desc(b_base, 8192, 1024) : sw128_desc(b_base, 0, 1024);
+          constexpr uint32_t a_step = ((SWAP && W_MN) ? 2048 : 32) >> 4, b_step = ((!SWAP && W_MN) ? 2048 : 32) >> 4;
 #pragma unroll
-          for (int j = 0; j < BK / 16; ++j) {
-            const uint64_t ad = (SWAP && W_MN) ? sw128_desc(a_base + j * 2048, 8192, 1024)
-                                               : sw128_desc(a_base + j * 32, 0, 1024);
-            const uint64_t bd = (!SWAP && W_MN) ? sw128_desc(b_base + j * 2048, 8192, 1024)
-                                                : sw128_desc(b_base + j * 32, 0, 1024);
-            mma_bf16_ss(dt, ad, bd, idesc, (i > 0 || j > 0) ? 1u : 0u);
-          }
+          for (int j = 0; j < BK / 16; ++j)
+            mma_bf16_ss(dt, ad0 + j * a_step, bd0 + j * b_step, idesc, (i > 0 || j > 0) ? 1u : 0u);
           mma_commit(bar(B_EMPTY + st));
         }
         if (!ok) break;

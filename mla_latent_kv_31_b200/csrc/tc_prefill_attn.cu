@@ -164,10 +164,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_kernel(const __grid_
         tc_fence_after();
         const uint32_t kst = sbase + OFF_K + ks * K_BYTES;
         const uint32_t d = tmem + BN * (JJ & 1);
+        // descriptors advance by adding (byte offset >> 4) to the start-address field (bits 0-13)
+        const uint64_t bk = sw128_desc(kst, 0, 1024);
 #pragma unroll
         for (int k = 0; k < DQK / 16; ++k)
-          mma_bf16_ts(d, tmem + T_Q + 8 * k, sw128_desc(kst + (k >> 2) * BOX + (k & 3) * 32, 0, 1024), idesc_qk,
-                      k ? 1u : 0u);
+          mma_bf16_ts(d, tmem + T_Q + 8 * k, bk + ((((k >> 2) * BOX) + (k & 3) * 32) >> 4), idesc_qk, k ? 1u : 0u);
         mma_commit(bar(B_SFULL + (JJ & 1)));
         mma_commit(bar(B_KEMPTY + ks));
         if (last) mma_commit(bar(B_QEMPTY));
@@ -190,10 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_kernel(const __grid_
           tc_fence_after();
           const uint32_t vst = sbase + OFF_V + vs * V_BYTES;
           const uint32_t pa = tmem + BN * (J & 1);
+          const uint64_t bv = sw128_desc(vst, BOX, 1024);
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
-            mma_bf16_ts(tmem + T_O, pa + 8 * kk, sw128_desc(vst + kk * 2048, BOX, 1024), idesc_pv,
-                        (n > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem + T_O, pa + 8 * kk, bv + (kk * 2048 >> 4), idesc_pv, (n > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(B_PVDONE));
           mma_commit(bar(B_VEMPTY + vs));
           ++jv;
