@@ -80,6 +80,25 @@ def recorded_traffic(kernel: str):
         return None
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity on one rank). Every rank must call
+    it at the same point. device: where the reduction tensor lives (the rank's GPU for NCCL, CPU for
+    gloo)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(world: int, units_per_rank: float, seconds_max: float) -> float:
+    """Units all ranks processed per second of the slowest rank (weak scaling: every rank does the
+    same amount of work on its own inputs)."""
+    return world * units_per_rank / seconds_max
+
+
 def workload_config():
     d = WORKLOAD.dims
     return {"workload": WORKLOAD.name, "batch": WORKLOAD.batch, "query_tokens_per_seq": WORKLOAD.tq,
@@ -187,11 +206,7 @@ def kernel_only_ms(fn, which, iters, warm, flush, world):
     finally:
         torch.cuda.synchronize()
         mla.mla_set_kernel_timing(False)
-    ms = torch.tensor([tot / iters], device=flush.device)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    return float(ms.item())
+    return max_over_ranks([tot / iters], flush.device)[0]
 
 
 def prefill_flops(dims, lens):
@@ -250,11 +265,7 @@ def run_prefill(args, m, dev, rank, world, flush, timed, peaks, peak_src):
     st = mla.mla_sync_status(h, device=dev.index)
     if st != 0:
         raise RuntimeError(f"device check failed after prefill timing: {mla.mla_status_string(st)}")
-    ms = torch.tensor([ms_full, ms_core], device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    ms_full, ms_core = (float(x) for x in ms.tolist())
+    ms_full, ms_core = max_over_ranks([ms_full, ms_core], dev)
     attn, proj = prefill_flops(dims, lens)
     sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -395,11 +406,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     st = mla.mla_sync_status(h, device=local_rank)
     if st != 0:
         raise RuntimeError(f"device check failed after timing: {mla.mla_status_string(st)}")
-    ms_step_max, ms_core_max, ms_e2e_max = ms_step, ms_core, ms_e2e
-    if world > 1:
-        t = torch.tensor([ms_step, ms_core, ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step_max, ms_core_max, ms_e2e_max = (float(x) for x in t.tolist())
+    ms_step_max, ms_core_max, ms_e2e_max = max_over_ranks([ms_step, ms_core, ms_e2e], dev)
     if rank != 0:
         return None
     cache_bytes = rows * ROW_BYTES
@@ -409,7 +416,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     kern_gbs = cache_bytes / (ms_kernel * 1e-3) / 1e9
     core_tflops = rows * tq * CORE_FLOP_PER_ROW / (ms_core_max * 1e-3) / 1e12
     step_bytes = cache_bytes + weight_bytes
-    value = world * cache_bytes / (ms_step_max * 1e-3) / 1e9
+    value = whole_job_rate(world, cache_bytes, ms_step_max * 1e-3) / 1e9
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step_max, 5), "higher_is_better": True, "scaling": "weak",
@@ -417,7 +424,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "N(0,1/fan_in) weights, DeepSeek-V3 sizes)",
         "config": dict(workload_config(), parallelism=f"replicas{world}", l2="flushed between steps (2x L2 write)",
                        step="mla_cache_append + mla_decode, CUDA-graph replay"),
-        "tokens_per_s": round(world * T / (ms_step_max * 1e-3), 1),
+        "tokens_per_s": round(whole_job_rate(world, T, ms_step_max * 1e-3), 1),
         "step_hbm_bytes": step_bytes,
         "step_roofline": {"bound": "hbm", "achieved": round(step_bytes / (ms_step_max * 1e-3) / 1e9, 1),
                           "peak": hbm, "unit": "GB/s", "frac": round(step_bytes / (ms_step_max * 1e-3) / 1e9 / hbm, 4),
@@ -429,7 +436,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      "kernel": "latent_core_kernel", "kernel_ms": round(ms_kernel, 5),
                      "timing": "CUDA events recorded by the library right around the kernel launch, L2 flushed",
                      "algorithmic_bytes": cache_bytes, "peak_source": peak_src},
-        "e2e": {"value": round(world * cache_bytes / (ms_e2e_max * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(whole_job_rate(world, cache_bytes, ms_e2e_max * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(ms_e2e_max, 5),
                 "h2d_bytes_per_step": int(h_np.size * 2 + pos_np.nbytes + slots_np.nbytes + cu_np.nbytes),
                 "d2h_bytes_per_step": int(T * dims.d * 2)},
