@@ -110,8 +110,33 @@ def test_calls_reject_bad_arguments_before_any_launch():
         with pytest.raises(mla.MLAError) as e:   # weights: misaligned pointer
             mla.mla_set_weights(h, {n: A + (2 if n == "w_o" else 0) for n in mla.WEIGHT_NAMES})
         assert e.value.status == 2
+        # prefill core alone: null k^C, capacity below the token count, max_seqlen 0, misaligned o
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_attn_prefill(h, A, A, None, A, 1, A, 64, 64, A, 64, A, stream=0)
+        assert e.value.status == 1
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_attn_prefill(h, A, A, A, A, 1, A, 64, 64, A, 63, A, stream=0)
+        assert e.value.status == 1
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_attn_prefill(h, A, A, A, A, 1, A, 64, 0, A, 64, A, stream=0)
+        assert e.value.status == 1
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_attn_prefill(h, A, A, A, A, 1, A, 64, 64, A, 64, A + 4, stream=0)
+        assert e.value.status == 2
     finally:
         mla.mla_destroy(h)
+
+
+def test_kernel_timing_calls_validate_without_a_launch():
+    mla.mla_set_kernel_timing(False)
+    for which in (-1, 2):
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_kernel_time_ms(which)
+        assert e.value.status == 1
+    # nothing has been bracketed in this process: no time to report
+    with pytest.raises(mla.MLAError) as e:
+        mla.mla_kernel_time_ms(mla.TIMED_PREFILL_CORE)
+    assert e.value.status == 1
 
 
 def test_tensor_core_routing_is_declared():
