@@ -133,7 +133,7 @@ mla_status_t mla_cache_append(mla_handle_t *h, const void *hidden, const int64_t
  * until the process exits.
  *   Same arguments, layouts and results as mla_cache_append, minus the workspace.
  *   Returns MLA_ERR_SCRATCH_LIMIT, before any launch, when the call would need more than
- *   4 MiB of scratch (at the DeepSeek-V3 sizes in bf16: 65 <= T <= 256 tokens; smaller and
+ *   4 MiB of scratch (at the DeepSeek-V3 sizes in bf16: 66 <= T <= 256 tokens; smaller and
  *   larger T need 4 MiB or less). MLA_ERR_NO_WEIGHTS if mla_set_weights() was not called.
  *   The first call on a device looks up the device address of the array (no allocation); make
  *   that first call outside any stream capture.
