@@ -78,7 +78,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-// ---- clusters (distributed shared memory; no multicast anywhere) ---------------------------
+// ---- clusters (distributed shared memory; every copy has a single destination) ------------
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
