@@ -29,6 +29,8 @@
  *     order, lengths, slots, positions) set a sticky error word in the handle and skip the
  *     offending rows; mla_sync_status() reports it.
  *   - Device pointers must be 16-byte aligned (MLA_ERR_ALIGNMENT otherwise).
+ *   - Calls make the handle's device current while they run and restore the calling thread's
+ *     current device before they return.
  *   - A handle may be used from several streams for different calls as long as calls that
  *     share a workspace or output buffer are ordered by the caller.
  */
@@ -94,7 +96,11 @@ typedef enum {
 typedef struct mla_handle mla_handle_t;
 
 /* Creates a handle for one device. Host-only: no CUDA call is made here.
- * dims must describe an MLA layer (all sizes > 0, d_r even); *out receives the handle. */
+ * dims must describe an MLA layer (all sizes > 0, d_r even); *out receives the handle.
+ * MLA_BF16 runs on the tcgen05/TMA kernels, which exist for the DeepSeek-V3 head layout only
+ * (n_h = 128, d_h = 128, d_c = 512, d_r = 64; d and d_cq multiples of 64): other BF16 sizes
+ * return MLA_ERR_UNSUPPORTED. MLA_FP32 runs on generic CUDA-core kernels at any sizes with
+ * d_c, d_h <= 512 (they exist for exact FP32 parity, not for speed). */
 mla_status_t mla_create(const mla_dims_t *dims, mla_dtype_t dtype, int device, mla_handle_t **out);
 
 /* Borrows the eight weight matrices (section 一(一)2 and 3). The first call on a device also
@@ -135,8 +141,10 @@ mla_status_t mla_cache_append(mla_handle_t *h, const void *hidden, const int64_t
  *   Returns MLA_ERR_SCRATCH_LIMIT, before any launch, when the call would need more than
  *   4 MiB of scratch (at the DeepSeek-V3 sizes in bf16: 66 <= T <= 256 tokens; smaller and
  *   larger T need 4 MiB or less). MLA_ERR_NO_WEIGHTS if mla_set_weights() was not called.
- *   The first call on a device looks up the device address of the array (no allocation); make
- *   that first call outside any stream capture.
+ *   The first call on a device looks up the device address of the array (no allocation) and
+ *   keeps it for the life of the process; make that first call outside any stream capture, and
+ *   do not reset the device (cudaDeviceReset) after it, since the address belongs to the
+ *   context that was current then.
  *   All calls share the one array and it keeps the last call's contents; nothing in it needs
  *   to start at zero, but calls that overlap on the GPU (different streams, no ordering)
  *   race on it. */
@@ -154,7 +162,7 @@ mla_status_t mla_cache_append_noalloc(mla_handle_t *h, const void *hidden, const
  *                                 cache rows cu[b] .. cu[b] + its position. len_b >= Tq.
  *   cache      [capacity, d_c + d_r]
  *   u_out      [B*Tq, d]          handle dtype
- * Tq is 1 or 2. */
+ * Tq is 1 or 2. Any B: the head-batched W^UK / W^UV projections run in chunks of 256 tokens. */
 mla_status_t mla_decode(mla_handle_t *h, const void *h_q, int64_t B, int32_t Tq,
                         const int64_t *cu_seqlens, const void *cache, int64_t capacity, void *u_out,
                         void *ws, size_t ws_bytes, mla_stream_t stream);

@@ -65,12 +65,29 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t elem_size(const mla_handle* h) { return h->dtype == MLA_BF16 ? 2 : 4; }
 
-// True when the tcgen05/TMA kernels cover this handle: BF16 at the DeepSeek-V3 sizes.
-bool tc_dims(const mla_handle* h) {
-  const mla_dims_t& d = h->dims;
-  return h->dtype == MLA_BF16 && d.n_h == 128 && d.d_h == 128 && d.d_c == 512 && d.d_r == 64 &&
-         d.d_cq % 64 == 0 && d.d % 64 == 0;
+// The sizes the tcgen05/TMA kernels are built for: the DeepSeek-V3 head layout, d and d_c'
+// multiples of 64. BF16 handles exist only at these sizes (mla_create).
+bool v3_dims(const mla_dims_t& d) {
+  return d.n_h == 128 && d.d_h == 128 && d.d_c == 512 && d.d_r == 64 && d.d_cq % 64 == 0 && d.d % 64 == 0;
 }
+
+// BF16 handles run on the tcgen05/TMA kernels; FP32 handles on the generic CUDA-core kernels.
+bool tc_dims(const mla_handle* h) { return h->dtype == MLA_BF16; }
+
+// Makes the handle's device current for the life of the guard and restores the caller's device
+// afterwards, so that no entry point changes the calling thread's current device.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int device) {
+    if (cudaGetDevice(&prev) != cudaSuccess) return;
+    ok = prev == device || cudaSetDevice(device) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
 
 struct Layout {
   size_t off[9];
@@ -130,8 +147,8 @@ mla_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA
     if (_e != cudaSuccess) return MLA_ERR_CUDA;    \
   } while (0)
 
+// Allocates the handle's error word on first use. The caller holds a DeviceGuard for h->device.
 mla_status_t ensure_device(mla_handle* h) {
-  MLA_TRY(cudaSetDevice(h->device));
   if (!h->d_err) {
     MLA_TRY(cudaMalloc(&h->d_err, sizeof(uint32_t)));
     MLA_TRY(cudaMemset(h->d_err, 0, sizeof(uint32_t)));
@@ -140,12 +157,6 @@ mla_status_t ensure_device(mla_handle* h) {
     h->num_sms = sms;
   }
   return MLA_OK;
-}
-
-mla_status_t check_ready(mla_handle* h) {
-  if (!h) return MLA_ERR_INVALID_ARG;
-  if (!h->has_weights) return MLA_ERR_NO_WEIGHTS;
-  return ensure_device(h);
 }
 
 // --- generic (CUDA-core) building blocks ----------------------------------------------------
@@ -167,9 +178,9 @@ SimtGemmArgs dense_nt(const void* A, int64_t lda, const void* W, void* C, int64_
   return a;
 }
 
-mla_status_t run_simt_gemm(const mla_handle* h, SimtGemmArgs a, cudaStream_t st, bool out_bf16) {
+mla_status_t run_simt_gemm(const mla_handle* h, SimtGemmArgs a, cudaStream_t st) {
   a.err = h->d_err;
-  return cuda_status(mla::simt_gemm(a, h->dtype == MLA_BF16, out_bf16, st));
+  return cuda_status(mla::simt_gemm(a, st));
 }
 
 // Steps (5), (7) + cache write: rows [c^KV | RoPE(W^KR h)] scattered to cache[rowmap[t]].
@@ -177,38 +188,36 @@ mla_status_t simt_cache_rows(const mla_handle* h, const void* hidden, const int6
                              int64_t T, void* cache, int64_t capacity, cudaStream_t st) {
   const mla_dims_t& d = h->dims;
   const size_t es = elem_size(h);
-  const bool bf = h->dtype == MLA_BF16;
   const int64_t R = d.d_c + d.d_r;
   SimtGemmArgs a = dense_nt(hidden, d.d, h->w.w_dkv, cache, R, T, d.d_c, d.d);
   a.rowmap = rowmap; a.rowmap_limit = capacity;
-  mla_status_t s = run_simt_gemm(h, a, st, bf);
+  mla_status_t s = run_simt_gemm(h, a, st);
   if (s != MLA_OK) return s;
   SimtGemmArgs b = dense_nt(hidden, d.d, h->w.w_kr, (char*)cache + (size_t)d.d_c * es, R, T, d.d_r, d.d);
   b.rowmap = rowmap; b.rowmap_limit = capacity;
   b.pos = pos; b.rope_col0 = 0; b.d_r = d.d_r; b.rope_base = d.rope_base;
-  return run_simt_gemm(h, b, st, bf);
+  return run_simt_gemm(h, b, st);
 }
 
 // Steps (1)-(3): c^Q, q^C and the rotated q^R of T tokens at positions pos.
 mla_status_t simt_queries(const mla_handle* h, const void* hidden, const int64_t* pos, int64_t T, void* cq,
                           void* qc, void* qr, cudaStream_t st) {
   const mla_dims_t& d = h->dims;
-  const bool bf = h->dtype == MLA_BF16;
-  mla_status_t s = run_simt_gemm(h, dense_nt(hidden, d.d, h->w.w_dq, cq, d.d_cq, T, d.d_cq, d.d), st, bf);
+  mla_status_t s = run_simt_gemm(h, dense_nt(hidden, d.d, h->w.w_dq, cq, d.d_cq, T, d.d_cq, d.d), st);
   if (s != MLA_OK) return s;
   s = run_simt_gemm(h, dense_nt(cq, d.d_cq, h->w.w_uq, qc, (int64_t)d.n_h * d.d_h, T, (int64_t)d.n_h * d.d_h,
-                                d.d_cq), st, bf);
+                                d.d_cq), st);
   if (s != MLA_OK) return s;
   SimtGemmArgs a = dense_nt(cq, d.d_cq, h->w.w_qr, qr, (int64_t)d.n_h * d.d_r, T, (int64_t)d.n_h * d.d_r, d.d_cq);
   a.pos = pos; a.rope_col0 = 0; a.d_r = d.d_r; a.rope_base = d.rope_base;
-  return run_simt_gemm(h, a, st, bf);
+  return run_simt_gemm(h, a, st);
 }
 
 // Step (10), second equation: u = W^O [o_1; ...; o_nh].
 mla_status_t simt_output(const mla_handle* h, const void* o, int64_t T, void* u, cudaStream_t st) {
   const mla_dims_t& d = h->dims;
   const int64_t HD = (int64_t)d.n_h * d.d_h;
-  return run_simt_gemm(h, dense_nt(o, HD, h->w.w_o, u, d.d, T, d.d, HD), st, h->dtype == MLA_BF16);
+  return run_simt_gemm(h, dense_nt(o, HD, h->w.w_o, u, d.d, T, d.d, HD), st);
 }
 
 // Latent attention core by CUDA cores: q~ [T, n_h, d_c], q^R [T, n_h, d_r] over the cache.
@@ -230,7 +239,8 @@ mla_status_t simt_latent_core(const mla_handle* h, const void* q_abs, const void
   a.cu = cu; a.B = B; a.tq = tq; a.T = B * tq; a.n_h = d.n_h; a.capacity = capacity;
   a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
   a.err = h->d_err;
-  return cuda_status(mla::simt_attention(a, h->dtype == MLA_BF16, o_f32, st));
+  (void)o_f32;
+  return cuda_status(mla::simt_attention(a, st));
 }
 
 }  // namespace
@@ -262,6 +272,8 @@ mla_status_t mla_create(const mla_dims_t* dims, mla_dtype_t dtype, int device, m
       !(d.rope_base > 1.0) || device < 0)
     return MLA_ERR_INVALID_ARG;
   if (dtype != MLA_BF16 && dtype != MLA_FP32) return MLA_ERR_INVALID_ARG;
+  // BF16 runs on the tcgen05 kernels, which are built for the DeepSeek-V3 head layout only.
+  if (dtype == MLA_BF16 && !v3_dims(d)) return MLA_ERR_UNSUPPORTED;
   // Generic kernels hold one latent row of q in shared memory and up to 512 value columns.
   if (d.d_c > 512 || d.d_h > 512 || d.d_c + d.d_r > 1024 || d.d_h + d.d_r > 1024) return MLA_ERR_UNSUPPORTED;
   mla_handle* h = new (std::nothrow) mla_handle;
@@ -281,6 +293,8 @@ mla_status_t mla_set_weights(mla_handle_t* h, const mla_weights_t* w) {
     if (!p) return MLA_ERR_INVALID_ARG;
     if (!aligned16(p)) return MLA_ERR_ALIGNMENT;
   }
+  DeviceGuard g(h->device);
+  if (!g.ok) return MLA_ERR_CUDA;
   mla_status_t s = ensure_device(h);
   if (s != MLA_OK) return s;
   h->w = *w;
@@ -314,8 +328,8 @@ mla_status_t mla_workspace_offset(const mla_handle_t* h, mla_op_t op, int64_t nu
 }
 
 int mla_uses_tensor_cores(const mla_handle_t* h, mla_op_t op) {
-  if (!h) return 0;
-  return tc_dims(h) && mla::tc_available(op) ? 1 : 0;
+  if (!h || op < MLA_OP_CACHE_APPEND || op > MLA_OP_ATTN_DECODE_LATENT) return 0;
+  return tc_dims(h) ? 1 : 0;
 }
 
 mla_status_t mla_cache_append(mla_handle_t* h, const void* hidden, const int64_t* positions, const int64_t* slots,
@@ -327,10 +341,13 @@ mla_status_t mla_cache_append(mla_handle_t* h, const void* hidden, const int64_t
     return MLA_ERR_ALIGNMENT;
   Layout L = layout(h, MLA_OP_CACHE_APPEND, 0, 1, T);
   if (ws_bytes < L.total || (L.total > 0 && !ws)) return MLA_ERR_WORKSPACE;
-  mla_status_t s = check_ready(h);
+  if (!h->has_weights) return MLA_ERR_NO_WEIGHTS;
+  DeviceGuard g(h->device);
+  if (!g.ok) return MLA_ERR_CUDA;
+  mla_status_t s = ensure_device(h);
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  if (tc_dims(h) && mla::tc_available(MLA_OP_CACHE_APPEND))
+  if (tc_dims(h))
     return cuda_status(mla::tc_cache_append(h->dims, h->w, hidden, positions, slots, T, cache, capacity,
                                             (char*)ws + L.tc_off, L.total - L.tc_off, h->d_err, st));
   return simt_cache_rows(h, hidden, positions, slots, T, cache, capacity, st);
@@ -347,14 +364,16 @@ mla_status_t mla_attn_decode_latent(mla_handle_t* h, const void* q_abs, const vo
     return MLA_ERR_ALIGNMENT;
   Layout L = layout(h, MLA_OP_ATTN_DECODE_LATENT, B, Tq, 0);
   if (ws_bytes < L.total || (L.total > 0 && !ws)) return MLA_ERR_WORKSPACE;
+  DeviceGuard g(h->device);
+  if (!g.ok) return MLA_ERR_CUDA;
   mla_status_t s = ensure_device(h);  // the core needs no weights
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   char* w = (char*)ws;
   MLA_TRY(mla::check_and_positions(cu_seqlens, B, Tq, B * Tq, capacity, 0, (int64_t*)(w + L.pos_off), h->d_err,
                                    st));
-  if (tc_dims(h) && mla::tc_available(MLA_OP_ATTN_DECODE_LATENT))
-    return cuda_status(mla::tc_latent_core(h->dims, q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, true,
+  if (tc_dims(h))
+    return cuda_status(mla::tc_latent_core_impl(q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, true,
                                            lse, w + L.tc_off, h->num_sms, h->d_err, st));
   return simt_latent_core(h, q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, true, lse, st);
 }
@@ -368,7 +387,10 @@ mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq,
     return MLA_ERR_ALIGNMENT;
   Layout L = layout(h, MLA_OP_DECODE, B, Tq, 0);
   if (ws_bytes < L.total) return MLA_ERR_WORKSPACE;
-  mla_status_t s = check_ready(h);
+  if (!h->has_weights) return MLA_ERR_NO_WEIGHTS;
+  DeviceGuard g(h->device);
+  if (!g.ok) return MLA_ERR_CUDA;
+  mla_status_t s = ensure_device(h);
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   const mla_dims_t& d = h->dims;
@@ -383,7 +405,7 @@ mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq,
   void* o = w + L.off[MLA_BUF_O];
   float* lse = (float*)(w + L.off[MLA_BUF_LSE]);
   MLA_TRY(mla::check_and_positions(cu_seqlens, B, Tq, T, capacity, 0, pos, h->d_err, st));
-  if (tc_dims(h) && mla::tc_available(MLA_OP_DECODE))
+  if (tc_dims(h))
     return cuda_status(mla::tc_decode(d, h->w, h_q, B, Tq, cu_seqlens, pos, cache, capacity, u_out, cq, qc, qr,
                                       qabs, olat, o, lse, w + L.tc_off, h->num_sms, h->d_err, st));
   // Steps (1)-(3)
@@ -395,7 +417,7 @@ mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq,
   a.B = h->w.w_uk; a.sbn = 1; a.sbk = d.d_c; a.sbb = (int64_t)d.d_h * d.d_c;
   a.C = qabs; a.scm = (int64_t)d.n_h * d.d_c; a.scn = 1; a.scb = d.d_c;
   a.M = T; a.N = d.d_c; a.K = d.d_h; a.batch = d.n_h;
-  s = run_simt_gemm(h, a, st, h->dtype == MLA_BF16);
+  s = run_simt_gemm(h, a, st);
   if (s != MLA_OK) return s;
   s = simt_latent_core(h, qabs, qr, B, Tq, cu_seqlens, cache, capacity, olat, h->dtype == MLA_FP32, lse, st);
   if (s != MLA_OK) return s;
@@ -405,7 +427,7 @@ mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq,
   v.B = h->w.w_uv; v.sbn = d.d_c; v.sbk = 1; v.sbb = (int64_t)d.d_h * d.d_c;
   v.C = o; v.scm = (int64_t)d.n_h * d.d_h; v.scn = 1; v.scb = d.d_h;
   v.M = T; v.N = d.d_h; v.K = d.d_c; v.batch = d.n_h;
-  s = run_simt_gemm(h, v, st, h->dtype == MLA_BF16);
+  s = run_simt_gemm(h, v, st);
   if (s != MLA_OK) return s;
   return simt_output(h, o, T, u_out, st);
 }
@@ -420,7 +442,10 @@ mla_status_t mla_prefill(mla_handle_t* h, const void* hidden, int64_t B, const i
     return MLA_ERR_ALIGNMENT;
   Layout L = layout(h, MLA_OP_PREFILL, B, 0, total_tokens);
   if (ws_bytes < L.total) return MLA_ERR_WORKSPACE;
-  mla_status_t s = check_ready(h);
+  if (!h->has_weights) return MLA_ERR_NO_WEIGHTS;
+  DeviceGuard g(h->device);
+  if (!g.ok) return MLA_ERR_CUDA;
+  mla_status_t s = ensure_device(h);
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   const mla_dims_t& d = h->dims;
@@ -435,18 +460,18 @@ mla_status_t mla_prefill(mla_handle_t* h, const void* hidden, int64_t B, const i
   void* kc = w + L.off[MLA_BUF_KC];
   void* vc = w + L.off[MLA_BUF_VC];
   MLA_TRY(mla::check_and_positions(cu_seqlens, B, 0, T, capacity, max_seqlen, pos, h->d_err, st));
-  if (tc_dims(h) && mla::tc_available(MLA_OP_PREFILL))
+  if (tc_dims(h))
     return cuda_status(mla::tc_prefill(d, h->w, hidden, B, cu_seqlens, T, max_seqlen, pos, cache, capacity, u_out,
-                                       cq, qc, qr, kc, vc, o, h->d_err, st));
+                                       cq, qc, qr, kc, vc, o, h->num_sms, h->d_err, st));
   // Steps (5), (7): cache rows of every token at row t (= cu[b] + position)
   s = simt_cache_rows(h, hidden, pos, nullptr, T, cache, capacity, st);
   if (s != MLA_OK) return s;
   s = simt_queries(h, hidden, pos, T, cq, qc, qr, st);
   if (s != MLA_OK) return s;
   // Steps (6), (9): k^C = W^UK c^KV, v^C = W^UV c^KV from the cache rows just written
-  s = run_simt_gemm(h, dense_nt(cache, R, h->w.w_uk, kc, HD, T, HD, d.d_c), st, h->dtype == MLA_BF16);
+  s = run_simt_gemm(h, dense_nt(cache, R, h->w.w_uk, kc, HD, T, HD, d.d_c), st);
   if (s != MLA_OK) return s;
-  s = run_simt_gemm(h, dense_nt(cache, R, h->w.w_uv, vc, HD, T, HD, d.d_c), st, h->dtype == MLA_BF16);
+  s = run_simt_gemm(h, dense_nt(cache, R, h->w.w_uv, vc, HD, T, HD, d.d_c), st);
   if (s != MLA_OK) return s;
   // Steps (4), (8), (10): causal attention per head with keys [k^C_i; k^R], values v^C_i
   SimtAttnArgs a;
@@ -461,7 +486,7 @@ mla_status_t mla_prefill(mla_handle_t* h, const void* hidden, int64_t B, const i
   a.cu = cu_seqlens; a.B = B; a.tq = 0; a.T = T; a.n_h = d.n_h; a.capacity = capacity;
   a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
   a.err = h->d_err;
-  MLA_TRY(mla::simt_attention(a, h->dtype == MLA_BF16, h->dtype == MLA_FP32, st));
+  MLA_TRY(mla::simt_attention(a, st));
   return simt_output(h, o, T, u_out, st);
 }
 
@@ -474,13 +499,15 @@ mla_status_t mla_attn_prefill(mla_handle_t* h, const void* q_c, const void* q_ro
   if (!aligned16(q_c) || !aligned16(q_rope) || !aligned16(k_c) || !aligned16(v_c) || !aligned16(cache) ||
       !aligned16(o) || !aligned16(cu_seqlens))
     return MLA_ERR_ALIGNMENT;
+  DeviceGuard g(h->device);
+  if (!g.ok) return MLA_ERR_CUDA;
   mla_status_t s = ensure_device(h);  // the core needs no weights
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   const mla_dims_t& d = h->dims;
   const int64_t T = total_tokens, R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
   MLA_TRY(mla::check_and_positions(cu_seqlens, B, 0, T, capacity, max_seqlen, nullptr, h->d_err, st));
-  if (tc_dims(h) && mla::tc_available(MLA_OP_PREFILL))
+  if (tc_dims(h))
     return cuda_status(mla::tc_prefill_attention(q_c, q_rope, k_c, v_c, cache, capacity, cu_seqlens, B, T, max_seqlen,
                                                  o, h->num_sms, h->d_err, st));
   SimtAttnArgs a;
@@ -495,13 +522,14 @@ mla_status_t mla_attn_prefill(mla_handle_t* h, const void* q_c, const void* q_ro
   a.cu = cu_seqlens; a.B = B; a.tq = 0; a.T = T; a.n_h = d.n_h; a.capacity = capacity;
   a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
   a.err = h->d_err;
-  return cuda_status(mla::simt_attention(a, h->dtype == MLA_BF16, h->dtype == MLA_FP32, st));
+  return cuda_status(mla::simt_attention(a, st));
 }
 
 mla_status_t mla_sync_status(mla_handle_t* h, mla_stream_t stream) {
   if (!h) return MLA_ERR_INVALID_ARG;
   if (!h->d_err) return MLA_OK;
-  MLA_TRY(cudaSetDevice(h->device));
+  DeviceGuard g(h->device);
+  if (!g.ok) return MLA_ERR_CUDA;
   MLA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
   uint32_t bits = 0;
   MLA_TRY(cudaMemcpy(&bits, h->d_err, sizeof(bits), cudaMemcpyDeviceToHost));
@@ -533,7 +561,7 @@ mla_status_t mla_kernel_time_ms(int which, float* ms) {
 void mla_destroy(mla_handle_t* h) {
   if (!h) return;
   if (h->d_err) {
-    cudaSetDevice(h->device);
+    DeviceGuard g(h->device);
     cudaFree(h->d_err);
   }
   delete h;
@@ -581,12 +609,13 @@ extern "C" mla_status_t mla_cache_append_noalloc(mla_handle_t* h, const void* hi
   if (!h->has_weights || !h->d_err) return MLA_ERR_NO_WEIGHTS;
   Layout L = layout(h, MLA_OP_CACHE_APPEND, 0, 1, T);
   if (L.total > kNoAllocScratchBytes) return MLA_ERR_SCRATCH_LIMIT;
-  MLA_TRY(cudaSetDevice(h->device));
+  DeviceGuard g(h->device);
+  if (!g.ok) return MLA_ERR_CUDA;
   void* scratch = nullptr;
   mla_status_t s = noalloc_scratch(h->device, &scratch);
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  if (tc_dims(h) && mla::tc_available(MLA_OP_CACHE_APPEND))
+  if (tc_dims(h))
     return cuda_status(mla::tc_cache_append(h->dims, h->w, hidden, positions, slots, T, cache, capacity,
                                             (char*)scratch + L.tc_off, L.total - L.tc_off, h->d_err, st));
   return simt_cache_rows(h, hidden, positions, slots, T, cache, capacity, st);

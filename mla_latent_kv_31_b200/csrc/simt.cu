@@ -186,24 +186,19 @@ __global__ void check_positions_kernel(const int64_t* cu, int64_t B, int32_t tq,
 
 }  // namespace
 
-cudaError_t simt_gemm(const SimtGemmArgs& a, bool in_bf16, bool out_bf16, cudaStream_t st) {
+cudaError_t simt_gemm(const SimtGemmArgs& a, cudaStream_t st) {
   if (a.M <= 0 || a.N <= 0) return cudaSuccess;
   dim3 grid((unsigned)((a.N + TN - 1) / TN), (unsigned)((a.M + TM - 1) / TM), (unsigned)a.batch);
-  if (in_bf16 && out_bf16) simt_gemm_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, st>>>(a);
-  else if (in_bf16) simt_gemm_kernel<__nv_bfloat16, float><<<grid, 256, 0, st>>>(a);
-  else if (out_bf16) simt_gemm_kernel<float, __nv_bfloat16><<<grid, 256, 0, st>>>(a);
-  else simt_gemm_kernel<float, float><<<grid, 256, 0, st>>>(a);
+  simt_gemm_kernel<float, float><<<grid, 256, 0, st>>>(a);
   note_launch();
   return cudaGetLastError();
 }
 
-cudaError_t simt_attention(const SimtAttnArgs& a, bool in_bf16, bool out_f32, cudaStream_t st) {
+cudaError_t simt_attention(const SimtAttnArgs& a, cudaStream_t st) {
   if (a.T <= 0) return cudaSuccess;
   if (a.dv > ATT_MAX_DV || a.d1 + a.d2 > ATT_MAX_Q) return cudaErrorInvalidValue;
   dim3 grid((unsigned)a.T, (unsigned)a.n_h);
-  if (in_bf16 && out_f32) simt_attention_kernel<__nv_bfloat16, float><<<grid, ATT_THREADS, 0, st>>>(a);
-  else if (in_bf16) simt_attention_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, ATT_THREADS, 0, st>>>(a);
-  else simt_attention_kernel<float, float><<<grid, ATT_THREADS, 0, st>>>(a);
+  simt_attention_kernel<float, float><<<grid, ATT_THREADS, 0, st>>>(a);
   note_launch();
   return cudaGetLastError();
 }

@@ -1,6 +1,6 @@
-// Generic CUDA-core kernels (any MLA sizes, fp32 or bf16 storage, fp32 arithmetic).
-// They serve the FP32 configuration, where tcgen05's tf32 rounding would miss a 1e-5 bound,
-// and any sizes the tensor-core kernels are not instantiated for.
+// Generic CUDA-core kernels (any MLA sizes, fp32 storage and arithmetic). They serve the FP32
+// configuration, where tcgen05's tf32 rounding would miss a 1e-5 bound. BF16 runs only on the
+// tcgen05 kernels (DeepSeek-V3 sizes); these kernels are not instantiated for it.
 #pragma once
 
 #include <stdint.h>
@@ -41,8 +41,8 @@ struct SimtAttnArgs {
   uint32_t* err;
 };
 
-cudaError_t simt_gemm(const SimtGemmArgs& a, bool in_bf16, bool out_bf16, cudaStream_t st);
-cudaError_t simt_attention(const SimtAttnArgs& a, bool in_bf16, bool out_f32, cudaStream_t st);
+cudaError_t simt_gemm(const SimtGemmArgs& a, cudaStream_t st);
+cudaError_t simt_attention(const SimtAttnArgs& a, cudaStream_t st);
 
 // Device-side checks of cu_seqlens; also writes per-token positions when pos_out != nullptr:
 // decode (tq > 0): pos = len_b - tq + k; prefill (tq == 0): pos = t - cu[b].

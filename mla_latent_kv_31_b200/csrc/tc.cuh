@@ -8,9 +8,6 @@
 
 namespace mla {
 
-// Whether this build routes `op` through the tensor-core kernels.
-bool tc_available(mla_op_t op);
-
 // Scratch bytes of the tensor-core decode path (split-K partials of the projections and the
 // split-KV partials of the latent core) for B sequences of tq query tokens.
 size_t tc_decode_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq);
@@ -23,10 +20,6 @@ cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const v
                             const int64_t* positions, const int64_t* slots, int64_t T, void* cache,
                             int64_t capacity, void* scratch, size_t scratch_bytes, uint32_t* err,
                             cudaStream_t st);
-
-cudaError_t tc_latent_core(const mla_dims_t& d, const void* q_abs, const void* q_rope, int64_t B, int32_t tq,
-                           const int64_t* cu, const void* cache, int64_t capacity, void* o_lat, bool o_f32,
-                           float* lse, void* scratch, int num_sms, uint32_t* err, cudaStream_t st);
 
 // The split-KV tcgen05 latent core (q~, q^R -> o^lat, lse); scratch of tc_core_scratch_bytes().
 cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
@@ -47,6 +40,6 @@ cudaError_t tc_prefill_attention(const void* qc, const void* qr, const void* kc,
 cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, int64_t B,
                        const int64_t* cu, int64_t T, int64_t max_seqlen, const int64_t* pos, void* cache,
                        int64_t capacity, void* u_out, void* cq, void* qc, void* qr, void* kc, void* vc, void* o,
-                       uint32_t* err, cudaStream_t st);
+                       int num_sms, uint32_t* err, cudaStream_t st);
 
 }  // namespace mla

@@ -450,7 +450,7 @@ void choose_splits(int64_t ctas, int kb_total, int slots, int* splits_out, int* 
 }  // namespace
 
 size_t tc_gemm_partial_bytes(int64_t T, int64_t f_tiles, int64_t f_total, int64_t K, int32_t batch) {
-  if (T <= 0 || T > 256 || batch != 1) return 0;
+  if (T <= 0 || T > kSwapMaxTokens || batch != 1) return 0;
   const int64_t ctas = f_tiles * ((T + swap_bn(T) - 1) / swap_bn(T));
   const int slots = swap_slots(swap_bn(T));
   int splits, kbps;
@@ -461,8 +461,9 @@ size_t tc_gemm_partial_bytes(int64_t T, int64_t f_tiles, int64_t f_total, int64_
 cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st) {
   if (g.T <= 0) return cudaSuccess;
   if (g.K % BK != 0 || g.nseg < 1 || g.nseg > 2 || g.d_r > 2 * kMaxRopePairs) return cudaErrorInvalidValue;
-  const bool swap = g.T <= 256;
-  if (g.w_mn && !swap) return cudaErrorInvalidValue;
+  const bool swap = g.T <= kSwapMaxTokens;
+  // head batching and MN-major weights exist only in the swap orientation
+  if ((g.w_mn || g.batch != 1) && !swap) return cudaErrorInvalidValue;
   const int BN = swap ? swap_bn(g.T) : 256;
   const int w_tile = swap ? 128 : BN, x_tile = swap ? BN : 128;
   GemmParams p;

@@ -16,6 +16,10 @@
 
 namespace mla {
 
+// Largest token count of the weight-streaming ("swap") orientation; head-batched and MN-major weight
+// launches exist only in that orientation, so their callers split larger token counts into chunks.
+constexpr int64_t kSwapMaxTokens = 256;
+
 struct TcMatrix {       // row-major bf16 matrix [rows, cols] with a row stride in elements
   const void* ptr;
   int64_t rows, cols, ld;

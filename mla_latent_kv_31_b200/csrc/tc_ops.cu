@@ -103,11 +103,6 @@ cudaError_t output(const mla_dims_t& d, const mla_weights_t& w, const void* o, i
 
 }  // namespace
 
-bool tc_available(mla_op_t op) {
-  (void)op;
-  return true;
-}
-
 size_t tc_decode_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq) {
   return decode_gemm_partials(d, B * tq) + align_up(tc_core_scratch_bytes(d, B, tq));
 }
@@ -123,51 +118,49 @@ cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const v
   return cache_rows(d, w, hidden, positions, slots, T, cache, capacity, scratch, scratch_bytes, err, st);
 }
 
-cudaError_t tc_latent_core(const mla_dims_t& d, const void* q_abs, const void* q_rope, int64_t B, int32_t tq,
-                           const int64_t* cu, const void* cache, int64_t capacity, void* o_lat, bool o_f32,
-                           float* lse, void* scratch, int num_sms, uint32_t* err, cudaStream_t st) {
-  (void)d;
-  return tc_latent_core_impl(q_abs, q_rope, B, tq, cu, cache, capacity, o_lat, o_f32, lse, scratch, num_sms, err,
-                             st);
-}
-
 cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const void* h_q, int64_t B, int32_t tq,
                       const int64_t* cu, const int64_t* pos, const void* cache, int64_t capacity, void* u_out,
                       void* cq, void* qc, void* qr, void* qabs, void* olat, void* o, float* lse, void* scratch,
                       int num_sms, uint32_t* err, cudaStream_t st) {
-  const int64_t T = B * tq, HD = (int64_t)d.n_h * d.d_h;
+  const int64_t T = B * tq, HD = (int64_t)d.n_h * d.d_h, HC = (int64_t)d.n_h * d.d_c;
   const size_t part_bytes = decode_gemm_partials(d, T);
   void* core_scratch = (char*)scratch + part_bytes;
   cudaError_t e = queries(d, w, h_q, pos, T, cq, qc, qr, scratch, part_bytes, err, st);
   if (e != cudaSuccess) return e;
-  // q~_i = W_i^UK^T q^C_i for every head i: the weight operand is W^UK read MN-major.
-  TcGemmDesc a = desc(mat(qc, T, HD, HD), T, d.d_h, err);
-  a.nseg = 1;
-  a.w_mn = true;
-  a.seg[0].w = mat(w.w_uk, HD, d.d_c, d.d_c);
-  a.seg[0].epi = epi(qabs, (int64_t)d.n_h * d.d_c, 1, d.d_c);
-  a.seg[0].epi.so_z = d.d_c;
-  a.batch = d.n_h; a.w_row_z = d.d_h; a.x_col_z = d.d_h;
-  e = tc_gemm(a, st);
+  // q~_i = W_i^UK^T q^C_i for every head i: the weight operand is W^UK read MN-major. The
+  // head-batched GEMM streams weights with the tokens on the MMA's N side, so it runs on chunks of
+  // at most kSwapMaxTokens tokens.
+  for (int64_t t0 = 0; t0 < T; t0 += kSwapMaxTokens) {
+    const int64_t n = T - t0 < kSwapMaxTokens ? T - t0 : kSwapMaxTokens;
+    TcGemmDesc a = desc(mat((const char*)qc + (size_t)t0 * HD * 2, n, HD, HD), n, d.d_h, err);
+    a.nseg = 1;
+    a.w_mn = true;
+    a.seg[0].w = mat(w.w_uk, HD, d.d_c, d.d_c);
+    a.seg[0].epi = epi((char*)qabs + (size_t)t0 * HC * 2, HC, 1, d.d_c);
+    a.seg[0].epi.so_z = d.d_c;
+    a.batch = d.n_h; a.w_row_z = d.d_h; a.x_col_z = d.d_h;
+    if ((e = tc_gemm(a, st)) != cudaSuccess) return e;
+  }
+  e = tc_latent_core_impl(qabs, qr, B, tq, cu, cache, capacity, olat, false, lse, core_scratch, num_sms, err, st);
   if (e != cudaSuccess) return e;
-  e = tc_latent_core(d, qabs, qr, B, tq, cu, cache, capacity, olat, false, lse, core_scratch, num_sms, err, st);
-  if (e != cudaSuccess) return e;
-  // o_i = W_i^UV o^lat_i for every head i.
-  TcGemmDesc v = desc(mat(olat, T, (int64_t)d.n_h * d.d_c, (int64_t)d.n_h * d.d_c), T, d.d_c, err);
-  v.nseg = 1;
-  v.seg[0].w = mat(w.w_uv, HD, d.d_c, d.d_c);
-  v.seg[0].epi = epi(o, HD, 1, d.d_h);
-  v.seg[0].epi.so_z = d.d_h;
-  v.batch = d.n_h; v.w_row_z = d.d_h; v.x_col_z = d.d_c;
-  e = tc_gemm(v, st);
-  if (e != cudaSuccess) return e;
+  // o_i = W_i^UV o^lat_i for every head i, in the same token chunks.
+  for (int64_t t0 = 0; t0 < T; t0 += kSwapMaxTokens) {
+    const int64_t n = T - t0 < kSwapMaxTokens ? T - t0 : kSwapMaxTokens;
+    TcGemmDesc v = desc(mat((const char*)olat + (size_t)t0 * HC * 2, n, HC, HC), n, d.d_c, err);
+    v.nseg = 1;
+    v.seg[0].w = mat(w.w_uv, HD, d.d_c, d.d_c);
+    v.seg[0].epi = epi((char*)o + (size_t)t0 * HD * 2, HD, 1, d.d_h);
+    v.seg[0].epi.so_z = d.d_h;
+    v.batch = d.n_h; v.w_row_z = d.d_h; v.x_col_z = d.d_c;
+    if ((e = tc_gemm(v, st)) != cudaSuccess) return e;
+  }
   return output(d, w, o, T, u_out, scratch, part_bytes, err, st);
 }
 
 cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, int64_t B,
                        const int64_t* cu, int64_t T, int64_t max_seqlen, const int64_t* pos, void* cache,
                        int64_t capacity, void* u_out, void* cq, void* qc, void* qr, void* kc, void* vc, void* o,
-                       uint32_t* err, cudaStream_t st) {
+                       int num_sms, uint32_t* err, cudaStream_t st) {
   const int64_t R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
   cudaError_t e = cache_rows(d, w, hidden, pos, nullptr, T, cache, capacity, nullptr, 0, err, st);
   if (e != cudaSuccess) return e;
@@ -183,10 +176,7 @@ cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* 
   e = tc_gemm(p3, st);
   if (e != cudaSuccess) return e;
   // Steps (4), (8), (10): causal attention per head, keys [k^C_i; k^R], values v^C_i.
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  e = tc_prefill_attention(qc, qr, kc, vc, cache, capacity, cu, B, T, max_seqlen, o, sms > 0 ? sms : 148, err, st);
+  e = tc_prefill_attention(qc, qr, kc, vc, cache, capacity, cu, B, T, max_seqlen, o, num_sms, err, st);
   if (e != cudaSuccess) return e;
   return output(d, w, o, T, u_out, nullptr, 0, err, st);
 }

@@ -111,6 +111,52 @@ def normal(seed: int, tensor_id: int, shape, std: float = 1.0, dtype: str = "bf1
     return out.reshape(shape)
 
 
+def _signed(x: int) -> int:
+    return x - (1 << 64) if x >= (1 << 63) else x
+
+
+def normal_torch(seed: int, tensor_id: int, shape, std: float = 1.0, dtype: str = "bf16", device="cpu"):
+    """The same draws as normal(), computed with torch on `device` (a GPU fills large synthetic caches in
+    milliseconds). uint64 arithmetic is done on int64 tensors: two's-complement products and sums wrap
+    exactly like uint64, and a logical right shift is an arithmetic shift with the sign bits masked off.
+    Returns a torch tensor of the dtype ('bf16' -> bfloat16, 'fp32' -> float32)."""
+    import torch
+    n = int(np.prod(shape))
+    key = torch.tensor(_signed(int(stream_key(seed, tensor_id))), dtype=torch.int64, device=device)
+    gamma = _signed(int(_GAMMA))
+    m1, m2 = _signed(int(_M1)), _signed(int(_M2))
+
+    def shr(z, k):
+        return (z >> k) & ((1 << (64 - k)) - 1)
+
+    def mix(z):
+        z = (z ^ shr(z, 30)) * m1
+        z = (z ^ shr(z, 27)) * m2
+        return z ^ shr(z, 31)
+
+    def uniform(c):
+        return shr(mix(key + (c + 1) * gamma), 11).to(torch.float64) * (2.0 ** -53)
+
+    out = torch.empty(n, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32, device=device)
+    step = 1 << 24
+    for lo in range(0, n, step):
+        hi = min(n, lo + step)
+        idx = torch.arange(lo, hi, dtype=torch.int64, device=device)
+        a = uniform(2 * idx)
+        b = uniform(2 * idx + 1)
+        x = torch.sqrt(-2.0 * torch.log1p(-a)) * torch.cos(2.0 * np.pi * b) * std
+        out[lo:hi] = x.to(torch.float32).to(out.dtype)
+    return out.reshape(shape)
+
+
+def latent_cache_torch(dims: "Dims", rows: int, seed: int = 0, dtype: str = "bf16", device="cpu"):
+    """latent_cache() drawn with torch on `device`: [rows, d_c + d_r], c^KV then k^R, each ~ N(0,1)."""
+    import torch
+    c = normal_torch(seed, TID_CACHE_C, (rows, dims.d_c), dtype=dtype, device=device)
+    kr = normal_torch(seed, TID_CACHE_KR, (rows, dims.d_r), dtype=dtype, device=device)
+    return torch.cat([c, kr], dim=1)
+
+
 @dataclass(frozen=True)
 class Dims:
     """MLA dimensions in the notes' symbols: d, n_h, d_h, d_c, d_c' (d_cq), d_h^R (d_r)."""

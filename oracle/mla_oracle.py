@@ -296,6 +296,40 @@ def mla_decode_absorbed(h_q, cache, cu_seqlens, tq, W, dims, seqs=None):
             "q_r": q_r, "q_c": q_c}
 
 
+def mla_prefill_absorbed(h, cu_seqlens, W, dims, query_rows, cache=None):
+    """Prefill outputs of the given query rows (global token indices) in the absorbed form.
+
+    The same exact rewrite as mla_decode_absorbed (section 2 【思考】), applied to prefill: the
+    cache rows of every token come from steps (5) and (7) (or `cache`, if the caller already has
+    them), each query row t at position p attends over its own sequence's rows 0..p through
+    q~ = W_i^UK^T q^C_i, and o = W_i^UV o^lat, u = W^O [o_1; ...; o_n_h] follow. The tests pin it
+    to mla_prefill to 1e-12; it costs O(d_c) per key instead of O(n_h d_h d_c) per cached row, so
+    u of a few rows of a 32K-token prefill can be checked on the host.
+    """
+    h = f64(h)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    T = h.shape[0]
+    pos = np.concatenate([np.arange(cu[b + 1] - cu[b]) for b in range(len(cu) - 1)]).astype(np.int64)
+    if cache is None:
+        c_kv, k_r = kv_compression(h, W, dims, pos)
+        cache = cache_rows(c_kv, k_r)
+    rows = np.sort(np.asarray(query_rows, dtype=np.int64))
+    _, q_c, q_r = query_projections(h[rows], W, dims, pos[rows])
+    q_abs = absorb_query(q_c, W, dims)
+    scale = 1.0 / np.sqrt(dims.d_h + dims.d_r)
+    o_lat = np.empty((len(rows), dims.n_h, dims.d_c))
+    lse = np.empty((len(rows), dims.n_h))
+    for n, t in enumerate(rows):
+        b = int(np.searchsorted(cu, t, side="right") - 1)
+        seq = f64(cache[cu[b]:t + 1])                    # the row's own sequence, keys 0..p
+        for i in range(dims.n_h):
+            q = np.concatenate([q_abs[n, i], f64(q_r[n, i])])[None, :]
+            lat, _, l, _ = causal_softmax_attend(q, seq, seq[:, :dims.d_c], None, np.array([t - cu[b]]), scale)
+            o_lat[n, i], lse[n, i] = lat[0], l[0]
+    o = value_up_projection(o_lat, W, dims)
+    return {"rows": rows, "cache": cache, "o_lat": o_lat, "lse": lse, "o": o, "u": output_projection(o, W)}
+
+
 def output_absorbed(o_lat, W, dims) -> np.ndarray:
     """u_t = sum_i W_i^O' o^lat_t,i with W_i^O' = W_i^O W_i^UV (section 2 【思考】, second absorption)."""
     w_o = f64(W["w_o"]).reshape(-1, dims.n_h, dims.d_h)          # [d, n_h, d_h]

@@ -59,6 +59,13 @@ def _decode_step(mod, W, name, sample):
     u_h = host(u)
     assert np.all(np.isfinite(u_h))
     assert rel(u_h[ref["rows"]], ref["u"]) <= TOL["bf16"]
+    # the latent core's own outputs for the sampled sequences (o^lat is stored as bf16 in the
+    # decode workspace, lse as fp32), before W^UV and W^O average over heads and columns
+    rows = mod.torch.from_numpy(ref["rows"]).to("cuda:0")
+    olat = mod.region(mla.OP_DECODE, mla.BUF_OLAT, (T, dims.n_h, dims.d_c), mod.torch.bfloat16, B, tq)
+    lse = mod.region(mla.OP_DECODE, mla.BUF_LSE, (T, dims.n_h), mod.torch.float32, B, tq)
+    assert rel(host(olat[rows]), ref["o_lat"]) <= TOL["bf16"]
+    assert rel(host(lse[rows]), ref["lse"]) <= TOL["bf16"]
 
 
 def test_decode_b16_l4096_full(mod, w0):
@@ -92,4 +99,9 @@ def test_prefill_l32768_full(mod, w0):
     o = mod.region(mla.OP_PREFILL, mla.BUF_O, (T, dims.n_h, dims.d_h), mod.torch.bfloat16, 1, 1, T)
     got = host(o[dev_i64(ref["rows"])][:, heads])
     assert rel(got, ref["o"]) <= TOL["bf16"]
-    assert np.all(np.isfinite(host(u[dev_i64(ref["rows"])])))
+    # u = W^O [o_1; ...; o_n_h] of the sampled rows over all heads: the tile-orientation W^O launch
+    # (28 weight tiles, raster groups 8/8/8/4) against the absorbed oracle on the same cache rows
+    ab = orc.mla_prefill_absorbed(h, cu, w0, dims, rows, cache=ref["cache"])
+    u_h = host(u)
+    assert np.all(np.isfinite(u_h))
+    assert rel(u_h[ab["rows"]], ab["u"]) <= TOL["bf16"]

@@ -191,6 +191,50 @@ def test_v3_prefill_bf16_two_sequences(v3_module, v3_weights):
     assert rel(host(u), ref["u"]) <= TOL["bf16"]
 
 
+def test_v3_prefill_bf16_three_sequences_past_the_swap_size(v3_module, v3_weights):
+    # T = 1129 > 256 tokens: every projection takes the tile orientation (128 tokens x 256 features),
+    # the token tiles straddle sequence starts, and RoPE takes each token's own position
+    dims = synth.V3
+    lens = [700, 300, 129]
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    h = synth.hidden(dims, T, seed=41, dtype="bf16")
+    ref = orc.mla_prefill(h, cu, v3_weights, dims)
+    cache = dev(np.zeros((T, dims.row)), "bf16")
+    u = v3_module.prefill(dev(h, "bf16"), 3, dev_i64(cu), max(lens), cache)
+    _status_ok(v3_module)
+    assert rel(host(cache), ref["cache"]) <= TOL["bf16"]
+    o = v3_module.region(mla.OP_PREFILL, mla.BUF_O, (T, dims.n_h, dims.d_h), v3_module.torch.bfloat16, 3, 1, T)
+    assert rel(host(o), ref["o"]) <= TOL["bf16"]
+    assert rel(host(u), ref["u"]) <= TOL["bf16"]
+
+
+def test_v3_decode_bf16_more_than_256_query_tokens(v3_module, v3_weights):
+    # B * Tq = 300 query tokens: the head-batched W^UK / W^UV projections run in chunks of at most
+    # 256 tokens, the other projections in the tile orientation
+    dims = synth.V3
+    tq = 2
+    lens = synth.ragged_lengths(150, tq, 90, seed=5)
+    cu = synth.cu_seqlens(lens)
+    B, T = len(lens), len(lens) * tq
+    cache = synth.latent_cache(dims, int(cu[-1]), seed=60, dtype="bf16")
+    h_q = synth.hidden(dims, T, seed=61, dtype="bf16")
+    seqs = [0, 1, 74, 127, 128, 149]
+    ref = orc.mla_decode_absorbed(h_q, cache, cu, tq, v3_weights, dims, seqs=seqs)
+    u = v3_module.decode(dev(h_q, "bf16"), B, tq, dev_i64(cu), dev(cache, "bf16"))
+    _status_ok(v3_module)
+    rows = v3_module.torch.from_numpy(ref["rows"]).to("cuda:0")
+    bf = v3_module.torch.bfloat16
+    qabs = v3_module.region(mla.OP_DECODE, mla.BUF_QABS, (T, dims.n_h, dims.d_c), bf, B, tq)
+    olat = v3_module.region(mla.OP_DECODE, mla.BUF_OLAT, (T, dims.n_h, dims.d_c), bf, B, tq)
+    o = v3_module.region(mla.OP_DECODE, mla.BUF_O, (T, dims.n_h, dims.d_h), bf, B, tq)
+    assert rel(host(qabs[rows]), ref["q_abs"]) <= TOL["bf16"]
+    assert rel(host(olat[rows]), ref["o_lat"]) <= TOL["bf16"]
+    assert rel(host(o[rows]), ref["o"]) <= TOL["bf16"]
+    assert rel(host(u)[ref["rows"]], ref["u"]) <= TOL["bf16"]
+    assert np.all(np.isfinite(host(u)))
+
+
 # ---------------------------------------------------------------------------
 # Device-side checks and determinism
 # ---------------------------------------------------------------------------

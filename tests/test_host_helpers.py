@@ -39,3 +39,13 @@ def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     assert bench.recorded_traffic("other") is None
     src.write_text("// kernel, changed\n")
     assert bench.recorded_traffic("k") is None
+
+
+def test_torch_draws_equal_numpy_draws():
+    # the benchmark fills its large caches with the torch form of the same generator
+    for dt in ("bf16", "fp32"):
+        a = synth.normal(5, synth.TID_CACHE_KR, (300, 77), std=1.5, dtype=dt)
+        b = synth.normal_torch(5, synth.TID_CACHE_KR, (300, 77), std=1.5, dtype=dt).float().numpy()
+        assert np.array_equal(a, b)
+    c = synth.latent_cache_torch(synth.TINY, 50, seed=2).float().numpy()
+    assert np.array_equal(c, synth.latent_cache(synth.TINY, 50, seed=2))

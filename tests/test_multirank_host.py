@@ -38,7 +38,7 @@ def _rank_main(rank, world, port, out):
 def test_two_gloo_ranks_reduce_timings_to_the_max_and_draw_their_own_inputs():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)

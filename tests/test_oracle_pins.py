@@ -73,9 +73,72 @@ def test_absorbed_core_matches_unabsorbed_prefill():
         assert _rel(lse[0], pre["lse"][t]) < 1e-12
 
 
+@pytest.mark.parametrize("dims", [synth.TINY, SMALL])
+def test_prefill_absorbed_equals_unabsorbed(dims):
+    W = _weights(dims, seed=13)
+    lens = [23, 1, 40]
+    cu = synth.cu_seqlens(lens)
+    h = synth.hidden(dims, int(cu[-1]), seed=14, dtype="fp32")
+    rows = [0, 5, 22, 23, 24, 40, 63]
+    un = orc.mla_prefill(h, cu, W, dims, query_rows=rows)
+    ab = orc.mla_prefill_absorbed(h, cu, W, dims, rows)
+    assert np.array_equal(ab["rows"], un["rows"])
+    for key in ("o_lat", "lse", "o", "u"):
+        assert _rel(ab[key], un[key]) < 1e-12, key
+    assert _rel(ab["cache"], un["cache"]) < 1e-15
+    # handing it the cache rows gives the same result
+    ab2 = orc.mla_prefill_absorbed(h, cu, W, dims, rows, cache=un["cache"])
+    assert _rel(ab2["u"], un["u"]) < 1e-12
+
+
 # ---------------------------------------------------------------------------
 # Softmax / single key / causality (section 一(一)1: Softmax_j over j = 1..t)
 # ---------------------------------------------------------------------------
+def test_lse_of_a_single_key_is_its_score():
+    # one visible key: the log of a one-term sum is that term's scaled score, written out here
+    # as q.k / sqrt(d_h + d_h^R) over the concatenated [q^C; q^R] and [k^C; k^R]
+    dims = synth.TINY
+    W = _weights(dims, seed=24)
+    h = synth.hidden(dims, 1, seed=25, dtype="fp32")
+    out = orc.mla_prefill(h, synth.cu_seqlens([1]), W, dims)
+    h64 = np.asarray(h[0], np.float64)
+    c_q = np.asarray(W["w_dq"], np.float64) @ h64
+    c_kv = np.asarray(W["w_dkv"], np.float64) @ h64
+    q_r = np.asarray(W["w_qr"], np.float64) @ c_q       # position 0: RoPE is the identity
+    k_r = np.asarray(W["w_kr"], np.float64) @ h64
+    for i in range(dims.n_h):
+        rows = slice(i * dims.d_h, (i + 1) * dims.d_h)
+        q_c = np.asarray(W["w_uq"], np.float64)[rows] @ c_q
+        k_c = np.asarray(W["w_uk"], np.float64)[rows] @ c_kv
+        s = (q_c @ k_c + q_r[i * dims.d_r:(i + 1) * dims.d_r] @ k_r) / math.sqrt(dims.d_h + dims.d_r)
+        assert abs(out["lse"][0, i] - s) <= 1e-12 * max(1.0, abs(s))
+
+
+def test_lse_equals_torch_logsumexp_of_the_scores():
+    # lse against torch.logsumexp over the causal scores formed explicitly in torch (float64)
+    dims = synth.TINY
+    W = _weights(dims, seed=26)
+    T = 20
+    h = synth.hidden(dims, T, seed=27, dtype="fp32")
+    ref = orc.mla_prefill(h, synth.cu_seqlens([T]), W, dims)
+    h64 = torch.tensor(np.asarray(h, np.float64))
+    Wt = {k: torch.tensor(np.asarray(v, np.float64)) for k, v in W.items()}
+    c_q = h64 @ Wt["w_dq"].T
+    c_kv = h64 @ Wt["w_dkv"].T
+    q_c = (c_q @ Wt["w_uq"].T).reshape(T, dims.n_h, dims.d_h)
+    k_c = (c_kv @ Wt["w_uk"].T).reshape(T, dims.n_h, dims.d_h)
+    pos = np.arange(T)
+    q_r = torch.tensor(orc.rope((c_q @ Wt["w_qr"].T).reshape(T, dims.n_h, dims.d_r).numpy(), pos[:, None],
+                                dims.rope_base))
+    k_r = torch.tensor(orc.rope((h64 @ Wt["w_kr"].T).numpy(), pos, dims.rope_base))
+    s = (torch.einsum("thd,jhd->htj", q_c, k_c) + torch.einsum("thd,jd->htj", q_r, k_r)) / math.sqrt(
+        dims.d_h + dims.d_r)
+    s = s.masked_fill(torch.triu(torch.ones(T, T, dtype=torch.bool), 1), float("-inf"))
+    lse = torch.logsumexp(s, dim=-1).transpose(0, 1).numpy()
+    assert _rel(ref["lse"], lse) < 1e-13
+
+
+
 def test_softmax_rows_sum_to_one():
     rng = np.random.default_rng(0)
     q = rng.standard_normal((3, 10))
