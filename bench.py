@@ -404,7 +404,9 @@ def decode_config_leg(args, m, wl, dev, rank, world, flush, timed, peaks, peak_s
         mla.mla_attn_decode_latent(h, ws_dec.data_ptr() + off_qabs, ws_dec.data_ptr() + off_qr, B, tq, cu_dev, cache,
                                    rows, o_lat, lse, ws_core, n_core, device=dev.index)
 
+    l0 = mla.mla_kernel_launches()
     step()
+    launches = mla.mla_kernel_launches() - l0
     torch.cuda.synchronize()
     st = mla.mla_sync_status(h, device=dev.index)
     if st != 0:
@@ -413,10 +415,6 @@ def decode_config_leg(args, m, wl, dev, rank, world, flush, timed, peaks, peak_s
     with torch.cuda.graph(g, capture_error_mode="relaxed"):
         step()
     iters = max(5, min(args.steps, 50))
-    l0 = mla.mla_kernel_launches()
-    g.replay()
-    torch.cuda.synchronize()
-    launches = mla.mla_kernel_launches() - l0
     ms_step = timed(g.replay, iters, 3)
     del g
     ms_kernel = kernel_only_ms(core, mla.TIMED_LATENT_CORE, iters, 2, flush, world)

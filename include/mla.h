@@ -227,6 +227,14 @@ int mla_uses_tensor_cores(const mla_handle_t *h, mla_op_t op);
 mla_status_t mla_set_kernel_timing(int enabled);
 mla_status_t mla_kernel_time_ms(int which, float *ms);
 
+/* Test hook for the bounded device-side waits (no counterpart on the pages). Arms the next launch
+ * of the decode latent core in this process (mla_attn_decode_latent or mla_decode, any handle) so
+ * that its first cluster waits for a cache tile that is never loaded, with a 20 ms wait limit
+ * instead of 1 s. Every role of that launch gives up after its limit and returns; the launch
+ * writes garbage outputs, and mla_sync_status() reports MLA_ERR_TIMEOUT. Nothing faults or hangs,
+ * and later calls run normally. Not thread-safe: arm it only while no other thread launches. */
+void mla_test_arm_stall(void);
+
 const char *mla_status_string(mla_status_t s);
 
 /* Frees the handle's own device memory (its error word). Borrowed tensors are untouched. */

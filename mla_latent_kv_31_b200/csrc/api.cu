@@ -544,6 +544,8 @@ uint32_t mla_device_error_bits(const mla_handle_t* h) { return h ? h->last_err_b
 
 uint64_t mla_kernel_launches(void) { return mla::g_launches.load(std::memory_order_relaxed); }
 
+void mla_test_arm_stall(void) { mla::tc_latent_core_arm_stall(); }
+
 mla_status_t mla_set_kernel_timing(int enabled) {
   mla::g_timing.store(enabled != 0, std::memory_order_relaxed);
   return MLA_OK;

@@ -21,6 +21,11 @@ cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const v
                             int64_t capacity, void* scratch, size_t scratch_bytes, uint32_t* err,
                             cudaStream_t st);
 
+// Test hook: the next latent-core launch in this process waits on a barrier that nothing signals
+// (the first cluster's first cache box is never loaded), with a 20 ms wait limit, so that its
+// bounded waits give up and the launch reports a timeout.
+void tc_latent_core_arm_stall();
+
 // The split-KV tcgen05 latent core (q~, q^R -> o^lat, lse); scratch of tc_core_scratch_bytes().
 cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
                                 const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse,

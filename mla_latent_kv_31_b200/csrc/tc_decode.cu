@@ -6,29 +6,29 @@
 //   s_j = (q~_t,i . c_j + q^R_t,i . k^R_j) / sqrt(d_h + d_h^R),  j <= pos_t,
 //   o^lat_t,i = sum_j softmax(s)_j c_j,   lse_t,i = log sum_j exp(s_j).
 //
-// Work split. Each sequence's cache rows form tiles of 64 keys; all tiles of all sequences are
-// cut into equal contiguous ranges, one per CTA pair (a 2-CTA cluster); a pair whose range
-// crosses a sequence boundary emits one partial result per sequence piece, and a final pass
-// merges the pieces of a sequence exactly (log-sum-exp). Within a pair, CTA r owns latent
-// columns [256 r, 256 r + 256) and k^R columns [32 r, 32 r + 32): it streams only those 288
-// columns of every cache row, computes the partial score over them, swaps the 128 x 64 partial
-// (as fp16) with its peer through distributed shared memory, and then both run the same softmax
-// and accumulate P . c into their own 256 TMEM columns of O. The 128 heads form the MMA M
-// dimension; one TMA-loaded cache tile is read K-major by QK^T and MN-major by P.V.
+// Work split. Each sequence's cache rows form tiles of 128 keys; all tiles of all sequences are
+// cut into equal contiguous ranges, one per 2-CTA cluster; a cluster whose range crosses a
+// sequence boundary emits one partial result per sequence piece, and a final pass merges the
+// pieces of a sequence exactly (log-sum-exp).
 //
-// Pipelining. Scores are double-buffered in TMEM and the peer's partials in shared memory, so QK^T
-// of tile j + 1 and the copy of its partial run while the softmax works on tile j; P.V of tile j
-// reads P from shared memory, which the softmax of tile j + 1 rewrites once that P.V is done.
-// Sending this CTA's partial scores to the peer has warps of its own: they read a tile's partial out
-// of TMEM as soon as QK^T is done, stage it in shared memory and copy it in bulk to the peer, while
-// the softmax warps work on the tile before it; the softmax adds the peer's partial to its own.
+// Roles inside a cluster. The 128 heads are the MMA's M rows, and O = P.C for 128 heads and 512
+// latent columns fills the whole TMEM (512 columns of fp32) of one SM, so a cluster pairs:
+//   * the score CTA (rank 0): q~ in TMEM (256 columns of bf16 pairs, the A operand), two
+//     128 x 128 fp32 score buffers; QK^T over the 576 cache columns (32 TS MMAs over the latent
+//     part, 4 SS MMAs over k^R with q^R in shared memory), N = 128 keys; the softmax (lazy
+//     rescale of the running max); P (bf16) plus per-head rescale factors go to the value CTA as
+//     one bulk shared-to-shared copy per tile;
+//   * the value CTA (rank 1): O in all 512 TMEM columns; per tile 16 SS MMAs (N = 256 latent
+//     columns, K = 16 keys) read P and the latent columns of the cache tile, which this CTA loads
+//     itself (the second read of the tile hits L2); it rescales O when the score CTA's running max
+//     moved, and writes o^lat at the end of each sequence piece.
+// The score CTA's tensor work per tile is 36 MMAs at N = 128 (about 2300 cycles), the value CTA's
+// 16 MMAs at N = 256 (about 2050), so the two stay busy together. Data flows one way (P), so the
+// two CTAs pipeline freely: two P buffers on the value side, two staging buffers on the score
+// side.
 //
-// Roles per CTA (448 threads): warps 0-3 and 10-13 softmax/epilogue (two warps per TMEM lane
-// quarter, thread = head = TMEM lane, one warp per half of a tile's keys), warp 4 TMA producer,
-// warp 5 TMEM owner + MMA issuer, warps 6-9 send this CTA's partial scores (warp w on TMEM lanes
-// 32 (w % 4) + [0, 32)). Every wait is bounded.
+// Every wait is bounded (a timeout sets the error word and the role returns).
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <string.h>
 
 #include "sm100.cuh"
@@ -41,73 +41,95 @@ namespace {
 using namespace sm100;
 
 constexpr int H = 128, DC = 512, DR = 64, ROW = DC + DR;
-constexpr int NK = 64;                       // keys per tile (the N of QK^T, the K of P.V)
-// Partial scores cross to the peer CTA as fp16; both CTAs add the same two fp16-rounded halves, so
-// they see identical scores (relative rounding 2^-11 per half, far inside the bf16 error budget).
-// Half the bytes of fp32 leave room for two receive buffers and four cache stages.
-constexpr bool kXHalf = true;
-constexpr int STAGES = 4;
-constexpr int kThreads = 448;
+constexpr int NK = 128;                        // keys per tile
+constexpr int kThreads = 384;
 constexpr int kMaxPairs = 74;
-constexpr float kRescaleLog2 = 8.f;          // lazy rescale: keep the running max until it grows by 2^8
+constexpr float kRescaleLog2 = 8.f;            // keep the running max until it grows by 2^8
 
-constexpr uint32_t KV_BOX = NK * 128;        // [64 keys x 64 latent cols] bf16, 128-byte swizzle: 8 KB
-constexpr uint32_t R_BOX = NK * 64;          // [64 keys x 32 k^R cols] bf16, 64-byte swizzle: 4 KB
-constexpr uint32_t STAGE_BYTES = 4 * KV_BOX + R_BOX;   // 36 KB
-constexpr uint32_t XE = kXHalf ? 2 : 4;      // bytes per exchanged score
-constexpr uint32_t X_BYTES = H * NK * XE;    // [128 x 64] partial scores: 32 KB (fp32) / 16 KB (fp16)
-constexpr int XPER = 16 / XE;                // scores per 16-byte chunk
-constexpr int XCH = NK / XPER;               // 16-byte chunks per head
-constexpr uint32_t P_BYTES = H * NK * 2;     // [128 x 64] bf16 probabilities, K-major, 128-byte swizzle
-constexpr uint32_t QR_BYTES = H * 32 * 2;    // [128 x 32] bf16 q^R half, K-major, 64-byte swizzle
-constexpr uint32_t OFF_KV = 0;
-constexpr uint32_t OFF_X = OFF_KV + STAGES * STAGE_BYTES;
-constexpr uint32_t OFF_XO = OFF_X + 2 * X_BYTES;  // two receive buffers, then this CTA's staged partial
-constexpr uint32_t OFF_P = OFF_XO + X_BYTES;
-constexpr uint32_t OFF_QR = OFF_P + P_BYTES;
-constexpr uint32_t OFF_RED = OFF_QR + QR_BYTES;   // per-head maxima / sums swapped between softmax halves
-constexpr uint32_t OFF_BAR = OFF_RED + 3 * 2 * H * 4;
-static_assert(STAGE_BYTES % 1024 == 0 && OFF_P % 1024 == 0 && OFF_QR % 1024 == 0, "swizzle atom alignment");
+// score CTA: ring of [128 keys x 64 columns] boxes (8 latent + 1 k^R per tile)
+constexpr uint32_t BOX = NK * 128;             // 16 KB, 128-byte swizzle, K-major rows of 64 bf16
+constexpr int S_BOXES = 9;
+constexpr int S_RING = 8;
+constexpr uint32_t P_BYTES = H * NK * 2;       // P [128 heads x 128 keys] bf16, K-major SW128: 2 blocks of 16 KB
+constexpr uint32_t HDR_BYTES = 2 * H * 4;      // alpha[128], inv_l[128]
+constexpr uint32_t PMSG = P_BYTES + HDR_BYTES; // one P message: 33 KB
+constexpr uint32_t QR_BYTES = H * DR * 2;      // q^R [128 x 64] bf16, K-major SW128
+// value CTA: ring of [64 keys x 256 columns] groups (4 boxes of [64 keys x 64 columns])
+constexpr uint32_t VBOX = 64 * 128;            // 8 KB
+constexpr uint32_t VGRP = 4 * VBOX;            // 32 KB
+constexpr int V_RING = 4;                      // one tile: (N-half, key-half) = 4 groups
 
-// barrier indices
-constexpr int B_FULL = 0, B_EMPTY = STAGES, B_SFULL = 2 * STAGES, B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2,
-              B_PVDONE = B_PFULL + 1, B_XFULL = B_PVDONE + 1, B_XFREE = B_XFULL + 2, B_QFULL = B_XFREE + 2,
-              B_QEMPTY = B_QFULL + 1, B_OFREE = B_QEMPTY + 1, B_XOFREE = B_OFREE + 1, B_XORDY = B_XOFREE + 1,
-              B_TMAX = B_XORDY + 1;
-constexpr int NBAR = B_TMAX + 4;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
+// Shared memory, from a 1024-byte aligned base (the same layout offsets in both CTAs for the
+// barrier block, which the value CTA's multicast commits and remote arrivals rely on).
+constexpr uint32_t OFF_BAR = 0;
+constexpr uint32_t OFF_RED = 512;              // score CTA: per-head maxima / sums swapped between halves
+constexpr uint32_t S_OFF_RING = 4096;
+constexpr uint32_t S_OFF_QR = S_OFF_RING + S_RING * BOX;
+constexpr uint32_t S_OFF_STG = S_OFF_QR + QR_BYTES;
+constexpr uint32_t S_END = S_OFF_STG + 2 * PMSG;
+constexpr uint32_t V_OFF_PBUF = 4096;
+constexpr uint32_t V_OFF_RING = V_OFF_PBUF + 2 * PMSG;
+constexpr uint32_t V_END = V_OFF_RING + V_RING * VGRP;
+constexpr uint32_t SMEM_BYTES = (S_END > V_END ? S_END : V_END) + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(S_OFF_RING % 1024 == 0 && S_OFF_QR % 1024 == 0 && S_OFF_STG % 1024 == 0 && PMSG % 1024 == 0 &&
+                  V_OFF_RING % 1024 == 0,
+              "swizzle atom alignment");
+static_assert(OFF_RED + 3 * 2 * H * 4 <= S_OFF_RING, "reduction buffer");
 
-// TMEM columns: O half [0, 256); q~ half as bf16 pairs [256, 384) (the A operand of QK^T);
-// two score buffers S0 [384, 448), S1 [448, 512).
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t T_Q = 256, T_S = 384;
-static_assert(T_S + 2 * NK <= TMEM_COLS, "TMEM budget");
+// barrier indices (one numbering for both CTAs)
+enum : int {
+  B_PVD = 0,                          // [2] value CTA's P.V of the tile in P buffer b done (multicast to both)
+  B_SFULL = 2,                        // [S_RING] score CTA ring
+  B_SEMPTY = B_SFULL + S_RING,        // [S_RING]
+  B_SCF = B_SEMPTY + S_RING,          // [2] scores ready
+  B_SCE = B_SCF + 2,                  // [2] scores read (256 softmax threads)
+  B_QFULL = B_SCE + 2,                // q~ / q^R of a piece loaded (256)
+  B_QEMPTY = B_QFULL + 1,             // last QK^T of a piece done
+  B_PSTG = B_QEMPTY + 1,              // [2] P message staged (256)
+  B_STGF = B_PSTG + 2,                // [2] staging buffer free again (remote arrival of the value CTA)
+  B_TMAX = B_STGF + 2,                // [4] the two softmax warps of a TMEM lane quarter (64)
+  B_GFULL = B_TMAX + 4,               // [V_RING] value CTA ring
+  B_GEMPTY = B_GFULL + V_RING,        // [V_RING]
+  B_PFULL = B_GEMPTY + V_RING,        // [2] P message landed (bytes)
+  B_OREADY = B_PFULL + 2,             // [2] O rescaled for the tile / nothing to rescale (128)
+  B_OFREE = B_OREADY + 2,             // O read out by the piece epilogue (128)
+  NBAR = B_OFREE + 1
+};
+static_assert(NBAR * 8 + 16 <= OFF_RED, "barrier block");
 
 struct CoreParams {
-  CUtensorMap cmap;   // cache as [capacity, ROW], box {64, NK}, 128-byte swizzle (latent columns)
-  CUtensorMap rmap;   // cache as [capacity, ROW], box {32, NK}, 64-byte swizzle (k^R columns)
+  CUtensorMap kmap;   // cache as [capacity, ROW], box {64, 128}, 128-byte swizzle (score CTA)
+  CUtensorMap vmap;   // cache as [capacity, ROW], box {64, 64}, 128-byte swizzle (value CTA)
   const __nv_bfloat16* q_abs;   // [T][H][DC]
   const __nv_bfloat16* q_rope;  // [T][H][DR]
   const int64_t* cu;
-  const int32_t* tile_start;  // [B+1]: first global tile of each sequence
-  const int32_t* slot_base;   // [B+1]: first partial slot of each sequence
+  const int32_t* tile_start;    // [B+1]: first global tile of each sequence
+  const int32_t* slot_base;     // [B+1]: first partial slot of each sequence
   int32_t B, tq, pairs, s_max;
-  float* part_o;     // [tq][s_max][H][DC]
-  float* part_lse;   // [tq][s_max][H]
-  void* o_lat;       // [T][H][DC] (fp32 or bf16)
-  float* lse;        // [T][H]
-  float scale_log2;  // log2(e) / sqrt(d_h + d_h^R)
+  float* part_o;      // [tq][s_max][H][DC]
+  float* part_lse;    // [tq][s_max][H]
+  void* o_lat;        // [T][H][DC] (fp32 or bf16)
+  float* lse;         // [T][H]
+  float scale_log2;   // log2(e) / sqrt(d_h + d_h^R)
+  uint64_t wait_ns;   // bounded-wait limit
+  int32_t stall;      // test hook: the first cluster's score-side producer skips its first box
   uint32_t* err;
 };
 
 __device__ __forceinline__ int32_t range_start(int64_t p, int64_t NT, int64_t P) { return (int32_t)(p * NT / P); }
 
-template <int V>
-struct IC {
-  static constexpr int value = V;
-};
-
+// Bounded waits with the launch's limit.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint64_t limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > limit) return false;
+  }
+}
 // The last sequence b in [0, B) with tile_start[b] <= x.
 __device__ __forceinline__ int find_seq(const int32_t* ts, int B, int32_t x) {
   int lo = 0, hi = B - 1;
@@ -137,30 +159,6 @@ struct SegWalk {
   }
 };
 
-// Walks the tiles of a range one by one: j (tile count), g (piece count), first/last of a piece.
-struct TileCursor {
-  SegWalk w;
-  int32_t xt;
-  int j, g;
-  __device__ void init(const int32_t* ts, int B, int32_t x0, int32_t x1) {
-    w.init(ts, B, x0, x1);
-    xt = w.x;
-    j = 0;
-    g = 0;
-  }
-  __device__ bool valid() const { return w.valid(); }
-  __device__ bool first() const { return xt == w.x; }
-  __device__ bool last() const { return xt == w.seg_end() - 1; }
-  __device__ void advance() {
-    ++j;
-    if (++xt >= w.seg_end()) {
-      w.next();
-      ++g;
-      xt = w.x;
-    }
-  }
-};
-
 template <bool OUT_F32>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     latent_core_kernel(const __grid_constant__ CoreParams p) {
@@ -169,45 +167,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
   const uint32_t sbase = smem_addr(smem);
-  auto bar = [&](int i) { return smem_addr(&bars[i]); };
+  auto bar = [&](int i) { return sbase + OFF_BAR + 8u * (uint32_t)i; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t r = cluster_rank();
-  const uint32_t peer = r ^ 1u;
   const int k = blockIdx.y;                          // query token within the sequence window
   const int pair = blockIdx.x >> 1;
   const int64_t NT = p.tile_start[p.B];
-  // Active pairs: never more than tiles, so that every active range holds at least one tile.
-  const int64_t npairs = NT < p.pairs ? NT : p.pairs;
+  const int64_t npairs = NT < p.pairs ? NT : p.pairs;   // every active pair holds >= 1 tile
   const int32_t t_begin = pair < npairs ? range_start(pair, NT, npairs) : 0;
   const int32_t t_end = pair < npairs ? range_start(pair + 1, NT, npairs) : 0;
+  const uint64_t lim = p.wait_ns;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
-      // counts: the 256 softmax threads (P, O, q hand-offs); SEMPTY: those plus the 128 exchange threads
-      // that also read a score buffer; XORDY: the exchange threads; XFREE: one arrival per softmax
-      // warp of the peer; TMAX: the two softmax warps of one TMEM lane quarter
       uint32_t cnt = 1;
-      if (i == B_PFULL || i == B_OFREE || i == B_QFULL) cnt = 256;
-      else if (i >= B_SEMPTY && i < B_SEMPTY + 2) cnt = 384;
-      else if (i == B_XORDY) cnt = 128;
-      else if (i == B_XFREE || i == B_XFREE + 1) cnt = 8;
+      if (i == B_SCE || i == B_SCE + 1 || i == B_QFULL || i == B_PSTG || i == B_PSTG + 1) cnt = 256;
       else if (i >= B_TMAX && i < B_TMAX + 4) cnt = 64;
+      else if (i == B_OREADY || i == B_OREADY + 1 || i == B_OFREE) cnt = 128;
       mbar_init(bar(i), cnt);
     }
-    // the exchange buffers' first phases: one arrival plus the bytes the peer's copy will bring
-    mbar_expect_tx(bar(B_XFULL), X_BYTES);
-    mbar_expect_tx(bar(B_XFULL + 1), X_BYTES);
+    if (r == 1) {
+      // the P buffers' first phases: one arrival plus the bytes of one message
+      mbar_expect_tx(bar(B_PFULL), PMSG);
+      mbar_expect_tx(bar(B_PFULL + 1), PMSG);
+    }
     fence_mbar_init();
   }
-  if (warp == 5) {
-    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&p.cmap);
-    prefetch_tmap(&p.rmap);
-  }
+  if (threadIdx.x == 0) prefetch_tmap(r == 0 ? &p.kmap : &p.vmap);
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
@@ -215,320 +206,353 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   SegWalk w;
   w.init(p.tile_start, p.B, t_begin, t_end);
+  const int ntiles = t_end - t_begin;
+  bool ok = true;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int j = 0, issued = 0;
-      bool ok = true;
-      const int xr = DC + 32 * (int)r;               // this CTA's k^R columns
-      for (; ok && w.valid(); w.next()) {
-        const int b = w.b;
-        const int32_t ts_b = p.tile_start[b];
-        const int32_t row_base = (int32_t)p.cu[b];
-        for (int32_t xt = w.x; xt < w.seg_end(); ++xt, ++j) {
-          const int st = j % STAGES;
-          if (!mbar_wait(bar(B_EMPTY + st), ((j / STAGES) & 1) ^ 1)) { ok = false; break; }
-          mbar_expect_tx(bar(B_FULL + st), STAGE_BYTES);
-          const int32_t row0 = row_base + (xt - ts_b) * NK;
-          const uint32_t dst = sbase + OFF_KV + st * STAGE_BYTES;
-          for (int c = 0; c < 4; ++c)
-            tma_load_2d(dst + c * KV_BOX, &p.cmap, 256 * (int)r + 64 * c, row0, bar(B_FULL + st));
-          tma_load_2d(dst + 4 * KV_BOX, &p.rmap, xr, row0, bar(B_FULL + st));
-          issued = j + 1;
-        }
-      }
-      if (!ok) {
-        flag_error(p.err, DEVERR_TIMEOUT);
-        for (int i = max(0, issued - STAGES); i < issued; ++i) mbar_wait(bar(B_FULL + i % STAGES), (i / STAGES) & 1);
-      }
-    }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA issuer
-    // Greedy: P.V for the oldest tile whose P is ready, else QK^T of the next tile once its cache
-    // tile has landed and its score buffer has been read out by the softmax. QK^T goes out in two
-    // halves of 9 MMAs, so that a P.V that becomes ready meanwhile does not wait for all of it.
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(128, NK, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
-      const uint32_t qr = sbase + OFF_QR;
-      TileCursor cq, cp;
-      cq.init(p.tile_start, p.B, t_begin, t_end);
-      cp.init(p.tile_start, p.B, t_begin, t_end);
-      uint64_t stall_since = 0;
-      bool ok = true;
-      int qk_half = 0;                               // halves of QK^T(cq.j) issued so far
-      while (cp.valid()) {
-        bool did = false;
-        if (cp.j < cq.j && mbar_test(bar(B_PFULL), cp.j & 1) &&
-            (!cp.first() || mbar_test(bar(B_OFREE), (cp.g & 1) ^ 1))) {
-          tc_fence_after();
-          const int st = cp.j % STAGES;
-          const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
-          const bool first = cp.first();
-          // descriptors advance by adding (byte offset >> 4) to the start-address field (bits 0-13,
-          // shared-memory addresses stay below 2^18): one add per MMA instead of a full encode
-          const uint64_t ap = sw128_desc(sbase + OFF_P, 0, 1024), bp = sw128_desc(kv, KV_BOX, 1024);
-#pragma unroll
-          for (int kk = 0; kk < NK / 16; ++kk)
-            mma_bf16_ss(tmem, ap + (kk * 32 >> 4), bp + (kk * 2048 >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
-          mma_commit(bar(B_PVDONE));
-          mma_commit(bar(B_EMPTY + st));
-          cp.advance();
-          did = true;
-        }
-        if (!did && cq.valid()) {
-          const int st = cq.j % STAGES, sb = cq.j & 1;
-          if (qk_half == 1 ||
-              (mbar_test(bar(B_FULL + st), (cq.j / STAGES) & 1) && mbar_test(bar(B_SEMPTY + sb), ((cq.j >> 1) & 1) ^ 1) &&
-               (!cq.first() || mbar_test(bar(B_QFULL), cq.g & 1)))) {
-            if (qk_half == 0) tc_fence_after();
-            const uint32_t kv = sbase + OFF_KV + st * STAGE_BYTES;
-            const uint32_t d = tmem + T_S + NK * sb;
-            // MMA m < 16: latent chunk m / 4, K step m % 4 (A from TMEM); m = 16, 17: the k^R half
-            // (A from shared memory). Descriptors: base + (byte offset >> 4), as for P.V.
-            const uint64_t bq = sw128_desc(kv, 0, 1024);
-            auto issue = [&](auto m_c) {
-              constexpr int m = decltype(m_c)::value;
-              if (m < 16)
-                mma_bf16_ts(d, tmem + T_Q + 8 * m, bq + (((m >> 2) * KV_BOX + (m & 3) * 32) >> 4), idesc_qk,
-                            m ? 1u : 0u);
-              else
-                mma_bf16_ss(d, sw64_desc(qr, 512) + (((m - 16) * 32) >> 4),
-                            sw64_desc(kv + 4 * KV_BOX, 512) + (((m - 16) * 32) >> 4), idesc_qk, 1u);
-            };
-            if (qk_half == 0) {
-              issue(IC<0>{}); issue(IC<1>{}); issue(IC<2>{}); issue(IC<3>{}); issue(IC<4>{});
-              issue(IC<5>{}); issue(IC<6>{}); issue(IC<7>{}); issue(IC<8>{});
-            } else {
-              issue(IC<9>{}); issue(IC<10>{}); issue(IC<11>{}); issue(IC<12>{}); issue(IC<13>{});
-              issue(IC<14>{}); issue(IC<15>{}); issue(IC<16>{}); issue(IC<17>{});
+  if (r == 0) {
+    // =========================================================== score CTA
+    if (warp == 0) {
+      // ------------------------------------------------ TMA producer: 9 boxes per tile
+      if (lane == 0) {
+        int n = 0, issued = 0;
+        const bool stall = p.stall && pair == 0 && k == 0;
+        for (; ok && w.valid(); w.next()) {
+          const int32_t ts_b = p.tile_start[w.b];
+          const int32_t row_base = (int32_t)p.cu[w.b];
+          for (int32_t xt = w.x; ok && xt < w.seg_end(); ++xt) {
+            const int32_t row0 = row_base + (xt - ts_b) * NK;
+            for (int c = 0; c < S_BOXES; ++c, ++n) {
+              const int slot = n % S_RING;
+              if (!wait_bar(bar(B_SEMPTY + slot), ((n / S_RING) & 1) ^ 1, lim)) { ok = false; break; }
+              if (stall && n == 0) continue;     // test hook: this box never arrives
+              mbar_expect_tx(bar(B_SFULL + slot), BOX);
+              tma_load_2d(sbase + S_OFF_RING + slot * BOX, &p.kmap, c < 8 ? 64 * c : DC, row0, bar(B_SFULL + slot));
+              issued = n + 1;
             }
-            if (qk_half == 1) {
-              mma_commit(bar(B_SFULL + sb));
-              if (cq.last()) mma_commit(bar(B_QEMPTY));
-              cq.advance();
-            }
-            qk_half ^= 1;
-            did = true;
           }
         }
-        if (did) {
-          stall_since = 0;
-        } else {
-          // back off so this polling warp leaves the issue slots of its sub-partition to the
-          // softmax warp that shares it
-          __nanosleep(40);
-          if (stall_since == 0) {
-            stall_since = globaltimer();
-          } else if (globaltimer() - stall_since > kWaitTimeoutNs) {
+        if (!ok) {
+          flag_error(p.err, DEVERR_TIMEOUT);
+          for (int i = max(0, issued - S_RING); i < issued; ++i)
+            if (!(p.stall && pair == 0 && k == 0 && i == 0)) wait_bar(bar(B_SFULL + i % S_RING), (i / S_RING) & 1, lim);
+        }
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------ MMA issuer: S = [q~ | q^R] [c | k^R]^T
+      if (lane == 0) {
+        constexpr uint32_t idesc = idesc_bf16(128, NK, 0, 0);
+        const uint64_t qr_desc = sw128_desc(sbase + S_OFF_QR, 0, 1024);
+        int j = 0, g = 0, n = 0;
+        for (; ok && w.valid(); w.next(), ++g) {
+          if (!wait_bar(bar(B_QFULL), g & 1, lim)) { ok = false; break; }
+          const int32_t send = w.seg_end();
+          for (int32_t xt = w.x; xt < send; ++xt, ++j) {
+            const int sb = j & 1;
+            if (!wait_bar(bar(B_SCE + sb), ((j >> 1) & 1) ^ 1, lim)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d = tmem + 256 + 128 * sb;
+            for (int c = 0; c < S_BOXES; ++c, ++n) {
+              const int slot = n % S_RING;
+              if (!wait_bar(bar(B_SFULL + slot), (n / S_RING) & 1, lim)) { ok = false; break; }
+              tc_fence_after();
+              // descriptors advance by (byte offset >> 4) in the start-address field: 32 bytes per
+              // K step of 16 bf16 inside the 128-byte swizzled row
+              const uint64_t bdesc = sw128_desc(sbase + S_OFF_RING + slot * BOX, 0, 1024);
+              if (c < 8) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_bf16_ts(d, tmem + 32 * c + 8 * kk, bdesc + 2 * kk, idesc, (c | kk) ? 1u : 0u);
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(d, qr_desc + 2 * kk, bdesc + 2 * kk, idesc, 1u);
+              }
+              mma_commit(bar(B_SEMPTY + slot));
+            }
+            if (!ok) break;
+            mma_commit(bar(B_SCF + sb));
+          }
+          if (!ok) break;
+          mma_commit(bar(B_QEMPTY));
+        }
+        if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
+      }
+    } else if (warp == 2) {
+      // ------------------------------------------------ sender: staged P message -> value CTA
+      if (lane == 0) {
+        const uint32_t pbuf_peer = map_peer(sbase + V_OFF_PBUF, 1);
+        const uint32_t pfull_peer = map_peer(bar(B_PFULL), 1);
+        int last = -1;
+        for (int j = 0; j < ntiles; ++j) {
+          const int b = j & 1;
+          if (!wait_bar(bar(B_PSTG + b), (j >> 1) & 1, lim) || !wait_bar(bar(B_PVD + b), ((j >> 1) & 1) ^ 1, lim)) {
             ok = false;
             break;
           }
+          bulk_copy_to_peer(pbuf_peer + b * PMSG, sbase + S_OFF_STG + b * PMSG, PMSG, pfull_peer + 8 * b);
+          last = j;
         }
+        // the value CTA acknowledges each message once its bytes have landed; wait for the last one
+        // so that no copy into its shared memory is in flight when the cluster exits
+        if (last >= 0) wait_bar(bar(B_STGF + (last & 1)), (last >> 1) & 1, lim);
+        if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
+      }
+    } else if (warp >= 4) {
+      // ------------------------------------------------ softmax: 8 warps, two per TMEM lane quarter
+      // Half 0 (warps 4-7) takes keys [0, 64) of every tile, half 1 (warps 8-11) keys [64, 128),
+      // for the same 32 heads (thread = head = TMEM lane); they agree on each tile's max through
+      // shared memory and a per-quarter barrier.
+      const int quarter = warp & 3, half = (warp - 4) >> 2;
+      const int i = 32 * quarter + lane;
+      const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
+      const uint32_t tmax_bar = bar(B_TMAX + quarter);
+      float* redbuf = reinterpret_cast<float*>(smem + OFF_RED);   // [3 slots][2 halves][128]
+      const float c2 = p.scale_log2;
+      const float thr_raw = kRescaleLog2 / c2;
+      auto wait_u = [&](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, wait_bar(b, par, lim)) != 0; };
+      int tph = 0;
+      auto swap_half = [&](float x, int slot, float& y) -> bool {
+        redbuf[(slot * 2 + half) * 128 + i] = x;
+        mbar_arrive(tmax_bar);
+        const bool okw = wait_u(tmax_bar, tph & 1);
+        ++tph;
+        y = redbuf[(slot * 2 + (half ^ 1)) * 128 + i];
+        return okw;
+      };
+      // q~ (this half's 256 latent columns -> TMEM columns [128 half, +128)) and q^R (this half's
+      // 32 columns -> the swizzled q^R tile) of sequence bq, once the previous piece's last QK^T is
+      // done with them.
+      int gq = 0;
+      auto load_q = [&](int bq) -> bool {
+        const int64_t t = (int64_t)bq * p.tq + k;
+        if (!wait_u(bar(B_QEMPTY), (gq & 1) ^ 1)) return false;
+        tc_fence_after();
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (t * H + i) * DC + 256 * half);
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint4 u = __ldg(src + 8 * cc + e);
+            v[4 * e] = u.x; v[4 * e + 1] = u.y; v[4 * e + 2] = u.z; v[4 * e + 3] = u.w;
+          }
+          tmem_st32(trow + 128 * half + 32 * cc, v);
+        }
+        const uint4* rsrc = reinterpret_cast<const uint4*>(p.q_rope + (t * H + i) * DR);
+        uint8_t* qrow = smem + S_OFF_QR + i * 128;
+#pragma unroll
+        for (int c = 4 * half; c < 4 * half + 4; ++c)
+          *reinterpret_cast<uint4*>(qrow + ((c ^ (i & 7)) << 4)) = __ldg(rsrc + c);
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(B_QFULL));
+        ++gq;
+        return true;
+      };
+      ok = !w.valid() || load_q(w.b);
+      int j = 0;
+      for (; ok && w.valid(); w.next()) {
+        const int b = w.b;
+        const int64_t len = p.cu[b + 1] - p.cu[b];
+        const int64_t vis = len - p.tq + k + 1;       // keys visible to this query token
+        const int32_t ts_b = p.tile_start[b];
+        const int32_t send = w.seg_end();
+        float m_ref = -INFINITY, l = 0.f;             // running max (raw score units); this half's sum
+        for (int32_t xt = w.x; xt < send; ++xt, ++j) {
+          const int sb = j & 1;
+          const bool first = xt == w.x, last = xt == send - 1;
+          if (!wait_u(bar(B_SCF + sb), (j >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          float s[64];
+          tmem_ld32(trow + 256 + 128 * sb + 64 * half, reinterpret_cast<uint32_t*>(s));
+          tmem_ld32(trow + 256 + 128 * sb + 64 * half + 32, reinterpret_cast<uint32_t*>(s) + 32);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(B_SCE + sb));
+          const int64_t key0 = (int64_t)(xt - ts_b) * NK + 64 * half;
+          const int nvis = (int)max((int64_t)0, min((int64_t)64, vis - key0));
+          if (nvis < 64) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] = c < nvis ? s[c] : -INFINITY;
+          }
+          float mx[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) mx[c] = fmaxf(fmaxf(s[4 * c], s[4 * c + 1]), fmaxf(s[4 * c + 2], s[4 * c + 3]));
+#pragma unroll
+          for (int w2 = 8; w2 > 0; w2 >>= 1)
+#pragma unroll
+            for (int c = 0; c < w2; ++c) mx[c] = fmaxf(mx[c], mx[c + w2]);
+          float pmax;
+          if (!swap_half(mx[0], j & 1, pmax)) { ok = false; break; }
+          const float tmax = fmaxf(mx[0], pmax);
+          // lazy rescale of the running max: the same decision in both halves (same tmax, m_ref)
+          float alpha = 1.f;
+          if (tmax > -INFINITY && (m_ref == -INFINITY || tmax > m_ref + thr_raw)) {
+            alpha = m_ref == -INFINITY ? 0.f : ex2_approx((m_ref - tmax) * c2);
+            l *= alpha;
+            m_ref = tmax;
+          }
+          // P = 2^((s - m_ref) c2) in bf16, packed in pairs
+          uint32_t pk[32];
+          if (m_ref > -INFINITY) {
+            const uint64_t cc = f2_pack(c2, c2), off = f2_pack(-m_ref * c2, -m_ref * c2);
+            uint64_t acc2[8];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              float a0, a1;
+              f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), cc, off), a0, a1);
+              const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
+              pk[c] = pack_bf16(e0, e1);
+              if (c < 8) acc2[c] = f2_pack(e0, e1);
+              else acc2[c & 7] = f2_add(acc2[c & 7], f2_pack(e0, e1));
+            }
+#pragma unroll
+            for (int w2 = 4; w2 > 0; w2 >>= 1)
+#pragma unroll
+              for (int c = 0; c < w2; ++c) acc2[c] = f2_add(acc2[c], acc2[c + w2]);
+            float l0, l1;
+            f2_unpack(acc2[0], l0, l1);
+            l += l0 + l1;
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pk[c] = 0u;
+          }
+          // staging buffer sb: the value CTA has received the message of tile j - 2 from it
+          if (!wait_u(bar(B_STGF + sb), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+          uint8_t* msg = smem + S_OFF_STG + sb * PMSG;
+          uint8_t* prow = msg + 16384 * half + i * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(prow + ((c ^ (i & 7)) << 4)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          float* hdr = reinterpret_cast<float*>(msg + P_BYTES);
+          if (half == 0) hdr[i] = first ? 1.f : alpha;
+          if (last) {
+            // piece end: both halves' sums -> 1/l for the value CTA, lse written here
+            float lp;
+            if (!swap_half(l, 2, lp)) { ok = false; break; }
+            const float lt = l + lp;
+            if (half == 0) {
+              hdr[H + i] = lt > 0.f ? 1.f / lt : 0.f;
+              const float lse_v = lt > 0.f ? (m_ref * c2 + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+              const int64_t t = (int64_t)b * p.tq + k;
+              const int32_t nseg = p.slot_base[b + 1] - p.slot_base[b];
+              if (nseg > 1) {
+                const int64_t slot =
+                    (int64_t)p.slot_base[b] + (pair - (int)(((int64_t)(ts_b + 1) * npairs - 1) / NT));
+                p.part_lse[((int64_t)k * p.s_max + slot) * H + i] = lse_v;
+              } else {
+                p.lse[t * H + i] = lse_v;
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(bar(B_PSTG + sb));
+        }
+        if (!ok) break;
+        // the next piece's query goes in now, so that its first QK^T overlaps the value CTA's epilogue
+        SegWalk nx = w;
+        nx.next();
+        if (nx.valid() && !load_q(nx.b)) { ok = false; break; }
       }
       if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
     }
-  } else if (warp >= 6 && warp < 10) {
-    // ------------------------------------------------------------------ score exchange (send side)
-    // Per tile: this CTA's partial scores TMEM -> registers -> the local staging buffer (chunk-major:
-    // chunk c of head i at (c * 128 + i) * 16), which one thread copies in bulk into the peer's
-    // exchange buffer once the peer's softmax has read the previous tile out of it (counted on the
-    // peer's x_full barrier). The staging buffer is rewritten only once the previous copy has read it.
-    const int e = threadIdx.x - 192;                 // exchange thread 0..127
-    const int i = 32 * (warp & 3) + lane;            // head = TMEM lane
-    const bool leader = e == 0;
-    const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    const uint32_t xin_peer = map_peer(sbase + OFF_X, peer);
-    const uint32_t xfull_peer = map_peer(bar(B_XFULL), peer);
-    uint4* xo = reinterpret_cast<uint4*>(smem + OFF_XO) + i;
-    auto wait_u = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(b, par)) != 0; };
-    const int ntiles = t_end - t_begin;
-    bool ok = true;
-    for (int jj = 0; jj < ntiles; ++jj) {
-      const int sb = jj & 1;
-      const uint32_t taddr = trow + T_S + NK * sb;
-      if (leader && jj > 0) {
-        bulk_wait_read0();                           // the previous copy has read the staging buffer
-        mbar_arrive(bar(B_XOFREE));
-      }
-      if (!wait_u(bar(B_SFULL + sb), (jj >> 1) & 1)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t v[NK];
-      tmem_ld32(taddr, v);
-      tmem_ld32(taddr + 32, v + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_SEMPTY + sb));
-      if (!wait_u(bar(B_XOFREE), (jj & 1) ^ 1)) { ok = false; break; }
-#pragma unroll
-      for (int c = 0; c < XCH; ++c) {
-        uint32_t w4[4];
-        if (kXHalf) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int k2 = XPER * c + 2 * q;
-            const __half2 h2 = __floats2half2_rn(__uint_as_float(v[k2]), __uint_as_float(v[k2 + 1]));
-            w4[q] = *reinterpret_cast<const uint32_t*>(&h2);
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) w4[q] = v[XPER * c + q];
-        }
-        xo[c * 128] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar(B_XORDY));
-      if (leader) {
-        // all 128 rows staged, and the peer's softmax has read the previous tile out of its buffer
-        const int xb = jj & 1;
-        if (mbar_wait(bar(B_XORDY), jj & 1) && mbar_wait_cluster(bar(B_XFREE + xb), ((jj >> 1) & 1) ^ 1)) {
-          bulk_copy_to_peer(xin_peer + xb * X_BYTES, sbase + OFF_XO, X_BYTES, xfull_peer + 8 * xb);
-          bulk_commit();
-        } else {
-          ok = false;
-        }
-      }
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-    }
-    if (leader) bulk_wait_read0();
-    if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
   } else {
-    // ------------------------------------------------------------------ softmax + epilogue
-    // Two warps per TMEM lane quarter: half 0 (warps 0-3) takes keys [0, 32) of every tile, half 1
-    // (warps 10-13) keys [32, 64), for the same 32 heads; they agree on each tile's max through
-    // shared memory and a per-quarter barrier. O columns (rescale, epilogue) and the query load are
-    // split between the halves the same way.
-    const int quarter = warp & 3, half = warp >= 10 ? 1 : 0;
-    const int i = 32 * quarter + lane;               // head
-    const int tid = 128 * half + i;                  // 0..255 over both halves
-    const int kc0 = 32 * half;                       // first key of this half within a tile
-    const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
-    const uint32_t xfree_peer = map_peer(bar(B_XFREE), peer);
-    const uint32_t tmax_bar = bar(B_TMAX + quarter);
-    float* redbuf = reinterpret_cast<float*>(smem + OFF_RED);   // [2 parity][2 half][128] maxima, then [2][128] sums
-    const float c2 = p.scale_log2;                   // raw score -> log2 units
-    const float thr_raw = kRescaleLog2 / c2;
-    // waits of the softmax warps are warp-uniform: a timeout on any lane fails the whole warp, so
-    // no lane can be left behind at a .sync.aligned tcgen05 instruction
-    auto wait_u = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(b, par)) != 0; };
-    auto wait_uc = [](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait_cluster(b, par)) != 0; };
-    int gq = 0, j = 0, tph = 0;
-    // one exchange of a value per head with the other half of this quarter: the partner's value in
-    // y; false if the wait gave up
-    auto swap_half = [&](float x, int slot, float& y) -> bool {
-      redbuf[(slot * 2 + half) * 128 + i] = x;
-      mbar_arrive(tmax_bar);
-      const bool okw = wait_u(tmax_bar, tph & 1);
-      ++tph;
-      y = redbuf[(slot * 2 + (half ^ 1)) * 128 + i];
-      return okw;
-    };
-    // q~ half -> TMEM (this half's 64 columns) and q^R half -> shared memory (64-byte swizzle, this
-    // half's two chunks) for the piece of sequence bq, once the previous piece's last QK^T is done.
-    auto load_q = [&](int bq) -> bool {
-      const int64_t t = (int64_t)bq * p.tq + k;
-      if (!wait_u(bar(B_QEMPTY), (gq & 1) ^ 1)) return false;
-      tc_fence_after();
-      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (t * H + i) * DC + 256 * r + 128 * half);
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
+    // =========================================================== value CTA
+    if (warp == 0) {
+      // ------------------------------------------------ TMA producer: 4 groups per tile
+      if (lane == 0) {
+        int n = 0, issued = 0;
+        for (; ok && w.valid(); w.next()) {
+          const int32_t ts_b = p.tile_start[w.b];
+          const int32_t row_base = (int32_t)p.cu[w.b];
+          for (int32_t xt = w.x; ok && xt < w.seg_end(); ++xt) {
+            const int32_t row0 = row_base + (xt - ts_b) * NK;
+            for (int s = 0; s < 4; ++s, ++n) {
+              const int g = n % V_RING;
+              if (!wait_bar(bar(B_GEMPTY + g), ((n / V_RING) & 1) ^ 1, lim)) { ok = false; break; }
+              mbar_expect_tx(bar(B_GFULL + g), VGRP);
+              const int nh = s & 1, kh = s >> 1;
+              const uint32_t dst = sbase + V_OFF_RING + g * VGRP;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint4 u = __ldg(src + 8 * c + e);
-          v[4 * e] = u.x; v[4 * e + 1] = u.y; v[4 * e + 2] = u.z; v[4 * e + 3] = u.w;
-        }
-        tmem_st32(trow + T_Q + 64 * half + 32 * c, v);
-      }
-      const uint4* rsrc = reinterpret_cast<const uint4*>(p.q_rope + (t * H + i) * DR + 32 * r);
-      uint8_t* qrow = smem + OFF_QR + i * 64;
-#pragma unroll
-      for (int c = 2 * half; c < 2 * half + 2; ++c)
-        *reinterpret_cast<uint4*>(qrow + ((c ^ ((i >> 1) & 3)) << 4)) = __ldg(rsrc + c);
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(B_QFULL));
-      ++gq;
-      return true;
-    };
-    bool ok = !w.valid() || load_q(w.b);
-    for (; ok && w.valid(); w.next()) {
-      const int b = w.b;
-      const int64_t len = p.cu[b + 1] - p.cu[b];
-      const int64_t vis = len - p.tq + k + 1;        // keys visible to this query token
-      const int32_t ts_b = p.tile_start[b];
-      const int32_t send = w.seg_end();
-      float m_ref = -INFINITY, l = 0.f;              // running max (raw score units); this half's sum
-      const int jfirst = j;
-      for (int32_t xt = w.x; xt < send; ++xt) {
-        // scores of this half's 32 keys: this CTA's partial (TMEM) plus the peer's (exchange buffer)
-        const int sb = j & 1, xb = j & 1;
-        if (!wait_u(bar(B_SFULL + sb), (j >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        float s[32];
-        tmem_ld32(trow + T_S + NK * sb + kc0, reinterpret_cast<uint32_t*>(s));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(B_SEMPTY + sb));
-        if (!wait_uc(bar(B_XFULL + xb), (j >> 1) & 1)) { ok = false; break; }
-        {
-          const uint4* xi = reinterpret_cast<const uint4*>(smem + OFF_X + xb * X_BYTES) + i;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 q = xi[(4 * half + c) * 128];
-            const uint32_t q4[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              // both CTAs add the two fp16-rounded partials, so they see the same scores
-              const int k2 = 8 * c + 2 * u;
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&q4[u]));
-              const float2 o = __half22float2(__floats2half2_rn(s[k2], s[k2 + 1]));
-              s[k2] = o.x + f.x;
-              s[k2 + 1] = o.y + f.y;
+              for (int bx = 0; bx < 4; ++bx)
+                tma_load_2d(dst + bx * VBOX, &p.vmap, 256 * nh + 64 * bx, row0 + 64 * kh, bar(B_GFULL + g));
+              issued = n + 1;
             }
           }
         }
-        // re-arm the buffer's next phase (one arrival + the bytes), then tell the peer it is free
-        if (tid == 0) mbar_expect_tx(bar(B_XFULL + xb), X_BYTES);
-        __syncwarp();
-        if (lane == 0) mbar_arrive_peer(xfree_peer + 8 * xb);
-        const int64_t key0 = (int64_t)(xt - ts_b) * NK;
-        const int nvis = (int)max((int64_t)0, min((int64_t)NK, vis - key0)) - kc0;
-        if (nvis < 32) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) s[c] = c < nvis ? s[c] : -INFINITY;
+        if (!ok) {
+          flag_error(p.err, DEVERR_TIMEOUT);
+          for (int i = max(0, issued - V_RING); i < issued; ++i) wait_bar(bar(B_GFULL + i % V_RING), (i / V_RING) & 1, lim);
         }
-        float mx[16];
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------ MMA issuer: O += P . C
+      if (lane == 0) {
+        constexpr uint32_t idesc = idesc_bf16(128, 256, 0, 1);
+        const uint32_t stgf_peer = map_peer(bar(B_STGF), 0);
+        int j = 0, g = 0, n = 0;
+        for (; ok && w.valid(); w.next(), ++g) {
+          const int32_t send = w.seg_end();
+          for (int32_t xt = w.x; xt < send; ++xt, ++j) {
+            const int pb = j & 1;
+            const bool first = xt == w.x;
+            if (!wait_bar(bar(B_PFULL + pb), (j >> 1) & 1, lim)) { ok = false; break; }
+            // re-arm the buffer's next phase, and let the score CTA reuse its staging buffer
+            mbar_expect_tx(bar(B_PFULL + pb), PMSG);
+            mbar_arrive_peer(stgf_peer + 8 * pb);
+            if (!wait_bar(bar(B_OREADY + pb), (j >> 1) & 1, lim)) { ok = false; break; }
+            if (first && !wait_bar(bar(B_OFREE), (g & 1) ^ 1, lim)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t pmsg = sbase + V_OFF_PBUF + pb * PMSG;
+            for (int s = 0; s < 4; ++s, ++n) {
+              const int gi = n % V_RING;
+              if (!wait_bar(bar(B_GFULL + gi), (n / V_RING) & 1, lim)) { ok = false; break; }
+              tc_fence_after();
+              const int nh = s & 1, kh = s >> 1;
+              const uint64_t adesc = sw128_desc(pmsg + 16384 * kh, 0, 1024);
+              const uint64_t bdesc = sw128_desc(sbase + V_OFF_RING + gi * VGRP, VBOX, 1024);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) mx[c] = fmaxf(s[2 * c], s[2 * c + 1]);
-#pragma unroll
-        for (int w2 = 8; w2 > 0; w2 >>= 1)
-#pragma unroll
-          for (int c = 0; c < w2; ++c) mx[c] = fmaxf(mx[c], mx[c + w2]);
-        float pmax;
-        if (!swap_half(mx[0], j & 1, pmax)) { ok = false; break; }
-        const float tmax = fmaxf(mx[0], pmax);
-        // rows of this stage past the sequence end: zero the latent half before P.V reads it
-        const int nrows = (int)max((int64_t)0, min((int64_t)NK, len - key0));
-        if (nrows < NK) {
-          uint8_t* kvs = smem + OFF_KV + (j % STAGES) * STAGE_BYTES;
-          const int chunks = (NK - nrows) * 4 * 8;   // 16-byte chunks over 4 boxes
-          for (int q = tid; q < chunks; q += 256) {
-            const int row = nrows + q / 32, box = (q / 8) & 3, c16 = q & 7;
-            *reinterpret_cast<uint4*>(kvs + box * KV_BOX + row * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tmem + 256 * nh, adesc + 2 * kk, bdesc + ((kk * 2048) >> 4), idesc,
+                            (first && kh == 0 && kk == 0) ? 0u : 1u);
+              mma_commit(bar(B_GEMPTY + gi));
+            }
+            if (!ok) break;
+            // P buffer pb free again / this tile's P.V done: both CTAs' B_PVD + pb
+            mma_commit_mc(bar(B_PVD + pb), 0x3);
           }
+          if (!ok) break;
         }
-        // lazy rescale of the running max (identical decision in both halves and both CTAs); O must
-        // be at rest, so P.V of the previous tile has to be done first
-        if (tmax > -INFINITY && (m_ref == -INFINITY || tmax > m_ref + thr_raw)) {
-          const float alpha = ex2_approx((m_ref - tmax) * c2);
-          if (j > jfirst) {
-            if (!wait_u(bar(B_PVDONE), (j - 1) & 1)) { ok = false; break; }
+        if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
+      }
+    } else if (warp >= 4 && warp < 8) {
+      // ------------------------------------------------ rescale + piece epilogue (thread = head = TMEM lane)
+      const int quarter = warp & 3;
+      const int i = 32 * quarter + lane;
+      const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
+      const int64_t total_rows = p.cu[p.B];
+      auto wait_u = [&](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, wait_bar(b, par, lim)) != 0; };
+      int j = 0, n = 0;
+      for (; ok && w.valid(); w.next()) {
+        const int b = w.b;
+        const int32_t ts_b = p.tile_start[b];
+        const int32_t send = w.seg_end();
+        const int64_t row_base = p.cu[b];
+        float inv_l = 0.f;
+        for (int32_t xt = w.x; xt < send; ++xt, ++j, n += 4) {
+          const int pb = j & 1;
+          const bool first = xt == w.x, last = xt == send - 1;
+          if (!wait_u(bar(B_PFULL + pb), (j >> 1) & 1)) { ok = false; break; }
+          const float* hdr = reinterpret_cast<const float*>(smem + V_OFF_PBUF + pb * PMSG + P_BYTES);
+          const float alpha = hdr[i];
+          if (last) inv_l = hdr[H + i];
+          if (__any_sync(0xffffffffu, !first && alpha != 1.f)) {
+            // O holds the previous tiles' sum at the old max: rescale once their P.V is done
+            if (!wait_u(bar(B_PVD + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 128 * half; c < 128 * half + 128; c += 32) {
+            for (int c = 0; c < DC; c += 32) {
               uint32_t v[32];
               tmem_ld32(trow + c, v);
               tmem_wait_ld();
@@ -539,111 +563,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tmem_wait_st();
             tc_fence_before();
           }
-          l *= alpha;
-          m_ref = tmax;
-        }
-        // P = 2^((s - m_ref) c2) in bf16: this half's 4 chunks of row i of the K-major P tile
-        uint32_t pk[16];
-        if (m_ref > -INFINITY) {
-          const uint64_t cc = f2_pack(c2, c2), off = f2_pack(-m_ref * c2, -m_ref * c2);
-          uint64_t acc2[8];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            float a0, a1;
-            f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), cc, off), a0, a1);
-            const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
-            pk[c] = pack_bf16(e0, e1);
-            if (c < 8) acc2[c] = f2_pack(e0, e1);
-            else acc2[c & 7] = f2_add(acc2[c & 7], f2_pack(e0, e1));
+          // cache rows past the last sequence may hold anything (even NaN): zero them in this tile's
+          // groups before P.V reads them (their P is zero, but 0 * NaN is not)
+          const int64_t row0 = row_base + (int64_t)(xt - ts_b) * NK;
+          if (row0 + NK > total_rows) {
+            const int nrows = (int)max((int64_t)0, total_rows - row0);
+            for (int s = 0; s < 4; ++s) {
+              const int gi = (n + s) % V_RING;
+              if (!wait_u(bar(B_GFULL + gi), ((n + s) / V_RING) & 1)) { ok = false; break; }
+              uint8_t* grp = smem + V_OFF_RING + gi * VGRP;
+              const int kh = s >> 1;
+              // rows 64 kh + rr >= nrows, 4 boxes x 8 chunks of 16 bytes each
+              for (int q = i; q < 64 * 32; q += 128) {
+                const int rr = q >> 5, bx = (q >> 3) & 3, c16 = q & 7;
+                if (64 * kh + rr >= nrows)
+                  *reinterpret_cast<uint4*>(grp + bx * VBOX + rr * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
+              }
+            }
+            if (!ok) break;
+            fence_proxy_async_smem();
           }
-#pragma unroll
-          for (int w2 = 4; w2 > 0; w2 >>= 1)
-#pragma unroll
-            for (int c = 0; c < w2; ++c) acc2[c] = f2_add(acc2[c], acc2[c + w2]);
-          float l0, l1;
-          f2_unpack(acc2[0], l0, l1);
-          l += l0 + l1;
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) pk[c] = 0u;
-        }
-        // the P tile was last read by P.V of tile j - 1
-        if (!wait_u(bar(B_PVDONE), (j - 1) & 1)) { ok = false; break; }
-        uint8_t* prow = smem + OFF_P + i * 128;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (i & 7)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        fence_proxy_async_smem();
-        mbar_arrive(bar(B_PFULL));
-        ++j;
-      }
-      if (!ok) break;
-      // the next piece's query goes in now, so that its first QK^T overlaps this epilogue
-      {
-        SegWalk nx = w;
-        nx.next();
-        if (nx.valid() && !load_q(nx.b)) { ok = false; break; }
-      }
-      // piece epilogue: O / l for this half's 128 of this CTA's 256 columns (+ lse from CTA 0)
-      float lp;
-      if (!swap_half(l, 2, lp)) { ok = false; break; }
-      const float lt = l + lp;                       // both halves' sums
-      const int jl = j - 1;
-      const float m_log2 = m_ref * c2;
-      if (!wait_u(bar(B_PVDONE), jl & 1)) { ok = false; break; }
-      tc_fence_after();
-      const int64_t t = (int64_t)b * p.tq + k;
-      const int32_t nseg = p.slot_base[b + 1] - p.slot_base[b];
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      const float lse_v = lt > 0.f ? (m_log2 + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-      float* po = nullptr;
-      if (nseg > 1) {
-        const int64_t slot = (int64_t)p.slot_base[b] + (pair - (int)(((int64_t)(ts_b + 1) * npairs - 1) / NT));
-        const int64_t row = ((int64_t)k * p.s_max + slot) * H + i;
-        po = p.part_o + row * DC + 256 * r;
-        if (r == 0 && half == 0) p.part_lse[row] = lse_v;
-      } else if (r == 0 && half == 0) {
-        p.lse[t * H + i] = lse_v;
-      }
+          mbar_arrive(bar(B_OREADY + pb));
+          if (last) {
+            // piece epilogue: o^lat = O / l for all 512 columns of head i
+            if (!wait_u(bar(B_PVD + pb), (j >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const int64_t t = (int64_t)b * p.tq + k;
+            const int32_t nseg = p.slot_base[b + 1] - p.slot_base[b];
+            float* po = nullptr;
+            if (nseg > 1) {
+              const int64_t slot = (int64_t)p.slot_base[b] + (pair - (int)(((int64_t)(ts_b + 1) * npairs - 1) / NT));
+              po = p.part_o + (((int64_t)k * p.s_max + slot) * H + i) * DC;
+            }
 #pragma unroll 1
-      for (int c = 128 * half; c < 128 * half + 128; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(trow + c, v);
-        tmem_wait_ld();
-        if (po) {
-          float4* dst = reinterpret_cast<float4*>(po + c);
+            for (int c = 0; c < DC; c += 32) {
+              uint32_t v[32];
+              tmem_ld32(trow + c, v);
+              tmem_wait_ld();
+              if (po || OUT_F32) {
+                float4* dst = po ? reinterpret_cast<float4*>(po + c)
+                                 : reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o_lat) + (t * H + i) * DC + c);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
-                                 __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
-        } else if (OUT_F32) {
-          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o_lat) + (t * H + i) * DC + 256 * r + c);
+                for (int e = 0; e < 8; ++e)
+                  dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv_l, __uint_as_float(v[4 * e + 1]) * inv_l,
+                                       __uint_as_float(v[4 * e + 2]) * inv_l, __uint_as_float(v[4 * e + 3]) * inv_l);
+              } else {
+                uint4* dst =
+                    reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o_lat) + (t * H + i) * DC + c);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
-                                 __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o_lat) + (t * H + i) * DC +
-                                                256 * r + c);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pack_bf16(__uint_as_float(v[8 * e]) * inv, __uint_as_float(v[8 * e + 1]) * inv),
-                                pack_bf16(__uint_as_float(v[8 * e + 2]) * inv, __uint_as_float(v[8 * e + 3]) * inv),
-                                pack_bf16(__uint_as_float(v[8 * e + 4]) * inv, __uint_as_float(v[8 * e + 5]) * inv),
-                                pack_bf16(__uint_as_float(v[8 * e + 6]) * inv, __uint_as_float(v[8 * e + 7]) * inv));
+                for (int e = 0; e < 4; ++e)
+                  dst[e] = make_uint4(pack_bf16(__uint_as_float(v[8 * e]) * inv_l, __uint_as_float(v[8 * e + 1]) * inv_l),
+                                      pack_bf16(__uint_as_float(v[8 * e + 2]) * inv_l, __uint_as_float(v[8 * e + 3]) * inv_l),
+                                      pack_bf16(__uint_as_float(v[8 * e + 4]) * inv_l, __uint_as_float(v[8 * e + 5]) * inv_l),
+                                      pack_bf16(__uint_as_float(v[8 * e + 6]) * inv_l, __uint_as_float(v[8 * e + 7]) * inv_l));
+              }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(B_OFREE));
+          }
         }
+        if (!ok) break;
       }
-      tc_fence_before();
-      mbar_arrive(bar(B_OFREE));
+      if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
     }
-    if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
   }
+  __syncwarp();
   tc_fence_before();
   cluster_sync();
-  if (warp == 5) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -672,9 +661,9 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
     if (lane == (int)(blockDim.x >> 5) - 1) *total = t;
   }
   __syncthreads();
-  const int32_t r = x - v + (wid > 0 ? warp_tot[wid - 1] : 0);
+  const int32_t res = x - v + (wid > 0 ? warp_tot[wid - 1] : 0);
   __syncthreads();
-  return r;
+  return res;
 }
 
 __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B, int32_t pairs, int32_t* ts,
@@ -766,15 +755,15 @@ struct CoreScratch {
 
 CoreScratch carve(void* scratch, int64_t B, int32_t tq) {
   CoreScratch c;
-  char* p = (char*)scratch;
+  char* ptr = (char*)scratch;
   c.s_max = (int32_t)(kMaxPairs + B);
-  c.ts = (int32_t*)p;
-  p += align1k((B + 1) * 4);
-  c.sb = (int32_t*)p;
-  p += align1k((B + 1) * 4);
-  c.part_lse = (float*)p;
-  p += align1k((size_t)tq * c.s_max * H * 4);
-  c.part_o = (float*)p;
+  c.ts = (int32_t*)ptr;
+  ptr += align1k((B + 1) * 4);
+  c.sb = (int32_t*)ptr;
+  ptr += align1k((B + 1) * 4);
+  c.part_lse = (float*)ptr;
+  ptr += align1k((size_t)tq * c.s_max * H * 4);
+  c.part_o = (float*)ptr;
   return c;
 }
 
@@ -794,7 +783,12 @@ cudaError_t launch_core(const CoreParams& p, dim3 grid, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// Test hook state (mla_test_stall_latent_core): consumed by the next launch.
+int g_stall_next = 0;
+
 }  // namespace
+
+void tc_latent_core_arm_stall() { g_stall_next = 1; }
 
 size_t tc_core_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq) {
   (void)d;
@@ -820,8 +814,8 @@ cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B
   memset(&p, 0, sizeof(p));
   p.q_abs = reinterpret_cast<const __nv_bfloat16*>(q_abs);
   p.q_rope = reinterpret_cast<const __nv_bfloat16*>(q_rope);
-  if ((e = make_tmap_bf16(&p.cmap, cache, ROW, capacity, ROW, 64, NK)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16(&p.rmap, cache, ROW, capacity, ROW, 32, NK, 64)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&p.kmap, cache, ROW, capacity, ROW, 64, NK)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&p.vmap, cache, ROW, capacity, ROW, 64, 64)) != cudaSuccess) return e;
   p.cu = cu;
   p.tile_start = c.ts;
   p.slot_base = c.sb;
@@ -834,6 +828,12 @@ cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B
   p.o_lat = o_lat;
   p.lse = lse;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt(128.0 + 64.0));
+  p.wait_ns = kWaitTimeoutNs;
+  if (g_stall_next) {
+    p.stall = 1;
+    p.wait_ns = 20000000ull;   // 20 ms, so that the stalled launch gives up quickly
+    g_stall_next = 0;
+  }
   p.err = err;
   dim3 grid((unsigned)(2 * pairs), (unsigned)tq);
   e = o_f32 ? launch_core<true>(p, grid, st) : launch_core<false>(p, grid, st);

@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
             "mla_set_kernel_timing": (c_int, [c_int]),
             "mla_kernel_time_ms": (c_int, [c_int, POINTER(ctypes.c_float)]),
             "mla_status_string": (c_char_p, [c_int]),
+            "mla_test_arm_stall": (None, []),
             "mla_destroy": (None, [H]),
         }
         for name, (res, args) in sigs.items():
@@ -188,6 +189,11 @@ def mla_kernel_time_ms(which: int) -> float:
     ms = ctypes.c_float(0.0)
     _check(lib().mla_kernel_time_ms(which, ctypes.byref(ms)), "mla_kernel_time_ms")
     return float(ms.value)
+
+
+def mla_test_arm_stall():
+    """Arms the next decode latent-core launch to give up on a wait nothing signals (20 ms limit)."""
+    lib().mla_test_arm_stall()
 
 
 def mla_kernel_launches() -> int:

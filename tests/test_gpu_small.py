@@ -255,6 +255,28 @@ def test_device_checks_flag_bad_cu_seqlens_and_slots(v3_module):
     assert mla.mla_device_error_bits(v3_module.handle) & 4
 
 
+def test_bounded_wait_gives_up_reports_timeout_and_the_next_call_recovers(v3_module):
+    # the armed launch waits for a cache tile that is never loaded; each role gives up after its
+    # 20 ms limit and returns, the error word says TIMEOUT, and the same handle then runs normally
+    dims = synth.V3
+    lens = np.array([300, 700])
+    cu = synth.cu_seqlens(lens)
+    cache = synth.latent_cache(dims, int(cu[-1]), seed=70, dtype="bf16")
+    q_abs = synth.normal(71, 20, (2, dims.n_h, dims.d_c), std=0.5, dtype="bf16")
+    q_rope = synth.normal(71, 21, (2, dims.n_h, dims.d_r), std=1.0, dtype="bf16")
+    args = (dev(q_abs, "bf16"), dev(q_rope, "bf16"), 2, 1, dev_i64(cu), dev(cache, "bf16"))
+    mla.mla_test_arm_stall()
+    v3_module.attn_decode_latent(*args)
+    s = v3_module.sync_status()
+    assert mla.STATUS_NAMES[s] == "MLA_ERR_TIMEOUT"
+    assert mla.mla_device_error_bits(v3_module.handle) & (1 << 6)
+    o_lat, lse = v3_module.attn_decode_latent(*args)
+    _status_ok(v3_module)
+    lat_ref, lse_ref = orc.attn_decode_latent(q_abs, q_rope, cache, cu, 1, dims)
+    assert rel(host(o_lat), lat_ref) <= TOL["bf16"]
+    assert rel(host(lse), lse_ref) <= TOL["bf16"]
+
+
 def test_decode_is_deterministic(v3_module):
     dims = synth.V3
     lens = np.array([700, 3000])
