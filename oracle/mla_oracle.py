@@ -233,6 +233,44 @@ def mla_prefill(h, cu_seqlens, W, dims, query_rows=None, heads=None):
     return out
 
 
+def mla_prefill_chunk(h, cu_q, cache, cu_kv, W, dims, heads=None):
+    """Chunked prefill against an existing latent cache (section 3 steps (1)-(10), with the sum of
+    step (10) running over every cached position j <= t, and the KV-cache reuse of the explainer's
+    "KV Cache的核心原理" paragraph).
+
+    Sequence b owns cache rows cache[cu_kv[b] : cu_kv[b+1]]. Its last Tc_b = cu_q[b+1] - cu_q[b] rows
+    belong to the chunk's new tokens h[cu_q[b] : cu_q[b+1]], at positions P_b .. P_b + Tc_b - 1 with
+    P_b = (cu_kv[b+1] - cu_kv[b]) - Tc_b; the first P_b rows are the cached prefix and are used as
+    given. The chunk's rows are computed by steps (5) and (7) and written into a copy of the cache;
+    every chunk token then attends over its sequence's rows 0 .. its position (unabsorbed form).
+    Returns dict: cache (with the chunk's rows), rows (chunk token indices), o, o_lat, lse and, when
+    all heads are computed, u.
+    """
+    h = f64(h)
+    cq = np.asarray(cu_q, dtype=np.int64)
+    ck = np.asarray(cu_kv, dtype=np.int64)
+    out_cache = f64(cache).copy()
+    rows, o_l, lat_l, lse_l = [], [], [], []
+    for b in range(len(cq) - 1):
+        tc = int(cq[b + 1] - cq[b])
+        if tc == 0:
+            continue
+        prefix = int(ck[b + 1] - ck[b]) - tc
+        pos = prefix + np.arange(tc, dtype=np.int64)
+        r = np.arange(cq[b], cq[b + 1])
+        c_kv, k_r = kv_compression(h[r], W, dims, pos)
+        out_cache[ck[b] + pos] = cache_rows(c_kv, k_r)
+        seq = out_cache[ck[b]:ck[b + 1]]
+        _, q_c, q_r = query_projections(h[r], W, dims, pos)
+        o, o_lat, lse = attend_unabsorbed(q_c, q_r, seq[:, :dims.d_c], seq[:, dims.d_c:], W, dims, pos, heads)
+        rows.append(r); o_l.append(o); lat_l.append(o_lat); lse_l.append(lse)
+    out = {"cache": out_cache, "rows": np.concatenate(rows), "o": np.concatenate(o_l),
+           "o_lat": np.concatenate(lat_l), "lse": np.concatenate(lse_l)}
+    if heads is None:
+        out["u"] = output_projection(out["o"], W)
+    return out
+
+
 # ---------------------------------------------------------------------------
 # The latent-attention core by its own definition (absorbed score, section 2 【思考】 + section 3)
 # ---------------------------------------------------------------------------

@@ -361,6 +361,38 @@ def test_decode_over_prefill_cache_matches_prefill():
     assert _rel(orc.cache_append(h, pos, W, dims), pre["cache"]) < 1e-15
 
 
+def test_chunked_prefill_equals_prefill_of_the_whole_sequence():
+    # prefill of [prefix; chunk] == prefill of the prefix, then the chunk against the cached prefix;
+    # two sequences with different prefix and chunk lengths, then a second chunk on top
+    dims = synth.TINY
+    W = _weights(dims, seed=61)
+    lens = [30, 19]
+    cu = synth.cu_seqlens(lens)
+    h = synth.hidden(dims, int(cu[-1]), seed=62, dtype="fp32")
+    full = orc.mla_prefill(h, cu, W, dims)
+    splits = [(12, 10), (5, 9)]           # per sequence: (prefix, first chunk); the rest is a second chunk
+    cache = np.zeros_like(full["cache"])
+    pre_rows = np.concatenate([np.arange(cu[b], cu[b] + splits[b][0]) for b in range(2)])
+    cache[pre_rows] = full["cache"][pre_rows]
+    step_cache = cache
+    done = [s[0] for s in splits]
+    for part in (0, 1):
+        take = [splits[b][1] if part == 0 else lens[b] - splits[b][0] - splits[b][1] for b in range(2)]
+        q_rows = np.concatenate([np.arange(cu[b] + done[b], cu[b] + done[b] + take[b]) for b in range(2)])
+        kv_lens = [done[b] + take[b] for b in range(2)]
+        # the cache of this call holds each sequence's first kv_lens[b] rows, packed
+        idx = np.concatenate([np.arange(cu[b], cu[b] + kv_lens[b]) for b in range(2)])
+        out = orc.mla_prefill_chunk(h[q_rows], synth.cu_seqlens(take), step_cache[idx], synth.cu_seqlens(kv_lens), W,
+                                    dims)
+        assert _rel(out["u"], full["u"][q_rows]) < 1e-12
+        assert _rel(out["o_lat"], full["o_lat"][q_rows]) < 1e-12
+        assert _rel(out["cache"], full["cache"][idx]) < 1e-15
+        step_cache = step_cache.copy()
+        step_cache[idx] = out["cache"]
+        done = kv_lens
+    assert done == lens
+
+
 # ---------------------------------------------------------------------------
 # Split-KV combine: exact identity of the softmax over disjoint key sets
 # ---------------------------------------------------------------------------
