@@ -39,6 +39,7 @@ TID_H, TID_WDQ, TID_WUQ, TID_WQR, TID_WDKV, TID_WKR, TID_WUK, TID_WUV, TID_WO = 
 TID_CACHE_C, TID_CACHE_KR, TID_LENGTHS = 9, 10, 11
 TID_POSITIONS, TID_SLOTS = 12, 13
 TID_QC, TID_QR, TID_KC, TID_VC = 14, 15, 16, 17   # inputs of the prefill attention core alone
+TID_GQ, TID_GKV = 18, 19                          # RMSNorm gains of c^Q and c^KV
 
 _CHUNK = 1 << 22
 
@@ -91,15 +92,15 @@ def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
     return (rounded.astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def normal(seed: int, tensor_id: int, shape, std: float = 1.0, dtype: str = "bf16") -> np.ndarray:
-    """N(0, std^2) draws rounded to dtype. Chunks are independent (counter based), so they are drawn
+def normal(seed: int, tensor_id: int, shape, std: float = 1.0, dtype: str = "bf16", mean: float = 0.0) -> np.ndarray:
+    """N(mean, std^2) draws rounded to dtype. Chunks are independent (counter based), so they are drawn
     on a thread pool; the values do not depend on the number of threads."""
     n = int(np.prod(shape))
     out = np.empty(n, dtype=np.float32)
 
     def fill(lo):
         hi = min(n, lo + _CHUNK)
-        out[lo:hi] = round_to(normal_f64(seed, tensor_id, hi - lo, start=lo) * std, dtype)
+        out[lo:hi] = round_to(normal_f64(seed, tensor_id, hi - lo, start=lo) * std + mean, dtype)
 
     starts = range(0, n, _CHUNK)
     if n <= _CHUNK:
@@ -167,6 +168,12 @@ class Dims:
     d_cq: int
     d_r: int
     rope_base: float = 10000.0
+    # YaRN context extension of the decoupled RoPE (s = 1: plain RoPE) and its original context
+    yarn_s: float = 1.0
+    yarn_alpha: float = 1.0
+    yarn_beta: float = 32.0
+    yarn_l0: int = 4096
+    rms_eps: float = 1e-6       # RMSNorm epsilon (the norm is on when the weights carry its gains)
 
     @property
     def row(self) -> int:
@@ -176,6 +183,11 @@ class Dims:
 
 TINY = Dims(d=256, n_h=4, d_h=32, d_c=64, d_cq=96, d_r=16)
 V3 = Dims(d=7168, n_h=128, d_h=128, d_c=512, d_cq=1536, d_r=64)
+# the DeepSeek-V3 long-context settings: YaRN with s = 40, alpha = 1, beta = 32 from a 4K context
+V3_YARN = Dims(d=7168, n_h=128, d_h=128, d_c=512, d_cq=1536, d_r=64, yarn_s=40.0, yarn_alpha=1.0, yarn_beta=32.0,
+               yarn_l0=4096)
+TINY_YARN = Dims(d=256, n_h=4, d_h=32, d_c=64, d_cq=96, d_r=16, yarn_s=40.0, yarn_alpha=1.0, yarn_beta=32.0,
+                 yarn_l0=64)
 
 # Weight name -> (tensor id, shape(dims) [out, in]); std = 1/sqrt(fan_in) with fan_in = in.
 WEIGHT_SPECS = {
@@ -198,6 +210,12 @@ def weights(dims: Dims, seed: int = 0, dtype: str = "bf16", names=None) -> dict:
         shape = shape_fn(dims)
         out[name] = normal(seed, tid, shape, std=1.0 / np.sqrt(shape[1]), dtype=dtype)
     return out
+
+
+def gains(dims: Dims, seed: int = 0, dtype: str = "bf16") -> dict:
+    """Synthetic RMSNorm gains g_q [d_cq] and g_kv [d_c]: 1 + 0.25 N(0,1) each."""
+    return {"g_q": normal(seed, TID_GQ, (dims.d_cq,), std=0.25, dtype=dtype, mean=1.0),
+            "g_kv": normal(seed, TID_GKV, (dims.d_c,), std=0.25, dtype=dtype, mean=1.0)}
 
 
 def hidden(dims: Dims, tokens: int, seed: int = 0, dtype: str = "bf16") -> np.ndarray:

@@ -16,6 +16,8 @@ Source. The definitions follow the notes "【论文解读】DeepSeek-V3"
                                  per head, shared k^R = RoPE(W^KR h), score scale
                                  1/sqrt(d_h + d_h^R), and the ten-step computation
                                  (1)-(10) that this file spells out.
+Section 三(二) "模型超参数" / "长上下文扩展" adds the RMSNorm after the latent
+compression and YaRN on the decoupled key (readings R4, R4').
 Decode semantics (cache the keys/values of past tokens, compute only the new
 query, attend over every cached position) follow the explainer at
 mlqm.cn/news/135256, paragraph "KV Cache的核心原理".
@@ -25,7 +27,18 @@ Readings where the pages leave a step open (each is also listed in the design doc):
      form, rotated by [[cos, -sin], [sin, cos]] with angle pos * base^(-2m/d_R).
   R2 Positions are 0-based within a sequence; packing does not shift them.
   R3 The scale is 1/sqrt(d_h + d_h^R) in both the absorbed and unabsorbed forms.
-  R4 No RMSNorm on c^Q / c^KV (no equation of the section has one) and no YaRN.
+  R4 RMSNorm and YaRN are opt-in (no equation of section 一(一) has them; section
+     三(二) names both). RMSNorm after the latent compression, when the weights carry
+     gains g_q [d_c'] and g_kv [d_c]: c^Q = RMSNorm(W^DQ h), c^KV = RMSNorm(W^DKV h)
+     with y = x / sqrt(mean(x^2) + eps) * g; k^R = RoPE(W^KR h) is not normalised
+     (its input is h). eps is not on the pages: 1e-6 by default.
+  R4' YaRN (section 三(二)3: s = 40, alpha = 1, beta = 32, sqrt(t) = 0.1 ln s + 1,
+     for the decoupled key only), when s > 1: the "NTK-by-parts" frequencies of the
+     YaRN paper from the original context L0 = 4096 (the 4K pre-training length),
+     r_m = L0 theta_m / (2 pi), gamma = clip((r - alpha) / (beta - alpha), 0, 1),
+     theta'_m = (1 - gamma) theta_m / s + gamma theta_m; the factor 0.1 ln s + 1
+     multiplies each rotated vector, q^R and k^R alike, so the RoPE term of the
+     score grows by its square and the latent term is untouched.
   R5 Decode: a sequence's cache length includes its Tq new tokens (appended
      first); query k sits at position len - Tq + k and sees rows j <= position.
   R6 A synthetic decode cache holds c^KV and an already-rotated k^R.
@@ -47,6 +60,33 @@ def f64(x) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # RoPE (section 3, the R_m block-diagonal rotation; reading R1)
 # ---------------------------------------------------------------------------
+def yarn_frequencies(d_r: int, base: float, s: float, alpha: float, beta: float, l0: int) -> np.ndarray:
+    """YaRN's interpolated RoPE frequencies (reading R4'), m = 0..d_r/2-1.
+
+    Pair m turns r_m = L0 / lambda_m times over the original context, lambda_m = 2 pi / theta_m.
+    Pairs that turn more than beta times keep theta_m, pairs that turn less than alpha times are
+    interpolated fully (theta_m / s), and the pairs in between are blended linearly in r.
+    """
+    m = np.arange(d_r // 2, dtype=np.float64)
+    theta = base ** (-2.0 * m / d_r)
+    r = l0 * theta / (2.0 * np.pi)
+    gamma = np.clip((r - alpha) / (beta - alpha), 0.0, 1.0)
+    return (1.0 - gamma) * theta / s + gamma * theta
+
+
+def rope_scale(dims) -> float:
+    """The factor on each rotated vector: 0.1 ln s + 1 with YaRN (s > 1), else 1 (reading R4')."""
+    return 0.1 * np.log(dims.yarn_s) + 1.0 if dims.yarn_s > 1.0 else 1.0
+
+
+def rope_frequencies(d_r: int, dims) -> np.ndarray:
+    """theta_m = base^(-2m/d_r) (reading R1), or YaRN's interpolated table when s > 1."""
+    if dims.yarn_s > 1.0:
+        return yarn_frequencies(d_r, dims.rope_base, dims.yarn_s, dims.yarn_alpha, dims.yarn_beta, dims.yarn_l0)
+    m = np.arange(d_r // 2, dtype=np.float64)
+    return dims.rope_base ** (-2.0 * m / d_r)
+
+
 def rope_angles(pos, d_r: int, base: float) -> np.ndarray:
     """Angles pos * theta_m with theta_m = base^(-2m/d_r), m = 0..d_r/2-1; shape pos.shape + (d_r/2,)."""
     m = np.arange(d_r // 2, dtype=np.float64)
@@ -54,18 +94,36 @@ def rope_angles(pos, d_r: int, base: float) -> np.ndarray:
     return f64(pos)[..., None] * theta
 
 
-def rope(x, pos, base: float) -> np.ndarray:
-    """Rotate each pair (x_2m, x_2m+1) of the last axis by the angle of position pos.
-
-    pos must broadcast against x.shape[:-1].
-    """
+def rotate(x, ang) -> np.ndarray:
+    """Rotate each pair (x_2m, x_2m+1) of the last axis by ang[..., m]."""
     x = f64(x)
-    ang = rope_angles(pos, x.shape[-1], base)
     c, s = np.cos(ang), np.sin(ang)
     x0, x1 = x[..., 0::2], x[..., 1::2]
     a = x0 * c - x1 * s
     b = x0 * s + x1 * c
     return np.stack([a, b], axis=-1).reshape(a.shape[:-1] + (2 * a.shape[-1],))
+
+
+def rope(x, pos, base: float) -> np.ndarray:
+    """Rotate each pair (x_2m, x_2m+1) of the last axis by the angle of position pos.
+
+    pos must broadcast against x.shape[:-1].
+    """
+    return rotate(x, rope_angles(pos, f64(x).shape[-1], base))
+
+
+def rope_dims(x, pos, dims) -> np.ndarray:
+    """The decoupled RoPE of a layer: plain (rope) or, with YaRN, its frequencies and factor."""
+    if dims.yarn_s <= 1.0:
+        return rope(x, pos, dims.rope_base)
+    ang = f64(pos)[..., None] * rope_frequencies(f64(x).shape[-1], dims)
+    return rope_scale(dims) * rotate(x, ang)
+
+
+def rms_norm(x, g, eps: float) -> np.ndarray:
+    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * g (reading R4)."""
+    x = f64(x)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * f64(g)
 
 
 # ---------------------------------------------------------------------------
@@ -74,22 +132,31 @@ def rope(x, pos, base: float) -> np.ndarray:
 def query_projections(h, W, dims, pos):
     """Steps (1)-(3): c^Q = W^DQ h; q^C = W^UQ c^Q split by heads; q^R = RoPE(W^QR c^Q) per head.
 
+    With gains W["g_q"], c^Q = RMSNorm(W^DQ h) (reading R4); RoPE follows dims (YaRN, reading R4').
+
     h [T, d], pos [T] -> c_q [T, d_cq], q_c [T, n_h, d_h], q_r [T, n_h, d_r].
     """
     h = f64(h)
     T = h.shape[0]
     c_q = h @ f64(W["w_dq"]).T
+    if "g_q" in W:
+        c_q = rms_norm(c_q, W["g_q"], dims.rms_eps)
     q_c = (c_q @ f64(W["w_uq"]).T).reshape(T, dims.n_h, dims.d_h)
     q_r_hat = (c_q @ f64(W["w_qr"]).T).reshape(T, dims.n_h, dims.d_r)
-    q_r = rope(q_r_hat, f64(pos)[:, None], dims.rope_base)
+    q_r = rope_dims(q_r_hat, f64(pos)[:, None], dims)
     return c_q, q_c, q_r
 
 
 def kv_compression(h, W, dims, pos):
-    """Steps (5) and (7): c^KV = W^DKV h and k^R = RoPE(W^KR h). Returns c_kv [T, d_c], k_r [T, d_r]."""
+    """Steps (5) and (7): c^KV = W^DKV h and k^R = RoPE(W^KR h). Returns c_kv [T, d_c], k_r [T, d_r].
+
+    With gains W["g_kv"], c^KV = RMSNorm(W^DKV h) (reading R4); RoPE follows dims (YaRN, reading R4').
+    """
     h = f64(h)
     c_kv = h @ f64(W["w_dkv"]).T
-    k_r = rope(h @ f64(W["w_kr"]).T, pos, dims.rope_base)
+    if "g_kv" in W:
+        c_kv = rms_norm(c_kv, W["g_kv"], dims.rms_eps)
+    k_r = rope_dims(h @ f64(W["w_kr"]).T, pos, dims)
     return c_kv, k_r
 
 

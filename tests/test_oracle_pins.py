@@ -394,6 +394,120 @@ def test_chunked_prefill_equals_prefill_of_the_whole_sequence():
 
 
 # ---------------------------------------------------------------------------
+# YaRN on the decoupled RoPE (section 三(二)3 "长上下文扩展": s = 40, alpha = 1, beta = 32,
+# sqrt(t) = 0.1 ln s + 1, for the decoupled key only) and the RMSNorm after the latent
+# compression (section 三(二)1 "模型超参数"); both opt-in
+# ---------------------------------------------------------------------------
+def test_yarn_with_s_one_is_plain_rope():
+    import dataclasses
+    d1 = dataclasses.replace(synth.V3_YARN, yarn_s=1.0)
+    x = np.random.default_rng(0).standard_normal((5, 64))
+    pos = np.array([0, 1, 77, 4095, 131071])[:, None]
+    assert np.array_equal(orc.rope_dims(x, pos, d1), orc.rope(x, pos, 10000.0))
+    theta = 10000.0 ** (-2.0 * np.arange(32) / 64)
+    assert _rel(orc.yarn_frequencies(64, 10000.0, 1.0, 1.0, 32.0, 4096), theta) < 1e-15
+    assert orc.rope_scale(d1) == 1.0
+
+
+def test_yarn_frequencies_by_parts_closed_form():
+    # d_r = 4, base 100: theta = [1, 0.1]; L0 chosen so that pair 1 turns 16.5 times over it, the
+    # middle of the ramp [1, 32]: gamma = 1/2 and theta' = (0.1 / 40 + 0.1) / 2 = 0.05125; pair 0 turns
+    # 165 times (> beta) and keeps theta = 1
+    l0 = 16.5 * 2.0 * math.pi / 0.1
+    th = orc.yarn_frequencies(4, 100.0, 40.0, 1.0, 32.0, l0)
+    assert abs(th[0] - 1.0) < 1e-15
+    assert abs(th[1] - 0.05125) < 1e-15
+    # the DeepSeek-V3 table: the fastest pair (lambda = 2 pi, 652 turns over 4K) unchanged, the slowest
+    # (lambda ~ 4.7e4 > 4K: under one turn) divided by s exactly, and every pair in between blended
+    th = orc.yarn_frequencies(64, 10000.0, 40.0, 1.0, 32.0, 4096)
+    theta = 10000.0 ** (-2.0 * np.arange(32) / 64)
+    turns = 4096 * theta / (2 * math.pi)
+    assert th[0] == theta[0]
+    assert np.all(th[turns > 32] == theta[turns > 32])
+    assert np.allclose(th[turns < 1], theta[turns < 1] / 40, rtol=1e-15, atol=0)
+    mid = (turns >= 1) & (turns <= 32)
+    assert mid.sum() >= 3
+    assert np.all((th[mid] <= theta[mid]) & (th[mid] >= theta[mid] / 40))
+    # blending is linear in the number of turns
+    g = (turns[mid] - 1) / 31
+    assert _rel(th[mid], (1 - g) * theta[mid] / 40 + g * theta[mid]) < 1e-15
+
+
+def test_yarn_scale_and_relative_position():
+    dims = synth.V3_YARN
+    m = orc.rope_scale(dims)
+    assert abs(m - (0.1 * math.log(40.0) + 1.0)) < 1e-15 and abs(m - 1.3688879454113936) < 1e-12
+    rng = np.random.default_rng(1)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    # every rotated pair keeps its length times the factor
+    rq = orc.rope_dims(q, np.array(1000), dims)
+    assert _rel(np.hypot(rq[0::2], rq[1::2]), m * np.hypot(q[0::2], q[1::2])) < 1e-13
+    # the RoPE score depends on the relative position only, and carries the factor squared
+    s1 = orc.rope_dims(q, np.array(70000), dims) @ orc.rope_dims(k, np.array(50000), dims)
+    s2 = orc.rope_dims(q, np.array(20123), dims) @ orc.rope_dims(k, np.array(123), dims)
+    assert abs(s1 - s2) < 1e-9 * abs(s1)
+    theta = orc.yarn_frequencies(64, 10000.0, 40.0, 1.0, 32.0, 4096)
+    ref = m * m * (orc.rotate(q, 20000.0 * theta) @ k)
+    assert abs(s1 - ref) < 1e-9 * abs(ref)
+
+
+def test_rms_norm_closed_forms():
+    # [3, 4]: mean square 12.5
+    assert _rel(orc.rms_norm([3.0, 4.0], [1.0, 1.0], 0.0), [3 / math.sqrt(12.5), 4 / math.sqrt(12.5)]) < 1e-15
+    # a constant row normalises to the gains; eps enters under the root
+    g = np.array([0.5, 2.0, -1.0])
+    assert _rel(orc.rms_norm([7.0, 7.0, 7.0], g, 0.0), g) < 1e-15
+    assert _rel(orc.rms_norm([2.0, 2.0, 2.0], g, 5.0), g * 2 / 3) < 1e-15
+    x = np.random.default_rng(2).standard_normal((4, 96))
+    assert _rel(orc.rms_norm(3.5 * x, np.ones(96), 0.0), orc.rms_norm(x, np.ones(96), 0.0)) < 1e-14
+    y = orc.rms_norm(x, np.ones(96), 0.0)
+    assert _rel(np.mean(y * y, axis=1), np.ones(4)) < 1e-14
+
+
+def test_rmsnorm_sits_on_the_latent_vectors_only():
+    # with the norm's gains and eps = 0, scaling h leaves c^Q, q^C, q^R and c^KV unchanged, while k^R
+    # (RoPE(W^KR h), not normalised) scales with h; without gains everything scales
+    import dataclasses
+    dims = dataclasses.replace(synth.TINY, rms_eps=0.0)
+    W = _weights(dims, seed=70)
+    Wn = dict(W, **synth.gains(dims, seed=71, dtype="fp32"))
+    h = synth.hidden(dims, 6, seed=72, dtype="fp32").astype(np.float64)
+    pos = np.arange(6) * 11
+    a, b = orc.query_projections(h, Wn, dims, pos), orc.query_projections(3.0 * h, Wn, dims, pos)
+    for x, y in zip(a, b):
+        assert _rel(y, x) < 1e-13
+    (c1, k1), (c2, k2) = orc.kv_compression(h, Wn, dims, pos), orc.kv_compression(3.0 * h, Wn, dims, pos)
+    assert _rel(c2, c1) < 1e-13
+    assert _rel(k2, 3.0 * k1) < 1e-13
+    # the gains act per latent column: c^KV / g_kv has mean square 1 in every row
+    r = c1 / Wn["g_kv"]
+    assert _rel(np.mean(r * r, axis=1), np.ones(6)) < 1e-13
+    cq = a[0] / Wn["g_q"]
+    assert _rel(np.mean(cq * cq, axis=1), np.ones(6)) < 1e-13
+    # no gains: the projections are linear in h
+    p1, p2 = orc.query_projections(h, W, dims, pos), orc.query_projections(3.0 * h, W, dims, pos)
+    assert _rel(p2[0], 3.0 * p1[0]) < 1e-13
+
+
+@pytest.mark.parametrize("tq", [1, 2])
+def test_absorbed_equals_unabsorbed_with_rmsnorm_and_yarn(tq):
+    dims = synth.TINY_YARN
+    W = dict(_weights(dims, seed=73), **synth.gains(dims, seed=74, dtype="fp32"))
+    lens = np.array([5, 70, 2 * tq, 40])
+    cu = synth.cu_seqlens(lens)
+    cache = synth.latent_cache(dims, int(cu[-1]), seed=75, dtype="fp32")
+    h_q = synth.hidden(dims, len(lens) * tq, seed=76, dtype="fp32")
+    un = orc.mla_decode(h_q, cache, cu, tq, W, dims)
+    ab = orc.mla_decode_absorbed(h_q, cache, cu, tq, W, dims)
+    assert _rel(ab["u"], un["u"]) < 1e-12
+    # decode over a prefill-built cache equals the prefill, with both options on
+    h = synth.hidden(dims, 90, seed=77, dtype="fp32")
+    pre = orc.mla_prefill(h, synth.cu_seqlens([90]), W, dims)
+    dec = orc.mla_decode(h[90 - tq:], pre["cache"], synth.cu_seqlens([90]), tq, W, dims)
+    assert _rel(dec["u"], pre["u"][90 - tq:]) < 1e-12
+
+
+# ---------------------------------------------------------------------------
 # Split-KV combine: exact identity of the softmax over disjoint key sets
 # ---------------------------------------------------------------------------
 def test_lse_combine_of_any_split_equals_unsplit():
@@ -464,10 +578,29 @@ def _attend_off_by_one(q, k, v, lat, qpos, scale):
 
 
 _ORIG_ATTEND = orc.causal_softmax_attend
+_ORIG_YARN = orc.yarn_frequencies
+
+
+def _yarn_ramp_inverted(d_r, base, s, alpha, beta, l0):
+    m = np.arange(d_r // 2, dtype=np.float64)
+    theta = base ** (-2.0 * m / d_r)
+    gamma = np.clip((2.0 * np.pi / (l0 * theta) - alpha) / (beta - alpha), 0.0, 1.0)   # wavelength ratio upside down
+    return (1.0 - gamma) * theta / s + gamma * theta
+
+
+def _yarn_scale_once(dims):
+    return math.sqrt(0.1 * math.log(dims.yarn_s) + 1.0) if dims.yarn_s > 1.0 else 1.0
+
+
+def _rms_norm_sum(x, g, eps):
+    x = np.asarray(x, np.float64)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps) * np.asarray(g, np.float64)
 
 PINS = [test_rope_closed_form_two_dims, test_rope_frequencies, lambda: test_oracle_equals_sdpa_on_tiny_prefill(),
         lambda: test_brute_force_tiny_random(0), lambda: test_brute_force_tiny_random(1),
-        lambda: test_zero_rope_weights_reduce_to_plain_mha(), test_causality_rows_after_position_do_not_matter]
+        lambda: test_zero_rope_weights_reduce_to_plain_mha(), test_causality_rows_after_position_do_not_matter,
+        test_yarn_frequencies_by_parts_closed_form, test_yarn_scale_and_relative_position, test_rms_norm_closed_forms,
+        test_rmsnorm_sits_on_the_latent_vectors_only]
 
 
 @pytest.mark.parametrize("name,attr,fake", [
@@ -476,6 +609,9 @@ PINS = [test_rope_closed_form_two_dims, test_rope_frequencies, lambda: test_orac
     ("W^UK head split transposed", "up_project_head", _up_project_transposed_heads),
     ("scale 1/sqrt(d_h)", "causal_softmax_attend", _attend_wrong_scale),
     ("causal window off by one", "causal_softmax_attend", _attend_off_by_one),
+    ("YaRN ramp on the wavelength ratio", "yarn_frequencies", _yarn_ramp_inverted),
+    ("YaRN factor on the score, not on each vector", "rope_scale", _yarn_scale_once),
+    ("RMSNorm over the sum of squares", "rms_norm", _rms_norm_sum),
 ])
 def test_planted_mistakes_are_caught(monkeypatch, name, attr, fake):
     monkeypatch.setattr(orc, attr, fake)
