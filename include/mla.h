@@ -107,6 +107,23 @@ mla_status_t mla_create(const mla_dims_t *dims, mla_dtype_t dtype, int device, m
  * allocates the handle's 4-byte device error word. */
 mla_status_t mla_set_weights(mla_handle_t *h, const mla_weights_t *w);
 
+/* Opt-in RMSNorm after the latent compression (section 三(二)1 of the notes): c^Q = RMSNorm(W^DQ h)
+ * and c^KV = RMSNorm(W^DKV h), y = x / sqrt(mean(x^2) + eps) * g, applied by every later call
+ * that computes c^Q or c^KV (the cache rows hold the normalised c^KV; k^R = RoPE(W^KR h) is not
+ * normalised). g_q [d_cq] and g_kv [d_c] are device pointers in the handle dtype, borrowed; both
+ * NULL turns the norm off (the default). Both or neither; eps >= 0. Host-only. */
+mla_status_t mla_set_rmsnorm(mla_handle_t *h, const void *g_q, const void *g_kv, double eps);
+
+/* Opt-in YaRN context extension of the decoupled RoPE (section 三(二)3 of the notes; the
+ * DeepSeek-V3 values are s = 40, alpha = 1, beta = 32 from a 4096-token original context).
+ * Pair m of the d_r-wide RoPE blocks turns r_m = original_len * theta_m / (2 pi) times over the
+ * original context (theta_m = rope_base^(-2m/d_r)); gamma = clamp((r_m - alpha) / (beta - alpha),
+ * 0, 1) and the frequency becomes (1 - gamma) theta_m / s + gamma theta_m. Each rotated vector,
+ * q^R and k^R alike, is multiplied by 0.1 ln s + 1, so the RoPE term of every score grows by its
+ * square. s = 1 turns it off (the default). s >= 1, beta > alpha, original_len > 0. Host-only;
+ * cache rows written under one setting must be read under the same one. */
+mla_status_t mla_set_yarn(mla_handle_t *h, double s, double alpha, double beta, double original_len);
+
 /* Workspace bytes for one call of `op` on num_seqs sequences with tq query tokens each
  * (decode, attention core) or total_tokens packed tokens (prefill, cache append).
  * Host-only arithmetic. */
@@ -178,6 +195,54 @@ mla_status_t mla_decode(mla_handle_t *h, const void *h_q, int64_t B, int32_t Tq,
 mla_status_t mla_prefill(mla_handle_t *h, const void *hidden, int64_t B, const int64_t *cu_seqlens,
                          int64_t total_tokens, int64_t max_seqlen, void *cache, int64_t capacity,
                          void *u_out, void *ws, size_t ws_bytes, mla_stream_t stream);
+
+/* The two forms a chunked prefill can take (mla_prefill_chunk). */
+typedef enum {
+  MLA_CHUNK_AUTO = 0,        /* chosen by the chunk / prefix ratio (see mla_prefill_chunk)            */
+  MLA_CHUNK_ABSORBED = 1,    /* the decode form: q~ = W^UK^T q^C, the latent core, W^UV; needs chunks  */
+                             /* of one length Tc <= 64 (total_q == B * max_q)                          */
+  MLA_CHUNK_UNABSORBED = 2   /* the prefill form: k^C, v^C = W^UK c^KV, W^UV c^KV for every key row    */
+} mla_chunk_form_t;
+
+/* Chunked prefill against an existing latent cache: step (10) of section 一(一)3 with the sum over
+ * every cached position j <= t, where the rows of the earlier positions are already in the cache
+ * and are reused as they are (the KV-cache reuse of mlqm.cn/news/135256, "KV Cache的核心原理").
+ * Sequence b owns cache rows cu_kv[b] .. cu_kv[b+1]; its chunk is the last Tc_b = cu_q[b+1] -
+ * cu_q[b] of them, at positions P_b .. P_b + Tc_b - 1 with P_b = (cu_kv[b+1] - cu_kv[b]) - Tc_b.
+ * The call writes the chunk's cache rows (steps (5), (7)), computes its queries (steps (1)-(3)),
+ * lets each chunk token attend to rows 0 .. its position of its sequence, and applies W^O.
+ * The first P_b rows of each sequence must hold the cache rows of its earlier tokens.
+ *   hidden   [total_q, d]            chunk tokens, packed by cu_q (cu_q[B] == total_q)
+ *   cu_q     [B + 1] device int64    chunk tokens per sequence (a chunk may be empty)
+ *   max_q    upper bound on any chunk length
+ *   cu_kv    [B + 1] device int64    cache rows per sequence INCLUDING its chunk (cu_kv[B] == total_kv)
+ *   cache    [capacity, d_c + d_r]   capacity >= total_kv
+ *   form     MLA_CHUNK_AUTO takes the absorbed form when the chunks share one length Tc <= 64
+ *            (total_q == B * max_q) and the key rows number at least twice the chunk tokens
+ *            (total_kv >= 2 total_q): its cost grows with Tc x rows, the unabsorbed form's with
+ *            the rows x the up-projection of every row, so short chunks on long prefixes favour it.
+ *            A forced MLA_CHUNK_ABSORBED with other chunk shapes returns MLA_ERR_INVALID_ARG.
+ *   u_out    [total_q, d]            handle dtype
+ *   ws       mla_prefill_chunk_workspace() bytes for the same arguments
+ * Device checks (MLA_ERR_DEVICE_CHECK through mla_sync_status): cu_q[0] = cu_kv[0] = 0, both
+ * non-decreasing, cu_kv[B] <= capacity, Tc_b <= len_b, Tc_b <= max_q, the two totals. */
+mla_status_t mla_prefill_chunk(mla_handle_t *h, const void *hidden, int64_t B, const int64_t *cu_q,
+                               int64_t total_q, int64_t max_q, const int64_t *cu_kv, int64_t total_kv,
+                               void *cache, int64_t capacity, mla_chunk_form_t form, void *u_out, void *ws,
+                               size_t ws_bytes, mla_stream_t stream);
+
+/* The form mla_prefill_chunk takes for these arguments (AUTO resolved) and its workspace bytes.
+ * Host-only arithmetic. */
+mla_status_t mla_prefill_chunk_workspace(const mla_handle_t *h, int64_t B, int64_t total_q, int64_t max_q,
+                                         int64_t total_kv, mla_chunk_form_t form, mla_chunk_form_t *chosen,
+                                         size_t *bytes);
+
+/* Byte offset of a named region of that workspace: CQ, QC, QR, O in both forms; QABS, OLAT, LSE in
+ * the absorbed form ([B * Tc] tokens); KC, VC in the unabsorbed form ([total_kv] key rows).
+ * MLA_ERR_INVALID_ARG if the chosen form has no such region. Host-only arithmetic. */
+mla_status_t mla_prefill_chunk_offset(const mla_handle_t *h, int64_t B, int64_t total_q, int64_t max_q,
+                                      int64_t total_kv, mla_chunk_form_t form, mla_buffer_t which,
+                                      size_t *offset);
 
 /* The latent attention core alone (decode semantics as mla_decode):
  *   q_abs  [B*Tq, n_h, d_c]  handle dtype (q~ = W_i^UK^T q^C_i)

@@ -23,6 +23,7 @@ struct mla_handle {
   uint32_t* d_err;         // device error word (sticky until mla_sync_status)
   uint32_t last_err_bits;  // last word read by mla_sync_status
   int num_sms;
+  mla::LayerOpts opts;     // RMSNorm gains and the RoPE (plain or YaRN)
 };
 
 namespace mla {
@@ -93,12 +94,16 @@ struct Layout {
   size_t off[9];
   bool has[9];
   size_t pos_off;     // int64 positions [T]
+  size_t slot_off;    // int64 cache rows [T] (chunked prefill only)
   size_t tc_off;      // tensor-core attention scratch
   size_t total;
 };
 
-// Workspace layout of one call; every region starts on a 1024-byte boundary.
-Layout layout(const mla_handle* h, mla_op_t op, int64_t B, int32_t tq, int64_t total_tokens) {
+// Workspace layout of one call; every region starts on a 1024-byte boundary. A chunked prefill
+// (kv_rows >= 0) takes the decode layout (absorbed form, B sequences of tq tokens) or the prefill
+// layout with k^C / v^C over kv_rows key rows (unabsorbed form), plus the chunk's cache rows.
+Layout layout(const mla_handle* h, mla_op_t op, int64_t B, int32_t tq, int64_t total_tokens,
+              int64_t kv_rows = -1) {
   Layout L;
   memset(&L, 0, sizeof(L));
   const mla_dims_t& d = h->dims;
@@ -122,16 +127,26 @@ Layout layout(const mla_handle* h, mla_op_t op, int64_t B, int32_t tq, int64_t t
     take(MLA_BUF_LSE, (size_t)T * d.n_h * sizeof(float));
   }
   if (op == MLA_OP_PREFILL) {
-    take(MLA_BUF_KC, (size_t)T * d.n_h * d.d_h * es);
-    take(MLA_BUF_VC, (size_t)T * d.n_h * d.d_h * es);
+    const int64_t KV = kv_rows >= 0 ? kv_rows : T;
+    take(MLA_BUF_KC, (size_t)KV * d.n_h * d.d_h * es);
+    take(MLA_BUF_VC, (size_t)KV * d.n_h * d.d_h * es);
   }
   if (op != MLA_OP_CACHE_APPEND) {
     L.pos_off = cur;
     cur = align_up(cur + (size_t)(T > 0 ? T : 1) * sizeof(int64_t));
   }
+  if (kv_rows >= 0) {
+    L.slot_off = cur;
+    cur = align_up(cur + (size_t)(T > 0 ? T : 1) * sizeof(int64_t));
+  }
   if (tc_dims(h)) {
     L.tc_off = cur;
-    if (op == MLA_OP_DECODE) cur = align_up(cur + mla::tc_decode_scratch_bytes(d, B, tq));
+    if (op == MLA_OP_DECODE && kv_rows >= 0) {
+      // the chunk's cache rows are written first, with the same scratch
+      const size_t a = mla::tc_decode_scratch_bytes(d, B, tq), b = mla::tc_append_scratch_bytes(d, T);
+      cur = align_up(cur + (a > b ? a : b));
+    }
+    if (op == MLA_OP_DECODE && kv_rows < 0) cur = align_up(cur + mla::tc_decode_scratch_bytes(d, B, tq));
     if (op == MLA_OP_ATTN_DECODE_LATENT) cur = align_up(cur + mla::tc_core_scratch_bytes(d, B, tq));
     if (op == MLA_OP_CACHE_APPEND) cur = align_up(cur + mla::tc_append_scratch_bytes(d, total_tokens));
   }
@@ -193,9 +208,12 @@ mla_status_t simt_cache_rows(const mla_handle* h, const void* hidden, const int6
   a.rowmap = rowmap; a.rowmap_limit = capacity;
   mla_status_t s = run_simt_gemm(h, a, st);
   if (s != MLA_OK) return s;
+  if (h->opts.g_kv)
+    MLA_TRY(mla::rmsnorm_rows(cache, h->dtype == MLA_BF16, R, rowmap, capacity, T, d.d_c, h->opts.g_kv, h->opts.eps,
+                              st));
   SimtGemmArgs b = dense_nt(hidden, d.d, h->w.w_kr, (char*)cache + (size_t)d.d_c * es, R, T, d.d_r, d.d);
   b.rowmap = rowmap; b.rowmap_limit = capacity;
-  b.pos = pos; b.rope_col0 = 0; b.d_r = d.d_r; b.rope_base = d.rope_base;
+  b.pos = pos; b.rope_col0 = 0; b.d_r = d.d_r; b.rope = h->opts.rope;
   return run_simt_gemm(h, b, st);
 }
 
@@ -205,11 +223,13 @@ mla_status_t simt_queries(const mla_handle* h, const void* hidden, const int64_t
   const mla_dims_t& d = h->dims;
   mla_status_t s = run_simt_gemm(h, dense_nt(hidden, d.d, h->w.w_dq, cq, d.d_cq, T, d.d_cq, d.d), st);
   if (s != MLA_OK) return s;
+  if (h->opts.g_q)
+    MLA_TRY(mla::rmsnorm_rows(cq, h->dtype == MLA_BF16, d.d_cq, nullptr, T, T, d.d_cq, h->opts.g_q, h->opts.eps, st));
   s = run_simt_gemm(h, dense_nt(cq, d.d_cq, h->w.w_uq, qc, (int64_t)d.n_h * d.d_h, T, (int64_t)d.n_h * d.d_h,
                                 d.d_cq), st);
   if (s != MLA_OK) return s;
   SimtGemmArgs a = dense_nt(cq, d.d_cq, h->w.w_qr, qr, (int64_t)d.n_h * d.d_r, T, (int64_t)d.n_h * d.d_r, d.d_cq);
-  a.pos = pos; a.rope_col0 = 0; a.d_r = d.d_r; a.rope_base = d.rope_base;
+  a.pos = pos; a.rope_col0 = 0; a.d_r = d.d_r; a.rope = h->opts.rope;
   return run_simt_gemm(h, a, st);
 }
 
@@ -282,7 +302,24 @@ mla_status_t mla_create(const mla_dims_t* dims, mla_dtype_t dtype, int device, m
   h->dims = d;
   h->dtype = dtype;
   h->device = device;
+  h->opts.eps = 1e-6f;
+  h->opts.rope = mla::RopeSpec{d.rope_base, 1.0, 1.0, 32.0, 4096.0};
   *out = h;
+  return MLA_OK;
+}
+
+mla_status_t mla_set_rmsnorm(mla_handle_t* h, const void* g_q, const void* g_kv, double eps) {
+  if (!h || (!g_q) != (!g_kv) || !(eps >= 0.0)) return MLA_ERR_INVALID_ARG;
+  if ((g_q && !aligned16(g_q)) || (g_kv && !aligned16(g_kv))) return MLA_ERR_ALIGNMENT;
+  h->opts.g_q = g_q;
+  h->opts.g_kv = g_kv;
+  h->opts.eps = (float)eps;
+  return MLA_OK;
+}
+
+mla_status_t mla_set_yarn(mla_handle_t* h, double s, double alpha, double beta, double original_len) {
+  if (!h || !(s >= 1.0) || !(beta > alpha) || !(original_len > 0.0)) return MLA_ERR_INVALID_ARG;
+  h->opts.rope = mla::RopeSpec{h->dims.rope_base, s, alpha, beta, original_len};
   return MLA_OK;
 }
 
@@ -327,6 +364,52 @@ mla_status_t mla_workspace_offset(const mla_handle_t* h, mla_op_t op, int64_t nu
   return MLA_OK;
 }
 
+namespace {
+
+constexpr int64_t kAbsorbedChunkMax = 64;   // the latent core runs one row of clusters per chunk token
+
+// Resolves the form of a chunked prefill; false if the arguments or the forced form do not fit.
+bool chunk_form(int64_t B, int64_t total_q, int64_t max_q, int64_t total_kv, mla_chunk_form_t form,
+                mla_chunk_form_t* chosen) {
+  if (B <= 0 || total_q <= 0 || max_q <= 0 || total_kv < total_q) return false;
+  if (form != MLA_CHUNK_AUTO && form != MLA_CHUNK_ABSORBED && form != MLA_CHUNK_UNABSORBED) return false;
+  const bool uniform = total_q == B * max_q && max_q <= kAbsorbedChunkMax;
+  if (form == MLA_CHUNK_ABSORBED && !uniform) return false;
+  if (form == MLA_CHUNK_AUTO) form = (uniform && total_kv >= 2 * total_q) ? MLA_CHUNK_ABSORBED : MLA_CHUNK_UNABSORBED;
+  *chosen = form;
+  return true;
+}
+
+Layout chunk_layout(const mla_handle* h, int64_t B, int64_t total_q, int64_t max_q, int64_t total_kv,
+                    mla_chunk_form_t chosen) {
+  return chosen == MLA_CHUNK_ABSORBED ? layout(h, MLA_OP_DECODE, B, (int32_t)max_q, 0, total_kv)
+                                      : layout(h, MLA_OP_PREFILL, B, 0, total_q, total_kv);
+}
+
+}  // namespace
+
+mla_status_t mla_prefill_chunk_workspace(const mla_handle_t* h, int64_t B, int64_t total_q, int64_t max_q,
+                                         int64_t total_kv, mla_chunk_form_t form, mla_chunk_form_t* chosen,
+                                         size_t* bytes) {
+  mla_chunk_form_t f;
+  if (!h || !bytes || !chunk_form(B, total_q, max_q, total_kv, form, &f)) return MLA_ERR_INVALID_ARG;
+  if (chosen) *chosen = f;
+  *bytes = chunk_layout(h, B, total_q, max_q, total_kv, f).total;
+  return MLA_OK;
+}
+
+mla_status_t mla_prefill_chunk_offset(const mla_handle_t* h, int64_t B, int64_t total_q, int64_t max_q,
+                                      int64_t total_kv, mla_chunk_form_t form, mla_buffer_t which,
+                                      size_t* offset) {
+  mla_chunk_form_t f;
+  if (!h || !offset || !chunk_form(B, total_q, max_q, total_kv, form, &f)) return MLA_ERR_INVALID_ARG;
+  if (which < MLA_BUF_CQ || which > MLA_BUF_LSE) return MLA_ERR_INVALID_ARG;
+  Layout L = chunk_layout(h, B, total_q, max_q, total_kv, f);
+  if (!L.has[which]) return MLA_ERR_INVALID_ARG;
+  *offset = L.off[which];
+  return MLA_OK;
+}
+
 int mla_uses_tensor_cores(const mla_handle_t* h, mla_op_t op) {
   if (!h || op < MLA_OP_CACHE_APPEND || op > MLA_OP_ATTN_DECODE_LATENT) return 0;
   return tc_dims(h) ? 1 : 0;
@@ -348,7 +431,7 @@ mla_status_t mla_cache_append(mla_handle_t* h, const void* hidden, const int64_t
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   if (tc_dims(h))
-    return cuda_status(mla::tc_cache_append(h->dims, h->w, hidden, positions, slots, T, cache, capacity,
+    return cuda_status(mla::tc_cache_append(h->dims, h->w, h->opts, hidden, positions, slots, T, cache, capacity,
                                             (char*)ws + L.tc_off, L.total - L.tc_off, h->d_err, st));
   return simt_cache_rows(h, hidden, positions, slots, T, cache, capacity, st);
 }
@@ -378,6 +461,95 @@ mla_status_t mla_attn_decode_latent(mla_handle_t* h, const void* q_abs, const vo
   return simt_latent_core(h, q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, true, lse, st);
 }
 
+namespace {
+
+// Decode steps after the position check (absorbed form, Tq tokens per sequence, positions in pos).
+mla_status_t decode_steps(mla_handle* h, const void* h_q, int64_t B, int32_t Tq, const int64_t* cu,
+                          const int64_t* pos, const void* cache, int64_t capacity, void* u_out, char* w,
+                          const Layout& L, cudaStream_t st) {
+  const mla_dims_t& d = h->dims;
+  const int64_t T = B * Tq;
+  void* cq = w + L.off[MLA_BUF_CQ];
+  void* qc = w + L.off[MLA_BUF_QC];
+  void* qr = w + L.off[MLA_BUF_QR];
+  void* qabs = w + L.off[MLA_BUF_QABS];
+  void* olat = w + L.off[MLA_BUF_OLAT];
+  void* o = w + L.off[MLA_BUF_O];
+  float* lse = (float*)(w + L.off[MLA_BUF_LSE]);
+  if (tc_dims(h))
+    return cuda_status(mla::tc_decode(d, h->w, h->opts, h_q, B, Tq, cu, pos, cache, capacity, u_out, cq, qc, qr, qabs,
+                                      olat, o, lse, w + L.tc_off, h->num_sms, h->d_err, st));
+  // Steps (1)-(3)
+  mla_status_t s = simt_queries(h, h_q, pos, T, cq, qc, qr, st);
+  if (s != MLA_OK) return s;
+  // q~_i = W_i^UK^T q^C_i (batched over heads): A(t, k) = q^C[t, i d_h + k], B(c, k) = W^UK[i d_h + k, c]
+  SimtGemmArgs a = gemm_args();
+  a.A = qc; a.sam = (int64_t)d.n_h * d.d_h; a.sak = 1; a.sab = d.d_h;
+  a.B = h->w.w_uk; a.sbn = 1; a.sbk = d.d_c; a.sbb = (int64_t)d.d_h * d.d_c;
+  a.C = qabs; a.scm = (int64_t)d.n_h * d.d_c; a.scn = 1; a.scb = d.d_c;
+  a.M = T; a.N = d.d_c; a.K = d.d_h; a.batch = d.n_h;
+  s = run_simt_gemm(h, a, st);
+  if (s != MLA_OK) return s;
+  s = simt_latent_core(h, qabs, qr, B, Tq, cu, cache, capacity, olat, h->dtype == MLA_FP32, lse, st);
+  if (s != MLA_OK) return s;
+  // o_i = W_i^UV o^lat_i: A(t, c) = o^lat[t, i, c], B(k, c) = W^UV[i d_h + k, c]
+  SimtGemmArgs v = gemm_args();
+  v.A = olat; v.sam = (int64_t)d.n_h * d.d_c; v.sak = 1; v.sab = d.d_c;
+  v.B = h->w.w_uv; v.sbn = d.d_c; v.sbk = 1; v.sbb = (int64_t)d.d_h * d.d_c;
+  v.C = o; v.scm = (int64_t)d.n_h * d.d_h; v.scn = 1; v.scb = d.d_h;
+  v.M = T; v.N = d.d_h; v.K = d.d_c; v.batch = d.n_h;
+  s = run_simt_gemm(h, v, st);
+  if (s != MLA_OK) return s;
+  return simt_output(h, o, T, u_out, st);
+}
+
+// Unabsorbed prefill steps after the position check: T query tokens packed by cu at positions pos,
+// their cache rows at slots (nullptr: row t); key rows packed by cu_kv (nullptr: cu_kv = cu).
+mla_status_t prefill_steps(mla_handle* h, const void* hidden, int64_t B, const int64_t* cu, const int64_t* cu_kv,
+                           int64_t T, int64_t T_kv, int64_t max_q, const int64_t* pos, const int64_t* slots,
+                           void* cache, int64_t capacity, void* u_out, char* w, const Layout& L, cudaStream_t st) {
+  const mla_dims_t& d = h->dims;
+  const size_t es = elem_size(h);
+  const int64_t R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
+  if (!cu_kv) T_kv = T;
+  void* cq = w + L.off[MLA_BUF_CQ];
+  void* qc = w + L.off[MLA_BUF_QC];
+  void* qr = w + L.off[MLA_BUF_QR];
+  void* o = w + L.off[MLA_BUF_O];
+  void* kc = w + L.off[MLA_BUF_KC];
+  void* vc = w + L.off[MLA_BUF_VC];
+  if (tc_dims(h))
+    return cuda_status(mla::tc_prefill(d, h->w, h->opts, hidden, B, cu, cu_kv, T, T_kv, max_q, pos, slots, cache,
+                                       capacity, u_out, cq, qc, qr, kc, vc, o, h->num_sms, h->d_err, st));
+  // Steps (5), (7): the tokens' cache rows
+  mla_status_t s = simt_cache_rows(h, hidden, pos, slots, T, cache, capacity, st);
+  if (s != MLA_OK) return s;
+  s = simt_queries(h, hidden, pos, T, cq, qc, qr, st);
+  if (s != MLA_OK) return s;
+  // Steps (6), (9): k^C = W^UK c^KV, v^C = W^UV c^KV from every key row
+  s = run_simt_gemm(h, dense_nt(cache, R, h->w.w_uk, kc, HD, T_kv, HD, d.d_c), st);
+  if (s != MLA_OK) return s;
+  s = run_simt_gemm(h, dense_nt(cache, R, h->w.w_uv, vc, HD, T_kv, HD, d.d_c), st);
+  if (s != MLA_OK) return s;
+  // Steps (4), (8), (10): causal attention per head with keys [k^C_i; k^R], values v^C_i
+  SimtAttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q1 = qc; a.sq1t = HD; a.sq1h = d.d_h; a.d1 = d.d_h;
+  a.q2 = qr; a.sq2t = (int64_t)d.n_h * d.d_r; a.sq2h = d.d_r; a.d2 = d.d_r;
+  a.k1 = kc; a.sk1 = HD; a.sk1h = d.d_h;
+  a.k2 = (const char*)cache + (size_t)d.d_c * es; a.sk2 = R;
+  a.v = vc; a.sv = HD; a.svh = d.d_h; a.dv = d.d_h;
+  a.o = o; a.sot = HD; a.soh = d.d_h;
+  a.lse = nullptr;
+  a.cu = cu; a.cu_kv = cu_kv; a.B = B; a.tq = 0; a.T = T; a.n_h = d.n_h; a.capacity = capacity;
+  a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
+  a.err = h->d_err;
+  MLA_TRY(mla::simt_attention(a, st));
+  return simt_output(h, o, T, u_out, st);
+}
+
+}  // namespace
+
 mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq, const int64_t* cu_seqlens,
                         const void* cache, int64_t capacity, void* u_out, void* ws, size_t ws_bytes,
                         mla_stream_t stream) {
@@ -393,43 +565,10 @@ mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq,
   mla_status_t s = ensure_device(h);
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  const mla_dims_t& d = h->dims;
   char* w = (char*)ws;
-  const int64_t T = B * Tq;
   int64_t* pos = (int64_t*)(w + L.pos_off);
-  void* cq = w + L.off[MLA_BUF_CQ];
-  void* qc = w + L.off[MLA_BUF_QC];
-  void* qr = w + L.off[MLA_BUF_QR];
-  void* qabs = w + L.off[MLA_BUF_QABS];
-  void* olat = w + L.off[MLA_BUF_OLAT];
-  void* o = w + L.off[MLA_BUF_O];
-  float* lse = (float*)(w + L.off[MLA_BUF_LSE]);
-  MLA_TRY(mla::check_and_positions(cu_seqlens, B, Tq, T, capacity, 0, pos, h->d_err, st));
-  if (tc_dims(h))
-    return cuda_status(mla::tc_decode(d, h->w, h_q, B, Tq, cu_seqlens, pos, cache, capacity, u_out, cq, qc, qr,
-                                      qabs, olat, o, lse, w + L.tc_off, h->num_sms, h->d_err, st));
-  // Steps (1)-(3)
-  s = simt_queries(h, h_q, pos, T, cq, qc, qr, st);
-  if (s != MLA_OK) return s;
-  // q~_i = W_i^UK^T q^C_i (batched over heads): A(t, k) = q^C[t, i d_h + k], B(c, k) = W^UK[i d_h + k, c]
-  SimtGemmArgs a = gemm_args();
-  a.A = qc; a.sam = (int64_t)d.n_h * d.d_h; a.sak = 1; a.sab = d.d_h;
-  a.B = h->w.w_uk; a.sbn = 1; a.sbk = d.d_c; a.sbb = (int64_t)d.d_h * d.d_c;
-  a.C = qabs; a.scm = (int64_t)d.n_h * d.d_c; a.scn = 1; a.scb = d.d_c;
-  a.M = T; a.N = d.d_c; a.K = d.d_h; a.batch = d.n_h;
-  s = run_simt_gemm(h, a, st);
-  if (s != MLA_OK) return s;
-  s = simt_latent_core(h, qabs, qr, B, Tq, cu_seqlens, cache, capacity, olat, h->dtype == MLA_FP32, lse, st);
-  if (s != MLA_OK) return s;
-  // o_i = W_i^UV o^lat_i: A(t, c) = o^lat[t, i, c], B(k, c) = W^UV[i d_h + k, c]
-  SimtGemmArgs v = gemm_args();
-  v.A = olat; v.sam = (int64_t)d.n_h * d.d_c; v.sak = 1; v.sab = d.d_c;
-  v.B = h->w.w_uv; v.sbn = d.d_c; v.sbk = 1; v.sbb = (int64_t)d.d_h * d.d_c;
-  v.C = o; v.scm = (int64_t)d.n_h * d.d_h; v.scn = 1; v.scb = d.d_h;
-  v.M = T; v.N = d.d_h; v.K = d.d_c; v.batch = d.n_h;
-  s = run_simt_gemm(h, v, st);
-  if (s != MLA_OK) return s;
-  return simt_output(h, o, T, u_out, st);
+  MLA_TRY(mla::check_and_positions(cu_seqlens, B, Tq, B * Tq, capacity, 0, pos, h->d_err, st));
+  return decode_steps(h, h_q, B, Tq, cu_seqlens, pos, cache, capacity, u_out, w, L, st);
 }
 
 mla_status_t mla_prefill(mla_handle_t* h, const void* hidden, int64_t B, const int64_t* cu_seqlens,
@@ -448,46 +587,50 @@ mla_status_t mla_prefill(mla_handle_t* h, const void* hidden, int64_t B, const i
   mla_status_t s = ensure_device(h);
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  const mla_dims_t& d = h->dims;
-  const size_t es = elem_size(h);
-  const int64_t T = total_tokens, R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
   char* w = (char*)ws;
   int64_t* pos = (int64_t*)(w + L.pos_off);
-  void* cq = w + L.off[MLA_BUF_CQ];
-  void* qc = w + L.off[MLA_BUF_QC];
-  void* qr = w + L.off[MLA_BUF_QR];
-  void* o = w + L.off[MLA_BUF_O];
-  void* kc = w + L.off[MLA_BUF_KC];
-  void* vc = w + L.off[MLA_BUF_VC];
-  MLA_TRY(mla::check_and_positions(cu_seqlens, B, 0, T, capacity, max_seqlen, pos, h->d_err, st));
-  if (tc_dims(h))
-    return cuda_status(mla::tc_prefill(d, h->w, hidden, B, cu_seqlens, T, max_seqlen, pos, cache, capacity, u_out,
-                                       cq, qc, qr, kc, vc, o, h->num_sms, h->d_err, st));
-  // Steps (5), (7): cache rows of every token at row t (= cu[b] + position)
-  s = simt_cache_rows(h, hidden, pos, nullptr, T, cache, capacity, st);
+  MLA_TRY(mla::check_and_positions(cu_seqlens, B, 0, total_tokens, capacity, max_seqlen, pos, h->d_err, st));
+  return prefill_steps(h, hidden, B, cu_seqlens, nullptr, total_tokens, total_tokens, max_seqlen, pos, nullptr, cache,
+                       capacity, u_out, w, L, st);
+}
+
+mla_status_t mla_prefill_chunk(mla_handle_t* h, const void* hidden, int64_t B, const int64_t* cu_q, int64_t total_q,
+                               int64_t max_q, const int64_t* cu_kv, int64_t total_kv, void* cache, int64_t capacity,
+                               mla_chunk_form_t form, void* u_out, void* ws, size_t ws_bytes, mla_stream_t stream) {
+  mla_chunk_form_t f;
+  if (!h || !hidden || !cu_q || !cu_kv || !cache || !u_out || !ws || capacity < total_kv ||
+      !chunk_form(B, total_q, max_q, total_kv, form, &f))
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(cache) || !aligned16(u_out) || !aligned16(ws) || !aligned16(cu_q) ||
+      !aligned16(cu_kv))
+    return MLA_ERR_ALIGNMENT;
+  Layout L = chunk_layout(h, B, total_q, max_q, total_kv, f);
+  if (ws_bytes < L.total) return MLA_ERR_WORKSPACE;
+  if (!h->has_weights) return MLA_ERR_NO_WEIGHTS;
+  DeviceGuard g(h->device);
+  if (!g.ok) return MLA_ERR_CUDA;
+  mla_status_t s = ensure_device(h);
   if (s != MLA_OK) return s;
-  s = simt_queries(h, hidden, pos, T, cq, qc, qr, st);
-  if (s != MLA_OK) return s;
-  // Steps (6), (9): k^C = W^UK c^KV, v^C = W^UV c^KV from the cache rows just written
-  s = run_simt_gemm(h, dense_nt(cache, R, h->w.w_uk, kc, HD, T, HD, d.d_c), st);
-  if (s != MLA_OK) return s;
-  s = run_simt_gemm(h, dense_nt(cache, R, h->w.w_uv, vc, HD, T, HD, d.d_c), st);
-  if (s != MLA_OK) return s;
-  // Steps (4), (8), (10): causal attention per head with keys [k^C_i; k^R], values v^C_i
-  SimtAttnArgs a;
-  memset(&a, 0, sizeof(a));
-  a.q1 = qc; a.sq1t = HD; a.sq1h = d.d_h; a.d1 = d.d_h;
-  a.q2 = qr; a.sq2t = (int64_t)d.n_h * d.d_r; a.sq2h = d.d_r; a.d2 = d.d_r;
-  a.k1 = kc; a.sk1 = HD; a.sk1h = d.d_h;
-  a.k2 = (const char*)cache + (size_t)d.d_c * es; a.sk2 = R;
-  a.v = vc; a.sv = HD; a.svh = d.d_h; a.dv = d.d_h;
-  a.o = o; a.sot = HD; a.soh = d.d_h;
-  a.lse = nullptr;
-  a.cu = cu_seqlens; a.B = B; a.tq = 0; a.T = T; a.n_h = d.n_h; a.capacity = capacity;
-  a.scale = (float)(1.0 / sqrt((double)(d.d_h + d.d_r)));
-  a.err = h->d_err;
-  MLA_TRY(mla::simt_attention(a, st));
-  return simt_output(h, o, T, u_out, st);
+  cudaStream_t st = (cudaStream_t)stream;
+  char* w = (char*)ws;
+  int64_t* pos = (int64_t*)(w + L.pos_off);
+  int64_t* slots = (int64_t*)(w + L.slot_off);
+  MLA_TRY(mla::check_chunk_positions(cu_q, cu_kv, B, total_q, total_kv, capacity, max_q, pos, slots, h->d_err, st));
+  if (f == MLA_CHUNK_UNABSORBED)
+    return prefill_steps(h, hidden, B, cu_q, cu_kv, total_q, total_kv, max_q, pos, slots, cache, capacity, u_out, w,
+                         L, st);
+  // Absorbed: the chunk's cache rows first (steps (5), (7)), then the decode steps with Tq = Tc,
+  // whose query k of sequence b sits at position len_b - Tc + k, the same position as above.
+  const int32_t tc = (int32_t)max_q;
+  if (tc_dims(h)) {
+    const size_t scratch = mla::tc_append_scratch_bytes(h->dims, total_q);
+    MLA_TRY(mla::tc_cache_append(h->dims, h->w, h->opts, hidden, pos, slots, total_q, cache, capacity, w + L.tc_off,
+                                 scratch, h->d_err, st));
+  } else {
+    s = simt_cache_rows(h, hidden, pos, slots, total_q, cache, capacity, st);
+    if (s != MLA_OK) return s;
+  }
+  return decode_steps(h, hidden, B, tc, cu_kv, pos, cache, capacity, u_out, w, L, st);
 }
 
 mla_status_t mla_attn_prefill(mla_handle_t* h, const void* q_c, const void* q_rope, const void* k_c, const void* v_c,
@@ -508,8 +651,8 @@ mla_status_t mla_attn_prefill(mla_handle_t* h, const void* q_c, const void* q_ro
   const int64_t T = total_tokens, R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
   MLA_TRY(mla::check_and_positions(cu_seqlens, B, 0, T, capacity, max_seqlen, nullptr, h->d_err, st));
   if (tc_dims(h))
-    return cuda_status(mla::tc_prefill_attention(q_c, q_rope, k_c, v_c, cache, capacity, cu_seqlens, B, T, max_seqlen,
-                                                 o, h->num_sms, h->d_err, st));
+    return cuda_status(mla::tc_prefill_attention(q_c, q_rope, k_c, v_c, cache, capacity, cu_seqlens, nullptr, B, T, T,
+                                                 max_seqlen, o, h->num_sms, h->d_err, st));
   SimtAttnArgs a;
   memset(&a, 0, sizeof(a));
   a.q1 = q_c; a.sq1t = HD; a.sq1h = d.d_h; a.d1 = d.d_h;
@@ -618,7 +761,7 @@ extern "C" mla_status_t mla_cache_append_noalloc(mla_handle_t* h, const void* hi
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   if (tc_dims(h))
-    return cuda_status(mla::tc_cache_append(h->dims, h->w, hidden, positions, slots, T, cache, capacity,
+    return cuda_status(mla::tc_cache_append(h->dims, h->w, h->opts, hidden, positions, slots, T, cache, capacity,
                                             (char*)scratch + L.tc_off, L.total - L.tc_off, h->d_err, st));
   return simt_cache_rows(h, hidden, positions, slots, T, cache, capacity, st);
 }

@@ -10,10 +10,10 @@ namespace mla {
 // Bits of the handle's sticky device error word.
 enum : uint32_t {
   DEVERR_CU_SEQLENS = 1u << 0,    // cu_seqlens[0] != 0, decreasing, or past the cache capacity
-  DEVERR_SHORT_SEQ = 1u << 1,     // a decode sequence holds fewer rows than its Tq query tokens
+  DEVERR_SHORT_SEQ = 1u << 1,     // a sequence holds fewer rows than its query tokens (decode Tq, chunk)
   DEVERR_SLOT = 1u << 2,          // a cache slot outside [0, capacity)
   DEVERR_POSITION = 1u << 3,      // a negative position
-  DEVERR_SEQ_TOO_LONG = 1u << 4,  // a prefill sequence longer than max_seqlen
+  DEVERR_SEQ_TOO_LONG = 1u << 4,  // a prefill sequence (or chunk) longer than max_seqlen (max_q)
   DEVERR_TOTAL = 1u << 5,         // cu_seqlens[B] differs from the token count given on the host
   DEVERR_TIMEOUT = 1u << 6,       // a bounded mbarrier wait gave up
 };
@@ -24,6 +24,36 @@ void note_launch(unsigned n = 1);
 enum TimedKernel { TIMED_LATENT_CORE = 0, TIMED_PREFILL_CORE = 1, TIMED_KERNELS = 2 };
 void timer_begin(TimedKernel k, cudaStream_t st);
 void timer_end(TimedKernel k, cudaStream_t st);
+
+// The decoupled RoPE of a layer (section 一(一)3 of the DeepSeek-V3 notes): pair m of a d_r-wide block
+// turns at theta_m = base^(-2m/d_r). With YaRN (section 三(二)3, yarn_s > 1) the frequencies are
+// interpolated by parts: pair m turns r_m = L0 theta_m / (2 pi) times over the original context
+// L0; gamma = clamp((r_m - alpha) / (beta - alpha), 0, 1) and theta'_m = (1 - gamma) theta_m / s +
+// gamma theta_m; each rotated vector (q^R and k^R) is multiplied by 0.1 ln s + 1.
+struct RopeSpec {
+  double base;
+  double yarn_s, yarn_alpha, yarn_beta, yarn_l0;   // yarn_s <= 1: plain RoPE
+};
+__host__ __device__ inline double rope_theta(const RopeSpec& r, int m, int d_r) {
+  const double theta = pow(r.base, -2.0 * (double)m / (double)d_r);
+  if (!(r.yarn_s > 1.0)) return theta;
+  const double turns = r.yarn_l0 * theta / 6.283185307179586;
+  double g = (turns - r.yarn_alpha) / (r.yarn_beta - r.yarn_alpha);
+  g = g < 0.0 ? 0.0 : (g > 1.0 ? 1.0 : g);
+  return (1.0 - g) * theta / r.yarn_s + g * theta;
+}
+__host__ __device__ inline float rope_mul(const RopeSpec& r) {
+  return r.yarn_s > 1.0 ? (float)(0.1 * log(r.yarn_s) + 1.0) : 1.0f;
+}
+
+// Opt-in parts of a layer: the RMSNorm after the latent compression (section 三(二)1 of the notes:
+// c^Q = RMSNorm(W^DQ h), c^KV = RMSNorm(W^DKV h), y = x / sqrt(mean(x^2) + eps) * g) and the RoPE.
+struct LayerOpts {
+  const void* g_q;    // [d_c'] gains of c^Q in the handle dtype; nullptr: no norm
+  const void* g_kv;   // [d_c] gains of c^KV
+  float eps;
+  RopeSpec rope;
+};
 
 __device__ __forceinline__ void flag_error(uint32_t* err, uint32_t bits) {
   if (err) atomicOr(err, bits);
@@ -74,15 +104,20 @@ __device__ __forceinline__ float block_sum(float v, float* scratch) {
   return warp_sum(r);
 }
 
-// RoPE angle for pair m of a d_r-wide block at position pos: pos * base^(-2m/d_r), in double,
-// then sine/cosine in double (CUDA's sincos) so long positions keep their precision.
-__device__ __forceinline__ void rope_cos_sin(int64_t pos, int m, int d_r, double base, float* c, float* s) {
-  const double theta = pow(base, -2.0 * (double)m / (double)d_r);
+// RoPE angle for pair m of a d_r-wide block at position pos: pos * theta_m, in double, then
+// sine/cosine in double (CUDA's sincos) so long positions keep their precision.
+__device__ __forceinline__ void rope_cos_sin(int64_t pos, int m, int d_r, const RopeSpec& r, float* c, float* s) {
+  const double theta = rope_theta(r, m, d_r);
   double sd, cd;
   sincos((double)pos * theta, &sd, &cd);
   *c = (float)cd;
   *s = (float)sd;
 }
+
+// In-place RMSNorm of `rows` rows of `cols` elements (row r at x + row(r) * ld, row(r) = rowmap ?
+// rowmap[r] : r; rows mapped outside [0, rowmap_limit) are skipped) with gains g.
+cudaError_t rmsnorm_rows(void* x, bool bf16, int64_t ld, const int64_t* rowmap, int64_t rowmap_limit, int64_t rows,
+                         int cols, const void* g, float eps, cudaStream_t st);
 
 // Sequence of a packed token t: the b with cu[b] <= t < cu[b+1] (cu non-decreasing, B >= 1).
 __device__ __forceinline__ int64_t seq_of_token(const int64_t* cu, int64_t B, int64_t t) {

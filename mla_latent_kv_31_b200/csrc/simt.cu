@@ -67,8 +67,9 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmArgs a) {
       if (a.pos && n >= a.rope_col0) {
         const int pair = (int)(((n - a.rope_col0) % a.d_r) >> 1);
         float c, s;
-        rope_cos_sin(p, pair, a.d_r, a.rope_base, &c, &s);
-        const float y0 = x0 * c - x1 * s, y1 = x0 * s + x1 * c;
+        rope_cos_sin(p, pair, a.d_r, a.rope, &c, &s);
+        const float mul = rope_mul(a.rope);
+        const float y0 = (x0 * c - x1 * s) * mul, y1 = (x0 * s + x1 * c) * mul;
         x0 = y0; x1 = y1;
       }
       if (n < a.N) C[r * a.scm + n * a.scn] = from_f<TC>(x0);
@@ -89,15 +90,21 @@ __global__ void __launch_bounds__(ATT_THREADS) simt_attention_kernel(SimtAttnArg
   const int64_t t = blockIdx.x;
   const int head = blockIdx.y;
   const int tid = threadIdx.x;
-  int64_t b, pos;
+  int64_t b, pos, row0;
   if (a.tq > 0) {
     b = t / a.tq;
     pos = (a.cu[b + 1] - a.cu[b]) - a.tq + (t % a.tq);
+    row0 = a.cu[b];
+  } else if (a.cu_kv) {
+    // a chunk: the sequence's query tokens are the last ones of its key rows
+    b = seq_of_token(a.cu, a.B, t);
+    row0 = a.cu_kv[b];
+    pos = (a.cu_kv[b + 1] - row0) - (a.cu[b + 1] - a.cu[b]) + (t - a.cu[b]);
   } else {
     b = seq_of_token(a.cu, a.B, t);
     pos = t - a.cu[b];
+    row0 = a.cu[b];
   }
-  const int64_t row0 = a.cu[b];
   const int64_t n = pos + 1;
   const bool bad = pos < 0 || row0 < 0 || row0 + n > a.capacity;
   TO* o = reinterpret_cast<TO*>(a.o) + t * a.sot + (int64_t)head * a.soh;
@@ -184,6 +191,26 @@ __global__ void check_positions_kernel(const int64_t* cu, int64_t B, int32_t tq,
   }
 }
 
+__global__ void check_chunk_kernel(const int64_t* cu_q, const int64_t* cu_kv, int64_t B, int64_t total_q,
+                                   int64_t total_kv, int64_t capacity, int64_t max_q, int64_t* pos_out,
+                                   int64_t* slot_out, uint32_t* err) {
+  // One block: sequence checks by a strided loop, then per-token positions and cache rows.
+  for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+    const int64_t q0 = cu_q[b], q1 = cu_q[b + 1], k0 = cu_kv[b], k1 = cu_kv[b + 1];
+    if (b == 0 && (q0 != 0 || k0 != 0)) flag_error(err, DEVERR_CU_SEQLENS);
+    if (q1 < q0 || k1 < k0 || k1 > capacity) flag_error(err, DEVERR_CU_SEQLENS);
+    if (q1 - q0 > k1 - k0) flag_error(err, DEVERR_SHORT_SEQ);
+    if (q1 - q0 > max_q) flag_error(err, DEVERR_SEQ_TOO_LONG);
+  }
+  if (threadIdx.x == 0 && (cu_q[B] != total_q || cu_kv[B] != total_kv)) flag_error(err, DEVERR_TOTAL);
+  for (int64_t t = threadIdx.x; t < total_q; t += blockDim.x) {
+    const int64_t b = seq_of_token(cu_q, B, t);
+    const int64_t pos = (cu_kv[b + 1] - cu_kv[b]) - (cu_q[b + 1] - cu_q[b]) + (t - cu_q[b]);
+    pos_out[t] = pos;
+    slot_out[t] = pos >= 0 ? cu_kv[b] + pos : -1;   // a negative row is skipped by the writers
+  }
+}
+
 }  // namespace
 
 cudaError_t simt_gemm(const SimtGemmArgs& a, cudaStream_t st) {
@@ -207,6 +234,14 @@ cudaError_t check_and_positions(const int64_t* cu, int64_t B, int32_t tq, int64_
                                 int64_t capacity, int64_t max_seqlen, int64_t* pos_out, uint32_t* err,
                                 cudaStream_t st) {
   check_positions_kernel<<<1, 512, 0, st>>>(cu, B, tq, total_tokens, capacity, max_seqlen, pos_out, err);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t check_chunk_positions(const int64_t* cu_q, const int64_t* cu_kv, int64_t B, int64_t total_q,
+                                  int64_t total_kv, int64_t capacity, int64_t max_q, int64_t* pos_out,
+                                  int64_t* slot_out, uint32_t* err, cudaStream_t st) {
+  check_chunk_kernel<<<1, 512, 0, st>>>(cu_q, cu_kv, B, total_q, total_kv, capacity, max_q, pos_out, slot_out, err);
   note_launch();
   return cudaGetLastError();
 }

@@ -20,7 +20,7 @@ struct SimtGemmArgs {
   void* C; int64_t scm, scn, scb;
   int64_t M, N, K, batch;
   const int64_t* rowmap; int64_t rowmap_limit;
-  const int64_t* pos; int64_t rope_col0; int32_t d_r; double rope_base;
+  const int64_t* pos; int64_t rope_col0; int32_t d_r; RopeSpec rope;
   uint32_t* err;
 };
 
@@ -36,6 +36,7 @@ struct SimtAttnArgs {
   void* o; int64_t sot, soh;
   float* lse;
   const int64_t* cu; int64_t B; int32_t tq;  // tq > 0: decode (token t of seq t/tq); tq == 0: prefill
+  const int64_t* cu_kv;  // prefill only, optional: key rows of each sequence, its query tokens the last ones
   int64_t T; int32_t n_h; int64_t capacity;
   float scale;
   uint32_t* err;
@@ -49,5 +50,12 @@ cudaError_t simt_attention(const SimtAttnArgs& a, cudaStream_t st);
 cudaError_t check_and_positions(const int64_t* cu, int64_t B, int32_t tq, int64_t total_tokens,
                                 int64_t capacity, int64_t max_seqlen, int64_t* pos_out, uint32_t* err,
                                 cudaStream_t st);
+
+// Device-side checks of a chunked prefill's cu_q / cu_kv (chunk b = the last cu_q[b+1] - cu_q[b] of
+// sequence b's cu_kv[b+1] - cu_kv[b] rows) and, per chunk token t of sequence b, its position
+// pos = len_kv_b - len_q_b + (t - cu_q[b]) and its cache row cu_kv[b] + pos.
+cudaError_t check_chunk_positions(const int64_t* cu_q, const int64_t* cu_kv, int64_t B, int64_t total_q,
+                                  int64_t total_kv, int64_t capacity, int64_t max_q, int64_t* pos_out,
+                                  int64_t* slot_out, uint32_t* err, cudaStream_t st);
 
 }  // namespace mla

@@ -4,6 +4,7 @@
 
 #include <stdint.h>
 
+#include "common.cuh"
 #include "mla.h"
 
 namespace mla {
@@ -16,7 +17,7 @@ size_t tc_core_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq);
 // Scratch bytes of mla_cache_append for T tokens (split-K partials when T is small).
 size_t tc_append_scratch_bytes(const mla_dims_t& d, int64_t T);
 
-cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const void* hidden,
+cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& o, const void* hidden,
                             const int64_t* positions, const int64_t* slots, int64_t T, void* cache,
                             int64_t capacity, void* scratch, size_t scratch_bytes, uint32_t* err,
                             cudaStream_t st);
@@ -31,20 +32,27 @@ cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B
                                 const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse,
                                 void* scratch, int num_sms, uint32_t* err, cudaStream_t st);
 
-cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const void* h_q, int64_t B, int32_t tq,
-                      const int64_t* cu, const int64_t* pos, const void* cache, int64_t capacity, void* u_out,
+cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& lo, const void* h_q, int64_t B,
+                      int32_t tq, const int64_t* cu, const int64_t* pos, const void* cache, int64_t capacity, void* u_out,
                       void* cq, void* qc, void* qr, void* qabs, void* olat, void* o, float* lse, void* scratch,
                       int num_sms, uint32_t* err, cudaStream_t st);
 
-// The causal prefill attention core (unabsorbed): q^C [T][H][128], q^R [T][H][64], k^C, v^C [T][H][128],
-// k^R in column 512 of the cache rows [capacity][576] (row = packed token index) -> o [T][H][128].
+// The causal prefill attention core (unabsorbed): q^C [T][H][128], q^R [T][H][64] of the query tokens
+// (packed by cu), k^C, v^C [T_kv][H][128] and k^R in column 512 of the cache rows [capacity][576] of
+// the key rows (packed by cu_kv; sequence b's query tokens are its last ones) -> o [T][H][128].
+// cu_kv == nullptr: the key rows are the query tokens themselves (cu_kv = cu, T_kv = T).
 cudaError_t tc_prefill_attention(const void* qc, const void* qr, const void* kc, const void* vc, const void* cache,
-                                 int64_t capacity, const int64_t* cu, int64_t B, int64_t T, int64_t max_seqlen,
-                                 void* o, int num_sms, uint32_t* err, cudaStream_t st);
+                                 int64_t capacity, const int64_t* cu, const int64_t* cu_kv, int64_t B, int64_t T,
+                                 int64_t T_kv, int64_t max_seqlen, void* o, int num_sms, uint32_t* err,
+                                 cudaStream_t st);
 
-cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, int64_t B,
-                       const int64_t* cu, int64_t T, int64_t max_seqlen, const int64_t* pos, void* cache,
-                       int64_t capacity, void* u_out, void* cq, void* qc, void* qr, void* kc, void* vc, void* o,
-                       int num_sms, uint32_t* err, cudaStream_t st);
+// Unabsorbed prefill of T query tokens (hidden states packed by cu) at positions pos, their cache
+// rows written at slots (nullptr: row t), k^C / v^C up-projected from the T_kv key rows packed by
+// cu_kv (nullptr: whole sequences, cu_kv = cu), then attention and W^O.
+cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& lo, const void* hidden, int64_t B,
+                       const int64_t* cu, const int64_t* cu_kv, int64_t T, int64_t T_kv, int64_t max_seqlen,
+                       const int64_t* pos, const int64_t* slots, void* cache, int64_t capacity, void* u_out,
+                       void* cq, void* qc, void* qr, void* kc, void* vc, void* o, int num_sms, uint32_t* err,
+                       cudaStream_t st);
 
 }  // namespace mla

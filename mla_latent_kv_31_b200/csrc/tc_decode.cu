@@ -21,7 +21,18 @@
 //   * the value CTA (rank 1): O in all 512 TMEM columns; per tile 16 SS MMAs (N = 256 latent
 //     columns, K = 16 keys) read P and the latent columns of the cache tile, which this CTA loads
 //     itself (the second read of the tile hits L2); it rescales O when the score CTA's running max
-//     moved, and writes o^lat at the end of each sequence piece.
+//     moved, and writes the piece's normalised partial o^lat at its end.
+// Each producer issues its TMA loads from four lanes: one issuing thread streams only about 40 GB/s.
+//
+// Queries. A piece's q~ (8 boxes of [128 heads x 64 columns]) and q^R (1 box) enter the score CTA's
+// ring ahead of its first tile, like a tile's boxes; the softmax warps copy q~ into TMEM and q^R
+// into its own shared-memory tile.
+//
+// Outputs. Every piece writes a partial: O = sum_j 2^((s_j - m) c) c_j unnormalised, its reference
+// m in natural units and its lse, O in a head-interleaved layout [token k][slot][column/4][head][4]
+// fp32, so that the 32 heads of a warp store 512 contiguous bytes per instruction. The merge pass
+// weights each partial by e^{m_s - lse} with lse = log sum_s e^{lse_s} and writes o^lat [T][H][DC]
+// and lse [T][H] (a one-piece sequence is a weighted copy).
 // The score CTA's tensor work per tile is 36 MMAs at N = 128 (about 2300 cycles), the value CTA's
 // 16 MMAs at N = 256 (about 2050), so the two stay busy together. Data flows one way (P), so the
 // two CTAs pipeline freely: two P buffers on the value side, two staging buffers on the score
@@ -45,13 +56,14 @@ constexpr int NK = 128;                        // keys per tile
 constexpr int kThreads = 384;
 constexpr int kMaxPairs = 74;
 constexpr float kRescaleLog2 = 8.f;            // keep the running max until it grows by 2^8
+constexpr int kIssuers = 4;                    // TMA issuing lanes per producer warp
 
 // score CTA: ring of [128 keys x 64 columns] boxes (8 latent + 1 k^R per tile)
 constexpr uint32_t BOX = NK * 128;             // 16 KB, 128-byte swizzle, K-major rows of 64 bf16
 constexpr int S_BOXES = 9;
 constexpr int S_RING = 8;
 constexpr uint32_t P_BYTES = H * NK * 2;       // P [128 heads x 128 keys] bf16, K-major SW128: 2 blocks of 16 KB
-constexpr uint32_t HDR_BYTES = 2 * H * 4;      // alpha[128], inv_l[128]
+constexpr uint32_t HDR_BYTES = 2 * H * 4;      // alpha[128] (+ reserve)
 constexpr uint32_t PMSG = P_BYTES + HDR_BYTES; // one P message: 33 KB
 constexpr uint32_t QR_BYTES = H * DR * 2;      // q^R [128 x 64] bf16, K-major SW128
 // value CTA: ring of [64 keys x 256 columns] groups (4 boxes of [64 keys x 64 columns])
@@ -76,6 +88,8 @@ static_assert(S_OFF_RING % 1024 == 0 && S_OFF_QR % 1024 == 0 && S_OFF_STG % 1024
                   V_OFF_RING % 1024 == 0,
               "swizzle atom alignment");
 static_assert(OFF_RED + 3 * 2 * H * 4 <= S_OFF_RING, "reduction buffer");
+static_assert(S_RING % kIssuers == 0 && V_RING % kIssuers == 0 && (kIssuers & (kIssuers - 1)) == 0,
+              "issuing lanes own whole ring slots");
 
 // barrier indices (one numbering for both CTAs)
 enum : int {
@@ -84,8 +98,8 @@ enum : int {
   B_SEMPTY = B_SFULL + S_RING,        // [S_RING]
   B_SCF = B_SEMPTY + S_RING,          // [2] scores ready
   B_SCE = B_SCF + 2,                  // [2] scores read (256 softmax threads)
-  B_QFULL = B_SCE + 2,                // q~ / q^R of a piece loaded (256)
-  B_QEMPTY = B_QFULL + 1,             // last QK^T of a piece done
+  B_QFULL = B_SCE + 2,                // q^R of a piece copied into its tile (256)
+  B_QEMPTY = B_QFULL + 1,             // last QK^T of a piece done (q~ TMEM and q^R tile free)
   B_PSTG = B_QEMPTY + 1,              // [2] P message staged (256)
   B_STGF = B_PSTG + 2,                // [2] staging buffer free again (remote arrival of the value CTA)
   B_TMAX = B_STGF + 2,                // [4] the two softmax warps of a TMEM lane quarter (64)
@@ -93,31 +107,31 @@ enum : int {
   B_GEMPTY = B_GFULL + V_RING,        // [V_RING]
   B_PFULL = B_GEMPTY + V_RING,        // [2] P message landed (bytes)
   B_OREADY = B_PFULL + 2,             // [2] O rescaled for the tile / nothing to rescale (128)
-  B_OFREE = B_OREADY + 2,             // O read out by the piece epilogue (128)
-  NBAR = B_OFREE + 1
+  B_OFREE = B_OREADY + 2,             // O read out by the piece epilogue (256: both column halves)
+  B_ODONE = B_OFREE + 1,              // the last P.V of a piece done (one phase per piece)
+  NBAR = B_ODONE + 1
 };
 static_assert(NBAR * 8 + 16 <= OFF_RED, "barrier block");
 
 struct CoreParams {
   CUtensorMap kmap;   // cache as [capacity, ROW], box {64, 128}, 128-byte swizzle (score CTA)
   CUtensorMap vmap;   // cache as [capacity, ROW], box {64, 64}, 128-byte swizzle (value CTA)
-  const __nv_bfloat16* q_abs;   // [T][H][DC]
-  const __nv_bfloat16* q_rope;  // [T][H][DR]
+  CUtensorMap qmap;   // q~ as [T * H, DC], box {64, 128}, 128-byte swizzle
+  CUtensorMap qrmap;  // q^R as [T * H, DR], box {64, 128}, 128-byte swizzle
   const int64_t* cu;
   const int32_t* tile_start;    // [B+1]: first global tile of each sequence
   const int32_t* slot_base;     // [B+1]: first partial slot of each sequence
+  const int4* pinfo;            // [pairs]: tile range [x, y), first sequence z, its partial slot w
   int32_t B, tq, pairs, s_max;
-  float* part_o;      // [tq][s_max][H][DC]
+  float* part_o;      // [tq][s_max][DC/4][H][4], unnormalised
   float* part_lse;    // [tq][s_max][H]
-  void* o_lat;        // [T][H][DC] (fp32 or bf16)
-  float* lse;         // [T][H]
+  float* part_m;      // [tq][s_max][H], the reference of part_o in natural units
   float scale_log2;   // log2(e) / sqrt(d_h + d_h^R)
   uint64_t wait_ns;   // bounded-wait limit
   int32_t stall;      // test hook: the first cluster's score-side producer skips its first box
   uint32_t* err;
 };
 
-__device__ __forceinline__ int32_t range_start(int64_t p, int64_t NT, int64_t P) { return (int32_t)(p * NT / P); }
 
 // Bounded waits with the launch's limit.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint64_t limit) {
@@ -130,25 +144,15 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint64_t
     if (globaltimer() - t0 > limit) return false;
   }
 }
-// The last sequence b in [0, B) with tile_start[b] <= x.
-__device__ __forceinline__ int find_seq(const int32_t* ts, int B, int32_t x) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (ts[mid] <= x) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
 // Iterates the sequence pieces of a tile range [x, end): b, [x, seg_end).
 struct SegWalk {
   const int32_t* ts;
   int B;
   int32_t x, end;
   int b;
-  __device__ void init(const int32_t* ts_, int B_, int32_t x0, int32_t x1) {
-    ts = ts_; B = B_; x = x0; end = x1;
-    b = x < end ? find_seq(ts, B, x) : 0;
+  // starts at tile x0, which belongs to sequence b0
+  __device__ void init_at(const int32_t* ts_, int B_, int32_t x0, int32_t x1, int b0) {
+    ts = ts_; B = B_; x = x0; end = x1; b = b0;
   }
   __device__ bool valid() const { return x < end; }
   __device__ int32_t seg_end() const { return min(end, ts[b + 1]); }
@@ -159,7 +163,6 @@ struct SegWalk {
   }
 };
 
-template <bool OUT_F32>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     latent_core_kernel(const __grid_constant__ CoreParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -173,18 +176,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t r = cluster_rank();
   const int k = blockIdx.y;                          // query token within the sequence window
   const int pair = blockIdx.x >> 1;
-  const int64_t NT = p.tile_start[p.B];
-  const int64_t npairs = NT < p.pairs ? NT : p.pairs;   // every active pair holds >= 1 tile
-  const int32_t t_begin = pair < npairs ? range_start(pair, NT, npairs) : 0;
-  const int32_t t_end = pair < npairs ? range_start(pair + 1, NT, npairs) : 0;
+  const int4 pi = p.pinfo[pair];
+  const int32_t t_begin = pi.x, t_end = pi.y;
   const uint64_t lim = p.wait_ns;
+  // partial slot of this cluster's piece of sequence b: the first piece's comes with the plan; a
+  // sequence that starts inside this cluster's range has this cluster as its first
+  auto piece_slot = [&](int b) -> int64_t { return b == pi.z ? (int64_t)pi.w : (int64_t)p.slot_base[b]; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
       if (i == B_SCE || i == B_SCE + 1 || i == B_QFULL || i == B_PSTG || i == B_PSTG + 1) cnt = 256;
       else if (i >= B_TMAX && i < B_TMAX + 4) cnt = 64;
-      else if (i == B_OREADY || i == B_OREADY + 1 || i == B_OFREE) cnt = 128;
+      else if (i == B_OREADY || i == B_OREADY + 1) cnt = 128;
+      else if (i == B_OFREE) cnt = 256;
       mbar_init(bar(i), cnt);
     }
     if (r == 1) {
@@ -198,43 +203,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_addr(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (threadIdx.x == 0) prefetch_tmap(r == 0 ? &p.kmap : &p.vmap);
+  if (threadIdx.x == 0) {
+    prefetch_tmap(r == 0 ? &p.kmap : &p.vmap);
+    if (r == 0) {
+      prefetch_tmap(&p.qmap);
+      prefetch_tmap(&p.qrmap);
+    }
+  }
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   SegWalk w;
-  w.init(p.tile_start, p.B, t_begin, t_end);
+  w.init_at(p.tile_start, p.B, t_begin, t_end, pi.z);
   const int ntiles = t_end - t_begin;
   bool ok = true;
 
   if (r == 0) {
     // =========================================================== score CTA
     if (warp == 0) {
-      // ------------------------------------------------ TMA producer: 9 boxes per tile
-      if (lane == 0) {
-        int n = 0, issued = 0;
+      // ------------------------------------------------ TMA producer: 9 entries per piece start and per tile
+      // A TMA issuing thread streams at most about 40 GB/s, so lanes 0-3 issue (lane l takes the
+      // entries n = l mod 4, slots l and l + 4 of the ring). Per piece: q~ in 8 boxes of
+      // [128 heads x 64 columns] and q^R in 1 box, then per tile the 8 latent boxes and the k^R box.
+      if (lane < kIssuers) {
+        int n = 0, last = -1;
         const bool stall = p.stall && pair == 0 && k == 0;
-        for (; ok && w.valid(); w.next()) {
-          const int32_t ts_b = p.tile_start[w.b];
-          const int32_t row_base = (int32_t)p.cu[w.b];
-          for (int32_t xt = w.x; ok && xt < w.seg_end(); ++xt) {
+        auto issue = [&](const CUtensorMap* map, int x, int y) -> bool {
+          const int cur = n++;
+          if ((cur & (kIssuers - 1)) != lane) return true;
+          const int slot = cur % S_RING;
+          if (!wait_bar(bar(B_SEMPTY + slot), ((cur / S_RING) & 1) ^ 1, lim)) return false;
+          if (stall && cur == 0) return true;     // test hook: entry 0 never arrives
+          mbar_expect_tx(bar(B_SFULL + slot), BOX);
+          tma_load_2d(sbase + S_OFF_RING + slot * BOX, map, x, y, bar(B_SFULL + slot));
+          last = cur;
+          return true;
+        };
+        for (SegWalk sw = w; ok && sw.valid(); sw.next()) {
+          const int32_t ts_b = p.tile_start[sw.b];
+          const int32_t row_base = (int32_t)p.cu[sw.b];
+          const int32_t qrow = (sw.b * p.tq + k) * H;
+          for (int c = 0; ok && c < 8; ++c) ok = issue(&p.qmap, 64 * c, qrow);
+          if (ok) ok = issue(&p.qrmap, 0, qrow);
+          for (int32_t xt = sw.x; ok && xt < sw.seg_end(); ++xt) {
             const int32_t row0 = row_base + (xt - ts_b) * NK;
-            for (int c = 0; c < S_BOXES; ++c, ++n) {
-              const int slot = n % S_RING;
-              if (!wait_bar(bar(B_SEMPTY + slot), ((n / S_RING) & 1) ^ 1, lim)) { ok = false; break; }
-              if (stall && n == 0) continue;     // test hook: this box never arrives
-              mbar_expect_tx(bar(B_SFULL + slot), BOX);
-              tma_load_2d(sbase + S_OFF_RING + slot * BOX, &p.kmap, c < 8 ? 64 * c : DC, row0, bar(B_SFULL + slot));
-              issued = n + 1;
-            }
+            for (int c = 0; ok && c < S_BOXES; ++c) ok = issue(&p.kmap, c < 8 ? 64 * c : DC, row0);
           }
         }
         if (!ok) {
           flag_error(p.err, DEVERR_TIMEOUT);
-          for (int i = max(0, issued - S_RING); i < issued; ++i)
-            if (!(p.stall && pair == 0 && k == 0 && i == 0)) wait_bar(bar(B_SFULL + i % S_RING), (i / S_RING) & 1, lim);
+          // this lane's entries still in flight: the last S_RING / kIssuers it issued
+          for (int i2 = max(lane, last - S_RING + 1); i2 <= last; ++i2)
+            if ((i2 & (kIssuers - 1)) == lane && !(p.stall && pair == 0 && k == 0 && i2 == 0))
+              wait_bar(bar(B_SFULL + i2 % S_RING), (i2 / S_RING) & 1, lim);
         }
       }
     } else if (warp == 1) {
@@ -244,6 +267,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint64_t qr_desc = sw128_desc(sbase + S_OFF_QR, 0, 1024);
         int j = 0, g = 0, n = 0;
         for (; ok && w.valid(); w.next(), ++g) {
+          // the piece's q~ / q^R entries are taken by the softmax warps (TMEM q~, q^R tile)
+          n += 9;
           if (!wait_bar(bar(B_QFULL), g & 1, lim)) { ok = false; break; }
           const int32_t send = w.seg_end();
           for (int32_t xt = w.x; xt < send; ++xt, ++j) {
@@ -318,38 +343,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         y = redbuf[(slot * 2 + (half ^ 1)) * 128 + i];
         return okw;
       };
-      // q~ (this half's 256 latent columns -> TMEM columns [128 half, +128)) and q^R (this half's
-      // 32 columns -> the swizzled q^R tile) of sequence bq, once the previous piece's last QK^T is
-      // done with them.
-      int gq = 0;
-      auto load_q = [&](int bq) -> bool {
-        const int64_t t = (int64_t)bq * p.tq + k;
-        if (!wait_u(bar(B_QEMPTY), (gq & 1) ^ 1)) return false;
+      // q~ and q^R of a piece from its 9 ring entries, once the previous piece's last QK^T is done with
+      // them: this half's 4 q~ boxes (its 256 latent columns) -> TMEM columns [128 half, +128) of row
+      // i as bf16 pairs; then this half's 4 chunks of q^R row i -> the q^R tile (the same swizzled
+      // offsets). The entries are released after a barrier over the 8 softmax warps. Both halves
+      // reach each barrier even when one of their waits gave up, and leave together if any did.
+      int gq = 0, nq = 0;                            // pieces seen; ring index of the next piece's q~
+      auto load_q = [&](int ntiles_prev) -> bool {
+        nq += ntiles_prev * S_BOXES;
+        const int n0 = nq;
+        nq += 9;
+        bool okq = wait_u(bar(B_QEMPTY), (gq & 1) ^ 1);
         tc_fence_after();
-        const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + (t * H + i) * DC + 256 * half);
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int c = 4 * half; okq && c < 4 * half + 4; ++c) {
+          const int e = n0 + c, slot = e % S_RING;
+          okq = wait_u(bar(B_SFULL + slot), (e / S_RING) & 1);
+          if (!okq) break;
+          const uint8_t* src = smem + S_OFF_RING + slot * BOX + i * 128;
           uint32_t v[32];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint4 u = __ldg(src + 8 * cc + e);
-            v[4 * e] = u.x; v[4 * e + 1] = u.y; v[4 * e + 2] = u.z; v[4 * e + 3] = u.w;
+          for (int q = 0; q < 8; ++q) {
+            const uint4 u = *reinterpret_cast<const uint4*>(src + ((q ^ (i & 7)) << 4));
+            v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
           }
-          tmem_st32(trow + 128 * half + 32 * cc, v);
+          tmem_st32(trow + 32 * c, v);
         }
-        const uint4* rsrc = reinterpret_cast<const uint4*>(p.q_rope + (t * H + i) * DR);
-        uint8_t* qrow = smem + S_OFF_QR + i * 128;
-#pragma unroll
-        for (int c = 4 * half; c < 4 * half + 4; ++c)
-          *reinterpret_cast<uint4*>(qrow + ((c ^ (i & 7)) << 4)) = __ldg(rsrc + c);
         tmem_wait_st();
-        fence_proxy_async_smem();
+        if (bar_sync_or(1, 256, !okq)) return false;   // all 8 q~ boxes read (or a wait gave up)
+        if (threadIdx.x == 128)
+          for (int c = 0; c < 8; ++c) mbar_arrive(bar(B_SEMPTY + (n0 + c) % S_RING));
+        {
+          const int e = n0 + 8, slot = e % S_RING;
+          okq = wait_u(bar(B_SFULL + slot), (e / S_RING) & 1);
+          if (okq) {
+            const uint8_t* src = smem + S_OFF_RING + slot * BOX + i * 128;
+            uint8_t* dst = smem + S_OFF_QR + i * 128;
+#pragma unroll
+            for (int c = 4 * half; c < 4 * half + 4; ++c) {
+              const int o = (c ^ (i & 7)) << 4;
+              *reinterpret_cast<uint4*>(dst + o) = *reinterpret_cast<const uint4*>(src + o);
+            }
+            fence_proxy_async_smem();
+          }
+          if (bar_sync_or(1, 256, !okq)) return false;   // the q^R entry read
+          if (threadIdx.x == 128) mbar_arrive(bar(B_SEMPTY + slot));
+        }
         tc_fence_before();
         mbar_arrive(bar(B_QFULL));
         ++gq;
         return true;
       };
-      ok = !w.valid() || load_q(w.b);
+      ok = !w.valid() || load_q(0);
       int j = 0;
       for (; ok && w.valid(); w.next()) {
         const int b = w.b;
@@ -428,32 +472,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           float* hdr = reinterpret_cast<float*>(msg + P_BYTES);
           if (half == 0) hdr[i] = first ? 1.f : alpha;
           if (last) {
-            // piece end: both halves' sums -> 1/l for the value CTA, lse written here
+            // piece end: lse of the piece and the reference of its unnormalised partial
             float lp;
             if (!swap_half(l, 2, lp)) { ok = false; break; }
             const float lt = l + lp;
             if (half == 0) {
-              hdr[H + i] = lt > 0.f ? 1.f / lt : 0.f;
-              const float lse_v = lt > 0.f ? (m_ref * c2 + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-              const int64_t t = (int64_t)b * p.tq + k;
-              const int32_t nseg = p.slot_base[b + 1] - p.slot_base[b];
-              if (nseg > 1) {
-                const int64_t slot =
-                    (int64_t)p.slot_base[b] + (pair - (int)(((int64_t)(ts_b + 1) * npairs - 1) / NT));
-                p.part_lse[((int64_t)k * p.s_max + slot) * H + i] = lse_v;
-              } else {
-                p.lse[t * H + i] = lse_v;
-              }
+              const int64_t row = ((int64_t)k * p.s_max + piece_slot(b)) * H + i;
+              p.part_lse[row] = lt > 0.f ? (m_ref * c2 + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+              p.part_m[row] = lt > 0.f ? m_ref * c2 * 0.69314718055994531f : -INFINITY;
             }
           }
           fence_proxy_async_smem();
           mbar_arrive(bar(B_PSTG + sb));
         }
         if (!ok) break;
-        // the next piece's query goes in now, so that its first QK^T overlaps the value CTA's epilogue
+        // the next piece's q^R goes in now, so that its first QK^T overlaps the value CTA's epilogue
         SegWalk nx = w;
         nx.next();
-        if (nx.valid() && !load_q(nx.b)) { ok = false; break; }
+        if (nx.valid() && !load_q(send - w.x)) { ok = false; break; }
       }
       if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
     }
@@ -461,14 +497,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // =========================================================== value CTA
     if (warp == 0) {
       // ------------------------------------------------ TMA producer: 4 groups per tile
-      if (lane == 0) {
-        int n = 0, issued = 0;
-        for (; ok && w.valid(); w.next()) {
-          const int32_t ts_b = p.tile_start[w.b];
-          const int32_t row_base = (int32_t)p.cu[w.b];
-          for (int32_t xt = w.x; ok && xt < w.seg_end(); ++xt) {
+      // lanes 0-3 issue, lane l the group (N-half l & 1, key-half l >> 1) of every tile (ring slot l)
+      if (lane < kIssuers) {
+        int n = 0, last = -1;
+        for (SegWalk sw = w; ok && sw.valid(); sw.next()) {
+          const int32_t ts_b = p.tile_start[sw.b];
+          const int32_t row_base = (int32_t)p.cu[sw.b];
+          for (int32_t xt = sw.x; ok && xt < sw.seg_end(); ++xt) {
             const int32_t row0 = row_base + (xt - ts_b) * NK;
             for (int s = 0; s < 4; ++s, ++n) {
+              if ((n & (kIssuers - 1)) != lane) continue;
               const int g = n % V_RING;
               if (!wait_bar(bar(B_GEMPTY + g), ((n / V_RING) & 1) ^ 1, lim)) { ok = false; break; }
               mbar_expect_tx(bar(B_GFULL + g), VGRP);
@@ -477,13 +515,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int bx = 0; bx < 4; ++bx)
                 tma_load_2d(dst + bx * VBOX, &p.vmap, 256 * nh + 64 * bx, row0 + 64 * kh, bar(B_GFULL + g));
-              issued = n + 1;
+              last = n;
             }
           }
         }
         if (!ok) {
           flag_error(p.err, DEVERR_TIMEOUT);
-          for (int i = max(0, issued - V_RING); i < issued; ++i) wait_bar(bar(B_GFULL + i % V_RING), (i / V_RING) & 1, lim);
+          for (int i = max(lane, last - V_RING + 1); i <= last; ++i)
+            if ((i & (kIssuers - 1)) == lane) wait_bar(bar(B_GFULL + i % V_RING), (i / V_RING) & 1, lim);
         }
       }
     } else if (warp == 1) {
@@ -523,30 +562,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mma_commit_mc(bar(B_PVD + pb), 0x3);
           }
           if (!ok) break;
+          mma_commit(bar(B_ODONE));
         }
         if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
       }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4) {
       // ------------------------------------------------ rescale + piece epilogue (thread = head = TMEM lane)
-      const int quarter = warp & 3;
+      // Warps 4-7 rescale O when the running max moved and zero cache rows past the last sequence
+      // (per tile); at a piece's end warps 4-7 write O's columns [0, 256) and warps 8-11 columns
+      // [256, 512) as the unnormalised partial.
+      const int quarter = warp & 3, ehalf = warp >= 8 ? 1 : 0;
       const int i = 32 * quarter + lane;
       const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
       const int64_t total_rows = p.cu[p.B];
       auto wait_u = [&](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, wait_bar(b, par, lim)) != 0; };
+      // the piece's partial, once its last P.V is done (B_ODONE moves once per piece, so neither half
+      // can see a stale phase however far behind it runs)
+      auto dump = [&](int b, int g) -> bool {
+        if (!wait_u(bar(B_ODONE), g & 1)) return false;
+        tc_fence_after();
+        float4* po = reinterpret_cast<float4*>(p.part_o) + ((int64_t)k * p.s_max + piece_slot(b)) * (DC / 4) * H + i;
+#pragma unroll 1
+        for (int c = 256 * ehalf; c < 256 * ehalf + 256; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(trow + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            po[(c / 4 + e) * H] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                              __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        }
+        tc_fence_before();
+        mbar_arrive(bar(B_OFREE));
+        return true;
+      };
       int j = 0, n = 0;
-      for (; ok && w.valid(); w.next()) {
+      for (int g = 0; ok && w.valid(); w.next(), ++g) {
         const int b = w.b;
         const int32_t ts_b = p.tile_start[b];
         const int32_t send = w.seg_end();
+        if (ehalf) {
+          // columns [256, 512) of the piece's partial
+          if (!dump(b, g)) { ok = false; break; }
+          continue;
+        }
         const int64_t row_base = p.cu[b];
-        float inv_l = 0.f;
         for (int32_t xt = w.x; xt < send; ++xt, ++j, n += 4) {
           const int pb = j & 1;
           const bool first = xt == w.x, last = xt == send - 1;
           if (!wait_u(bar(B_PFULL + pb), (j >> 1) & 1)) { ok = false; break; }
           const float* hdr = reinterpret_cast<const float*>(smem + V_OFF_PBUF + pb * PMSG + P_BYTES);
           const float alpha = hdr[i];
-          if (last) inv_l = hdr[H + i];
           if (__any_sync(0xffffffffu, !first && alpha != 1.f)) {
             // O holds the previous tiles' sum at the old max: rescale once their P.V is done
             if (!wait_u(bar(B_PVD + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) { ok = false; break; }
@@ -568,11 +634,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int64_t row0 = row_base + (int64_t)(xt - ts_b) * NK;
           if (row0 + NK > total_rows) {
             const int nrows = (int)max((int64_t)0, total_rows - row0);
-            for (int s = 0; s < 4; ++s) {
-              const int gi = (n + s) % V_RING;
-              if (!wait_u(bar(B_GFULL + gi), ((n + s) / V_RING) & 1)) { ok = false; break; }
+            for (int s2 = 0; s2 < 4; ++s2) {
+              const int gi = (n + s2) % V_RING;
+              if (!wait_u(bar(B_GFULL + gi), ((n + s2) / V_RING) & 1)) { ok = false; break; }
               uint8_t* grp = smem + V_OFF_RING + gi * VGRP;
-              const int kh = s >> 1;
+              const int kh = s2 >> 1;
               // rows 64 kh + rr >= nrows, 4 boxes x 8 chunks of 16 bytes each
               for (int q = i; q < 64 * 32; q += 128) {
                 const int rr = q >> 5, bx = (q >> 3) & 3, c16 = q & 7;
@@ -584,43 +650,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
           }
           mbar_arrive(bar(B_OREADY + pb));
-          if (last) {
-            // piece epilogue: o^lat = O / l for all 512 columns of head i
-            if (!wait_u(bar(B_PVD + pb), (j >> 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-            const int64_t t = (int64_t)b * p.tq + k;
-            const int32_t nseg = p.slot_base[b + 1] - p.slot_base[b];
-            float* po = nullptr;
-            if (nseg > 1) {
-              const int64_t slot = (int64_t)p.slot_base[b] + (pair - (int)(((int64_t)(ts_b + 1) * npairs - 1) / NT));
-              po = p.part_o + (((int64_t)k * p.s_max + slot) * H + i) * DC;
-            }
-#pragma unroll 1
-            for (int c = 0; c < DC; c += 32) {
-              uint32_t v[32];
-              tmem_ld32(trow + c, v);
-              tmem_wait_ld();
-              if (po || OUT_F32) {
-                float4* dst = po ? reinterpret_cast<float4*>(po + c)
-                                 : reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o_lat) + (t * H + i) * DC + c);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                  dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv_l, __uint_as_float(v[4 * e + 1]) * inv_l,
-                                       __uint_as_float(v[4 * e + 2]) * inv_l, __uint_as_float(v[4 * e + 3]) * inv_l);
-              } else {
-                uint4* dst =
-                    reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o_lat) + (t * H + i) * DC + c);
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  dst[e] = make_uint4(pack_bf16(__uint_as_float(v[8 * e]) * inv_l, __uint_as_float(v[8 * e + 1]) * inv_l),
-                                      pack_bf16(__uint_as_float(v[8 * e + 2]) * inv_l, __uint_as_float(v[8 * e + 3]) * inv_l),
-                                      pack_bf16(__uint_as_float(v[8 * e + 4]) * inv_l, __uint_as_float(v[8 * e + 5]) * inv_l),
-                                      pack_bf16(__uint_as_float(v[8 * e + 6]) * inv_l, __uint_as_float(v[8 * e + 7]) * inv_l));
-              }
-            }
-            tc_fence_before();
-            mbar_arrive(bar(B_OFREE));
-          }
+          if (last && !dump(b, g)) { ok = false; break; }
         }
         if (!ok) break;
       }
@@ -667,7 +697,7 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
 }
 
 __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B, int32_t pairs, int32_t* ts,
-                                                   int32_t* sb) {
+                                                   int32_t* sb, int4* pinfo) {
   __shared__ int32_t warp_tot[8];
   __shared__ int32_t total;
   const int tid = threadIdx.x;
@@ -695,60 +725,107 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
   acc = block_exclusive_scan(acc, warp_tot, &total);
   for (int b = lo; b < hi; ++b) { sb[b] = acc; acc += nseg(b); }
   if (tid == 0) sb[B] = total;
+  __syncthreads();
+  // per cluster: its tile range, the sequence of its first tile and that piece's partial slot
+  for (int pp = tid; pp < pairs; pp += blockDim.x) {
+    int4 v = make_int4(0, 0, 0, 0);
+    if (pp < npairs) {
+      v.x = (int32_t)((int64_t)pp * NT / npairs);
+      v.y = (int32_t)((int64_t)(pp + 1) * NT / npairs);
+      int lo2 = 0, hi2 = B - 1;               // the last b with ts[b] <= v.x
+      while (lo2 < hi2) {
+        const int mid = (lo2 + hi2 + 1) >> 1;
+        if (ts[mid] <= v.x) lo2 = mid; else hi2 = mid - 1;
+      }
+      // the first sequence with tiles: skip empty sequences that share the start
+      while (lo2 < B - 1 && ts[lo2 + 1] <= v.x) ++lo2;
+      v.z = lo2;
+      v.w = sb[lo2] + (int32_t)(pp - pair_of(ts[lo2]));
+    }
+    pinfo[pp] = v;
+  }
 }
 
-// Exact merge of a sequence's pieces: lse = log sum_s e^{lse_s}, o = sum_s e^{lse_s - lse} o_s.
-// One block of 128 threads per (token, head); sequences in a single piece were written directly.
+// Exact merge of a sequence's pieces: lse = log sum_s e^{lse_s}, o = sum_s e^{m_s - lse} O_s from the
+// unnormalised head-interleaved partials O_s (O_s / l_s is the piece's own softmax average and
+// e^{lse_s} = e^{m_s} l_s, so the weight e^{lse_s - lse} / l_s is e^{m_s - lse}). One block per (token, group of 32 heads, group of 128 columns): the
+// reads of a (piece, 4-column group) are 512 contiguous bytes over the 32 heads; the block's
+// [32 heads x 128 columns] result goes through shared memory so that each head's row is written as
+// contiguous 512-byte runs.
+constexpr int kCombHeads = 32, kCombCols = 128;
 template <bool OUT_F32>
-__global__ void __launch_bounds__(128) combine_kernel(const int32_t* sb, int32_t tq, int32_t s_max,
-                                                      const float* part_o, const float* part_lse, void* o_lat,
-                                                      float* lse) {
-  __shared__ float wts[kMaxPairs + 64];
-  __shared__ float red[32];
+__global__ void __launch_bounds__(256) combine_kernel(const int32_t* sb, int32_t tq, int32_t s_max,
+                                                      const float* part_o, const float* part_lse,
+                                                      const float* part_m, void* o_lat, float* lse) {
+  __shared__ float wts[kMaxPairs][kCombHeads];
+  __shared__ float tile[kCombHeads][kCombCols + 4];
   const int64_t t = blockIdx.x;
-  const int h = blockIdx.y;
+  const int h0 = kCombHeads * blockIdx.y, c0 = kCombCols * blockIdx.z;
   const int b = (int)(t / tq), k = (int)(t % tq);
-  const int32_t s0 = sb[b], ns = min(sb[b + 1] - s0, kMaxPairs + 64);
-  if (ns == 1) return;
-  const int64_t row0 = ((int64_t)k * s_max + s0) * H + h;
-  float lmax = -INFINITY;
-  for (int s = threadIdx.x; s < ns; s += 128) {
-    const float v = part_lse[row0 + (int64_t)s * H];
-    wts[s] = v;
-    lmax = fmaxf(lmax, v);
+  const int32_t s0 = sb[b], ns = min(sb[b + 1] - s0, kMaxPairs);
+  const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
+  const int64_t slot0 = (int64_t)k * s_max + s0;
+  if (tid < kCombHeads) {
+    // weights of head h0 + tid over the pieces
+    const int h = h0 + tid;
+    float mx = -INFINITY;
+    for (int sl = 0; sl < ns; ++sl) mx = fmaxf(mx, part_lse[(slot0 + sl) * H + h]);
+    float sum = 0.f;
+    for (int sl = 0; sl < ns; ++sl) sum += mx > -INFINITY ? __expf(part_lse[(slot0 + sl) * H + h] - mx) : 0.f;
+    const float tot = sum > 0.f ? mx + logf(sum) : -INFINITY;     // lse over all pieces
+    for (int sl = 0; sl < ns; ++sl) {
+      const float ms = part_m[(slot0 + sl) * H + h];
+      wts[sl][tid] = (tot > -INFINITY && ms > -INFINITY) ? __expf(ms - tot) : 0.f;
+    }
+    if (blockIdx.z == 0) lse[t * H + h] = tot;
   }
-  const float mx = block_max(lmax, red);
-  float wpart = 0.f;
-  for (int s = threadIdx.x; s < ns; s += 128) {
-    const float wv = mx > -INFINITY ? __expf(wts[s] - mx) : 0.f;
-    wts[s] = wv;
-    wpart += wv;
+  __syncthreads();
+  // thread (lane = head, grp): 4-column groups c4 = c0/4 + 4 grp + q, q = 0..3
+  float4 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4* src = reinterpret_cast<const float4*>(part_o) + (c0 / 4 + 4 * grp) * H + h0 + lane;
+  for (int sl = 0; sl < ns; ++sl) {
+    const float wgt = wts[sl][lane];
+    const float4* ps = src + (slot0 + sl) * (DC / 4) * H;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = ps[q * H];
+      acc[q].x += wgt * v.x; acc[q].y += wgt * v.y; acc[q].z += wgt * v.z; acc[q].w += wgt * v.w;
+    }
   }
-  const float wsum = block_sum(wpart, red);   // includes a __syncthreads: wts[] is complete
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int s = 0; s < ns; ++s) {
-    const float wgt = wts[s];
-    const float4 v = reinterpret_cast<const float4*>(part_o + (row0 + (int64_t)s * H) * DC)[threadIdx.x];
-    acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
-  }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) *reinterpret_cast<float4*>(&tile[lane][16 * grp + 4 * q]) = acc[q];
+  __syncthreads();
+  // row h0 + r, columns c0 .. c0 + 127: 8 threads per row, 16 columns each
+  const int r = tid >> 3, cc = 16 * (tid & 7);
+  const int64_t dst = (t * H + h0 + r) * DC + c0 + cc;
   if (OUT_F32) {
-    reinterpret_cast<float4*>(reinterpret_cast<float*>(o_lat) + (t * H + h) * DC)[threadIdx.x] = acc;
+    float4* d4 = reinterpret_cast<float4*>(reinterpret_cast<float*>(o_lat) + dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d4[q] = *reinterpret_cast<const float4*>(&tile[r][cc + 4 * q]);
   } else {
-    uint2 v2 = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
-    reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(o_lat) + (t * H + h) * DC)[threadIdx.x] = v2;
+    uint4* d4 = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(o_lat) + dst);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const float* x = &tile[r][cc + 8 * q];
+      d4[q] = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+    }
   }
-  if (threadIdx.x == 0) lse[t * H + h] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
 }
 
 size_t align1k(size_t x) { return (x + 1023) / 1024 * 1024; }
 
+// Clusters per query token: each query token k takes its own row of clusters, and all rows
+// together hold at most kMaxPairs clusters (one CTA per SM).
+int32_t pairs_cap(int32_t tq) { return kMaxPairs / tq > 1 ? kMaxPairs / tq : 1; }
+
 struct CoreScratch {
   int32_t* ts;
   int32_t* sb;
+  int4* pinfo;
   float* part_lse;
+  float* part_m;
   float* part_o;
   int32_t s_max;
 };
@@ -756,28 +833,31 @@ struct CoreScratch {
 CoreScratch carve(void* scratch, int64_t B, int32_t tq) {
   CoreScratch c;
   char* ptr = (char*)scratch;
-  c.s_max = (int32_t)(kMaxPairs + B);
+  c.s_max = (int32_t)(pairs_cap(tq) + B);
   c.ts = (int32_t*)ptr;
   ptr += align1k((B + 1) * 4);
   c.sb = (int32_t*)ptr;
   ptr += align1k((B + 1) * 4);
+  c.pinfo = (int4*)ptr;
+  ptr += align1k(kMaxPairs * sizeof(int4));
   c.part_lse = (float*)ptr;
+  ptr += align1k((size_t)tq * c.s_max * H * 4);
+  c.part_m = (float*)ptr;
   ptr += align1k((size_t)tq * c.s_max * H * 4);
   c.part_o = (float*)ptr;
   return c;
 }
 
-template <bool OUT_F32>
 cudaError_t launch_core(const CoreParams& p, dim3 grid, cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(latent_core_kernel<OUT_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+    cudaError_t e =
+        cudaFuncSetAttribute(latent_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   timer_begin(TIMED_LATENT_CORE, st);
-  latent_core_kernel<OUT_F32><<<grid, kThreads, SMEM_BYTES, st>>>(p);
+  latent_core_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p);
   timer_end(TIMED_LATENT_CORE, st);
   note_launch();
   return cudaGetLastError();
@@ -792,41 +872,43 @@ void tc_latent_core_arm_stall() { g_stall_next = 1; }
 
 size_t tc_core_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq) {
   (void)d;
-  const int64_t s_max = kMaxPairs + B;
-  return 2 * align1k((B + 1) * 4) + align1k((size_t)tq * s_max * H * 4) + (size_t)tq * s_max * H * DC * 4;
+  const int64_t s_max = pairs_cap(tq) + B;
+  return 2 * align1k((B + 1) * 4) + align1k(kMaxPairs * sizeof(int4)) + 2 * align1k((size_t)tq * s_max * H * 4) +
+         (size_t)tq * s_max * H * DC * 4;
 }
 
 cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
                                 const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse,
                                 void* scratch, int num_sms, uint32_t* err, cudaStream_t st) {
   if (B <= 0) return cudaSuccess;
-  if (B > (int64_t)1 << 20 || capacity > INT32_MAX || B * tq * H > INT32_MAX) return cudaErrorInvalidValue;
+  if (B > (int64_t)1 << 20 || tq < 1 || tq > kMaxPairs || capacity > INT32_MAX || B * tq * H > INT32_MAX)
+    return cudaErrorInvalidValue;
   const int64_t T = B * tq;
   CoreScratch c = carve(scratch, B, tq);
   int pairs = num_sms / (2 * tq);
-  pairs = pairs < kMaxPairs ? pairs : kMaxPairs;
+  pairs = pairs < pairs_cap(tq) ? pairs : pairs_cap(tq);
   pairs = pairs < 1 ? 1 : pairs;
-  plan_kernel<<<1, 256, 0, st>>>(cu, (int32_t)B, pairs, c.ts, c.sb);
+  plan_kernel<<<1, 256, 0, st>>>(cu, (int32_t)B, pairs, c.ts, c.sb, c.pinfo);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CoreParams p;
   memset(&p, 0, sizeof(p));
-  p.q_abs = reinterpret_cast<const __nv_bfloat16*>(q_abs);
-  p.q_rope = reinterpret_cast<const __nv_bfloat16*>(q_rope);
   if ((e = make_tmap_bf16(&p.kmap, cache, ROW, capacity, ROW, 64, NK)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&p.vmap, cache, ROW, capacity, ROW, 64, 64)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&p.qmap, q_abs, DC, T * H, DC, 64, H)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&p.qrmap, q_rope, DR, T * H, DR, 64, H)) != cudaSuccess) return e;
   p.cu = cu;
   p.tile_start = c.ts;
   p.slot_base = c.sb;
+  p.pinfo = c.pinfo;
   p.B = (int32_t)B;
   p.tq = tq;
   p.pairs = pairs;
   p.s_max = c.s_max;
   p.part_o = c.part_o;
   p.part_lse = c.part_lse;
-  p.o_lat = o_lat;
-  p.lse = lse;
+  p.part_m = c.part_m;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt(128.0 + 64.0));
   p.wait_ns = kWaitTimeoutNs;
   if (g_stall_next) {
@@ -836,11 +918,11 @@ cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B
   }
   p.err = err;
   dim3 grid((unsigned)(2 * pairs), (unsigned)tq);
-  e = o_f32 ? launch_core<true>(p, grid, st) : launch_core<false>(p, grid, st);
+  e = launch_core(p, grid, st);
   if (e != cudaSuccess) return e;
-  dim3 cg((unsigned)T, (unsigned)H);
-  if (o_f32) combine_kernel<true><<<cg, 128, 0, st>>>(c.sb, tq, c.s_max, c.part_o, c.part_lse, o_lat, lse);
-  else combine_kernel<false><<<cg, 128, 0, st>>>(c.sb, tq, c.s_max, c.part_o, c.part_lse, o_lat, lse);
+  dim3 cg((unsigned)T, (unsigned)(H / kCombHeads), (unsigned)(DC / kCombCols));
+  if (o_f32) combine_kernel<true><<<cg, 256, 0, st>>>(c.sb, tq, c.s_max, c.part_o, c.part_lse, c.part_m, o_lat, lse);
+  else combine_kernel<false><<<cg, 256, 0, st>>>(c.sb, tq, c.s_max, c.part_o, c.part_lse, c.part_m, o_lat, lse);
   note_launch();
   return cudaGetLastError();
 }

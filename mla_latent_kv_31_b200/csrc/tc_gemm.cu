@@ -22,6 +22,7 @@ constexpr int kThreads = 192;    // warp 0: TMA producer, warp 1: TMEM owner + M
 constexpr int kMaxSplits = 64;
 constexpr int kMaxRopePairs = 64;
 constexpr int kRasterW = 8;      // weight tiles per raster group (large token counts)
+constexpr int kIssuers = 4;      // TMA issuing lanes of the producer warp (every ring has 4 stages)
 
 struct GemmParams {
   CUtensorMap wmap[2];
@@ -34,7 +35,8 @@ struct GemmParams {
   int32_t w_row_z, w_col_z, x_col_z;
   const int64_t* pos;
   int32_t d_r;
-  double theta[kMaxRopePairs];     // RoPE frequencies base^(-2m/d_r)
+  double theta[kMaxRopePairs];     // RoPE frequencies theta_m (plain or YaRN)
+  float rope_mul;                  // factor on each rotated vector (YaRN; else 1)
   float* partial;
   int64_t f_total;
   uint32_t* err;
@@ -56,14 +58,15 @@ __device__ __forceinline__ void store_out(const TcEpiSeg& E, uint32_t* err, int 
 }
 
 // RoPE of one element of the pair (2m, 2m+1) that holds feature f (segment-local): `own` is x_f,
-// `partner` is x_{f^1}. The angle pos * theta_m is reduced modulo 2 pi in double, then sincosf.
+// `partner` is x_{f^1}. The angle pos * theta_m is reduced modulo 2 pi in double, then sincosf;
+// the rotated value is multiplied by `mul`.
 __device__ __forceinline__ float rope_one(int64_t f, int64_t pos, float own, float partner, int d_r,
-                                          const double* theta) {
+                                          const double* theta, float mul) {
   const double a = (double)pos * theta[(f % d_r) >> 1];
   const double red = a - 6.283185307179586 * rint(a * 0.15915494309189535);
   float s, c;
   sincosf((float)red, &s, &c);
-  return (f & 1) ? (partner * s + own * c) : (own * c - partner * s);
+  return ((f & 1) ? (partner * s + own * c) : (own * c - partner * s)) * mul;
 }
 
 template <int BN, bool SWAP, bool W_MN, int STAGES>
@@ -144,14 +147,17 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
   };
 
   if (warp == 0) {
-    if (lane == 0) {
-      int it = 0, issued = 0;
+    // One TMA issuing thread streams only about 40 GB/s, so lanes 0 .. kIssuers-1 issue: lane l
+    // loads the k-blocks it = l mod kIssuers (ring stages l, l + kIssuers, ...).
+    if (lane < kIssuers) {
+      int it = 0, last = -1;
       bool ok = true;
       for (int idx = blockIdx.x; ok && idx < p.tiles; idx += gridDim.x) {
         const Tile d = decode_tile(idx);
         const CUtensorMap* wm = &p.wmap[d.s];
         const int64_t f0 = (int64_t)d.wt * W_TILE, t0 = (int64_t)d.tt * X_TILE;
         for (int i = 0; i < d.nkb; ++i, ++it) {
+          if ((it % kIssuers) != lane) continue;
           const int st = it % STAGES;
           if (!mbar_wait(bar(B_EMPTY + st), ((it / STAGES) & 1) ^ 1)) { ok = false; break; }
           const uint32_t full = bar(B_FULL + st);
@@ -167,12 +173,13 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
             tma_load_2d(w_dst, wm, k0 + d.z * p.w_col_z, (int)f0 + d.z * p.w_row_z, full);
           }
           tma_load_2d(x_dst, &p.xmap, k0 + d.z * p.x_col_z, (int)t0, full);
-          issued = it + 1;
+          last = it;
         }
       }
       if (!ok) {
         flag_error(p.err, DEVERR_TIMEOUT);
-        for (int i = max(0, issued - STAGES); i < issued; ++i) mbar_wait(bar(B_FULL + i % STAGES), (i / STAGES) & 1);
+        for (int i = max(lane, last - STAGES + 1); i <= last; ++i)
+          if ((i % kIssuers) == lane) mbar_wait(bar(B_FULL + i % STAGES), (i / STAGES) & 1);
       }
     }
   } else if (warp == 1) {
@@ -242,8 +249,8 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
             for (int j = 0; j < 32; j += 2) {
               float a = __uint_as_float(v[j]), b2 = __uint_as_float(v[j + 1]);
               if (E.rope) {
-                const float a2 = rope_one(f + j, ps, a, b2, p.d_r, p.theta);
-                const float b3 = rope_one(f + j + 1, ps, b2, a, p.d_r, p.theta);
+                const float a2 = rope_one(f + j, ps, a, b2, p.d_r, p.theta, p.rope_mul);
+                const float b3 = rope_one(f + j + 1, ps, b2, a, p.d_r, p.theta, p.rope_mul);
                 a = a2;
                 b2 = b3;
               }
@@ -276,7 +283,7 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
               flag_error(p.err, DEVERR_POSITION);
               continue;
             }
-            y = rope_one(f, ps, x, partner, p.d_r, p.theta);
+            y = rope_one(f, ps, x, partner, p.d_r, p.theta, p.rope_mul);
           }
           store_out(E, p.err, d.z, f, t, y);
         }
@@ -302,6 +309,7 @@ struct ReduceParams {
   const int64_t* pos;
   int32_t d_r;
   double theta[kMaxRopePairs];
+  float rope_mul;
   uint32_t* err;
 };
 
@@ -341,8 +349,8 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constan
       flag_error(p.err, DEVERR_POSITION);
       return;
     }
-    const float a2 = rope_one(fl, ps, a, b, p.d_r, p.theta);
-    const float b2 = rope_one(fl + 1, ps, b, a, p.d_r, p.theta);
+    const float a2 = rope_one(fl, ps, a, b, p.d_r, p.theta, p.rope_mul);
+    const float b2 = rope_one(fl + 1, ps, b, a, p.d_r, p.theta, p.rope_mul);
     a = a2;
     b = b2;
   }
@@ -506,7 +514,8 @@ cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st) {
   p.x_col_z = (int32_t)g.x_col_z;
   p.pos = g.pos;
   p.d_r = g.d_r;
-  for (int m = 0; m < g.d_r / 2; ++m) p.theta[m] = pow(g.rope_base, -2.0 * m / g.d_r);
+  for (int m = 0; m < g.d_r / 2; ++m) p.theta[m] = rope_theta(g.rope, m, g.d_r);
+  p.rope_mul = rope_mul(g.rope);
   p.partial = g.partial;
   p.f_total = f_total;
   p.err = g.err;
@@ -540,6 +549,7 @@ cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st) {
   r.pos = g.pos;
   r.d_r = g.d_r;
   memcpy(r.theta, p.theta, sizeof(r.theta));
+  r.rope_mul = p.rope_mul;
   r.err = g.err;
   int L = 2;
   while (L < p.splits && L < 32) L <<= 1;

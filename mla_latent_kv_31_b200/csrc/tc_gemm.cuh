@@ -14,6 +14,8 @@
 #include <cuda.h>
 #include <stdint.h>
 
+#include "common.cuh"
+
 namespace mla {
 
 // Largest token count of the weight-streaming ("swap") orientation; head-batched and MN-major weight
@@ -51,7 +53,7 @@ struct TcGemmDesc {
   int32_t batch;
   int64_t w_row_z, w_col_z;   // per-batch offsets of the weight operand (elements)
   int64_t x_col_z;            // per-batch column offset of X
-  const int64_t* pos; int32_t d_r; double rope_base;
+  const int64_t* pos; int32_t d_r; RopeSpec rope;   // RoPE epilogue (segments with epi.rope)
   float* partial;             // split-K scratch (fp32), may be null when splits == 1
   size_t partial_bytes;
   uint32_t* err;

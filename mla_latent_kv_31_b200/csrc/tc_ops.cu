@@ -44,10 +44,11 @@ size_t decode_gemm_partials(const mla_dims_t& d, int64_t T) {
   return align_up(ab > c ? ab : c);
 }
 
-// Steps (5) and (7) with the cache write: rows [c^KV | RoPE(W^KR h)] -> cache[rowmap[t]].
-cudaError_t cache_rows(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, const int64_t* pos,
-                       const int64_t* rowmap, int64_t T, void* cache, int64_t capacity, void* scratch,
-                       size_t scratch_bytes, uint32_t* err, cudaStream_t st) {
+// Steps (5) and (7) with the cache write: rows [c^KV | RoPE(W^KR h)] -> cache[rowmap[t]], then the
+// optional RMSNorm of c^KV in place.
+cudaError_t cache_rows(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& o, const void* hidden,
+                       const int64_t* pos, const int64_t* rowmap, int64_t T, void* cache, int64_t capacity,
+                       void* scratch, size_t scratch_bytes, uint32_t* err, cudaStream_t st) {
   const int64_t R = d.d_c + d.d_r;
   TcGemmDesc g = desc(mat(hidden, T, d.d, d.d), T, d.d, err);
   g.nseg = 2;
@@ -60,15 +61,17 @@ cudaError_t cache_rows(const mla_dims_t& d, const mla_weights_t& w, const void* 
     g.seg[s].epi.rowmap = rowmap;
     g.seg[s].epi.rowmap_limit = capacity;
   }
-  g.pos = pos; g.d_r = d.d_r; g.rope_base = d.rope_base;
+  g.pos = pos; g.d_r = d.d_r; g.rope = o.rope;
   g.partial = (float*)scratch; g.partial_bytes = scratch_bytes;
-  return tc_gemm(g, st);
+  cudaError_t e = tc_gemm(g, st);
+  if (e != cudaSuccess || !o.g_kv) return e;
+  return rmsnorm_rows(cache, true, R, rowmap, capacity, T, d.d_c, o.g_kv, o.eps, st);
 }
 
-// Steps (1)-(3): c^Q = W^DQ h; q^C = W^UQ c^Q; q^R = RoPE(W^QR c^Q).
-cudaError_t queries(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, const int64_t* pos, int64_t T,
-                    void* cq, void* qc, void* qr, void* scratch, size_t scratch_bytes, uint32_t* err,
-                    cudaStream_t st) {
+// Steps (1)-(3): c^Q = W^DQ h (then the optional RMSNorm); q^C = W^UQ c^Q; q^R = RoPE(W^QR c^Q).
+cudaError_t queries(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& o, const void* hidden,
+                    const int64_t* pos, int64_t T, void* cq, void* qc, void* qr, void* scratch, size_t scratch_bytes,
+                    uint32_t* err, cudaStream_t st) {
   const int64_t HD = (int64_t)d.n_h * d.d_h, HR = (int64_t)d.n_h * d.d_r;
   TcGemmDesc a = desc(mat(hidden, T, d.d, d.d), T, d.d, err);
   a.nseg = 1;
@@ -77,6 +80,7 @@ cudaError_t queries(const mla_dims_t& d, const mla_weights_t& w, const void* hid
   a.partial = (float*)scratch; a.partial_bytes = scratch_bytes;
   cudaError_t e = tc_gemm(a, st);
   if (e != cudaSuccess) return e;
+  if (o.g_q && (e = rmsnorm_rows(cq, true, d.d_cq, nullptr, T, T, d.d_cq, o.g_q, o.eps, st)) != cudaSuccess) return e;
   TcGemmDesc b = desc(mat(cq, T, d.d_cq, d.d_cq), T, d.d_cq, err);
   b.nseg = 2;
   b.seg[0].w = mat(w.w_uq, HD, d.d_cq, d.d_cq);
@@ -84,7 +88,7 @@ cudaError_t queries(const mla_dims_t& d, const mla_weights_t& w, const void* hid
   b.seg[1].w = mat(w.w_qr, HR, d.d_cq, d.d_cq);
   b.seg[1].epi = epi(qr, HR, 1, HR);
   b.seg[1].epi.rope = 1;
-  b.pos = pos; b.d_r = d.d_r; b.rope_base = d.rope_base;
+  b.pos = pos; b.d_r = d.d_r; b.rope = o.rope;
   b.partial = (float*)scratch; b.partial_bytes = scratch_bytes;
   return tc_gemm(b, st);
 }
@@ -111,21 +115,22 @@ size_t tc_append_scratch_bytes(const mla_dims_t& d, int64_t T) {
   return align_up(tc_gemm_partial_bytes(T, tiles128(d.d_c) + tiles128(d.d_r), d.d_c + d.d_r, d.d, 1));
 }
 
-cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const void* hidden,
+cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& o, const void* hidden,
                             const int64_t* positions, const int64_t* slots, int64_t T, void* cache,
                             int64_t capacity, void* scratch, size_t scratch_bytes, uint32_t* err,
                             cudaStream_t st) {
-  return cache_rows(d, w, hidden, positions, slots, T, cache, capacity, scratch, scratch_bytes, err, st);
+  return cache_rows(d, w, o, hidden, positions, slots, T, cache, capacity, scratch, scratch_bytes, err, st);
 }
 
-cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const void* h_q, int64_t B, int32_t tq,
+cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& lo, const void* h_q, int64_t B,
+                      int32_t tq,
                       const int64_t* cu, const int64_t* pos, const void* cache, int64_t capacity, void* u_out,
                       void* cq, void* qc, void* qr, void* qabs, void* olat, void* o, float* lse, void* scratch,
                       int num_sms, uint32_t* err, cudaStream_t st) {
   const int64_t T = B * tq, HD = (int64_t)d.n_h * d.d_h, HC = (int64_t)d.n_h * d.d_c;
   const size_t part_bytes = decode_gemm_partials(d, T);
   void* core_scratch = (char*)scratch + part_bytes;
-  cudaError_t e = queries(d, w, h_q, pos, T, cq, qc, qr, scratch, part_bytes, err, st);
+  cudaError_t e = queries(d, w, lo, h_q, pos, T, cq, qc, qr, scratch, part_bytes, err, st);
   if (e != cudaSuccess) return e;
   // q~_i = W_i^UK^T q^C_i for every head i: the weight operand is W^UK read MN-major. The
   // head-batched GEMM streams weights with the tokens on the MMA's N side, so it runs on chunks of
@@ -157,17 +162,20 @@ cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const void* h
   return output(d, w, o, T, u_out, scratch, part_bytes, err, st);
 }
 
-cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* hidden, int64_t B,
-                       const int64_t* cu, int64_t T, int64_t max_seqlen, const int64_t* pos, void* cache,
-                       int64_t capacity, void* u_out, void* cq, void* qc, void* qr, void* kc, void* vc, void* o,
-                       int num_sms, uint32_t* err, cudaStream_t st) {
+cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& lo, const void* hidden, int64_t B,
+                       const int64_t* cu, const int64_t* cu_kv, int64_t T, int64_t T_kv, int64_t max_seqlen,
+                       const int64_t* pos, const int64_t* slots, void* cache, int64_t capacity, void* u_out,
+                       void* cq, void* qc, void* qr, void* kc, void* vc, void* o, int num_sms, uint32_t* err,
+                       cudaStream_t st) {
   const int64_t R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
-  cudaError_t e = cache_rows(d, w, hidden, pos, nullptr, T, cache, capacity, nullptr, 0, err, st);
+  if (!cu_kv) T_kv = T;
+  cudaError_t e = cache_rows(d, w, lo, hidden, pos, slots, T, cache, capacity, nullptr, 0, err, st);
   if (e != cudaSuccess) return e;
-  e = queries(d, w, hidden, pos, T, cq, qc, qr, nullptr, 0, err, st);
+  e = queries(d, w, lo, hidden, pos, T, cq, qc, qr, nullptr, 0, err, st);
   if (e != cudaSuccess) return e;
-  // Steps (6), (9): [k^C; v^C] = [W^UK; W^UV] c^KV from the cache rows just written.
-  TcGemmDesc p3 = desc(mat(cache, T, d.d_c, R), T, d.d_c, err);
+  // Steps (6), (9): [k^C; v^C] = [W^UK; W^UV] c^KV from every key row (a chunk's cached prefix and
+  // the rows just written).
+  TcGemmDesc p3 = desc(mat(cache, T_kv, d.d_c, R), T_kv, d.d_c, err);
   p3.nseg = 2;
   p3.seg[0].w = mat(w.w_uk, HD, d.d_c, d.d_c);
   p3.seg[0].epi = epi(kc, HD, 1, HD);
@@ -176,7 +184,7 @@ cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const void* 
   e = tc_gemm(p3, st);
   if (e != cudaSuccess) return e;
   // Steps (4), (8), (10): causal attention per head, keys [k^C_i; k^R], values v^C_i.
-  e = tc_prefill_attention(qc, qr, kc, vc, cache, capacity, cu, B, T, max_seqlen, o, num_sms, err, st);
+  e = tc_prefill_attention(qc, qr, kc, vc, cache, capacity, cu, cu_kv, B, T, T_kv, max_seqlen, o, num_sms, err, st);
   if (e != cudaSuccess) return e;
   return output(d, w, o, T, u_out, nullptr, 0, err, st);
 }

@@ -5,9 +5,13 @@
 // head i and query token t at position p of its sequence,
 //   q = [q^C_t,i ; q^R_t,i] (192),  k_j = [k^C_j,i ; k^R_j] (192, k^R shared by the heads),
 //   o_t,i = sum_{j <= p} softmax_j(q . k_j / sqrt(d_h + d_h^R)) v^C_j,i   (128).
+// The query tokens of sequence b may be the last Tc_b of its len_b key rows (a chunk after a cached
+// prefix of P_b = len_b - Tc_b rows, whose keys are reused as they are): query token r of the chunk
+// sits at position P_b + r. A whole-sequence prefill is the case P_b = 0.
 //
 // Work unit: one head and one tile of 128 query rows of one sequence; it walks the key tiles of
-// 128 rows up to its diagonal (flash-attention online softmax). The kernel is persistent (one CTA
+// 128 rows up to the last one its rows can see (flash-attention online softmax), masking the keys
+// past each row's position. The kernel is persistent (one CTA
 // per SM); units run head-major with query tiles in descending order, so that the CTAs running at
 // the same time share one head's k^C / v^C in L2 and the long units start first.
 //
@@ -57,13 +61,14 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t T_O = 256, T_Q = 384;
 
 struct PrefillParams {
-  CUtensorMap kc_map;   // k^C as [T, H * 128], box {64, 128}
+  CUtensorMap kc_map;   // k^C as [T_kv, H * 128], box {64, 128}
   CUtensorMap kr_map;   // cache as [capacity, 576], box {64, 128} (k^R at column 512)
-  CUtensorMap vc_map;   // v^C as [T, H * 128], box {64, 128}
+  CUtensorMap vc_map;   // v^C as [T_kv, H * 128], box {64, 128}
   const __nv_bfloat16* qc;   // [T][H][128]
   const __nv_bfloat16* qr;   // [T][H][64]
   __nv_bfloat16* o;          // [T][H][128]
-  const int64_t* cu;         // [B + 1]
+  const int64_t* cu;         // [B + 1] query tokens of each sequence
+  const int64_t* cu_kv;      // [B + 1] key rows of each sequence (k^C, v^C and cache rows)
   int32_t B, M;              // sequences; query tiles of the longest sequence
   int64_t T;
   float scale_log2;          // log2(e) / sqrt(d_h + d_h^R)
@@ -73,7 +78,9 @@ struct PrefillParams {
 // Unit u -> head, query tile (descending), sequence; false when the sequence has no such tile.
 struct Unit {
   int h, m, b;
-  int64_t row0, len;   // first packed row of the sequence, its length
+  int nt;               // key tiles the unit's rows see
+  int64_t row0, len;    // first packed query row of the sequence, its query count
+  int64_t kv0, pre;     // first key row of the sequence, its prefix (position of query row 0)
 };
 __device__ __forceinline__ bool unit_of(const PrefillParams& p, int64_t u, Unit& x) {
   const int64_t per_head = (int64_t)p.B * p.M;
@@ -83,7 +90,11 @@ __device__ __forceinline__ bool unit_of(const PrefillParams& p, int64_t u, Unit&
   x.b = (int)(rem % p.B);
   x.row0 = p.cu[x.b];
   x.len = p.cu[x.b + 1] - x.row0;
-  return (int64_t)x.m * BM < x.len;
+  x.kv0 = p.cu_kv[x.b];
+  x.pre = (p.cu_kv[x.b + 1] - x.kv0) - x.len;
+  const int64_t r_last = min((int64_t)x.m * BM + BM - 1, x.len - 1);   // the tile's last valid row
+  x.nt = (int)((x.pre + r_last) / BN) + 1;
+  return (int64_t)x.m * BM < x.len && x.pre >= 0;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) prefill_attn_kernel(const __grid_constant__ PrefillParams p) {
@@ -131,11 +142,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_kernel(const __grid_
       for (int64_t u = blockIdx.x; ok && u < U; u += gridDim.x) {
         Unit x;
         if (!unit_of(p, u, x)) continue;
-        for (int n = 0; n <= x.m; ++n, ++j) {
+        for (int n = 0; n < x.nt; ++n, ++j) {
           const int s = j % nst;
           if (!mbar_wait(bar(b_empty + s), ((j / nst) & 1) ^ 1)) { ok = false; break; }
           mbar_expect_tx(bar(b_full + s), bytes);
-          const int32_t y = (int32_t)(x.row0 + (int64_t)n * BN);
+          const int32_t y = (int32_t)(x.kv0 + (int64_t)n * BN);
           const uint32_t dst = base + s * bytes;
           const CUtensorMap* map = keys ? &p.kc_map : &p.vc_map;
           tma_load_2d(dst, map, DH * x.h, y, bar(b_full + s));
@@ -179,9 +190,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_kernel(const __grid_
         Unit x;
         if (!unit_of(p, u, x)) continue;
         if (!mbar_wait(bar(B_QFULL), g & 1)) { ok = false; break; }
-        if (!qk(J, x.m == 0)) { ok = false; break; }
-        for (int n = 0; n <= x.m; ++n, ++J) {
-          if (n < x.m && !qk(J + 1, n + 1 == x.m)) { ok = false; break; }
+        if (!qk(J, x.nt == 1)) { ok = false; break; }
+        for (int n = 0; n < x.nt; ++n, ++J) {
+          if (n + 1 < x.nt && !qk(J + 1, n + 2 == x.nt)) { ok = false; break; }
           const int vs = jv % VSTAGES;
           if (!mbar_wait(bar(B_PFULL + (J & 1)), (J >> 1) & 1) || !mbar_wait(bar(B_VFULL + vs), (jv / VSTAGES) & 1) ||
               (n == 0 && !mbar_wait(bar(B_OFREE), (g & 1) ^ 1))) {
@@ -248,7 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_kernel(const __grid_
     if (u < U && !load_q(x, 0)) ok = false;
     for (; ok && u < U; ++g) {
       float m_ref = -INFINITY, l = 0.f;              // running max (raw score units) and row sum
-      for (int n = 0; n <= x.m; ++n, ++J) {
+      // row i sits at position pre + 128 m + i: key c of tile n is visible while 128 n + c <= that
+      const int64_t rpos = x.pre + (int64_t)x.m * BM + i;
+      for (int n = 0; n < x.nt; ++n, ++J) {
         const int sb = J & 1;
         if (!wait_u(bar(B_SFULL + sb), (J >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
@@ -256,9 +269,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_kernel(const __grid_
 #pragma unroll
         for (int c = 0; c < BN; c += 32) tmem_ld32(trow + BN * sb + c, reinterpret_cast<uint32_t*>(s + c));
         tmem_wait_ld();
-        if (n == x.m) {                              // diagonal tile: key c of the tile sees rows >= c
+        const int64_t lim = rpos - (int64_t)n * BN;   // the last visible key column of this tile
+        if (lim < BN - 1) {
+          const int li = (int)max(lim, (int64_t)-1);
 #pragma unroll
-          for (int c = 0; c < BN; ++c) s[c] = c <= i ? s[c] : -INFINITY;
+          for (int c = 0; c < BN; ++c) s[c] = c <= li ? s[c] : -INFINITY;
         }
         float mx[BN / 2];
 #pragma unroll
@@ -361,20 +376,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_kernel(const __grid_
 }  // namespace
 
 cudaError_t tc_prefill_attention(const void* qc, const void* qr, const void* kc, const void* vc, const void* cache,
-                                 int64_t capacity, const int64_t* cu, int64_t B, int64_t T, int64_t max_seqlen,
-                                 void* o, int num_sms, uint32_t* err, cudaStream_t st) {
+                                 int64_t capacity, const int64_t* cu, const int64_t* cu_kv, int64_t B, int64_t T,
+                                 int64_t T_kv, int64_t max_seqlen, void* o, int num_sms, uint32_t* err,
+                                 cudaStream_t st) {
   if (B <= 0 || T <= 0 || max_seqlen <= 0) return cudaSuccess;
-  if (T > INT32_MAX || capacity > INT32_MAX || B > INT32_MAX) return cudaErrorInvalidValue;
+  if (!cu_kv) { cu_kv = cu; T_kv = T; }
+  if (T > INT32_MAX || T_kv > INT32_MAX || T_kv <= 0 || capacity > INT32_MAX || B > INT32_MAX)
+    return cudaErrorInvalidValue;
   PrefillParams p;
   memset(&p, 0, sizeof(p));
   cudaError_t e;
-  if ((e = make_tmap_bf16(&p.kc_map, kc, (int64_t)H * DH, T, (int64_t)H * DH, 64, BN)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16(&p.vc_map, vc, (int64_t)H * DH, T, (int64_t)H * DH, 64, BN)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&p.kc_map, kc, (int64_t)H * DH, T_kv, (int64_t)H * DH, 64, BN)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&p.vc_map, vc, (int64_t)H * DH, T_kv, (int64_t)H * DH, 64, BN)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&p.kr_map, cache, CROW, capacity, CROW, 64, BN)) != cudaSuccess) return e;
   p.qc = reinterpret_cast<const __nv_bfloat16*>(qc);
   p.qr = reinterpret_cast<const __nv_bfloat16*>(qr);
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.cu = cu;
+  p.cu_kv = cu_kv;
   p.B = (int32_t)B;
   p.M = (int32_t)((max_seqlen + BM - 1) / BM);
   p.T = T;

@@ -15,6 +15,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so"
 MLA_BF16, MLA_FP32 = 0, 1
 OP_CACHE_APPEND, OP_DECODE, OP_PREFILL, OP_ATTN_DECODE_LATENT = 0, 1, 2, 3
 BUF_CQ, BUF_QC, BUF_QR, BUF_QABS, BUF_OLAT, BUF_O, BUF_KC, BUF_VC, BUF_LSE = range(9)
+CHUNK_AUTO, CHUNK_ABSORBED, CHUNK_UNABSORBED = 0, 1, 2
 STATUS_NAMES = ["MLA_OK", "MLA_ERR_INVALID_ARG", "MLA_ERR_ALIGNMENT", "MLA_ERR_UNSUPPORTED", "MLA_ERR_WORKSPACE",
                 "MLA_ERR_CUDA", "MLA_ERR_TIMEOUT", "MLA_ERR_DEVICE_CHECK", "MLA_ERR_NO_WEIGHTS",
                 "MLA_ERR_SCRATCH_LIMIT"]
@@ -60,10 +61,18 @@ def lib() -> ctypes.CDLL:
                                    c_size_t, c_void_p]),
             "mla_prefill": (c_int, [H, c_void_p, c_int64, c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p,
                                     c_void_p, c_size_t, c_void_p]),
+            "mla_prefill_chunk": (c_int, [H, c_void_p, c_int64, c_void_p, c_int64, c_int64, c_void_p, c_int64,
+                                          c_void_p, c_int64, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
+            "mla_prefill_chunk_workspace": (c_int, [H, c_int64, c_int64, c_int64, c_int64, c_int, POINTER(c_int),
+                                                    POINTER(c_size_t)]),
+            "mla_prefill_chunk_offset": (c_int, [H, c_int64, c_int64, c_int64, c_int64, c_int, c_int,
+                                                 POINTER(c_size_t)]),
             "mla_attn_decode_latent": (c_int, [H, c_void_p, c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_int64,
                                                c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
             "mla_attn_prefill": (c_int, [H, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_int64,
                                          c_int64, c_void_p, c_int64, c_void_p, c_void_p]),
+            "mla_set_rmsnorm": (c_int, [H, c_void_p, c_void_p, c_double]),
+            "mla_set_yarn": (c_int, [H, c_double, c_double, c_double, c_double]),
             "mla_sync_status": (c_int, [H, c_void_p]),
             "mla_device_error_bits": (c_uint32, [H]),
             "mla_uses_tensor_cores": (c_int, [H, c_int]),
@@ -152,6 +161,28 @@ def mla_prefill(handle, hidden, B, cu_seqlens, total_tokens, max_seqlen, cache, 
                              capacity, _ptr(u_out), _ptr(ws), ws_bytes, _stream(stream, device)), "mla_prefill")
 
 
+def mla_prefill_chunk(handle, hidden, B, cu_q, total_q, max_q, cu_kv, total_kv, cache, capacity, form, u_out, ws,
+                      ws_bytes, stream=None, device=0):
+    _check(lib().mla_prefill_chunk(handle, _ptr(hidden), B, _ptr(cu_q), total_q, max_q, _ptr(cu_kv), total_kv,
+                                   _ptr(cache), capacity, form, _ptr(u_out), _ptr(ws), ws_bytes,
+                                   _stream(stream, device)), "mla_prefill_chunk")
+
+
+def mla_prefill_chunk_workspace(handle, B, total_q, max_q, total_kv, form=CHUNK_AUTO) -> tuple[int, int]:
+    """(bytes, the form the call takes) for these arguments."""
+    n, f = c_size_t(), c_int()
+    _check(lib().mla_prefill_chunk_workspace(handle, B, total_q, max_q, total_kv, form, ctypes.byref(f),
+                                             ctypes.byref(n)), "mla_prefill_chunk_workspace")
+    return n.value, f.value
+
+
+def mla_prefill_chunk_offset(handle, B, total_q, max_q, total_kv, form, which) -> int:
+    n = c_size_t()
+    _check(lib().mla_prefill_chunk_offset(handle, B, total_q, max_q, total_kv, form, which, ctypes.byref(n)),
+           "mla_prefill_chunk_offset")
+    return n.value
+
+
 def mla_attn_decode_latent(handle, q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, lse, ws, ws_bytes,
                            stream=None, device=0):
     _check(lib().mla_attn_decode_latent(handle, _ptr(q_abs), _ptr(q_rope), B, Tq, _ptr(cu_seqlens), _ptr(cache),
@@ -164,6 +195,15 @@ def mla_attn_prefill(handle, q_c, q_rope, k_c, v_c, B, cu_seqlens, total_tokens,
     _check(lib().mla_attn_prefill(handle, _ptr(q_c), _ptr(q_rope), _ptr(k_c), _ptr(v_c), B, _ptr(cu_seqlens),
                                   total_tokens, max_seqlen, _ptr(cache), capacity, _ptr(o), _stream(stream, device)),
            "mla_attn_prefill")
+
+
+def mla_set_rmsnorm(handle, g_q, g_kv, eps: float = 1e-6):
+    """RMSNorm gains of c^Q and c^KV (device tensors in the handle dtype), or None, None to turn it off."""
+    _check(lib().mla_set_rmsnorm(handle, _ptr(g_q), _ptr(g_kv), eps), "mla_set_rmsnorm")
+
+
+def mla_set_yarn(handle, s: float, alpha: float = 1.0, beta: float = 32.0, original_len: float = 4096.0):
+    _check(lib().mla_set_yarn(handle, s, alpha, beta, original_len), "mla_set_yarn")
 
 
 def mla_sync_status(handle, stream=None, device=0) -> int:
@@ -220,6 +260,12 @@ class MLA:
         self.handle = mla_create(dims, dtype, device)
         self.weights = {n: weights[n] for n in WEIGHT_NAMES}
         mla_set_weights(self.handle, self.weights)
+        # opt-in parts of the layer: RMSNorm gains among the weights, YaRN settings in the dims
+        if "g_q" in weights or "g_kv" in weights:
+            self.gains = (weights["g_q"], weights["g_kv"])
+            mla_set_rmsnorm(self.handle, *self.gains, getattr(dims, "rms_eps", 1e-6))
+        if getattr(dims, "yarn_s", 1.0) > 1.0:
+            mla_set_yarn(self.handle, dims.yarn_s, dims.yarn_alpha, dims.yarn_beta, dims.yarn_l0)
         self._ws = None
 
     def close(self):
@@ -276,6 +322,28 @@ class MLA:
         mla_prefill(self.handle, hidden, B, cu_seqlens, T, max_seqlen, cache, cache.shape[0], u_out, ws, ws.numel(),
                     device=self.device)
         return u_out
+
+    def prefill_chunk(self, hidden, B, cu_q, max_q, cu_kv, total_kv, cache, form=CHUNK_AUTO, u_out=None):
+        """Chunked prefill; returns (u, the form taken)."""
+        torch = self.torch
+        T = hidden.shape[0]
+        if u_out is None:
+            u_out = torch.empty(T, self.dims.d, dtype=self.tdtype, device=hidden.device)
+        n, chosen = mla_prefill_chunk_workspace(self.handle, B, T, max_q, total_kv, form)
+        ws = self.workspace(n)
+        mla_prefill_chunk(self.handle, hidden, B, cu_q, T, max_q, cu_kv, total_kv, cache, cache.shape[0], form, u_out,
+                          ws, ws.numel(), device=self.device)
+        return u_out, chosen
+
+    def chunk_region(self, B, total_q, max_q, total_kv, form, which, shape, dtype):
+        """A view of a named workspace region after a prefill_chunk call."""
+        torch = self.torch
+        off = mla_prefill_chunk_offset(self.handle, B, total_q, max_q, total_kv, form, which)
+        n = 1
+        for s in shape:
+            n *= s
+        es = torch.tensor([], dtype=dtype).element_size()
+        return self._ws[off:off + n * es].view(dtype).view(*shape)
 
     def attn_decode_latent(self, q_abs, q_rope, B, Tq, cu_seqlens, cache, o_lat=None, lse=None):
         torch = self.torch

@@ -187,7 +187,7 @@ V3 = Dims(d=7168, n_h=128, d_h=128, d_c=512, d_cq=1536, d_r=64)
 V3_YARN = Dims(d=7168, n_h=128, d_h=128, d_c=512, d_cq=1536, d_r=64, yarn_s=40.0, yarn_alpha=1.0, yarn_beta=32.0,
                yarn_l0=4096)
 TINY_YARN = Dims(d=256, n_h=4, d_h=32, d_c=64, d_cq=96, d_r=16, yarn_s=40.0, yarn_alpha=1.0, yarn_beta=32.0,
-                 yarn_l0=64)
+                 yarn_l0=256)   # pair turns over L0: 40.7, 12.9, 4.1, 1.3, 0.41, ...: all three regimes
 
 # Weight name -> (tensor id, shape(dims) [out, in]); std = 1/sqrt(fan_in) with fan_in = in.
 WEIGHT_SPECS = {

@@ -149,3 +149,73 @@ def test_tensor_core_routing_is_declared():
     finally:
         mla.mla_destroy(bf)
         mla.mla_destroy(f32)
+
+
+def test_chunked_prefill_form_choice_workspace_and_validation():
+    h = mla.mla_create(synth.V3, mla.MLA_BF16)
+    d = synth.V3
+    try:
+        ws = mla.mla_prefill_chunk_workspace
+        # uniform short chunks on long prefixes: absorbed; ragged, long or prefix-light: unabsorbed
+        assert ws(h, 4, 16, 4, 4000)[1] == mla.CHUNK_ABSORBED
+        assert ws(h, 4, 15, 4, 4000)[1] == mla.CHUNK_UNABSORBED
+        assert ws(h, 2, 200, 100, 40000)[1] == mla.CHUNK_UNABSORBED
+        assert ws(h, 4, 16, 4, 31)[1] == mla.CHUNK_UNABSORBED
+        assert ws(h, 4, 16, 4, 32)[1] == mla.CHUNK_ABSORBED
+        assert ws(h, 4, 16, 4, 4000, mla.CHUNK_UNABSORBED)[1] == mla.CHUNK_UNABSORBED
+        with pytest.raises(mla.MLAError) as e:          # forced absorbed on ragged chunks
+            ws(h, 4, 15, 4, 4000, mla.CHUNK_ABSORBED)
+        assert e.value.status == 1
+        with pytest.raises(mla.MLAError) as e:          # fewer key rows than chunk tokens
+            ws(h, 1, 16, 16, 15)
+        assert e.value.status == 1
+        # regions: the absorbed form has q~ and no k^C; the unabsorbed form's k^C spans every key row
+        off = mla.mla_prefill_chunk_offset
+        assert off(h, 4, 16, 4, 4000, mla.CHUNK_ABSORBED, mla.BUF_QABS) >= 0
+        with pytest.raises(mla.MLAError):
+            off(h, 4, 16, 4, 4000, mla.CHUNK_ABSORBED, mla.BUF_KC)
+        with pytest.raises(mla.MLAError):
+            off(h, 4, 15, 4, 4000, mla.CHUNK_AUTO, mla.BUF_QABS)
+        kc = off(h, 4, 15, 4, 4000, mla.CHUNK_AUTO, mla.BUF_KC)
+        vc = off(h, 4, 15, 4, 4000, mla.CHUNK_AUTO, mla.BUF_VC)
+        assert vc - kc >= 4000 * d.n_h * d.d_h * 2
+        assert ws(h, 4, 15, 4, 4000)[0] >= vc + 4000 * d.n_h * d.d_h * 2
+        A = 1 << 20
+        call = mla.mla_prefill_chunk
+        with pytest.raises(mla.MLAError) as e:          # capacity below the key rows
+            call(h, A, 2, A, 8, 4, A, 100, A, 99, mla.CHUNK_AUTO, A, A, 1 << 40, stream=0)
+        assert e.value.status == 1
+        with pytest.raises(mla.MLAError) as e:          # misaligned cu_kv
+            call(h, A, 2, A, 8, 4, A + 8, 100, A, 100, mla.CHUNK_AUTO, A, A, 1 << 40, stream=0)
+        assert e.value.status == 2
+        with pytest.raises(mla.MLAError) as e:          # workspace too small
+            call(h, A, 2, A, 8, 4, A, 100, A, 100, mla.CHUNK_AUTO, A, A, 1024, stream=0)
+        assert e.value.status == 4
+        with pytest.raises(mla.MLAError) as e:          # no weights given yet
+            call(h, A, 2, A, 8, 4, A, 100, A, 100, mla.CHUNK_AUTO, A, A, 1 << 40, stream=0)
+        assert e.value.status == 8
+        with pytest.raises(mla.MLAError) as e:          # unknown form
+            call(h, A, 2, A, 8, 4, A, 100, A, 100, 7, A, A, 1 << 40, stream=0)
+        assert e.value.status == 1
+    finally:
+        mla.mla_destroy(h)
+
+
+def test_option_setters_validate_on_the_host():
+    h = mla.mla_create(synth.V3, mla.MLA_BF16)
+    A = 1 << 20
+    try:
+        mla.mla_set_rmsnorm(h, A, A + 1024, 1e-6)
+        mla.mla_set_rmsnorm(h, None, None, 1e-6)            # off again
+        for args, status in (((A, None, 1e-6), 1), ((A, A, -1.0), 1), ((A + 8, A, 1e-6), 2)):
+            with pytest.raises(mla.MLAError) as e:
+                mla.mla_set_rmsnorm(h, *args)
+            assert e.value.status == status
+        mla.mla_set_yarn(h, 40.0, 1.0, 32.0, 4096.0)
+        mla.mla_set_yarn(h, 1.0)                             # plain RoPE again
+        for args in ((0.5,), (40.0, 32.0, 1.0), (40.0, 1.0, 32.0, 0.0)):
+            with pytest.raises(mla.MLAError) as e:
+                mla.mla_set_yarn(h, *args)
+            assert e.value.status == 1
+    finally:
+        mla.mla_destroy(h)

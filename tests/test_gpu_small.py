@@ -97,6 +97,7 @@ def test_tiny_cache_append_fp32_scattered_slots():
 # BF16 at the DeepSeek-V3 sizes, small batches with ragged tails
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("tq,lens", [(1, [1, 63, 64, 65, 129, 1000, 4097]), (2, [2, 63, 64, 65, 129, 1000, 4097]),
+                                     (1, [127, 128, 256, 257, 383, 2]), (2, [128, 129, 255, 256, 2, 3]),
                                      (1, [1, 40, 100]), (2, [33, 2, 97])])
 def test_v3_attn_core_bf16_ragged(v3_module, tq, lens):
     # the last two cases hold fewer key tiles than there are CTA pairs
@@ -110,6 +111,28 @@ def test_v3_attn_core_bf16_ragged(v3_module, tq, lens):
     lat_ref, lse_ref = orc.attn_decode_latent(q_abs, q_rope, cache, cu, tq, dims)
     o_lat, lse = v3_module.attn_decode_latent(dev(q_abs, "bf16"), dev(q_rope, "bf16"), B, tq, dev_i64(cu),
                                               dev(cache, "bf16"))
+    _status_ok(v3_module)
+    assert rel(host(o_lat), lat_ref) <= TOL["bf16"]
+    assert rel(host(lse), lse_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("tq", [1, 2])
+def test_v3_attn_core_rows_past_the_last_sequence_are_never_read(v3_module, tq):
+    # the cache holds NaN in every row after the last sequence; the last key tile of that sequence
+    # reaches into them, and nothing of them may reach the outputs
+    dims = synth.V3
+    lens = np.array([200, 77])
+    cu = synth.cu_seqlens(lens)
+    B, T = len(lens), len(lens) * tq
+    total = int(cu[-1])
+    cache = synth.latent_cache(dims, total, seed=80 + tq, dtype="bf16")
+    q_abs = synth.normal(81, 20, (T, dims.n_h, dims.d_c), std=0.5, dtype="bf16")
+    q_rope = synth.normal(81, 21, (T, dims.n_h, dims.d_r), std=1.0, dtype="bf16")
+    lat_ref, lse_ref = orc.attn_decode_latent(q_abs, q_rope, cache, cu, tq, dims)
+    padded = np.full((total + 300, dims.row), np.nan, dtype=np.float32)
+    padded[:total] = cache
+    o_lat, lse = v3_module.attn_decode_latent(dev(q_abs, "bf16"), dev(q_rope, "bf16"), B, tq, dev_i64(cu),
+                                              dev(padded, "bf16"))
     _status_ok(v3_module)
     assert rel(host(o_lat), lat_ref) <= TOL["bf16"]
     assert rel(host(lse), lse_ref) <= TOL["bf16"]
