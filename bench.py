@@ -477,6 +477,117 @@ def tiny_prefill_leg(dev, timed):
             "latency_us": round(ms * 1e3, 2), "note": "latency-bound by construction (2080 causal pairs)"}
 
 
+def next_rows_leg(args, W, dev, rank, world, flush, timed, peaks, peak_src):
+    """The rows built after the hot path, each timed on its own:
+    - chunked prefill, unabsorbed form: one sequence, a 4096-token chunk after a 28672-row cached
+      prefix (the 32K prefill shape taken in chunks);
+    - chunked prefill, absorbed form: 16 sequences, 4-token chunks after 4092 cached rows each;
+    - the decode_b16_l4096 step with RMSNorm and YaRN (s = 40) on, next to the same step without."""
+    import torch
+    from mla_latent_kv_31_b200 import mla
+    dims = synth.V3
+    out = {}
+    m = mla.MLA(dims, W, mla.MLA_BF16, device=dev.index)
+    h = m.handle
+    sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    hd = dims.n_h * dims.d_h
+
+    def chunk_case(name, kv_lens, q_lens, form):
+        B = len(kv_lens)
+        cu_kv, cu_q = synth.cu_seqlens(kv_lens), synth.cu_seqlens(q_lens)
+        tkv, tq_tot, mq = int(cu_kv[-1]), int(cu_q[-1]), int(max(q_lens))
+        cache = synth.latent_cache_torch(dims, tkv, seed=rank, device=dev)
+        hid = synth.normal_torch(rank, synth.TID_H, (tq_tot, dims.d), device=dev)
+        cq_d, ck_d = torch.from_numpy(cu_q).to(dev), torch.from_numpy(cu_kv).to(dev)
+        u = torch.empty(tq_tot, dims.d, dtype=torch.bfloat16, device=dev)
+        n, chosen = mla.mla_prefill_chunk_workspace(h, B, tq_tot, mq, tkv, form)
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+
+        def call():
+            mla.mla_prefill_chunk(h, hid, B, cq_d, tq_tot, mq, ck_d, tkv, cache, tkv, form, u, ws, n, device=dev.index)
+
+        l0 = mla.mla_kernel_launches()
+        call()
+        launches = mla.mla_kernel_launches() - l0
+        torch.cuda.synchronize()
+        st = mla.mla_sync_status(h, device=dev.index)
+        if st != 0:
+            raise RuntimeError(f"device check failed in {name}: {mla.mla_status_string(st)}")
+        ms = max_over_ranks([timed(call, 10 if chosen == mla.CHUNK_UNABSORBED else 50, 3)], dev)[0]
+        pre = [int(k) - int(q) for k, q in zip(kv_lens, q_lens)]
+        # attention: every chunk token against its visible rows; projections of the chunk tokens
+        vis = sum(sum(p + i + 1 for i in range(int(q))) for p, q in zip(pre, q_lens))
+        proj_tok = 2 * tq_tot * (dims.d * (dims.d_c + dims.d_r) + dims.d * dims.d_cq +
+                                 dims.d_cq * (hd + dims.n_h * dims.d_r) + hd * dims.d)
+        if chosen == mla.CHUNK_UNABSORBED:
+            flops = vis * dims.n_h * 2 * (dims.d_h + dims.d_r + dims.d_h) + proj_tok + 2 * tkv * dims.d_c * 2 * hd
+            form_name = "unabsorbed: k^C / v^C of every key row, then causal attention"
+        else:
+            flops = vis * CORE_FLOP_PER_ROW + proj_tok + 2 * tq_tot * 2 * hd * dims.d_c
+            form_name = "absorbed: q~ = W^UK^T q^C, the latent core with Tq = the chunk, W^UV"
+        tf = flops / (ms * 1e-3) / 1e12
+        return {"workload": name, "batch": B, "chunk_tokens": q_lens[0] if len(set(q_lens)) == 1 else list(q_lens),
+                "prefix_rows": pre[0] if len(set(pre)) == 1 else pre, "form": form_name,
+                "call": "mla_prefill_chunk, L2 flushed before each call", "ms": round(ms, 4),
+                "tokens_per_s": round(whole_job_rate(world, tq_tot, ms * 1e-3), 1), "flops_per_call": flops,
+                "tflops": round(world * tf, 1), "gpu_launches_per_call": int(launches),
+                "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": sus, "unit": "TFLOP/s",
+                             "frac": round(tf / sus, 4), "peak_source": f"{peak_src} sustained"}}
+
+    out["chunk_prefill_l32768_c4096"] = chunk_case("chunk_prefill_l32768_c4096", [32768], [4096], mla.CHUNK_AUTO)
+    ab = chunk_case("chunk_prefill_b16_l4096_c4", [4096] * 16, [4] * 16, mla.CHUNK_AUTO)
+    cb = 16 * 4096 * ROW_BYTES
+    ab["cache_gbs"] = round(whole_job_rate(world, cb, ab["ms"] * 1e-3) / 1e9, 1)
+    ab["note"] = f"cache {cb} B read once per chunk token by the latent core; {peak_src} HBM peak {hbm}"
+    out["chunk_prefill_b16_l4096_c4"] = ab
+    m.close()
+
+    # decode_b16_l4096 with and without RMSNorm + YaRN: the same step on two handles
+    wl = synth.WORKLOADS["decode_b16_l4096"]
+    lens, cu_np, rows, cache, h_np, pos_np, slots_np = decode_inputs(wl, rank, dev, on_device=True)
+    B, T = len(lens), len(lens) * wl.tq
+    h_dev = torch.from_numpy(h_np).to(dev, torch.bfloat16)
+    cu_dev, pos_dev, slots_dev = (torch.from_numpy(x).to(dev) for x in (cu_np, pos_np, slots_np))
+    u_dev = torch.empty(T, dims.d, dtype=torch.bfloat16, device=dev)
+    gains = {k: torch.from_numpy(v).to(dev, torch.bfloat16) for k, v in synth.gains(dims, seed=0).items()}
+    res = {}
+    for label, d_use, extra in (("plain", dims, {}), ("rmsnorm_yarn", synth.V3_YARN, gains)):
+        mm = mla.MLA(d_use, dict(W, **extra), mla.MLA_BF16, device=dev.index)
+        hh = mm.handle
+        n_app = mla.mla_workspace_size(hh, mla.OP_CACHE_APPEND, 0, 1, T)
+        n_dec = mla.mla_workspace_size(hh, mla.OP_DECODE, B, wl.tq, 0)
+        ws_app = torch.empty(max(n_app, 1024), dtype=torch.uint8, device=dev)
+        ws_dec = torch.empty(n_dec, dtype=torch.uint8, device=dev)
+
+        def step():
+            mla.mla_cache_append(hh, h_dev, pos_dev, slots_dev, T, cache, rows, ws_app, n_app, device=dev.index)
+            mla.mla_decode(hh, h_dev, B, wl.tq, cu_dev, cache, rows, u_dev, ws_dec, n_dec, device=dev.index)
+
+        l0 = mla.mla_kernel_launches()
+        step()
+        launches = mla.mla_kernel_launches() - l0
+        torch.cuda.synchronize()
+        if mla.mla_sync_status(hh, device=dev.index) != 0:
+            raise RuntimeError(f"device check failed in the {label} step")
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            step()
+        res[label] = (max_over_ranks([timed(g.replay, max(5, min(args.steps, 200)), 3)], dev)[0], int(launches))
+        del g
+        mm.close()
+    out["decode_b16_l4096_rmsnorm_yarn"] = {
+        "workload": "decode_b16_l4096 with RMSNorm (gains on c^Q, c^KV) and YaRN (s = 40, alpha = 1, beta = 32)",
+        "step": "mla_cache_append + mla_decode, CUDA-graph replay, L2 flushed",
+        "ms_per_step": round(res["rmsnorm_yarn"][0], 5), "ms_per_step_without": round(res["plain"][0], 5),
+        "overhead_ms": round(res["rmsnorm_yarn"][0] - res["plain"][0], 5),
+        "gpu_launches_per_step": res["rmsnorm_yarn"][1], "gpu_launches_per_step_without": res["plain"][1],
+        "note": "YaRN changes only the RoPE table and factor in the projection epilogues; RMSNorm adds one row-norm "
+                "kernel after W^DQ and one after the cache append"}
+    return out
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -589,6 +700,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             others[name] = decode_config_leg(args, m, synth.WORKLOADS[name], dev, rank, world, flush, timed, peaks,
                                              peak_src)
         others["tiny_prefill_fp32"] = tiny_prefill_leg(dev, timed)
+        others["next_rows"] = next_rows_leg(args, W, dev, rank, world, flush, timed, peaks, peak_src)
     prefill = (run_prefill(args, m, dev, rank, world, flush, timed, peaks, peak_src) if args.prefill_iters > 0
                else {"status": "skipped (--prefill-iters 0)"})
     st = mla.mla_sync_status(h, device=local_rank)

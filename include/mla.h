@@ -22,7 +22,8 @@
  *     the rotated k^R in columns [d_c, d_c + d_r). At the V3 sizes a row is 1152 bytes in bf16.
  *   - Sequences are packed and addressed by cu_seqlens: device int64 [B + 1], cu[0] = 0,
  *     non-decreasing; sequence b owns cache rows [cu[b], cu[b+1]). Positions are 0-based
- *     within a sequence. RoPE rotates interleaved pairs (2m, 2m+1) by pos * base^(-2m/d_r).
+ *     within a sequence. RoPE rotates interleaved pairs (2m, 2m+1) by pos * base^(-2m/d_r)
+ *     (or YaRN's frequencies, mla_set_yarn).
  *   - Every call is asynchronous on the given stream and returns a status; it never throws.
  *     Host-side validation (null pointers, sizes, alignment, workspace) runs before any launch:
  *     on failure nothing is launched and nothing is written. Device-side checks (cu_seqlens
@@ -32,7 +33,8 @@
  *   - Calls make the handle's device current while they run and restore the calling thread's
  *     current device before they return.
  *   - A handle may be used from several streams for different calls as long as calls that
- *     share a workspace or output buffer are ordered by the caller.
+ *     share a workspace or output buffer are ordered by the caller (they also share the handle's
+ *     error word, which then reports the union of their device-side errors).
  */
 #ifndef MLA_H
 #define MLA_H
@@ -294,7 +296,8 @@ mla_status_t mla_kernel_time_ms(int which, float *ms);
 
 /* Test hook for the bounded device-side waits (no counterpart on the pages). Arms the next launch
  * of the decode latent core in this process (mla_attn_decode_latent or mla_decode, any handle) so
- * that its first cluster waits for a cache tile that is never loaded, with a 20 ms wait limit
+ * that the cluster holding the first cache tile waits for a box of it that is never loaded (the
+ * query's first box), with a 20 ms wait limit
  * instead of 1 s. Every role of that launch gives up after its limit and returns; the launch
  * writes garbage outputs, and mla_sync_status() reports MLA_ERR_TIMEOUT. Nothing faults or hangs,
  * and later calls run normally. Not thread-safe: arm it only while no other thread launches. */

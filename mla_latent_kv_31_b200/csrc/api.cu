@@ -453,11 +453,14 @@ mla_status_t mla_attn_decode_latent(mla_handle_t* h, const void* q_abs, const vo
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   char* w = (char*)ws;
+  if (tc_dims(h)) {
+    // the device checks ride in the core's plan launch
+    MLA_TRY(mla::tc_core_prepare(cu_seqlens, B, Tq, capacity, nullptr, w + L.tc_off, h->num_sms, h->d_err, st));
+    return cuda_status(mla::tc_core_run(q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, true, lse,
+                                        w + L.tc_off, h->num_sms, h->d_err, st));
+  }
   MLA_TRY(mla::check_and_positions(cu_seqlens, B, Tq, B * Tq, capacity, 0, (int64_t*)(w + L.pos_off), h->d_err,
                                    st));
-  if (tc_dims(h))
-    return cuda_status(mla::tc_latent_core_impl(q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, true,
-                                           lse, w + L.tc_off, h->num_sms, h->d_err, st));
   return simt_latent_core(h, q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, true, lse, st);
 }
 
@@ -567,7 +570,8 @@ mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq,
   cudaStream_t st = (cudaStream_t)stream;
   char* w = (char*)ws;
   int64_t* pos = (int64_t*)(w + L.pos_off);
-  MLA_TRY(mla::check_and_positions(cu_seqlens, B, Tq, B * Tq, capacity, 0, pos, h->d_err, st));
+  // the tensor-core path runs the device checks and writes the positions in its core's plan launch
+  if (!tc_dims(h)) MLA_TRY(mla::check_and_positions(cu_seqlens, B, Tq, B * Tq, capacity, 0, pos, h->d_err, st));
   return decode_steps(h, h_q, B, Tq, cu_seqlens, pos, cache, capacity, u_out, w, L, st);
 }
 

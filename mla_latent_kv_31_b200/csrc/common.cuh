@@ -129,4 +129,32 @@ __device__ __forceinline__ int64_t seq_of_token(const int64_t* cu, int64_t B, in
   return lo;
 }
 
+// Device-side checks of cu_seqlens by one block (strided loops), and per-token positions when
+// pos_out != nullptr: decode (tq > 0): pos = len_b - tq + k for token k of sequence b; prefill
+// (tq == 0): pos = t - cu[b]. Offending sequences set bits of the error word.
+__device__ inline void check_seqs_and_positions(const int64_t* cu, int64_t B, int32_t tq, int64_t total,
+                                                int64_t capacity, int64_t max_seqlen, int64_t* pos_out,
+                                                uint32_t* err) {
+  for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+    const int64_t lo = cu[b], hi = cu[b + 1];
+    if (b == 0 && lo != 0) flag_error(err, DEVERR_CU_SEQLENS);
+    if (hi < lo || hi > capacity) flag_error(err, DEVERR_CU_SEQLENS);
+    if (tq > 0 && hi - lo < tq) flag_error(err, DEVERR_SHORT_SEQ);
+    if (tq == 0 && max_seqlen > 0 && hi - lo > max_seqlen) flag_error(err, DEVERR_SEQ_TOO_LONG);
+  }
+  if (threadIdx.x == 0 && tq == 0 && total >= 0 && cu[B] != total) flag_error(err, DEVERR_TOTAL);
+  if (!pos_out) return;
+  if (tq > 0) {
+    for (int64_t t = threadIdx.x; t < B * tq; t += blockDim.x) {
+      const int64_t b = t / tq;
+      pos_out[t] = (cu[b + 1] - cu[b]) - tq + (t % tq);
+    }
+  } else {
+    for (int64_t t = threadIdx.x; t < total; t += blockDim.x) {
+      const int64_t b = seq_of_token(cu, B, t);
+      pos_out[t] = t - cu[b];
+    }
+  }
+}
+
 }  // namespace mla

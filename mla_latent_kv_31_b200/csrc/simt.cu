@@ -168,27 +168,7 @@ __global__ void __launch_bounds__(ATT_THREADS) simt_attention_kernel(SimtAttnArg
 __global__ void check_positions_kernel(const int64_t* cu, int64_t B, int32_t tq, int64_t total,
                                        int64_t capacity, int64_t max_seqlen, int64_t* pos_out,
                                        uint32_t* err) {
-  // One block: sequence checks by a strided loop, then per-token positions.
-  for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
-    const int64_t lo = cu[b], hi = cu[b + 1];
-    if (b == 0 && lo != 0) flag_error(err, DEVERR_CU_SEQLENS);
-    if (hi < lo || hi > capacity) flag_error(err, DEVERR_CU_SEQLENS);
-    if (tq > 0 && hi - lo < tq) flag_error(err, DEVERR_SHORT_SEQ);
-    if (tq == 0 && max_seqlen > 0 && hi - lo > max_seqlen) flag_error(err, DEVERR_SEQ_TOO_LONG);
-  }
-  if (threadIdx.x == 0 && tq == 0 && total >= 0 && cu[B] != total) flag_error(err, DEVERR_TOTAL);
-  if (!pos_out) return;
-  if (tq > 0) {
-    for (int64_t t = threadIdx.x; t < B * tq; t += blockDim.x) {
-      const int64_t b = t / tq;
-      pos_out[t] = (cu[b + 1] - cu[b]) - tq + (t % tq);
-    }
-  } else {
-    for (int64_t t = threadIdx.x; t < total; t += blockDim.x) {
-      const int64_t b = seq_of_token(cu, B, t);
-      pos_out[t] = t - cu[b];
-    }
-  }
+  check_seqs_and_positions(cu, B, tq, total, capacity, max_seqlen, pos_out, err);
 }
 
 __global__ void check_chunk_kernel(const int64_t* cu_q, const int64_t* cu_kv, int64_t B, int64_t total_q,
@@ -205,9 +185,10 @@ __global__ void check_chunk_kernel(const int64_t* cu_q, const int64_t* cu_kv, in
   if (threadIdx.x == 0 && (cu_q[B] != total_q || cu_kv[B] != total_kv)) flag_error(err, DEVERR_TOTAL);
   for (int64_t t = threadIdx.x; t < total_q; t += blockDim.x) {
     const int64_t b = seq_of_token(cu_q, B, t);
-    const int64_t pos = (cu_kv[b + 1] - cu_kv[b]) - (cu_q[b + 1] - cu_q[b]) + (t - cu_q[b]);
+    const int64_t kb = cu_kv[b], qb = cu_q[b];
+    const int64_t pos = (cu_kv[b + 1] - kb) - (cu_q[b + 1] - qb) + (t - qb);
     pos_out[t] = pos;
-    slot_out[t] = pos >= 0 ? cu_kv[b] + pos : -1;   // a negative row is skipped by the writers
+    slot_out[t] = pos >= 0 ? kb + pos : -1;   // a negative row is skipped by the writers
   }
 }
 

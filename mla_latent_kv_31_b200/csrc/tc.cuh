@@ -23,14 +23,19 @@ cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const L
                             cudaStream_t st);
 
 // Test hook: the next latent-core launch in this process waits on a barrier that nothing signals
-// (the first cluster's first cache box is never loaded), with a 20 ms wait limit, so that its
+// (the first box of the cluster holding tile 0 is never loaded), with a 20 ms wait limit, so that its
 // bounded waits give up and the launch reports a timeout.
 void tc_latent_core_arm_stall();
 
-// The split-KV tcgen05 latent core (q~, q^R -> o^lat, lse); scratch of tc_core_scratch_bytes().
-cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
-                                const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse,
-                                void* scratch, int num_sms, uint32_t* err, cudaStream_t st);
+// The split-KV tcgen05 latent core (q~, q^R -> o^lat, lse) on scratch of tc_core_scratch_bytes(), in two
+// launches: tc_core_prepare (one block: the device checks of cu_seqlens, the decode positions when pos is
+// not null, and the plan of the clusters' tile ranges and partial slots), then tc_core_run (the core and
+// the log-sum-exp merge of the partials) with the same B, tq, scratch and num_sms.
+cudaError_t tc_core_prepare(const int64_t* cu, int64_t B, int32_t tq, int64_t capacity, int64_t* pos, void* scratch,
+                            int num_sms, uint32_t* err, cudaStream_t st);
+cudaError_t tc_core_run(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
+                        const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse, void* scratch,
+                        int num_sms, uint32_t* err, cudaStream_t st);
 
 cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& lo, const void* h_q, int64_t B,
                       int32_t tq, const int64_t* cu, const int64_t* pos, const void* cache, int64_t capacity, void* u_out,

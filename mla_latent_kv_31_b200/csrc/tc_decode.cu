@@ -16,13 +16,16 @@
 //   * the score CTA (rank 0): q~ in TMEM (256 columns of bf16 pairs, the A operand), two
 //     128 x 128 fp32 score buffers; QK^T over the 576 cache columns (32 TS MMAs over the latent
 //     part, 4 SS MMAs over k^R with q^R in shared memory), N = 128 keys; the softmax (lazy
-//     rescale of the running max); P (bf16) plus per-head rescale factors go to the value CTA as
-//     one bulk shared-to-shared copy per tile;
+//     rescale of the running max); the softmax warps store P (bf16) and the per-head rescale
+//     factors straight into the value CTA's shared memory (st.async, counted on its mbarrier);
 //   * the value CTA (rank 1): O in all 512 TMEM columns; per tile 16 SS MMAs (N = 256 latent
 //     columns, K = 16 keys) read P and the latent columns of the cache tile, which this CTA loads
 //     itself (the second read of the tile hits L2); it rescales O when the score CTA's running max
 //     moved, and writes the piece's normalised partial o^lat at its end.
 // Each producer issues its TMA loads from four lanes: one issuing thread streams only about 40 GB/s.
+// The score CTA's ring holds 12 boxes (192 KB): at the 2-3 us of HBM latency under load, the bytes
+// in flight per SM set its streaming rate (Little's law), so the ring takes all the shared memory
+// the P hand-off no longer needs.
 //
 // Queries. A piece's q~ (8 boxes of [128 heads x 64 columns]) and q^R (1 box) enter the score CTA's
 // ring ahead of its first tile, like a tile's boxes; the softmax warps copy q~ into TMEM and q^R
@@ -30,13 +33,14 @@
 //
 // Outputs. Every piece writes a partial: O = sum_j 2^((s_j - m) c) c_j unnormalised, its reference
 // m in natural units and its lse, O in a head-interleaved layout [token k][slot][column/4][head][4]
-// fp32, so that the 32 heads of a warp store 512 contiguous bytes per instruction. The merge pass
+// bf16 (fp32 accumulation, one rounding before the merge), so that the 32 heads of a warp store 256
+// contiguous bytes per instruction. The merge pass
 // weights each partial by e^{m_s - lse} with lse = log sum_s e^{lse_s} and writes o^lat [T][H][DC]
 // and lse [T][H] (a one-piece sequence is a weighted copy).
 // The score CTA's tensor work per tile is 36 MMAs at N = 128 (about 2300 cycles), the value CTA's
 // 16 MMAs at N = 256 (about 2050), so the two stay busy together. Data flows one way (P), so the
-// two CTAs pipeline freely: two P buffers on the value side, two staging buffers on the score
-// side.
+// two CTAs pipeline freely: two P buffers on the value side; the score side writes P of tile j
+// once the value CTA's P.V of tile j - 2 (the same buffer) is done.
 //
 // Every wait is bounded (a timeout sets the error word and the role returns).
 #include <cuda_bf16.h>
@@ -57,14 +61,16 @@ constexpr int kThreads = 384;
 constexpr int kMaxPairs = 74;
 constexpr float kRescaleLog2 = 8.f;            // keep the running max until it grows by 2^8
 constexpr int kIssuers = 4;                    // TMA issuing lanes per producer warp
+constexpr int kStartCost = 3;                  // a sequence piece's fixed cost, in half tiles (plan)
 
 // score CTA: ring of [128 keys x 64 columns] boxes (8 latent + 1 k^R per tile)
 constexpr uint32_t BOX = NK * 128;             // 16 KB, 128-byte swizzle, K-major rows of 64 bf16
 constexpr int S_BOXES = 9;
-constexpr int S_RING = 8;
+constexpr int S_RING = 12;
 constexpr uint32_t P_BYTES = H * NK * 2;       // P [128 heads x 128 keys] bf16, K-major SW128: 2 blocks of 16 KB
 constexpr uint32_t HDR_BYTES = 2 * H * 4;      // alpha[128] (+ reserve)
-constexpr uint32_t PMSG = P_BYTES + HDR_BYTES; // one P message: 33 KB
+constexpr uint32_t PMSG = P_BYTES + HDR_BYTES; // one P buffer: 33 KB
+constexpr uint32_t PMSG_TX = P_BYTES + H * 4;  // the bytes stored into it per tile: P and alpha
 constexpr uint32_t QR_BYTES = H * DR * 2;      // q^R [128 x 64] bf16, K-major SW128
 // value CTA: ring of [64 keys x 256 columns] groups (4 boxes of [64 keys x 64 columns])
 constexpr uint32_t VBOX = 64 * 128;            // 8 KB
@@ -77,15 +83,13 @@ constexpr uint32_t OFF_BAR = 0;
 constexpr uint32_t OFF_RED = 512;              // score CTA: per-head maxima / sums swapped between halves
 constexpr uint32_t S_OFF_RING = 4096;
 constexpr uint32_t S_OFF_QR = S_OFF_RING + S_RING * BOX;
-constexpr uint32_t S_OFF_STG = S_OFF_QR + QR_BYTES;
-constexpr uint32_t S_END = S_OFF_STG + 2 * PMSG;
+constexpr uint32_t S_END = S_OFF_QR + QR_BYTES;
 constexpr uint32_t V_OFF_PBUF = 4096;
 constexpr uint32_t V_OFF_RING = V_OFF_PBUF + 2 * PMSG;
 constexpr uint32_t V_END = V_OFF_RING + V_RING * VGRP;
 constexpr uint32_t SMEM_BYTES = (S_END > V_END ? S_END : V_END) + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(S_OFF_RING % 1024 == 0 && S_OFF_QR % 1024 == 0 && S_OFF_STG % 1024 == 0 && PMSG % 1024 == 0 &&
-                  V_OFF_RING % 1024 == 0,
+static_assert(S_OFF_RING % 1024 == 0 && S_OFF_QR % 1024 == 0 && PMSG % 1024 == 0 && V_OFF_RING % 1024 == 0,
               "swizzle atom alignment");
 static_assert(OFF_RED + 3 * 2 * H * 4 <= S_OFF_RING, "reduction buffer");
 static_assert(S_RING % kIssuers == 0 && V_RING % kIssuers == 0 && (kIssuers & (kIssuers - 1)) == 0,
@@ -100,12 +104,10 @@ enum : int {
   B_SCE = B_SCF + 2,                  // [2] scores read (256 softmax threads)
   B_QFULL = B_SCE + 2,                // q^R of a piece copied into its tile (256)
   B_QEMPTY = B_QFULL + 1,             // last QK^T of a piece done (q~ TMEM and q^R tile free)
-  B_PSTG = B_QEMPTY + 1,              // [2] P message staged (256)
-  B_STGF = B_PSTG + 2,                // [2] staging buffer free again (remote arrival of the value CTA)
-  B_TMAX = B_STGF + 2,                // [4] the two softmax warps of a TMEM lane quarter (64)
+  B_TMAX = B_QEMPTY + 1,              // [4] the two softmax warps of a TMEM lane quarter (64)
   B_GFULL = B_TMAX + 4,               // [V_RING] value CTA ring
   B_GEMPTY = B_GFULL + V_RING,        // [V_RING]
-  B_PFULL = B_GEMPTY + V_RING,        // [2] P message landed (bytes)
+  B_PFULL = B_GEMPTY + V_RING,        // [2] P and alpha of a tile landed (bytes stored by the score CTA)
   B_OREADY = B_PFULL + 2,             // [2] O rescaled for the tile / nothing to rescale (128)
   B_OFREE = B_OREADY + 2,             // O read out by the piece epilogue (256: both column halves)
   B_ODONE = B_OFREE + 1,              // the last P.V of a piece done (one phase per piece)
@@ -123,12 +125,12 @@ struct CoreParams {
   const int32_t* slot_base;     // [B+1]: first partial slot of each sequence
   const int4* pinfo;            // [pairs]: tile range [x, y), first sequence z, its partial slot w
   int32_t B, tq, pairs, s_max;
-  float* part_o;      // [tq][s_max][DC/4][H][4], unnormalised
+  uint2* part_o;      // [tq][s_max][DC/4][H] x 4 bf16, unnormalised
   float* part_lse;    // [tq][s_max][H]
   float* part_m;      // [tq][s_max][H], the reference of part_o in natural units
   float scale_log2;   // log2(e) / sqrt(d_h + d_h^R)
   uint64_t wait_ns;   // bounded-wait limit
-  int32_t stall;      // test hook: the first cluster's score-side producer skips its first box
+  int32_t stall;      // test hook: the score-side producer of the cluster holding tile 0 skips its first box
   uint32_t* err;
 };
 
@@ -141,6 +143,16 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint64_t
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > limit) return false;
+  }
+}
+__device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, uint64_t limit) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
     if (globaltimer() - t0 > limit) return false;
   }
 }
@@ -176,26 +188,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t r = cluster_rank();
   const int k = blockIdx.y;                          // query token within the sequence window
   const int pair = blockIdx.x >> 1;
-  const int4 pi = p.pinfo[pair];
-  const int32_t t_begin = pi.x, t_end = pi.y;
   const uint64_t lim = p.wait_ns;
   // partial slot of this cluster's piece of sequence b: the first piece's comes with the plan; a
   // sequence that starts inside this cluster's range has this cluster as its first
-  auto piece_slot = [&](int b) -> int64_t { return b == pi.z ? (int64_t)pi.w : (int64_t)p.slot_base[b]; };
-
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
-      if (i == B_SCE || i == B_SCE + 1 || i == B_QFULL || i == B_PSTG || i == B_PSTG + 1) cnt = 256;
+      if (i == B_SCE || i == B_SCE + 1 || i == B_QFULL) cnt = 256;
       else if (i >= B_TMAX && i < B_TMAX + 4) cnt = 64;
       else if (i == B_OREADY || i == B_OREADY + 1) cnt = 128;
       else if (i == B_OFREE) cnt = 256;
       mbar_init(bar(i), cnt);
     }
     if (r == 1) {
-      // the P buffers' first phases: one arrival plus the bytes of one message
-      mbar_expect_tx(bar(B_PFULL), PMSG);
-      mbar_expect_tx(bar(B_PFULL + 1), PMSG);
+      // the P buffers' first phases: one arrival plus the bytes of one tile
+      mbar_expect_tx(bar(B_PFULL), PMSG_TX);
+      mbar_expect_tx(bar(B_PFULL + 1), PMSG_TX);
     }
     fence_mbar_init();
   }
@@ -214,10 +222,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int4 pi = p.pinfo[pair];
+  const int32_t t_begin = pi.x, t_end = pi.y;
+  auto piece_slot = [&](int b) -> int64_t { return b == pi.z ? (int64_t)pi.w : (int64_t)p.slot_base[b]; };
 
   SegWalk w;
   w.init_at(p.tile_start, p.B, t_begin, t_end, pi.z);
-  const int ntiles = t_end - t_begin;
   bool ok = true;
 
   if (r == 0) {
@@ -229,7 +239,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // [128 heads x 64 columns] and q^R in 1 box, then per tile the 8 latent boxes and the k^R box.
       if (lane < kIssuers) {
         int n = 0, last = -1;
-        const bool stall = p.stall && pair == 0 && k == 0;
+        const bool stall = p.stall && k == 0 && t_begin == 0 && t_end > 0;
         auto issue = [&](const CUtensorMap* map, int x, int y) -> bool {
           const int cur = n++;
           if ((cur & (kIssuers - 1)) != lane) return true;
@@ -256,7 +266,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           flag_error(p.err, DEVERR_TIMEOUT);
           // this lane's entries still in flight: the last S_RING / kIssuers it issued
           for (int i2 = max(lane, last - S_RING + 1); i2 <= last; ++i2)
-            if ((i2 & (kIssuers - 1)) == lane && !(p.stall && pair == 0 && k == 0 && i2 == 0))
+            if ((i2 & (kIssuers - 1)) == lane && !(stall && i2 == 0))
               wait_bar(bar(B_SFULL + i2 % S_RING), (i2 / S_RING) & 1, lim);
         }
       }
@@ -301,26 +311,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
       }
-    } else if (warp == 2) {
-      // ------------------------------------------------ sender: staged P message -> value CTA
-      if (lane == 0) {
-        const uint32_t pbuf_peer = map_peer(sbase + V_OFF_PBUF, 1);
-        const uint32_t pfull_peer = map_peer(bar(B_PFULL), 1);
-        int last = -1;
-        for (int j = 0; j < ntiles; ++j) {
-          const int b = j & 1;
-          if (!wait_bar(bar(B_PSTG + b), (j >> 1) & 1, lim) || !wait_bar(bar(B_PVD + b), ((j >> 1) & 1) ^ 1, lim)) {
-            ok = false;
-            break;
-          }
-          bulk_copy_to_peer(pbuf_peer + b * PMSG, sbase + S_OFF_STG + b * PMSG, PMSG, pfull_peer + 8 * b);
-          last = j;
-        }
-        // the value CTA acknowledges each message once its bytes have landed; wait for the last one
-        // so that no copy into its shared memory is in flight when the cluster exits
-        if (last >= 0) wait_bar(bar(B_STGF + (last & 1)), (last >> 1) & 1, lim);
-        if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
-      }
     } else if (warp >= 4) {
       // ------------------------------------------------ softmax: 8 warps, two per TMEM lane quarter
       // Half 0 (warps 4-7) takes keys [0, 64) of every tile, half 1 (warps 8-11) keys [64, 128),
@@ -333,6 +323,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       float* redbuf = reinterpret_cast<float*>(smem + OFF_RED);   // [3 slots][2 halves][128]
       const float c2 = p.scale_log2;
       const float thr_raw = kRescaleLog2 / c2;
+      const uint32_t pbuf_peer = map_peer(sbase + V_OFF_PBUF, 1);
+      const uint32_t pfull_peer = map_peer(bar(B_PFULL), 1);
       auto wait_u = [&](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, wait_bar(b, par, lim)) != 0; };
       int tph = 0;
       auto swap_half = [&](float x, int slot, float& y) -> bool {
@@ -461,16 +453,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c) pk[c] = 0u;
           }
-          // staging buffer sb: the value CTA has received the message of tile j - 2 from it
-          if (!wait_u(bar(B_STGF + sb), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
-          uint8_t* msg = smem + S_OFF_STG + sb * PMSG;
-          uint8_t* prow = msg + 16384 * half + i * 128;
+          // the value CTA's P buffer sb: its P.V of tile j - 2 is done; this half's 64 keys of row i
+          // go straight into it (the same 128-byte swizzle the MMA descriptor reads), alpha too
+          if (!wait_u(bar(B_PVD + sb), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+          const uint32_t pbuf = pbuf_peer + sb * PMSG, pfull = pfull_peer + 8 * sb;
+          const uint32_t prow = pbuf + 16384 * half + i * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(prow + ((c ^ (i & 7)) << 4)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-          float* hdr = reinterpret_cast<float*>(msg + P_BYTES);
-          if (half == 0) hdr[i] = first ? 1.f : alpha;
+            st_async_v4(prow + ((c ^ (i & 7)) << 4), make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]),
+                        pfull);
+          if (half == 0) st_async_b32(pbuf + P_BYTES + 4 * i, __float_as_uint(first ? 1.f : alpha), pfull);
           if (last) {
             // piece end: lse of the piece and the reference of its unnormalised partial
             float lp;
@@ -482,8 +474,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               p.part_m[row] = lt > 0.f ? m_ref * c2 * 0.69314718055994531f : -INFINITY;
             }
           }
-          fence_proxy_async_smem();
-          mbar_arrive(bar(B_PSTG + sb));
         }
         if (!ok) break;
         // the next piece's q^R goes in now, so that its first QK^T overlaps the value CTA's epilogue
@@ -500,6 +490,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // lanes 0-3 issue, lane l the group (N-half l & 1, key-half l >> 1) of every tile (ring slot l)
       if (lane < kIssuers) {
         int n = 0, last = -1;
+        // The first tile's groups wait for the first P message: at launch the score CTAs' q~ and
+        // first boxes then have the memory system to themselves, and these loads hit L2 behind them.
+        if (w.valid() && !wait_bar_cluster(bar(B_PFULL), 0, lim)) ok = false;
         for (SegWalk sw = w; ok && sw.valid(); sw.next()) {
           const int32_t ts_b = p.tile_start[sw.b];
           const int32_t row_base = (int32_t)p.cu[sw.b];
@@ -529,20 +522,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ------------------------------------------------ MMA issuer: O += P . C
       if (lane == 0) {
         constexpr uint32_t idesc = idesc_bf16(128, 256, 0, 1);
-        const uint32_t stgf_peer = map_peer(bar(B_STGF), 0);
         int j = 0, g = 0, n = 0;
         for (; ok && w.valid(); w.next(), ++g) {
           const int32_t send = w.seg_end();
           for (int32_t xt = w.x; xt < send; ++xt, ++j) {
             const int pb = j & 1;
             const bool first = xt == w.x;
-            if (!wait_bar(bar(B_PFULL + pb), (j >> 1) & 1, lim)) { ok = false; break; }
-            // re-arm the buffer's next phase, and let the score CTA reuse its staging buffer
-            mbar_expect_tx(bar(B_PFULL + pb), PMSG);
-            mbar_arrive_peer(stgf_peer + 8 * pb);
+            if (!wait_bar_cluster(bar(B_PFULL + pb), (j >> 1) & 1, lim)) { ok = false; break; }
+            // re-arm the buffer's next phase (tile j + 2: the score CTA writes it after this tile's P.V)
+            mbar_expect_tx(bar(B_PFULL + pb), PMSG_TX);
             if (!wait_bar(bar(B_OREADY + pb), (j >> 1) & 1, lim)) { ok = false; break; }
             if (first && !wait_bar(bar(B_OFREE), (g & 1) ^ 1, lim)) { ok = false; break; }
             tc_fence_after();
+            // P came in through the score CTA's generic stores: order them before the MMAs' reads
+            fence_proxy_async_smem();
             const uint32_t pmsg = sbase + V_OFF_PBUF + pb * PMSG;
             for (int s = 0; s < 4; ++s, ++n) {
               const int gi = n % V_RING;
@@ -581,7 +574,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       auto dump = [&](int b, int g) -> bool {
         if (!wait_u(bar(B_ODONE), g & 1)) return false;
         tc_fence_after();
-        float4* po = reinterpret_cast<float4*>(p.part_o) + ((int64_t)k * p.s_max + piece_slot(b)) * (DC / 4) * H + i;
+        uint2* po = p.part_o + ((int64_t)k * p.s_max + piece_slot(b)) * (DC / 4) * H + i;
 #pragma unroll 1
         for (int c = 256 * ehalf; c < 256 * ehalf + 256; c += 32) {
           uint32_t v[32];
@@ -589,8 +582,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            po[(c / 4 + e) * H] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                              __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+            po[(c / 4 + e) * H] = make_uint2(pack_bf16(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1])),
+                                             pack_bf16(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
         }
         tc_fence_before();
         mbar_arrive(bar(B_OFREE));
@@ -610,7 +603,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int32_t xt = w.x; xt < send; ++xt, ++j, n += 4) {
           const int pb = j & 1;
           const bool first = xt == w.x, last = xt == send - 1;
-          if (!wait_u(bar(B_PFULL + pb), (j >> 1) & 1)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, wait_bar_cluster(bar(B_PFULL + pb), (j >> 1) & 1, lim))) { ok = false; break; }
           const float* hdr = reinterpret_cast<const float*>(smem + V_OFF_PBUF + pb * PMSG + P_BYTES);
           const float alpha = hdr[i];
           if (__any_sync(0xffffffffu, !first && alpha != 1.f)) {
@@ -696,8 +689,12 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return res;
 }
 
+// The same block first runs the device checks of cu_seqlens and writes the decode positions
+// (len_b - tq + k), so that a decode step needs one small launch for both.
 __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B, int32_t pairs, int32_t* ts,
-                                                   int32_t* sb, int4* pinfo) {
+                                                   int32_t* sb, int4* pinfo, int32_t tq, int64_t capacity,
+                                                   int64_t* pos_out, uint32_t* err) {
+  check_seqs_and_positions(cu, B, tq, (int64_t)B * tq, capacity, 0, pos_out, err);
   __shared__ int32_t warp_tot[8];
   __shared__ int32_t total;
   const int tid = threadIdx.x;
@@ -714,11 +711,47 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
   if (tid == 0) ts[B] = total;
   __syncthreads();
   const int64_t NT = total;
-  const int64_t npairs = NT < pairs ? NT : pairs;   // every active pair holds >= 1 tile
-  auto pair_of = [&](int64_t x) -> int64_t { return ((x + 1) * npairs - 1) / NT; };
+  // Cost-aware ranges. Besides its tiles, a cluster pays once per sequence piece (the piece's q load
+  // and its partial write, about kStartCost / 2 tiles), so every sequence start weighs kStartCost
+  // half-tiles: in half-tile units sequence b starts at vs(b) = 2 ts[b] + kStartCost b and its tile
+  // x covers [vs(b) + kStartCost + 2 (x - ts[b]), +2). The clusters split [0, V) evenly; cluster
+  // pp's range begins at the first tile at or after half-unit pp V / pairs. A range can be empty.
+  const int64_t V = 2 * NT + kStartCost * (int64_t)B;
+  auto bound = [&](int pp) -> int32_t {
+    const int64_t v = (int64_t)pp * V / pairs;
+    int b0 = 0, b1 = B;                       // the last b in [0, B] with vs(b) <= v
+    while (b0 < b1) {
+      const int mid = (b0 + b1 + 1) >> 1;
+      if (2 * (int64_t)ts[mid] + kStartCost * (int64_t)mid <= v) b0 = mid; else b1 = mid - 1;
+    }
+    if (b0 == B) return ts[B];
+    const int64_t off = v - (2 * (int64_t)ts[b0] + kStartCost * (int64_t)b0) - kStartCost;
+    const int64_t x = ts[b0] + (off <= 0 ? 0 : (off + 1) / 2);
+    return (int32_t)min(x, (int64_t)ts[b0 + 1]);
+  };
+  // the cluster owning tile x: the last pp with bound(pp) <= x (empty clusters never win a tie)
+  auto pair_of = [&](int32_t x) -> int {
+    int p0 = 0, p1 = pairs - 1;
+    while (p0 < p1) {
+      const int mid = (p0 + p1 + 1) >> 1;
+      if (bound(mid) <= x) p0 = mid; else p1 = mid - 1;
+    }
+    return p0;
+  };
+  // rank of each cluster among the clusters with a non-empty range
+  __shared__ int32_t arank[kMaxPairs + 1];
+  if (tid == 0) {
+    int32_t r = 0;
+    for (int pp = 0; pp < pairs; ++pp) {
+      arank[pp] = r;
+      if (bound(pp + 1) > bound(pp)) ++r;
+    }
+    arank[pairs] = r;
+  }
+  __syncthreads();
   auto nseg = [&](int b) -> int32_t {
     const int32_t a = ts[b], e = ts[b + 1];
-    return e > a ? (int32_t)(pair_of(e - 1) - pair_of(a) + 1) : 0;
+    return e > a ? arank[pair_of(e - 1)] - arank[pair_of(a)] + 1 : 0;
   };
   acc = 0;
   for (int b = lo; b < hi; ++b) acc += nseg(b);
@@ -729,18 +762,19 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
   // per cluster: its tile range, the sequence of its first tile and that piece's partial slot
   for (int pp = tid; pp < pairs; pp += blockDim.x) {
     int4 v = make_int4(0, 0, 0, 0);
-    if (pp < npairs) {
-      v.x = (int32_t)((int64_t)pp * NT / npairs);
-      v.y = (int32_t)((int64_t)(pp + 1) * NT / npairs);
-      int lo2 = 0, hi2 = B - 1;               // the last b with ts[b] <= v.x
+    const int32_t x0 = bound(pp), x1 = bound(pp + 1);
+    if (x1 > x0) {
+      v.x = x0;
+      v.y = x1;
+      int lo2 = 0, hi2 = B - 1;               // the last b with ts[b] <= x0
       while (lo2 < hi2) {
         const int mid = (lo2 + hi2 + 1) >> 1;
-        if (ts[mid] <= v.x) lo2 = mid; else hi2 = mid - 1;
+        if (ts[mid] <= x0) lo2 = mid; else hi2 = mid - 1;
       }
       // the first sequence with tiles: skip empty sequences that share the start
-      while (lo2 < B - 1 && ts[lo2 + 1] <= v.x) ++lo2;
+      while (lo2 < B - 1 && ts[lo2 + 1] <= x0) ++lo2;
       v.z = lo2;
-      v.w = sb[lo2] + (int32_t)(pp - pair_of(ts[lo2]));
+      v.w = sb[lo2] + arank[pp] - arank[pair_of(ts[lo2])];
     }
     pinfo[pp] = v;
   }
@@ -755,7 +789,7 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
 constexpr int kCombHeads = 32, kCombCols = 128;
 template <bool OUT_F32>
 __global__ void __launch_bounds__(256) combine_kernel(const int32_t* sb, int32_t tq, int32_t s_max,
-                                                      const float* part_o, const float* part_lse,
+                                                      const uint2* part_o, const float* part_lse,
                                                       const float* part_m, void* o_lat, float* lse) {
   __shared__ float wts[kMaxPairs][kCombHeads];
   __shared__ float tile[kCombHeads][kCombCols + 4];
@@ -784,14 +818,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* sb, int32_t
   float4 acc[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float4* src = reinterpret_cast<const float4*>(part_o) + (c0 / 4 + 4 * grp) * H + h0 + lane;
+  const uint2* src = part_o + (c0 / 4 + 4 * grp) * H + h0 + lane;
   for (int sl = 0; sl < ns; ++sl) {
     const float wgt = wts[sl][lane];
-    const float4* ps = src + (slot0 + sl) * (DC / 4) * H;
+    const uint2* ps = src + (slot0 + sl) * (DC / 4) * H;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float4 v = ps[q * H];
-      acc[q].x += wgt * v.x; acc[q].y += wgt * v.y; acc[q].z += wgt * v.z; acc[q].w += wgt * v.w;
+      const uint2 u = ps[q * H];
+      acc[q].x += wgt * bf16_lo(u.x); acc[q].y += wgt * bf16_hi(u.x);
+      acc[q].z += wgt * bf16_lo(u.y); acc[q].w += wgt * bf16_hi(u.y);
     }
   }
 #pragma unroll
@@ -826,7 +861,7 @@ struct CoreScratch {
   int4* pinfo;
   float* part_lse;
   float* part_m;
-  float* part_o;
+  uint2* part_o;
   int32_t s_max;
 };
 
@@ -844,7 +879,7 @@ CoreScratch carve(void* scratch, int64_t B, int32_t tq) {
   ptr += align1k((size_t)tq * c.s_max * H * 4);
   c.part_m = (float*)ptr;
   ptr += align1k((size_t)tq * c.s_max * H * 4);
-  c.part_o = (float*)ptr;
+  c.part_o = (uint2*)ptr;
   return c;
 }
 
@@ -863,7 +898,7 @@ cudaError_t launch_core(const CoreParams& p, dim3 grid, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// Test hook state (mla_test_stall_latent_core): consumed by the next launch.
+// Test hook state (mla_test_arm_stall): consumed by the next launch.
 int g_stall_next = 0;
 
 }  // namespace
@@ -874,24 +909,37 @@ size_t tc_core_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq) {
   (void)d;
   const int64_t s_max = pairs_cap(tq) + B;
   return 2 * align1k((B + 1) * 4) + align1k(kMaxPairs * sizeof(int4)) + 2 * align1k((size_t)tq * s_max * H * 4) +
-         (size_t)tq * s_max * H * DC * 4;
+         (size_t)tq * s_max * H * DC * 2;
 }
 
-cudaError_t tc_latent_core_impl(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
-                                const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse,
-                                void* scratch, int num_sms, uint32_t* err, cudaStream_t st) {
+namespace {
+int32_t core_pairs(int32_t tq, int num_sms) {
+  int pairs = num_sms / (2 * tq);
+  pairs = pairs < pairs_cap(tq) ? pairs : pairs_cap(tq);
+  return pairs < 1 ? 1 : pairs;
+}
+}  // namespace
+
+cudaError_t tc_core_prepare(const int64_t* cu, int64_t B, int32_t tq, int64_t capacity, int64_t* pos, void* scratch,
+                            int num_sms, uint32_t* err, cudaStream_t st) {
+  if (B <= 0) return cudaSuccess;
+  if (B > (int64_t)1 << 20 || tq < 1 || tq > kMaxPairs) return cudaErrorInvalidValue;
+  CoreScratch c = carve(scratch, B, tq);
+  plan_kernel<<<1, 256, 0, st>>>(cu, (int32_t)B, core_pairs(tq, num_sms), c.ts, c.sb, c.pinfo, tq, capacity, pos, err);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t tc_core_run(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
+                        const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse, void* scratch,
+                        int num_sms, uint32_t* err, cudaStream_t st) {
   if (B <= 0) return cudaSuccess;
   if (B > (int64_t)1 << 20 || tq < 1 || tq > kMaxPairs || capacity > INT32_MAX || B * tq * H > INT32_MAX)
     return cudaErrorInvalidValue;
   const int64_t T = B * tq;
   CoreScratch c = carve(scratch, B, tq);
-  int pairs = num_sms / (2 * tq);
-  pairs = pairs < pairs_cap(tq) ? pairs : pairs_cap(tq);
-  pairs = pairs < 1 ? 1 : pairs;
-  plan_kernel<<<1, 256, 0, st>>>(cu, (int32_t)B, pairs, c.ts, c.sb, c.pinfo);
-  note_launch();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  const int pairs = core_pairs(tq, num_sms);
+  cudaError_t e;
   CoreParams p;
   memset(&p, 0, sizeof(p));
   if ((e = make_tmap_bf16(&p.kmap, cache, ROW, capacity, ROW, 64, NK)) != cudaSuccess) return e;

@@ -130,7 +130,10 @@ cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const LayerOp
   const int64_t T = B * tq, HD = (int64_t)d.n_h * d.d_h, HC = (int64_t)d.n_h * d.d_c;
   const size_t part_bytes = decode_gemm_partials(d, T);
   void* core_scratch = (char*)scratch + part_bytes;
-  cudaError_t e = queries(d, w, lo, h_q, pos, T, cq, qc, qr, scratch, part_bytes, err, st);
+  // device checks of cu_seqlens, the query positions and the latent core's plan: one launch
+  cudaError_t e = tc_core_prepare(cu, B, tq, capacity, const_cast<int64_t*>(pos), core_scratch, num_sms, err, st);
+  if (e != cudaSuccess) return e;
+  e = queries(d, w, lo, h_q, pos, T, cq, qc, qr, scratch, part_bytes, err, st);
   if (e != cudaSuccess) return e;
   // q~_i = W_i^UK^T q^C_i for every head i: the weight operand is W^UK read MN-major. The
   // head-batched GEMM streams weights with the tokens on the MMA's N side, so it runs on chunks of
@@ -146,7 +149,7 @@ cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const LayerOp
     a.batch = d.n_h; a.w_row_z = d.d_h; a.x_col_z = d.d_h;
     if ((e = tc_gemm(a, st)) != cudaSuccess) return e;
   }
-  e = tc_latent_core_impl(qabs, qr, B, tq, cu, cache, capacity, olat, false, lse, core_scratch, num_sms, err, st);
+  e = tc_core_run(qabs, qr, B, tq, cu, cache, capacity, olat, false, lse, core_scratch, num_sms, err, st);
   if (e != cudaSuccess) return e;
   // o_i = W_i^UV o^lat_i for every head i, in the same token chunks.
   for (int64_t t0 = 0; t0 < T; t0 += kSwapMaxTokens) {
