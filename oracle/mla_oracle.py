@@ -39,6 +39,10 @@ Readings where the pages leave a step open (each is also listed in the design doc):
      theta'_m = (1 - gamma) theta_m / s + gamma theta_m; the factor 0.1 ln s + 1
      multiplies each rotated vector, q^R and k^R alike, so the RoPE term of the
      score grows by its square and the latent term is untouched.
+  R15 FP8 latent cache (opt-in): one fp32 scale per cached row, s = max(amax(c^KV) / 448,
+     amax(k^R) / 32768); c^KV stored as e4m3 codes of c^KV / s (round to nearest, ties to
+     even, saturating at 448) and k^R as f16 of k^R / s, both divisions in fp32. Attention
+     over an FP8 cache is attention over the dequantized rows [codes s | k^R' s].
   R5 Decode: a sequence's cache length includes its Tq new tokens (appended
      first); query k sits at position len - Tq + k and sees rows j <= position.
   R6 A synthetic decode cache holds c^KV and an already-rotated k^R.
@@ -467,3 +471,64 @@ def mha_cache_elements_per_token(dims, layers: int) -> int:
 def mla_cache_elements_per_token(dims, layers: int) -> int:
     """(d_c + d_h^R) l elements per token for MLA with the decoupled RoPE key."""
     return (dims.d_c + dims.d_r) * layers
+
+
+# ---------------------------------------------------------------------------
+# FP8 (e4m3) latent cache (opt-in; reading R15). The notes' FP8 section scales 1 x 128 tiles for
+# training GEMMs; for the cache this build takes one fp32 scale per cached row.
+# ---------------------------------------------------------------------------
+E4M3_MAX = 448.0
+KR_F16_RANGE = 32768.0
+
+
+def e4m3_positive_values() -> np.ndarray:
+    """The 127 non-negative finite e4m3 values in code order 0x00 .. 0x7E (1 sign, 4 exponent bits
+    with bias 7, 3 mantissa bits; no infinities, 0x7F is NaN): code e * 8 + m is m/8 * 2^-6 for e = 0
+    and (1 + m/8) * 2^(e - 7) otherwise. Codes increase with the value."""
+    out = []
+    for code in range(0x7F):
+        e, m = code >> 3, code & 7
+        out.append(m / 8.0 * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return np.array(out)
+
+
+def round_to_e4m3(x) -> np.ndarray:
+    """x rounded to the nearest e4m3 value, ties to the even code (even mantissa), magnitudes past
+    448 saturated to 448. Works on the magnitude and puts the sign back."""
+    x = f64(x)
+    grid = e4m3_positive_values()
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(grid, a, side="left"), 0, len(grid) - 1)
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - grid[lo], grid[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    return np.sign(x) * np.where(pick_hi, grid[hi], grid[lo])
+
+
+def round_to_f16(x) -> np.ndarray:
+    """IEEE half precision, round to nearest even (numpy's float16 conversion)."""
+    return f64(np.asarray(x, dtype=np.float64).astype(np.float16))
+
+
+def quantize_cache_rows_fp8(rows, dims):
+    """FP8 cache rows from bf16 cache rows [n, d_c + d_r] (reading R15).
+
+    Per row: s = max(amax(c^KV) / 448, amax(k^R) / 32768) in fp32 (1 if the row is all zero);
+    codes = e4m3(c^KV / s) and k^R' = f16(k^R / s), each division in fp32. Returns (codes [n, d_c] as
+    the e4m3 values, kr_scaled [n, d_r] as the f16 values, s [n]) in float64.
+    """
+    rows = np.asarray(rows, dtype=np.float32)
+    c, kr = rows[:, :dims.d_c], rows[:, dims.d_c:]
+    amax_c = np.abs(c).max(axis=1).astype(np.float32)
+    amax_r = np.abs(kr).max(axis=1).astype(np.float32)
+    s = np.maximum(amax_c / np.float32(E4M3_MAX), amax_r / np.float32(KR_F16_RANGE)).astype(np.float32)
+    s = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    codes = round_to_e4m3((c / s[:, None]).astype(np.float32))
+    kr_scaled = round_to_f16((kr / s[:, None]).astype(np.float32))
+    return codes, kr_scaled, f64(s)
+
+
+def dequantize_cache_rows_fp8(codes, kr_scaled, s) -> np.ndarray:
+    """The cache rows an FP8 cache stands for: [codes * s | k^R' * s], exactly in float64."""
+    s = f64(s)[:, None]
+    return np.concatenate([f64(codes) * s, f64(kr_scaled) * s], axis=1)

@@ -508,6 +508,59 @@ def test_absorbed_equals_unabsorbed_with_rmsnorm_and_yarn(tq):
 
 
 # ---------------------------------------------------------------------------
+# FP8 (e4m3) latent cache (reading R15; the notes' FP8 section, 二（三）, scales values into the
+# e4m3 range with fp32 scales)
+# ---------------------------------------------------------------------------
+def test_e4m3_grid_matches_the_format_and_torch():
+    g = orc.e4m3_positive_values()
+    assert len(g) == 127 and np.all(np.diff(g) > 0)
+    assert g[0x01] == 2.0 ** -9 and g[0x07] == 7 * 2.0 ** -9 and g[0x08] == 2.0 ** -6 and g[0x7E] == 448.0
+    assert g[0x38] == 1.0 and g[0x39] == 1.125
+    ref = torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(g, ref)
+
+
+def test_round_to_e4m3_is_round_to_nearest_even_and_saturates():
+    g = orc.e4m3_positive_values()
+    mids = (g[1:] + g[:-1]) / 2
+    x = np.concatenate([mids, -mids, g, np.random.default_rng(5).uniform(-448, 448, 20000),
+                        np.random.default_rng(6).standard_normal(20000) * 0.01])
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(orc.round_to_e4m3(x.astype(np.float32)), ref)
+    # ties go to the even code: 1 + 1/16 -> 1 (code 0x38), 1 + 3/16 -> 1.25 (0x3A)
+    assert orc.round_to_e4m3([1.0625, 1.1875]).tolist() == [1.0, 1.25]
+    # beyond the range: 448 (torch gives NaN past 464; the format's saturating conversion gives 448)
+    assert orc.round_to_e4m3([500.0, -1e6, 464.0]).tolist() == [448.0, -448.0, 448.0]
+
+
+def test_fp8_cache_rows_scale_codes_and_error_bounds():
+    dims = synth.V3
+    rng = np.random.default_rng(7)
+    rows = synth.latent_cache(dims, 64, seed=8, dtype="bf16").astype(np.float64)
+    rows[0] = 0.0                                   # an all-zero row: scale 1, codes 0
+    rows[1, :dims.d_c] *= 1e-3                      # k^R sets the scale
+    rows[2, dims.d_c:] *= 1e4                       # |k^R| / s would pass f16's range without the second term
+    rows = rows.astype(np.float32)
+    codes, krs, s = orc.quantize_cache_rows_fp8(rows, dims)
+    c, kr = rows[:, :dims.d_c].astype(np.float64), rows[:, dims.d_c:].astype(np.float64)
+    assert s[0] == 1.0 and np.all(codes[0] == 0) and np.all(krs[0] == 0)
+    amax_c, amax_r = np.abs(c).max(1), np.abs(kr).max(1)
+    expect = np.maximum(np.float32(amax_c) / np.float32(448), np.float32(amax_r) / np.float32(32768))
+    assert np.array_equal(s[1:], expect[1:].astype(np.float64))
+    assert np.all(np.abs(codes) <= 448) and np.all(np.abs(krs) <= 32768 * (1 + 2 ** -10))
+    assert np.all(np.isin(np.abs(codes), orc.e4m3_positive_values()))
+    deq = orc.dequantize_cache_rows_fp8(codes, krs, s)
+    # e4m3: half an ulp, relative 2^-4 for normals, 2^-10 s absolute in the subnormal range
+    err_c = np.abs(deq[:, :dims.d_c] - c)
+    assert np.all(err_c <= np.maximum(2.0 ** -4 * np.abs(c), 2.0 ** -10 * s[:, None]) * (1 + 1e-6))
+    # f16: relative 2^-11 for normals (|k^R| / s >= 2^-14), plus the fp32 division's own rounding
+    err_r = np.abs(deq[:, dims.d_c:] - kr)
+    assert np.all(err_r <= np.maximum(2.0 ** -11 * np.abs(kr), 2.0 ** -25 * s[:, None]) * (1 + 1e-6) + 1e-300)
+    # the row whose k^R sets the scale keeps k^R exactly to f16 precision with codes far below 448
+    assert np.abs(codes[1]).max() < 448 and np.abs(krs[1]).max() == 32768
+
+
+# ---------------------------------------------------------------------------
 # Split-KV combine: exact identity of the softmax over disjoint key sets
 # ---------------------------------------------------------------------------
 def test_lse_combine_of_any_split_equals_unsplit():
@@ -592,6 +645,15 @@ def _yarn_scale_once(dims):
     return math.sqrt(0.1 * math.log(dims.yarn_s) + 1.0) if dims.yarn_s > 1.0 else 1.0
 
 
+def _round_e4m3_ties_away(x):
+    x = np.asarray(x, np.float64)
+    grid = orc.e4m3_positive_values()
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.clip(np.searchsorted(grid, a, side="left"), 0, len(grid) - 1)
+    lo = np.maximum(hi - 1, 0)
+    return np.sign(x) * np.where(grid[hi] - a <= a - grid[lo], grid[hi], grid[lo])
+
+
 def _rms_norm_sum(x, g, eps):
     x = np.asarray(x, np.float64)
     return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps) * np.asarray(g, np.float64)
@@ -600,7 +662,7 @@ PINS = [test_rope_closed_form_two_dims, test_rope_frequencies, lambda: test_orac
         lambda: test_brute_force_tiny_random(0), lambda: test_brute_force_tiny_random(1),
         lambda: test_zero_rope_weights_reduce_to_plain_mha(), test_causality_rows_after_position_do_not_matter,
         test_yarn_frequencies_by_parts_closed_form, test_yarn_scale_and_relative_position, test_rms_norm_closed_forms,
-        test_rmsnorm_sits_on_the_latent_vectors_only]
+        test_rmsnorm_sits_on_the_latent_vectors_only, test_round_to_e4m3_is_round_to_nearest_even_and_saturates]
 
 
 @pytest.mark.parametrize("name,attr,fake", [
@@ -612,6 +674,7 @@ PINS = [test_rope_closed_form_two_dims, test_rope_frequencies, lambda: test_orac
     ("YaRN ramp on the wavelength ratio", "yarn_frequencies", _yarn_ramp_inverted),
     ("YaRN factor on the score, not on each vector", "rope_scale", _yarn_scale_once),
     ("RMSNorm over the sum of squares", "rms_norm", _rms_norm_sum),
+    ("e4m3 ties away from zero", "round_to_e4m3", _round_e4m3_ties_away),
 ])
 def test_planted_mistakes_are_caught(monkeypatch, name, attr, fake):
     monkeypatch.setattr(orc, attr, fake)
