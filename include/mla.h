@@ -126,6 +126,30 @@ mla_status_t mla_set_rmsnorm(mla_handle_t *h, const void *g_q, const void *g_kv,
  * cache rows written under one setting must be read under the same one. */
 mla_status_t mla_set_yarn(mla_handle_t *h, double s, double alpha, double beta, double original_len);
 
+/* The format of the latent cache the handle's calls read and write. */
+typedef enum {
+  MLA_CACHE_BF16 = 0,   /* rows [d_c + d_r] in the handle dtype (the default)                  */
+  MLA_CACHE_FP8 = 1     /* 656-byte rows at the DeepSeek-V3 sizes, see mla_set_cache_format     */
+} mla_cache_format_t;
+
+/* Opt-in FP8 (e4m3) latent cache (the notes' FP8 section 二（三） keeps e4m3 values with fp32 scales;
+ * here one scale per cached row). Row layout, 656 bytes, 16-byte aligned:
+ *   bytes [0, 512)    e4m3 codes of c^KV / s, round to nearest even, saturating at 448
+ *   bytes [512, 640)  f16 of k^R / s, round to nearest even
+ *   bytes [640, 644)  s as fp32: s = max(amax(c^KV) / 448, amax(k^R) / 32768), or 1 for a zero row
+ *   bytes [644, 656)  zero
+ * A row stands for [codes * s | (k^R / s) * s]; every division is an IEEE fp32 division. With FP8 the
+ * cache argument of mla_cache_append points to such rows (capacity rows of 656 bytes); the decode,
+ * prefill and attention calls and mla_cache_append_noalloc return MLA_ERR_UNSUPPORTED for now.
+ * BF16 handles only (MLA_ERR_UNSUPPORTED otherwise). Host-only. */
+mla_status_t mla_set_cache_format(mla_handle_t *h, mla_cache_format_t format);
+
+/* Converts n bf16 cache rows [n, 576] to FP8 rows [n, 656 bytes] (the layout above), for example to
+ * move an existing cache to FP8. Device pointers, 16-byte aligned. BF16 handles at the DeepSeek-V3
+ * sizes. */
+mla_status_t mla_cache_quantize_fp8(mla_handle_t *h, const void *rows, int64_t n, void *out,
+                                    mla_stream_t stream);
+
 /* Workspace bytes for one call of `op` on num_seqs sequences with tq query tokens each
  * (decode, attention core) or total_tokens packed tokens (prefill, cache append).
  * Host-only arithmetic. */

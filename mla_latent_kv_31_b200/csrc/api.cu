@@ -148,7 +148,8 @@ Layout layout(const mla_handle* h, mla_op_t op, int64_t B, int32_t tq, int64_t t
     }
     if (op == MLA_OP_DECODE && kv_rows < 0) cur = align_up(cur + mla::tc_decode_scratch_bytes(d, B, tq));
     if (op == MLA_OP_ATTN_DECODE_LATENT) cur = align_up(cur + mla::tc_core_scratch_bytes(d, B, tq));
-    if (op == MLA_OP_CACHE_APPEND) cur = align_up(cur + mla::tc_append_scratch_bytes(d, total_tokens));
+    if (op == MLA_OP_CACHE_APPEND)
+      cur = align_up(cur + mla::tc_append_scratch_bytes(d, total_tokens, h->opts.cache_fp8 != 0));
   }
   L.total = cur;
   return L;
@@ -317,6 +318,24 @@ mla_status_t mla_set_rmsnorm(mla_handle_t* h, const void* g_q, const void* g_kv,
   return MLA_OK;
 }
 
+mla_status_t mla_set_cache_format(mla_handle_t* h, mla_cache_format_t format) {
+  if (!h || (format != MLA_CACHE_BF16 && format != MLA_CACHE_FP8)) return MLA_ERR_INVALID_ARG;
+  if (format == MLA_CACHE_FP8 && !tc_dims(h)) return MLA_ERR_UNSUPPORTED;
+  h->opts.cache_fp8 = format == MLA_CACHE_FP8 ? 1 : 0;
+  return MLA_OK;
+}
+
+mla_status_t mla_cache_quantize_fp8(mla_handle_t* h, const void* rows, int64_t n, void* out, mla_stream_t stream) {
+  if (!h || !rows || !out || n <= 0) return MLA_ERR_INVALID_ARG;
+  if (!tc_dims(h)) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(rows) || !aligned16(out)) return MLA_ERR_ALIGNMENT;
+  DeviceGuard g(h->device);
+  if (!g.ok) return MLA_ERR_CUDA;
+  mla_status_t s = ensure_device(h);
+  if (s != MLA_OK) return s;
+  return cuda_status(mla::fp8_quantize_rows(rows, n, nullptr, n, out, (cudaStream_t)stream));
+}
+
 mla_status_t mla_set_yarn(mla_handle_t* h, double s, double alpha, double beta, double original_len) {
   if (!h || !(s >= 1.0) || !(beta > alpha) || !(original_len > 0.0)) return MLA_ERR_INVALID_ARG;
   h->opts.rope = mla::RopeSpec{h->dims.rope_base, s, alpha, beta, original_len};
@@ -442,6 +461,7 @@ mla_status_t mla_attn_decode_latent(mla_handle_t* h, const void* q_abs, const vo
   if (!h || !q_abs || !q_rope || !cu_seqlens || !cache || !o_lat || !lse || B <= 0 || capacity <= 0)
     return MLA_ERR_INVALID_ARG;
   if (Tq != 1 && Tq != 2) return MLA_ERR_INVALID_ARG;
+  if (h->opts.cache_fp8) return MLA_ERR_UNSUPPORTED;   // FP8 latent core not built yet
   if (!aligned16(q_abs) || !aligned16(q_rope) || !aligned16(cache) || !aligned16(o_lat) || !aligned16(lse) ||
       !aligned16(cu_seqlens) || (ws && !aligned16(ws)))
     return MLA_ERR_ALIGNMENT;
@@ -558,6 +578,7 @@ mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq,
                         mla_stream_t stream) {
   if (!h || !h_q || !cu_seqlens || !cache || !u_out || !ws || B <= 0 || capacity <= 0) return MLA_ERR_INVALID_ARG;
   if (Tq != 1 && Tq != 2) return MLA_ERR_INVALID_ARG;
+  if (h->opts.cache_fp8) return MLA_ERR_UNSUPPORTED;   // FP8 latent core not built yet
   if (!aligned16(h_q) || !aligned16(cache) || !aligned16(u_out) || !aligned16(ws) || !aligned16(cu_seqlens))
     return MLA_ERR_ALIGNMENT;
   Layout L = layout(h, MLA_OP_DECODE, B, Tq, 0);
@@ -578,6 +599,7 @@ mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq,
 mla_status_t mla_prefill(mla_handle_t* h, const void* hidden, int64_t B, const int64_t* cu_seqlens,
                          int64_t total_tokens, int64_t max_seqlen, void* cache, int64_t capacity, void* u_out,
                          void* ws, size_t ws_bytes, mla_stream_t stream) {
+  if (h && h->opts.cache_fp8) return MLA_ERR_UNSUPPORTED;   // FP8 caches: append and decode only
   if (!h || !hidden || !cu_seqlens || !cache || !u_out || !ws || B <= 0 || total_tokens <= 0 || max_seqlen <= 0 ||
       capacity < total_tokens)
     return MLA_ERR_INVALID_ARG;
@@ -601,6 +623,7 @@ mla_status_t mla_prefill(mla_handle_t* h, const void* hidden, int64_t B, const i
 mla_status_t mla_prefill_chunk(mla_handle_t* h, const void* hidden, int64_t B, const int64_t* cu_q, int64_t total_q,
                                int64_t max_q, const int64_t* cu_kv, int64_t total_kv, void* cache, int64_t capacity,
                                mla_chunk_form_t form, void* u_out, void* ws, size_t ws_bytes, mla_stream_t stream) {
+  if (h && h->opts.cache_fp8) return MLA_ERR_UNSUPPORTED;   // FP8 caches: append and decode only
   mla_chunk_form_t f;
   if (!h || !hidden || !cu_q || !cu_kv || !cache || !u_out || !ws || capacity < total_kv ||
       !chunk_form(B, total_q, max_q, total_kv, form, &f))
@@ -640,6 +663,7 @@ mla_status_t mla_prefill_chunk(mla_handle_t* h, const void* hidden, int64_t B, c
 mla_status_t mla_attn_prefill(mla_handle_t* h, const void* q_c, const void* q_rope, const void* k_c, const void* v_c,
                               int64_t B, const int64_t* cu_seqlens, int64_t total_tokens, int64_t max_seqlen,
                               const void* cache, int64_t capacity, void* o, mla_stream_t stream) {
+  if (h && h->opts.cache_fp8) return MLA_ERR_UNSUPPORTED;   // FP8 caches: append and decode only
   if (!h || !q_c || !q_rope || !k_c || !v_c || !cu_seqlens || !cache || !o || B <= 0 || total_tokens <= 0 ||
       max_seqlen <= 0 || capacity < total_tokens)
     return MLA_ERR_INVALID_ARG;
@@ -751,6 +775,7 @@ mla_status_t noalloc_scratch(int device, void** out) {
 extern "C" mla_status_t mla_cache_append_noalloc(mla_handle_t* h, const void* hidden, const int64_t* positions,
                                                  const int64_t* slots, int64_t T, void* cache, int64_t capacity,
                                                  mla_stream_t stream) {
+  if (h && h->opts.cache_fp8) return MLA_ERR_UNSUPPORTED;   // FP8 caches: append and decode only
   if (!h || !hidden || !positions || !slots || !cache || T <= 0 || capacity <= 0) return MLA_ERR_INVALID_ARG;
   if (!aligned16(hidden) || !aligned16(cache) || !aligned16(positions) || !aligned16(slots))
     return MLA_ERR_ALIGNMENT;

@@ -53,6 +53,7 @@ struct LayerOpts {
   const void* g_kv;   // [d_c] gains of c^KV
   float eps;
   RopeSpec rope;
+  int cache_fp8;      // the latent cache holds FP8 rows (656 bytes) instead of bf16 rows
 };
 
 __device__ __forceinline__ void flag_error(uint32_t* err, uint32_t bits) {

@@ -14,8 +14,20 @@ namespace mla {
 size_t tc_decode_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq);
 // Scratch bytes of the latent core alone.
 size_t tc_core_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq);
-// Scratch bytes of mla_cache_append for T tokens (split-K partials when T is small).
-size_t tc_append_scratch_bytes(const mla_dims_t& d, int64_t T);
+// Scratch bytes of mla_cache_append for T tokens (split-K partials when T is small; with an FP8 cache,
+// then the bf16 rows staged before quantization).
+size_t tc_append_scratch_bytes(const mla_dims_t& d, int64_t T, bool fp8 = false);
+
+// FP8 latent cache rows (mla_set_cache_format): 656 bytes = 512 e4m3 codes of c^KV / s, 64 f16 of
+// k^R / s, the fp32 scale s and 12 zero bytes.
+constexpr int kFp8RowBytes = 656;
+constexpr int kFp8RowLatent = 576;   // bf16 elements of the cache row it is made from
+// bf16 cache rows [n][576] -> FP8 rows at out + row(r) * 656, row(r) = rowmap ? rowmap[r] : r (rows
+// mapped outside [0, limit) are skipped).
+cudaError_t fp8_quantize_rows(const void* rows, int64_t n, const int64_t* rowmap, int64_t limit, void* out,
+                              cudaStream_t st);
+// Scratch bytes of the bf16 rows an FP8 append stages before quantizing them.
+inline size_t fp8_staging_bytes(int64_t T) { return (size_t)(T > 0 ? T : 1) * kFp8RowLatent * 2; }
 
 cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& o, const void* hidden,
                             const int64_t* positions, const int64_t* slots, int64_t T, void* cache,

@@ -729,12 +729,16 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
     const int64_t x = ts[b0] + (off <= 0 ? 0 : (off + 1) / 2);
     return (int32_t)min(x, (int64_t)ts[b0 + 1]);
   };
-  // the cluster owning tile x: the last pp with bound(pp) <= x (empty clusters never win a tie)
+  // every cluster's first tile, one thread each (each a binary search over the sequences)
+  __shared__ int32_t bnd[kMaxPairs + 1];
+  for (int pp = tid; pp <= pairs; pp += blockDim.x) bnd[pp] = bound(pp);
+  __syncthreads();
+  // the cluster owning tile x: the last pp with bnd[pp] <= x (empty clusters never win a tie)
   auto pair_of = [&](int32_t x) -> int {
     int p0 = 0, p1 = pairs - 1;
     while (p0 < p1) {
       const int mid = (p0 + p1 + 1) >> 1;
-      if (bound(mid) <= x) p0 = mid; else p1 = mid - 1;
+      if (bnd[mid] <= x) p0 = mid; else p1 = mid - 1;
     }
     return p0;
   };
@@ -744,7 +748,7 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
     int32_t r = 0;
     for (int pp = 0; pp < pairs; ++pp) {
       arank[pp] = r;
-      if (bound(pp + 1) > bound(pp)) ++r;
+      if (bnd[pp + 1] > bnd[pp]) ++r;
     }
     arank[pairs] = r;
   }
@@ -762,7 +766,7 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
   // per cluster: its tile range, the sequence of its first tile and that piece's partial slot
   for (int pp = tid; pp < pairs; pp += blockDim.x) {
     int4 v = make_int4(0, 0, 0, 0);
-    const int32_t x0 = bound(pp), x1 = bound(pp + 1);
+    const int32_t x0 = bnd[pp], x1 = bnd[pp + 1];
     if (x1 > x0) {
       v.x = x0;
       v.y = x1;

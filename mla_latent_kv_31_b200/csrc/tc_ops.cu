@@ -45,27 +45,33 @@ size_t decode_gemm_partials(const mla_dims_t& d, int64_t T) {
 }
 
 // Steps (5) and (7) with the cache write: rows [c^KV | RoPE(W^KR h)] -> cache[rowmap[t]], then the
-// optional RMSNorm of c^KV in place.
+// optional RMSNorm of c^KV in place. With an FP8 cache the rows go to `staging` ([T][576] bf16) first,
+// are normalised there, and are quantized into the cache rows.
 cudaError_t cache_rows(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& o, const void* hidden,
                        const int64_t* pos, const int64_t* rowmap, int64_t T, void* cache, int64_t capacity,
-                       void* scratch, size_t scratch_bytes, uint32_t* err, cudaStream_t st) {
+                       void* scratch, size_t scratch_bytes, void* staging, uint32_t* err, cudaStream_t st) {
   const int64_t R = d.d_c + d.d_r;
+  const bool fp8 = o.cache_fp8 && staging;
+  void* dst = fp8 ? staging : cache;
+  const int64_t* map = fp8 ? nullptr : rowmap;
+  const int64_t limit = fp8 ? T : capacity;
   TcGemmDesc g = desc(mat(hidden, T, d.d, d.d), T, d.d, err);
   g.nseg = 2;
   g.seg[0].w = mat(w.w_dkv, d.d_c, d.d, d.d);
-  g.seg[0].epi = epi(cache, R, 1, d.d_c);
+  g.seg[0].epi = epi(dst, R, 1, d.d_c);
   g.seg[1].w = mat(w.w_kr, d.d_r, d.d, d.d);
-  g.seg[1].epi = epi((char*)cache + (size_t)d.d_c * 2, R, 1, d.d_r);
+  g.seg[1].epi = epi((char*)dst + (size_t)d.d_c * 2, R, 1, d.d_r);
   g.seg[1].epi.rope = 1;
   for (int s = 0; s < 2; ++s) {
-    g.seg[s].epi.rowmap = rowmap;
-    g.seg[s].epi.rowmap_limit = capacity;
+    g.seg[s].epi.rowmap = map;
+    g.seg[s].epi.rowmap_limit = limit;
   }
   g.pos = pos; g.d_r = d.d_r; g.rope = o.rope;
   g.partial = (float*)scratch; g.partial_bytes = scratch_bytes;
   cudaError_t e = tc_gemm(g, st);
-  if (e != cudaSuccess || !o.g_kv) return e;
-  return rmsnorm_rows(cache, true, R, rowmap, capacity, T, d.d_c, o.g_kv, o.eps, st);
+  if (e != cudaSuccess) return e;
+  if (o.g_kv && (e = rmsnorm_rows(dst, true, R, map, limit, T, d.d_c, o.g_kv, o.eps, st)) != cudaSuccess) return e;
+  return fp8 ? fp8_quantize_rows(staging, T, rowmap, capacity, cache, st) : cudaSuccess;
 }
 
 // Steps (1)-(3): c^Q = W^DQ h (then the optional RMSNorm); q^C = W^UQ c^Q; q^R = RoPE(W^QR c^Q).
@@ -111,15 +117,21 @@ size_t tc_decode_scratch_bytes(const mla_dims_t& d, int64_t B, int32_t tq) {
   return decode_gemm_partials(d, B * tq) + align_up(tc_core_scratch_bytes(d, B, tq));
 }
 
-size_t tc_append_scratch_bytes(const mla_dims_t& d, int64_t T) {
-  return align_up(tc_gemm_partial_bytes(T, tiles128(d.d_c) + tiles128(d.d_r), d.d_c + d.d_r, d.d, 1));
+size_t tc_append_scratch_bytes(const mla_dims_t& d, int64_t T, bool fp8) {
+  return align_up(tc_gemm_partial_bytes(T, tiles128(d.d_c) + tiles128(d.d_r), d.d_c + d.d_r, d.d, 1)) +
+         (fp8 ? align_up(fp8_staging_bytes(T)) : 0);
 }
 
 cudaError_t tc_cache_append(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& o, const void* hidden,
                             const int64_t* positions, const int64_t* slots, int64_t T, void* cache,
                             int64_t capacity, void* scratch, size_t scratch_bytes, uint32_t* err,
                             cudaStream_t st) {
-  return cache_rows(d, w, o, hidden, positions, slots, T, cache, capacity, scratch, scratch_bytes, err, st);
+  // FP8: the bf16 rows are staged at the end of the scratch, after the split-K partials
+  const size_t stage = o.cache_fp8 ? align_up(fp8_staging_bytes(T)) : 0;
+  if (scratch_bytes < stage) return cudaErrorInvalidValue;
+  void* staging = o.cache_fp8 ? (char*)scratch + (scratch_bytes - stage) : nullptr;
+  return cache_rows(d, w, o, hidden, positions, slots, T, cache, capacity, scratch, scratch_bytes - stage, staging, err,
+                    st);
 }
 
 cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& lo, const void* h_q, int64_t B,
@@ -172,7 +184,7 @@ cudaError_t tc_prefill(const mla_dims_t& d, const mla_weights_t& w, const LayerO
                        cudaStream_t st) {
   const int64_t R = d.d_c + d.d_r, HD = (int64_t)d.n_h * d.d_h;
   if (!cu_kv) T_kv = T;
-  cudaError_t e = cache_rows(d, w, lo, hidden, pos, slots, T, cache, capacity, nullptr, 0, err, st);
+  cudaError_t e = cache_rows(d, w, lo, hidden, pos, slots, T, cache, capacity, nullptr, 0, nullptr, err, st);
   if (e != cudaSuccess) return e;
   e = queries(d, w, lo, hidden, pos, T, cq, qc, qr, nullptr, 0, err, st);
   if (e != cudaSuccess) return e;
