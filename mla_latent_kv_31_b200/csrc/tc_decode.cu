@@ -690,7 +690,11 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
 }
 
 // The same block first runs the device checks of cu_seqlens and writes the decode positions
-// (len_b - tq + k), so that a decode step needs one small launch for both.
+// (len_b - tq + k), so that a decode step needs one small launch for both. The plan is a chain of
+// dependent lookups, so up to kPlanShSeqs sequences keep their tile and slot prefixes in (dynamic)
+// shared memory besides the global copies the core reads.
+constexpr int kPlanShSeqs = 4096;
+static_assert(kMaxPairs < 96, "the active-cluster ranks take three ballots");
 __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B, int32_t pairs, int32_t* ts,
                                                    int32_t* sb, int4* pinfo, int32_t tq, int64_t capacity,
                                                    int64_t* pos_out, uint32_t* err) {
@@ -704,11 +708,15 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
     const int64_t len = cu[b + 1] - cu[b];
     return len > 0 ? (int32_t)((len + NK - 1) / NK) : 0;
   };
+  extern __shared__ int32_t plan_sh[];
+  const bool in_sh = B + 1 <= kPlanShSeqs;
+  int32_t* tsr = in_sh ? plan_sh : ts;
+  int32_t* sbr = in_sh ? plan_sh + (B + 1) : sb;
   int32_t acc = 0;
   for (int b = lo; b < hi; ++b) acc += ntiles(b);
   acc = block_exclusive_scan(acc, warp_tot, &total);
-  for (int b = lo; b < hi; ++b) { ts[b] = acc; acc += ntiles(b); }
-  if (tid == 0) ts[B] = total;
+  for (int b = lo; b < hi; ++b) { ts[b] = acc; tsr[b] = acc; acc += ntiles(b); }
+  if (tid == 0) { ts[B] = total; tsr[B] = total; }
   __syncthreads();
   const int64_t NT = total;
   // Cost-aware ranges. Besides its tiles, a cluster pays once per sequence piece (the piece's q load
@@ -722,12 +730,12 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
     int b0 = 0, b1 = B;                       // the last b in [0, B] with vs(b) <= v
     while (b0 < b1) {
       const int mid = (b0 + b1 + 1) >> 1;
-      if (2 * (int64_t)ts[mid] + kStartCost * (int64_t)mid <= v) b0 = mid; else b1 = mid - 1;
+      if (2 * (int64_t)tsr[mid] + kStartCost * (int64_t)mid <= v) b0 = mid; else b1 = mid - 1;
     }
-    if (b0 == B) return ts[B];
-    const int64_t off = v - (2 * (int64_t)ts[b0] + kStartCost * (int64_t)b0) - kStartCost;
-    const int64_t x = ts[b0] + (off <= 0 ? 0 : (off + 1) / 2);
-    return (int32_t)min(x, (int64_t)ts[b0 + 1]);
+    if (b0 == B) return tsr[B];
+    const int64_t off = v - (2 * (int64_t)tsr[b0] + kStartCost * (int64_t)b0) - kStartCost;
+    const int64_t x = tsr[b0] + (off <= 0 ? 0 : (off + 1) / 2);
+    return (int32_t)min(x, (int64_t)tsr[b0 + 1]);
   };
   // every cluster's first tile, one thread each (each a binary search over the sequences)
   __shared__ int32_t bnd[kMaxPairs + 1];
@@ -742,26 +750,29 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
     }
     return p0;
   };
-  // rank of each cluster among the clusters with a non-empty range
+  // rank of each cluster among the clusters with a non-empty range: a ballot of the non-empty ones
   __shared__ int32_t arank[kMaxPairs + 1];
-  if (tid == 0) {
-    int32_t r = 0;
-    for (int pp = 0; pp < pairs; ++pp) {
-      arank[pp] = r;
-      if (bnd[pp + 1] > bnd[pp]) ++r;
-    }
-    arank[pairs] = r;
+  __shared__ uint32_t active[3];
+  if (tid < 96) {
+    const uint32_t m = __ballot_sync(0xffffffffu, tid < pairs && bnd[tid + 1] > bnd[tid]);
+    if ((tid & 31) == 0) active[tid >> 5] = m;
+  }
+  __syncthreads();
+  for (int pp = tid; pp <= pairs; pp += blockDim.x) {
+    int32_t r = __popc(active[pp >> 5] & ((1u << (pp & 31)) - 1u));
+    for (int w = 0; w < (pp >> 5); ++w) r += __popc(active[w]);
+    arank[pp] = r;
   }
   __syncthreads();
   auto nseg = [&](int b) -> int32_t {
-    const int32_t a = ts[b], e = ts[b + 1];
+    const int32_t a = tsr[b], e = tsr[b + 1];
     return e > a ? arank[pair_of(e - 1)] - arank[pair_of(a)] + 1 : 0;
   };
   acc = 0;
   for (int b = lo; b < hi; ++b) acc += nseg(b);
   acc = block_exclusive_scan(acc, warp_tot, &total);
-  for (int b = lo; b < hi; ++b) { sb[b] = acc; acc += nseg(b); }
-  if (tid == 0) sb[B] = total;
+  for (int b = lo; b < hi; ++b) { sb[b] = acc; sbr[b] = acc; acc += nseg(b); }
+  if (tid == 0) { sb[B] = total; sbr[B] = total; }
   __syncthreads();
   // per cluster: its tile range, the sequence of its first tile and that piece's partial slot
   for (int pp = tid; pp < pairs; pp += blockDim.x) {
@@ -773,29 +784,32 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
       int lo2 = 0, hi2 = B - 1;               // the last b with ts[b] <= x0
       while (lo2 < hi2) {
         const int mid = (lo2 + hi2 + 1) >> 1;
-        if (ts[mid] <= x0) lo2 = mid; else hi2 = mid - 1;
+        if (tsr[mid] <= x0) lo2 = mid; else hi2 = mid - 1;
       }
       // the first sequence with tiles: skip empty sequences that share the start
-      while (lo2 < B - 1 && ts[lo2 + 1] <= x0) ++lo2;
+      while (lo2 < B - 1 && tsr[lo2 + 1] <= x0) ++lo2;
       v.z = lo2;
-      v.w = sb[lo2] + arank[pp] - arank[pair_of(ts[lo2])];
+      v.w = sbr[lo2] + arank[pp] - arank[pair_of(tsr[lo2])];
     }
     pinfo[pp] = v;
   }
 }
 
 // Exact merge of a sequence's pieces: lse = log sum_s e^{lse_s}, o = sum_s e^{m_s - lse} O_s from the
-// unnormalised head-interleaved partials O_s (O_s / l_s is the piece's own softmax average and
-// e^{lse_s} = e^{m_s} l_s, so the weight e^{lse_s - lse} / l_s is e^{m_s - lse}). One block per (token, group of 32 heads, group of 128 columns): the
-// reads of a (piece, 4-column group) are 512 contiguous bytes over the 32 heads; the block's
-// [32 heads x 128 columns] result goes through shared memory so that each head's row is written as
-// contiguous 512-byte runs.
-constexpr int kCombHeads = 32, kCombCols = 128;
+// unnormalised head-interleaved bf16 partials O_s (O_s / l_s is the piece's own softmax average and
+// e^{lse_s} = e^{m_s} l_s, so the weight e^{lse_s - lse} / l_s is e^{m_s - lse}). One block per (token,
+// group of 32 heads, group of 128 columns): the reads of a (piece, 4-column group) are 256 contiguous
+// bytes over the 32 heads; the block's [32 heads x 128 columns] result goes through shared memory so
+// that each head's row is written as contiguous runs. The kernel is latency-bound (a few MB of L2-hot
+// partials), so the partials of up to kCombBatch pieces are in flight at once, the first batch issued
+// before the pieces' m and lse are staged, and the staging takes one parallel pass over the pieces.
+constexpr int kCombHeads = 32, kCombCols = 128, kCombBatch = 8;
 template <bool OUT_F32>
 __global__ void __launch_bounds__(256) combine_kernel(const int32_t* sb, int32_t tq, int32_t s_max,
                                                       const uint2* part_o, const float* part_lse,
                                                       const float* part_m, void* o_lat, float* lse) {
-  __shared__ float wts[kMaxPairs][kCombHeads];
+  __shared__ float s_lse[kMaxPairs][kCombHeads];
+  __shared__ float s_m[kMaxPairs][kCombHeads];
   __shared__ float tile[kCombHeads][kCombCols + 4];
   const int64_t t = blockIdx.x;
   const int h0 = kCombHeads * blockIdx.y, c0 = kCombCols * blockIdx.z;
@@ -803,35 +817,48 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* sb, int32_t
   const int32_t s0 = sb[b], ns = min(sb[b + 1] - s0, kMaxPairs);
   const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
   const int64_t slot0 = (int64_t)k * s_max + s0;
-  if (tid < kCombHeads) {
-    // weights of head h0 + tid over the pieces
-    const int h = h0 + tid;
-    float mx = -INFINITY;
-    for (int sl = 0; sl < ns; ++sl) mx = fmaxf(mx, part_lse[(slot0 + sl) * H + h]);
-    float sum = 0.f;
-    for (int sl = 0; sl < ns; ++sl) sum += mx > -INFINITY ? __expf(part_lse[(slot0 + sl) * H + h] - mx) : 0.f;
-    const float tot = sum > 0.f ? mx + logf(sum) : -INFINITY;     // lse over all pieces
-    for (int sl = 0; sl < ns; ++sl) {
-      const float ms = part_m[(slot0 + sl) * H + h];
-      wts[sl][tid] = (tot > -INFINITY && ms > -INFINITY) ? __expf(ms - tot) : 0.f;
-    }
-    if (blockIdx.z == 0) lse[t * H + h] = tot;
+  // thread (lane = head, grp): 4-column groups c4 = c0/4 + 4 grp + q, q = 0..3
+  const uint2* src = part_o + (slot0 * (DC / 4) + c0 / 4 + 4 * grp) * H + h0 + lane;
+  uint2 v[kCombBatch][4];
+  auto load_batch = [&](int sl0) {
+#pragma unroll
+    for (int j = 0; j < kCombBatch; ++j)
+      if (sl0 + j < ns) {
+        const uint2* ps = src + (int64_t)(sl0 + j) * (DC / 4) * H;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[j][q] = ps[q * H];
+      }
+  };
+  load_batch(0);
+  for (int sl = grp; sl < ns; sl += 8) {
+    s_lse[sl][lane] = part_lse[(slot0 + sl) * H + h0 + lane];
+    s_m[sl][lane] = part_m[(slot0 + sl) * H + h0 + lane];
   }
   __syncthreads();
-  // thread (lane = head, grp): 4-column groups c4 = c0/4 + 4 grp + q, q = 0..3
+  // lse over all pieces of head h0 + lane
+  float mx = -INFINITY;
+  for (int sl = 0; sl < ns; ++sl) mx = fmaxf(mx, s_lse[sl][lane]);
+  float sum = 0.f;
+  for (int sl = 0; sl < ns; ++sl) sum += mx > -INFINITY ? __expf(s_lse[sl][lane] - mx) : 0.f;
+  const float tot = sum > 0.f ? mx + logf(sum) : -INFINITY;
+  if (blockIdx.z == 0 && grp == 0) lse[t * H + h0 + lane] = tot;
   float4 acc[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  const uint2* src = part_o + (c0 / 4 + 4 * grp) * H + h0 + lane;
-  for (int sl = 0; sl < ns; ++sl) {
-    const float wgt = wts[sl][lane];
-    const uint2* ps = src + (slot0 + sl) * (DC / 4) * H;
+  for (int sl0 = 0; sl0 < ns; sl0 += kCombBatch) {
+    if (sl0 > 0) load_batch(sl0);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint2 u = ps[q * H];
-      acc[q].x += wgt * bf16_lo(u.x); acc[q].y += wgt * bf16_hi(u.x);
-      acc[q].z += wgt * bf16_lo(u.y); acc[q].w += wgt * bf16_hi(u.y);
-    }
+    for (int j = 0; j < kCombBatch; ++j)
+      if (sl0 + j < ns) {
+        const float ms = s_m[sl0 + j][lane];
+        const float wgt = (tot > -INFINITY && ms > -INFINITY) ? __expf(ms - tot) : 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint2 u = v[j][q];
+          acc[q].x += wgt * bf16_lo(u.x); acc[q].y += wgt * bf16_hi(u.x);
+          acc[q].z += wgt * bf16_lo(u.y); acc[q].w += wgt * bf16_hi(u.y);
+        }
+      }
   }
 #pragma unroll
   for (int q = 0; q < 4; ++q) *reinterpret_cast<float4*>(&tile[lane][16 * grp + 4 * q]) = acc[q];
@@ -929,7 +956,8 @@ cudaError_t tc_core_prepare(const int64_t* cu, int64_t B, int32_t tq, int64_t ca
   if (B <= 0) return cudaSuccess;
   if (B > (int64_t)1 << 20 || tq < 1 || tq > kMaxPairs) return cudaErrorInvalidValue;
   CoreScratch c = carve(scratch, B, tq);
-  plan_kernel<<<1, 256, 0, st>>>(cu, (int32_t)B, core_pairs(tq, num_sms), c.ts, c.sb, c.pinfo, tq, capacity, pos, err);
+  const size_t plan_sh = B + 1 <= kPlanShSeqs ? 2 * (size_t)(B + 1) * sizeof(int32_t) : 0;
+  plan_kernel<<<1, 256, plan_sh, st>>>(cu, (int32_t)B, core_pairs(tq, num_sms), c.ts, c.sb, c.pinfo, tq, capacity, pos, err);
   note_launch();
   return cudaGetLastError();
 }

@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
                                          c_int64, c_void_p, c_int64, c_void_p, c_void_p]),
             "mla_set_rmsnorm": (c_int, [H, c_void_p, c_void_p, c_double]),
             "mla_set_yarn": (c_int, [H, c_double, c_double, c_double, c_double]),
+            "mla_set_cache_format": (c_int, [H, c_int]),
+            "mla_cache_quantize_fp8": (c_int, [H, c_void_p, c_int64, c_void_p, c_void_p]),
             "mla_sync_status": (c_int, [H, c_void_p]),
             "mla_device_error_bits": (c_uint32, [H]),
             "mla_uses_tensor_cores": (c_int, [H, c_int]),
@@ -206,6 +208,19 @@ def mla_set_yarn(handle, s: float, alpha: float = 1.0, beta: float = 32.0, origi
     _check(lib().mla_set_yarn(handle, s, alpha, beta, original_len), "mla_set_yarn")
 
 
+CACHE_BF16, CACHE_FP8 = 0, 1
+FP8_ROW_BYTES = 656   # e4m3 codes [512] | f16 k^R / s [64] | fp32 s | zero padding
+
+
+def mla_set_cache_format(handle, fmt: int):
+    _check(lib().mla_set_cache_format(handle, fmt), "mla_set_cache_format")
+
+
+def mla_cache_quantize_fp8(handle, rows, n, out, stream=None, device=0):
+    _check(lib().mla_cache_quantize_fp8(handle, _ptr(rows), n, _ptr(out), _stream(stream, device)),
+           "mla_cache_quantize_fp8")
+
+
 def mla_sync_status(handle, stream=None, device=0) -> int:
     return lib().mla_sync_status(handle, _stream(stream, device))
 
@@ -294,6 +309,15 @@ class MLA:
             n *= s
         es = torch.tensor([], dtype=dtype).element_size()
         return self._ws[off:off + n * es].view(dtype).view(*shape)
+
+    def set_cache_format(self, fmt: int):
+        mla_set_cache_format(self.handle, fmt)
+
+    def quantize_fp8(self, rows):
+        """FP8 rows [n, 656] (uint8) of bf16 cache rows [n, 576]."""
+        out = self.torch.empty(rows.shape[0], FP8_ROW_BYTES, dtype=self.torch.uint8, device=rows.device)
+        mla_cache_quantize_fp8(self.handle, rows, rows.shape[0], out, device=self.device)
+        return out
 
     def cache_append(self, hidden, positions, slots, cache):
         T = hidden.shape[0]

@@ -219,3 +219,41 @@ def test_option_setters_validate_on_the_host():
             assert e.value.status == 1
     finally:
         mla.mla_destroy(h)
+
+
+def test_cache_format_setter_and_fp8_guards():
+    A = 1 << 20
+    h32 = mla.mla_create(synth.TINY, mla.MLA_FP32)
+    try:
+        with pytest.raises(mla.MLAError) as e:   # FP8 rows are laid out for the DeepSeek-V3 sizes in bf16
+            mla.mla_set_cache_format(h32, mla.CACHE_FP8)
+        assert e.value.status == 3
+        mla.mla_set_cache_format(h32, mla.CACHE_BF16)
+    finally:
+        mla.mla_destroy(h32)
+    h = mla.mla_create(synth.V3, mla.MLA_BF16)
+    try:
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_set_cache_format(h, 2)
+        assert e.value.status == 1
+        mla.mla_set_cache_format(h, mla.CACHE_FP8)
+        # the calls that read the cache as bf16 rows refuse an FP8 handle before any launch
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_prefill(h, A, 1, A, 64, 64, A, 64, A, A, 1 << 30, stream=0)
+        assert e.value.status == 3
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_cache_append_noalloc(h, A, A, A, 4, A, 10, stream=0)
+        assert e.value.status == 3
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_attn_prefill(h, A, A, A, A, 1, A, 64, 64, A, 64, A, stream=0)
+        assert e.value.status == 3
+        # the quantizer validates its arguments on the host
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_cache_quantize_fp8(h, A, 0, A, stream=0)
+        assert e.value.status == 1
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_cache_quantize_fp8(h, A + 8, 4, A, stream=0)
+        assert e.value.status == 2
+        mla.mla_set_cache_format(h, mla.CACHE_BF16)
+    finally:
+        mla.mla_destroy(h)

@@ -1,0 +1,122 @@
+"""GPU parity of the FP8 (e4m3) latent cache rows: the quantizer against the oracle's
+`quantize_cache_rows_fp8` (same codes, scaled k^R and scale on every row, the values compared
+exactly; +0 and -0 compare equal), and the cache append writing FP8 rows against the oracle's
+float64 append within the format's rounding bound. The row layout is 656 bytes: e4m3 codes [0, 512),
+f16 k^R / s [512, 640), fp32 s [640, 644), zero [644, 656)."""
+import numpy as np
+import pytest
+
+from mla_testlib import dev, dev_i64, host, make_module, mla, orc, synth
+
+pytestmark = pytest.mark.gpu
+
+V3 = synth.V3
+E4M3 = orc.e4m3_positive_values()
+
+
+def decode_rows(raw: np.ndarray):
+    """(codes as values [n, 512], k^R' [n, 64], s [n], padding bytes [n, 12]) of FP8 rows [n, 656]."""
+    raw = np.ascontiguousarray(raw, dtype=np.uint8)
+    codes = raw[:, :512]
+    assert not np.any((codes & 0x7F) == 0x7F), "NaN code"
+    vals = np.where(codes & 0x80, -1.0, 1.0) * E4M3[codes & 0x7F]
+    kr = raw[:, 512:640].copy().view(np.float16).astype(np.float64)
+    s = raw[:, 640:644].copy().view(np.float32)[:, 0].astype(np.float64)
+    return vals, kr, s, raw[:, 644:656]
+
+
+def bf16(x):
+    """x rounded to bf16 (round to nearest even), as float64."""
+    import torch
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def stress_rows(n: int, seed: int) -> np.ndarray:
+    """bf16 cache rows [n, 576] that reach every branch of the format: N(0, 1) rows at scales from
+    1e-30 to 1e30, an all-zero row, rows whose k^R sets the scale (so k^R / s is at the f16 range's
+    end and c^KV / s lands in e4m3 subnormals), and rows with amax(c^KV) = 448 (s = 1) whose other
+    entries are exact midpoints between neighbouring e4m3 values (ties to the even code)."""
+    rng = np.random.default_rng(seed)
+    rows = rng.standard_normal((n, 576))
+    scale = 10.0 ** rng.integers(-30, 31, size=n)
+    rows *= scale[:, None]
+    rows[0] = 0.0
+    kr_big = np.arange(1, n, 7)
+    rows[kr_big, 512:] *= 1e5
+    rows[kr_big, :512] *= 1e-3
+    tie_rows = np.arange(2, n, 11)
+    mid = (E4M3[1:] + E4M3[:-1]) / 2          # every midpoint of the positive grid is bf16-exact
+    for r in tie_rows:
+        pick = rng.integers(0, len(mid), size=511)
+        rows[r, 1:512] = np.where(rng.random(511) < 0.5, -1.0, 1.0) * mid[pick]
+        rows[r, 0] = 448.0
+        rows[r, 512:] = rng.standard_normal(64)
+    return bf16(rows)
+
+
+@pytest.fixture(scope="module")
+def v3():
+    W = synth.weights(V3, seed=60, dtype="bf16")
+    m = make_module(V3, W, "bf16")
+    yield m, W
+    m.close()
+
+
+@pytest.mark.parametrize("n", [1, 8, 1037])
+def test_quantizer_matches_the_oracle_exactly(v3, n):
+    import torch
+    m, _ = v3
+    rows = stress_rows(n, seed=61 + n)
+    assert np.all(bf16(rows) == rows)
+    mid = (E4M3[1:] + E4M3[:-1]) / 2
+    assert np.all(bf16(mid) == mid)
+    got = m.quantize_fp8(dev(rows, "bf16"))
+    torch.cuda.synchronize()
+    vals, kr, s, pad = decode_rows(got.cpu().numpy())
+    codes_ref, kr_ref, s_ref = orc.quantize_cache_rows_fp8(rows, V3)
+    assert np.array_equal(s, s_ref)
+    assert np.array_equal(vals, codes_ref)
+    assert np.array_equal(kr, kr_ref)
+    assert not pad.any()
+
+
+def _fp8_bound(ref, s):
+    """Per-element bound of |dequantized - ref| for rows that went fp64 -> bf16 -> FP8: bf16 rounding
+    (2^-8 relative) then e4m3 rounding (2^-4 relative; s 2^-10 absolute in the subnormals) of the
+    c^KV part, f16 rounding (2^-11 relative) of the k^R part, and the projection's fp32 accumulation."""
+    b = np.empty_like(ref)
+    b[:, :512] = (2.0 ** -4 + 2.0 ** -7) * np.abs(ref[:, :512]) + s[:, None] * 2.0 ** -9
+    b[:, 512:] = 2.0 ** -7 * np.abs(ref[:, 512:]) + s[:, None] * 2.0 ** -20
+    return b + 1e-5 * np.abs(ref).max(axis=1, keepdims=True)
+
+
+@pytest.mark.parametrize("T,cap", [(45, 64), (700, 1024)])
+def test_cache_append_writes_fp8_rows(v3, T, cap):
+    import torch
+    m, W = v3
+    h = synth.hidden(V3, T, seed=62, dtype="bf16")
+    pos = np.concatenate([[0, 1, 4095, 4096, 32767], np.arange(T - 5) * 131 + 3])
+    slots = np.random.default_rng(4).permutation(cap)[:T]
+    ref = orc.cache_append(h, pos, W, V3)
+    m.set_cache_format(mla.CACHE_FP8)
+    try:
+        cache8 = torch.zeros(cap, mla.FP8_ROW_BYTES, dtype=torch.uint8, device="cuda:0")
+        m.cache_append(dev(h, "bf16"), dev_i64(pos), dev_i64(slots), cache8)
+        assert m.sync_status() == 0
+    finally:
+        m.set_cache_format(mla.CACHE_BF16)
+    raw = cache8.cpu().numpy()
+    untouched = np.setdiff1d(np.arange(cap), slots)
+    assert not raw[untouched].any()
+    vals, kr, s, pad = decode_rows(raw[slots])
+    assert not pad.any()
+    deq = orc.dequantize_cache_rows_fp8(vals, kr, s)
+    err = np.abs(deq - ref)
+    assert np.all(err <= _fp8_bound(ref, s)), float((err / _fp8_bound(ref, s)).max())
+    # the rows the bf16 format writes for the same call, put through the library's own quantizer,
+    # are the same bytes (the FP8 append quantizes the very rows the bf16 append would store)
+    cache16 = torch.zeros(cap, 576, dtype=torch.bfloat16, device="cuda:0")
+    m.cache_append(dev(h, "bf16"), dev_i64(pos), dev_i64(slots), cache16)
+    q = m.quantize_fp8(cache16[dev_i64(slots)].contiguous())
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), raw[slots])
