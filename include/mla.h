@@ -139,9 +139,10 @@ typedef enum {
  *   bytes [640, 644)  s as fp32: s = max(amax(c^KV) / 448, amax(k^R) / 32768), or 1 for a zero row
  *   bytes [644, 656)  zero
  * A row stands for [codes * s | (k^R / s) * s]; every division is an IEEE fp32 division. With FP8 the
- * cache argument of mla_cache_append points to such rows (capacity rows of 656 bytes); the decode,
- * prefill and attention calls and mla_cache_append_noalloc return MLA_ERR_UNSUPPORTED for now.
- * BF16 handles only (MLA_ERR_UNSUPPORTED otherwise). Host-only. */
+ * cache arguments of mla_cache_append, mla_decode and mla_attn_decode_latent point to such rows
+ * (capacity rows of 656 bytes), and the decode attends over the rows they stand for; the prefill
+ * calls and mla_cache_append_noalloc return MLA_ERR_UNSUPPORTED. BF16 handles only
+ * (MLA_ERR_UNSUPPORTED otherwise). Host-only. */
 mla_status_t mla_set_cache_format(mla_handle_t *h, mla_cache_format_t format);
 
 /* Converts n bf16 cache rows [n, 576] to FP8 rows [n, 656 bytes] (the layout above), for example to

@@ -461,7 +461,6 @@ mla_status_t mla_attn_decode_latent(mla_handle_t* h, const void* q_abs, const vo
   if (!h || !q_abs || !q_rope || !cu_seqlens || !cache || !o_lat || !lse || B <= 0 || capacity <= 0)
     return MLA_ERR_INVALID_ARG;
   if (Tq != 1 && Tq != 2) return MLA_ERR_INVALID_ARG;
-  if (h->opts.cache_fp8) return MLA_ERR_UNSUPPORTED;   // FP8 latent core not built yet
   if (!aligned16(q_abs) || !aligned16(q_rope) || !aligned16(cache) || !aligned16(o_lat) || !aligned16(lse) ||
       !aligned16(cu_seqlens) || (ws && !aligned16(ws)))
     return MLA_ERR_ALIGNMENT;
@@ -476,8 +475,8 @@ mla_status_t mla_attn_decode_latent(mla_handle_t* h, const void* q_abs, const vo
   if (tc_dims(h)) {
     // the device checks ride in the core's plan launch
     MLA_TRY(mla::tc_core_prepare(cu_seqlens, B, Tq, capacity, nullptr, w + L.tc_off, h->num_sms, h->d_err, st));
-    return cuda_status(mla::tc_core_run(q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, o_lat, true, lse,
-                                        w + L.tc_off, h->num_sms, h->d_err, st));
+    return cuda_status(mla::tc_core_run(q_abs, q_rope, B, Tq, cu_seqlens, cache, capacity, h->opts.cache_fp8 != 0,
+                                        o_lat, true, lse, w + L.tc_off, h->num_sms, h->d_err, st));
   }
   MLA_TRY(mla::check_and_positions(cu_seqlens, B, Tq, B * Tq, capacity, 0, (int64_t*)(w + L.pos_off), h->d_err,
                                    st));
@@ -578,7 +577,6 @@ mla_status_t mla_decode(mla_handle_t* h, const void* h_q, int64_t B, int32_t Tq,
                         mla_stream_t stream) {
   if (!h || !h_q || !cu_seqlens || !cache || !u_out || !ws || B <= 0 || capacity <= 0) return MLA_ERR_INVALID_ARG;
   if (Tq != 1 && Tq != 2) return MLA_ERR_INVALID_ARG;
-  if (h->opts.cache_fp8) return MLA_ERR_UNSUPPORTED;   // FP8 latent core not built yet
   if (!aligned16(h_q) || !aligned16(cache) || !aligned16(u_out) || !aligned16(ws) || !aligned16(cu_seqlens))
     return MLA_ERR_ALIGNMENT;
   Layout L = layout(h, MLA_OP_DECODE, B, Tq, 0);

@@ -68,8 +68,8 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
   }
   *reinterpret_cast<uint4*>(row + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
   const __half2 kh = __halves2half2(__float2half_rn(__fdiv_rn(k0, s)), __float2half_rn(__fdiv_rn(k1, s)));
-  *reinterpret_cast<__half2*>(row + 512 + 4 * lane) = kh;
-  if (lane == 0) *reinterpret_cast<uint4*>(row + 640) = make_uint4(__float_as_uint(s), 0u, 0u, 0u);
+  *reinterpret_cast<__half2*>(row + kFp8KrOffset + 4 * lane) = kh;
+  if (lane == 0) *reinterpret_cast<uint4*>(row + kFp8ScaleOffset) = make_uint4(__float_as_uint(s), 0u, 0u, 0u);
 }
 
 }  // namespace

@@ -22,6 +22,8 @@ size_t tc_append_scratch_bytes(const mla_dims_t& d, int64_t T, bool fp8 = false)
 // k^R / s, the fp32 scale s and 12 zero bytes.
 constexpr int kFp8RowBytes = 656;
 constexpr int kFp8RowLatent = 576;   // bf16 elements of the cache row it is made from
+constexpr int kFp8KrOffset = 512;    // byte offsets of k^R / s and of s in the row
+constexpr int kFp8ScaleOffset = 640;
 // bf16 cache rows [n][576] -> FP8 rows at out + row(r) * 656, row(r) = rowmap ? rowmap[r] : r (rows
 // mapped outside [0, limit) are skipped).
 cudaError_t fp8_quantize_rows(const void* rows, int64_t n, const int64_t* rowmap, int64_t limit, void* out,
@@ -45,9 +47,10 @@ void tc_latent_core_arm_stall();
 // the log-sum-exp merge of the partials) with the same B, tq, scratch and num_sms.
 cudaError_t tc_core_prepare(const int64_t* cu, int64_t B, int32_t tq, int64_t capacity, int64_t* pos, void* scratch,
                             int num_sms, uint32_t* err, cudaStream_t st);
+// cache_fp8: the cache rows are FP8 rows of kFp8RowBytes (e4m3 codes, f16 k^R / s, fp32 s).
 cudaError_t tc_core_run(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
-                        const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse, void* scratch,
-                        int num_sms, uint32_t* err, cudaStream_t st);
+                        const void* cache, int64_t capacity, bool cache_fp8, void* o_lat, bool o_f32, float* lse,
+                        void* scratch, int num_sms, uint32_t* err, cudaStream_t st);
 
 cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const LayerOpts& lo, const void* h_q, int64_t B,
                       int32_t tq, const int64_t* cu, const int64_t* pos, const void* cache, int64_t capacity, void* u_out,

@@ -58,6 +58,7 @@ using namespace sm100;
 constexpr int H = 128, DC = 512, DR = 64, ROW = DC + DR;
 constexpr int NK = 128;                        // keys per tile
 constexpr int kThreads = 384;
+constexpr int kConvThreads = 64;               // FP8 cache: warps 2-3 convert the codes to f16
 constexpr int kMaxPairs = 74;
 constexpr float kRescaleLog2 = 8.f;            // keep the running max until it grows by 2^8
 constexpr int kIssuers = 4;                    // TMA issuing lanes per producer warp
@@ -80,15 +81,19 @@ constexpr int V_RING = 4;                      // one tile: (N-half, key-half) =
 // Shared memory, from a 1024-byte aligned base (the same layout offsets in both CTAs for the
 // barrier block, which the value CTA's multicast commits and remote arrivals rely on).
 constexpr uint32_t OFF_BAR = 0;
-constexpr uint32_t OFF_RED = 512;              // score CTA: per-head maxima / sums swapped between halves
+constexpr uint32_t OFF_RED = 1024;             // score CTA: per-head maxima / sums swapped between halves
 constexpr uint32_t S_OFF_RING = 4096;
 constexpr uint32_t S_OFF_QR = S_OFF_RING + S_RING * BOX;
 constexpr uint32_t S_END = S_OFF_QR + QR_BYTES;
+constexpr uint32_t S_OFF_SC = S_END;           // FP8: per-key s, log2 s, 1/s of the two tiles in flight
+constexpr uint32_t SC_BYTES = 3 * NK * 4;
+constexpr uint32_t S_END8 = S_OFF_SC + 2 * SC_BYTES;
 constexpr uint32_t V_OFF_PBUF = 4096;
 constexpr uint32_t V_OFF_RING = V_OFF_PBUF + 2 * PMSG;
 constexpr uint32_t V_END = V_OFF_RING + V_RING * VGRP;
 constexpr uint32_t SMEM_BYTES = (S_END > V_END ? S_END : V_END) + 1024;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+constexpr uint32_t SMEM_BYTES8 = (S_END8 > V_END ? S_END8 : V_END) + 1024;
+static_assert(SMEM_BYTES <= 232448 && SMEM_BYTES8 <= 232448, "shared memory budget");
 static_assert(S_OFF_RING % 1024 == 0 && S_OFF_QR % 1024 == 0 && PMSG % 1024 == 0 && V_OFF_RING % 1024 == 0,
               "swizzle atom alignment");
 static_assert(OFF_RED + 3 * 2 * H * 4 <= S_OFF_RING, "reduction buffer");
@@ -111,16 +116,24 @@ enum : int {
   B_OREADY = B_PFULL + 2,             // [2] O rescaled for the tile / nothing to rescale (128)
   B_OFREE = B_OREADY + 2,             // O read out by the piece epilogue (256: both column halves)
   B_ODONE = B_OFREE + 1,              // the last P.V of a piece done (one phase per piece)
-  NBAR = B_ODONE + 1
+  // FP8 cache only
+  B_CF = B_ODONE + 1,                 // [8] code box m of a tile of parity t converted to f16: m + 4 t (64)
+  B_SCR = B_CF + 8,                   // [2] per-key scale values of the tile written (64)
+  B_SCX = B_SCR + 2,                  // [2] per-key scale values of the tile read (256 softmax threads)
+  B_VCF = B_SCX + 2,                  // [V_RING] value CTA: group converted to f16 (64)
+  NBAR = B_VCF + V_RING
 };
 static_assert(NBAR * 8 + 16 <= OFF_RED, "barrier block");
 
 struct CoreParams {
-  CUtensorMap kmap;   // cache as [capacity, ROW], box {64, 128}, 128-byte swizzle (score CTA)
-  CUtensorMap vmap;   // cache as [capacity, ROW], box {64, 64}, 128-byte swizzle (value CTA)
+  // bf16 cache: [capacity, ROW] bf16, kmap box {64, 128}, vmap box {64, 64};
+  // FP8 cache: [capacity, 656] bytes, kmap box {128, 128}, vmap box {128, 64}; 128-byte swizzle
+  CUtensorMap kmap;   // score CTA
+  CUtensorMap vmap;   // value CTA
   CUtensorMap qmap;   // q~ as [T * H, DC], box {64, 128}, 128-byte swizzle
   CUtensorMap qrmap;  // q^R as [T * H, DR], box {64, 128}, 128-byte swizzle
   const int64_t* cu;
+  const uint8_t* cache8;        // FP8: the cache rows (the scale of row r at byte 656 r + 640)
   const int32_t* tile_start;    // [B+1]: first global tile of each sequence
   const int32_t* slot_base;     // [B+1]: first partial slot of each sequence
   const int4* pinfo;            // [pairs]: tile range [x, y), first sequence z, its partial slot w
@@ -175,6 +188,42 @@ struct SegWalk {
   }
 };
 
+// FP8 cache: row r of a [rows x 128 codes] box (128-byte swizzle, the layout TMA writes) becomes
+// the 128 f16 values of those codes: columns 0-63 go to row r of box `lo`, columns 64-127 over the
+// codes' own row (both 128-byte swizzled K-major rows of 64 f16, the layout the MMA reads). The
+// thread reads its whole row before writing, and rows are 128-byte lines of their own, so the
+// in-place half is safe. `zero` writes zeros instead (cache rows that belong to no sequence).
+__device__ __forceinline__ void convert_code_row(uint8_t* codes, uint8_t* lo, int r, bool zero) {
+  uint8_t* crow = codes + r * 128;
+  uint8_t* lrow = lo + r * 128;
+  const int sw = r & 7;
+  uint4 in[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) in[c] = *reinterpret_cast<const uint4*>(crow + ((c ^ sw) << 4));
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    // codes 16 c .. 16 c + 15: f16 columns 16 c .. 16 c + 15, output chunks 2 c and 2 c + 1
+    uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
+    if (!zero) {
+      o0 = make_uint4(e4m3x2_to_f16x2(in[c].x & 0xffffu), e4m3x2_to_f16x2(in[c].x >> 16),
+                      e4m3x2_to_f16x2(in[c].y & 0xffffu), e4m3x2_to_f16x2(in[c].y >> 16));
+      o1 = make_uint4(e4m3x2_to_f16x2(in[c].z & 0xffffu), e4m3x2_to_f16x2(in[c].z >> 16),
+                      e4m3x2_to_f16x2(in[c].w & 0xffffu), e4m3x2_to_f16x2(in[c].w >> 16));
+    }
+    uint8_t* dst = c < 4 ? lrow : crow;
+    const int q0 = (2 * c) & 7;
+    *reinterpret_cast<uint4*>(dst + ((q0 ^ sw) << 4)) = o0;
+    *reinterpret_cast<uint4*>(dst + (((q0 + 1) ^ sw) << 4)) = o1;
+  }
+}
+
+// F8 = the FP8 cache (e4m3 codes with one fp32 scale per row, k^R / s in f16). The codes are
+// converted to f16 in shared memory (exactly) and the MMAs run in f16: q~ and q^R of a head are
+// scaled by one power of two into f16's range, and the score of key j is s_j times the score over
+// (codes_j, k^R_j / s_j). The softmax tracks w_j = log2(p_j s_j) (p_j the unnormalised softmax
+// weight), so that P'_j = 2^(w_j - m) = p_j s_j 2^-m is the f16 weight of the codes in P'.C, and
+// the sum l = sum_j P'_j / s_j = sum_j p_j 2^-m shares the reference m.
+template <bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     latent_core_kernel(const __grid_constant__ CoreParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -198,6 +247,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       else if (i >= B_TMAX && i < B_TMAX + 4) cnt = 64;
       else if (i == B_OREADY || i == B_OREADY + 1) cnt = 128;
       else if (i == B_OFREE) cnt = 256;
+      else if (i >= B_CF && i < B_SCX) cnt = kConvThreads;
+      else if (i == B_SCX || i == B_SCX + 1) cnt = 256;
+      else if (i >= B_VCF && i < B_VCF + V_RING) cnt = kConvThreads;
       mbar_init(bar(i), cnt);
     }
     if (r == 1) {
@@ -240,12 +292,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane < kIssuers) {
         int n = 0, last = -1;
         const bool stall = p.stall && k == 0 && t_begin == 0 && t_end > 0;
+        // map == nullptr (FP8): no load; the free slot is handed to the code converters, which write
+        // the low half of a code box's f16 columns into it
         auto issue = [&](const CUtensorMap* map, int x, int y) -> bool {
           const int cur = n++;
           if ((cur & (kIssuers - 1)) != lane) return true;
           const int slot = cur % S_RING;
           if (!wait_bar(bar(B_SEMPTY + slot), ((cur / S_RING) & 1) ^ 1, lim)) return false;
           if (stall && cur == 0) return true;     // test hook: entry 0 never arrives
+          if (map == nullptr) {
+            mbar_arrive(bar(B_SFULL + slot));
+            return true;
+          }
           mbar_expect_tx(bar(B_SFULL + slot), BOX);
           tma_load_2d(sbase + S_OFF_RING + slot * BOX, map, x, y, bar(B_SFULL + slot));
           last = cur;
@@ -259,7 +317,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (ok) ok = issue(&p.qrmap, 0, qrow);
           for (int32_t xt = sw.x; ok && xt < sw.seg_end(); ++xt) {
             const int32_t row0 = row_base + (xt - ts_b) * NK;
-            for (int c = 0; ok && c < S_BOXES; ++c) ok = issue(&p.kmap, c < 8 ? 64 * c : DC, row0);
+            if (F8) {
+              // entries 2m, 2m + 1: code box m (columns 128 m .. 128 m + 127) lands in entry 2m + 1's
+              // slot; entry 8: k^R / s (f16, bytes 512 .. 639 of the row)
+              for (int c = 0; ok && c < S_BOXES; ++c)
+                ok = c == 8 ? issue(&p.kmap, DC, row0) : (c & 1) ? issue(&p.kmap, 128 * (c >> 1), row0)
+                                                                  : issue(nullptr, 0, 0);
+            } else {
+              for (int c = 0; ok && c < S_BOXES; ++c) ok = issue(&p.kmap, c < 8 ? 64 * c : DC, row0);
+            }
           }
         }
         if (!ok) {
@@ -273,7 +339,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       // ------------------------------------------------ MMA issuer: S = [q~ | q^R] [c | k^R]^T
       if (lane == 0) {
-        constexpr uint32_t idesc = idesc_bf16(128, NK, 0, 0);
+        constexpr uint32_t idesc = F8 ? idesc_f16(128, NK, 0, 0) : idesc_bf16(128, NK, 0, 0);
         const uint64_t qr_desc = sw128_desc(sbase + S_OFF_QR, 0, 1024);
         int j = 0, g = 0, n = 0;
         for (; ok && w.valid(); w.next(), ++g) {
@@ -288,7 +354,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t d = tmem + 256 + 128 * sb;
             for (int c = 0; c < S_BOXES; ++c, ++n) {
               const int slot = n % S_RING;
-              if (!wait_bar(bar(B_SFULL + slot), (n / S_RING) & 1, lim)) { ok = false; break; }
+              if (F8 && c < 8) {
+                // both f16 halves of code box c / 2 written by the converters
+                if ((c & 1) == 0 && !wait_bar(bar(B_CF + (c >> 1) + 4 * sb), (j >> 1) & 1, lim)) { ok = false; break; }
+              } else if (!wait_bar(bar(B_SFULL + slot), (n / S_RING) & 1, lim)) {
+                ok = false;
+                break;
+              }
               tc_fence_after();
               // descriptors advance by (byte offset >> 4) in the start-address field: 32 bytes per
               // K step of 16 bf16 inside the 128-byte swizzled row
@@ -311,6 +383,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
       }
+    } else if (F8 && (warp == 2 || warp == 3)) {
+      // ------------------------------------------------ FP8 code converters (64 threads, key rows ct, ct + 64)
+      // Per tile: the scales of its two keys (s, log2 s, 1/s into the tile's scale buffer; a row past
+      // the last sequence gets s = 0: weight 0), then the 4 code boxes of the tile, its two rows of
+      // each, into f16 in place (the low half into the slot of the box's even entry).
+      const int ct = threadIdx.x - 64;
+      float* scb = reinterpret_cast<float*>(smem + S_OFF_SC);
+      const int64_t total_rows = p.cu[p.B];
+      int j = 0, n = 0;
+      for (; ok && w.valid(); w.next()) {
+        n += 9;                                      // the piece's q~ / q^R entries
+        const int b = w.b;
+        const int32_t ts_b = p.tile_start[b];
+        const int64_t row_base = p.cu[b];
+        const int32_t send = w.seg_end();
+        for (int32_t xt = w.x; xt < send; ++xt, ++j, n += S_BOXES) {
+          const int sb = j & 1;
+          const int64_t row = row_base + (int64_t)(xt - ts_b) * NK + ct;
+          float sv[2];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int64_t r2 = row + 64 * h2;
+            sv[h2] = r2 < total_rows ? *reinterpret_cast<const float*>(p.cache8 + r2 * kFp8RowBytes + kFp8ScaleOffset) : 0.f;
+            if (!(sv[h2] > 0.f && sv[h2] < INFINITY)) sv[h2] = 0.f;
+          }
+          if (!wait_bar(bar(B_SCX + sb), ((j >> 1) & 1) ^ 1, lim)) { ok = false; break; }
+          float* sc = scb + sb * (3 * NK);
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int key = ct + 64 * h2;
+            sc[key] = sv[h2];
+            sc[NK + key] = sv[h2] > 0.f ? log2f(sv[h2]) : -INFINITY;
+            sc[2 * NK + key] = sv[h2] > 0.f ? 1.f / sv[h2] : 0.f;
+          }
+          mbar_arrive(bar(B_SCR + sb));
+          for (int m = 0; m < 4; ++m) {
+            const int e0 = n + 2 * m, e1 = e0 + 1;
+            const int s0 = e0 % S_RING, s1 = e1 % S_RING;
+            if (!wait_bar(bar(B_SFULL + s0), (e0 / S_RING) & 1, lim) ||
+                !wait_bar(bar(B_SFULL + s1), (e1 / S_RING) & 1, lim)) {
+              ok = false;
+              break;
+            }
+            convert_code_row(smem + S_OFF_RING + s1 * BOX, smem + S_OFF_RING + s0 * BOX, ct, false);
+            convert_code_row(smem + S_OFF_RING + s1 * BOX, smem + S_OFF_RING + s0 * BOX, ct + 64, false);
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_CF + m + 4 * sb));
+          }
+          if (!ok) break;
+        }
+      }
+      if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
     } else if (warp >= 4) {
       // ------------------------------------------------ softmax: 8 warps, two per TMEM lane quarter
       // Half 0 (warps 4-7) takes keys [0, 64) of every tile, half 1 (warps 8-11) keys [64, 128),
@@ -322,7 +446,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t tmax_bar = bar(B_TMAX + quarter);
       float* redbuf = reinterpret_cast<float*>(smem + OFF_RED);   // [3 slots][2 halves][128]
       const float c2 = p.scale_log2;
-      const float thr_raw = kRescaleLog2 / c2;
+      // bf16: the running max is in raw score units and P = 2^((s - m) c2); FP8: the softmax works on
+      // w = log2(p s) directly (c2 and the head's q scale folded into kq), P' = 2^(w - m)
+      const float cw = F8 ? 1.f : c2;
+      const float thr_raw = kRescaleLog2 / cw;
+      float kq = c2;
+      const float* scb = reinterpret_cast<const float*>(smem + S_OFF_SC);
       const uint32_t pbuf_peer = map_peer(sbase + V_OFF_PBUF, 1);
       const uint32_t pfull_peer = map_peer(bar(B_PFULL), 1);
       auto wait_u = [&](uint32_t b, uint32_t par) { return __all_sync(0xffffffffu, wait_bar(b, par, lim)) != 0; };
@@ -347,24 +476,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         nq += 9;
         bool okq = wait_u(bar(B_QEMPTY), (gq & 1) ^ 1);
         tc_fence_after();
-        for (int c = 4 * half; okq && c < 4 * half + 4; ++c) {
-          const int e = n0 + c, slot = e % S_RING;
-          okq = wait_u(bar(B_SFULL + slot), (e / S_RING) & 1);
-          if (!okq) break;
-          const uint8_t* src = smem + S_OFF_RING + slot * BOX + i * 128;
-          uint32_t v[32];
+        if constexpr (F8) {
+          // f16 operands: q~ and q^R of head i scaled by fq = 2^(14 - e), e the exponent of the row's
+          // largest magnitude, so that the row's values are f16 normals up to 2^15 (exact for bf16
+          // values down to 2^-14 of the largest); the scores are multiplied back by kq = c2 / fq
+          for (int c = 0; okq && c < 9; ++c) okq = wait_u(bar(B_SFULL + (n0 + c) % S_RING), ((n0 + c) / S_RING) & 1);
+          float amax = 0.f;
+          if (okq) {
+            for (int c = 0; c < 9; ++c) {
+              const uint8_t* src = smem + S_OFF_RING + ((n0 + c) % S_RING) * BOX + i * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint4 u = *reinterpret_cast<const uint4*>(src + ((q ^ (i & 7)) << 4));
-            v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
+              for (int q = 0; q < 8; ++q) {
+                const uint4 u = *reinterpret_cast<const uint4*>(src + 16 * q);
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(u.x)), fabsf(bf16_hi(u.x))),
+                                         fmaxf(fabsf(bf16_lo(u.y)), fabsf(bf16_hi(u.y)))));
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(u.z)), fabsf(bf16_hi(u.z))),
+                                         fmaxf(fabsf(bf16_lo(u.w)), fabsf(bf16_hi(u.w)))));
+              }
+            }
           }
-          tmem_st32(trow + 32 * c, v);
-        }
-        tmem_wait_st();
-        if (bar_sync_or(1, 256, !okq)) return false;   // all 8 q~ boxes read (or a wait gave up)
-        if (threadIdx.x == 128)
-          for (int c = 0; c < 8; ++c) mbar_arrive(bar(B_SEMPTY + (n0 + c) % S_RING));
-        {
+          int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xffu) - 127 : 0;
+          e = max(-100, min(100, e));
+          const float fq = __uint_as_float((uint32_t)(127 + 14 - e) << 23);
+          kq = c2 * __uint_as_float((uint32_t)(127 - 14 + e) << 23);
+          if (okq) {
+            for (int c = 4 * half; c < 4 * half + 4; ++c) {
+              const uint8_t* src = smem + S_OFF_RING + ((n0 + c) % S_RING) * BOX + i * 128;
+              uint32_t v[32];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const uint4 u = *reinterpret_cast<const uint4*>(src + ((q ^ (i & 7)) << 4));
+                v[4 * q] = pack_f16(bf16_lo(u.x) * fq, bf16_hi(u.x) * fq);
+                v[4 * q + 1] = pack_f16(bf16_lo(u.y) * fq, bf16_hi(u.y) * fq);
+                v[4 * q + 2] = pack_f16(bf16_lo(u.z) * fq, bf16_hi(u.z) * fq);
+                v[4 * q + 3] = pack_f16(bf16_lo(u.w) * fq, bf16_hi(u.w) * fq);
+              }
+              tmem_st32(trow + 32 * c, v);
+            }
+            tmem_wait_st();
+            const uint8_t* src = smem + S_OFF_RING + ((n0 + 8) % S_RING) * BOX + i * 128;
+            uint8_t* dst = smem + S_OFF_QR + i * 128;
+#pragma unroll
+            for (int c = 4 * half; c < 4 * half + 4; ++c) {
+              const int o = (c ^ (i & 7)) << 4;
+              const uint4 u = *reinterpret_cast<const uint4*>(src + o);
+              *reinterpret_cast<uint4*>(dst + o) =
+                  make_uint4(pack_f16(bf16_lo(u.x) * fq, bf16_hi(u.x) * fq), pack_f16(bf16_lo(u.y) * fq, bf16_hi(u.y) * fq),
+                             pack_f16(bf16_lo(u.z) * fq, bf16_hi(u.z) * fq), pack_f16(bf16_lo(u.w) * fq, bf16_hi(u.w) * fq));
+            }
+            fence_proxy_async_smem();
+          }
+          if (bar_sync_or(1, 256, !okq)) return false;   // all 9 entries read (or a wait gave up)
+          if (threadIdx.x == 128)
+            for (int c = 0; c < 9; ++c) mbar_arrive(bar(B_SEMPTY + (n0 + c) % S_RING));
+        } else {
+          for (int c = 4 * half; okq && c < 4 * half + 4; ++c) {
+            const int e = n0 + c, slot = e % S_RING;
+            okq = wait_u(bar(B_SFULL + slot), (e / S_RING) & 1);
+            if (!okq) break;
+            const uint8_t* src = smem + S_OFF_RING + slot * BOX + i * 128;
+            uint32_t v[32];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint4 u = *reinterpret_cast<const uint4*>(src + ((q ^ (i & 7)) << 4));
+              v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
+            }
+            tmem_st32(trow + 32 * c, v);
+          }
+          tmem_wait_st();
+          if (bar_sync_or(1, 256, !okq)) return false;   // all 8 q~ boxes read (or a wait gave up)
+          if (threadIdx.x == 128)
+            for (int c = 0; c < 8; ++c) mbar_arrive(bar(B_SEMPTY + (n0 + c) % S_RING));
           const int e = n0 + 8, slot = e % S_RING;
           okq = wait_u(bar(B_SFULL + slot), (e / S_RING) & 1);
           if (okq) {
@@ -405,6 +587,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           tc_fence_before();
           mbar_arrive(bar(B_SCE + sb));
+          const float* sc = scb + sb * (3 * NK) + 64 * half;   // FP8: this half's keys' s, log2 s, 1/s
+          if constexpr (F8) {
+            // w_j = s_j S'_j kq + log2 s_j (S' the score over the codes and k^R / s in f16 units)
+            if (!wait_u(bar(B_SCR + sb), (j >> 1) & 1)) { ok = false; break; }
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              const float2 sv = *reinterpret_cast<const float2*>(sc + c);
+              const float2 lv = *reinterpret_cast<const float2*>(sc + NK + c);
+              s[c] = fmaf(s[c] * sv.x, kq, lv.x);
+              s[c + 1] = fmaf(s[c + 1] * sv.y, kq, lv.y);
+            }
+          }
           const int64_t key0 = (int64_t)(xt - ts_b) * NK + 64 * half;
           const int nvis = (int)max((int64_t)0, min((int64_t)64, vis - key0));
           if (nvis < 64) {
@@ -424,23 +618,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // lazy rescale of the running max: the same decision in both halves (same tmax, m_ref)
           float alpha = 1.f;
           if (tmax > -INFINITY && (m_ref == -INFINITY || tmax > m_ref + thr_raw)) {
-            alpha = m_ref == -INFINITY ? 0.f : ex2_approx((m_ref - tmax) * c2);
+            alpha = m_ref == -INFINITY ? 0.f : ex2_approx((m_ref - tmax) * cw);
             l *= alpha;
             m_ref = tmax;
           }
-          // P = 2^((s - m_ref) c2) in bf16, packed in pairs
+          // P = 2^((s - m_ref) c2) in bf16 (FP8: P' = 2^(w - m_ref) in f16, l sums P' / s), packed in pairs
           uint32_t pk[32];
           if (m_ref > -INFINITY) {
-            const uint64_t cc = f2_pack(c2, c2), off = f2_pack(-m_ref * c2, -m_ref * c2);
+            const uint64_t cc = f2_pack(cw, cw), off = f2_pack(-m_ref * cw, -m_ref * cw);
             uint64_t acc2[8];
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               float a0, a1;
               f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), cc, off), a0, a1);
               const float e0 = ex2_approx(a0), e1 = ex2_approx(a1);
-              pk[c] = pack_bf16(e0, e1);
-              if (c < 8) acc2[c] = f2_pack(e0, e1);
-              else acc2[c & 7] = f2_add(acc2[c & 7], f2_pack(e0, e1));
+              uint64_t le = f2_pack(e0, e1);
+              if constexpr (F8) {
+                pk[c] = pack_f16(e0, e1);
+                const float2 iv = *reinterpret_cast<const float2*>(sc + 2 * NK + 2 * c);
+                le = f2_mul(le, f2_pack(iv.x, iv.y));
+              } else {
+                pk[c] = pack_bf16(e0, e1);
+              }
+              if (c < 8) acc2[c] = le;
+              else acc2[c & 7] = f2_add(acc2[c & 7], le);
             }
 #pragma unroll
             for (int w2 = 4; w2 > 0; w2 >>= 1)
@@ -453,6 +654,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c) pk[c] = 0u;
           }
+          if (F8) mbar_arrive(bar(B_SCX + sb));      // done with the tile's scale values
           // the value CTA's P buffer sb: its P.V of tile j - 2 is done; this half's 64 keys of row i
           // go straight into it (the same 128-byte swizzle the MMA descriptor reads), alpha too
           if (!wait_u(bar(B_PVD + sb), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
@@ -470,8 +672,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const float lt = l + lp;
             if (half == 0) {
               const int64_t row = ((int64_t)k * p.s_max + piece_slot(b)) * H + i;
-              p.part_lse[row] = lt > 0.f ? (m_ref * c2 + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-              p.part_m[row] = lt > 0.f ? m_ref * c2 * 0.69314718055994531f : -INFINITY;
+              p.part_lse[row] = lt > 0.f ? (m_ref * cw + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+              p.part_m[row] = lt > 0.f ? m_ref * cw * 0.69314718055994531f : -INFINITY;
             }
           }
         }
@@ -502,12 +704,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               if ((n & (kIssuers - 1)) != lane) continue;
               const int g = n % V_RING;
               if (!wait_bar(bar(B_GEMPTY + g), ((n / V_RING) & 1) ^ 1, lim)) { ok = false; break; }
-              mbar_expect_tx(bar(B_GFULL + g), VGRP);
               const int nh = s & 1, kh = s >> 1;
               const uint32_t dst = sbase + V_OFF_RING + g * VGRP;
+              if (F8) {
+                // the group's 256 columns as two code boxes of [64 keys x 128 codes], into boxes 1 and 3
+                // (the converters spread them over all four as f16)
+                mbar_expect_tx(bar(B_GFULL + g), VGRP / 2);
+                tma_load_2d(dst + VBOX, &p.vmap, 256 * nh, row0 + 64 * kh, bar(B_GFULL + g));
+                tma_load_2d(dst + 3 * VBOX, &p.vmap, 256 * nh + 128, row0 + 64 * kh, bar(B_GFULL + g));
+              } else {
+                mbar_expect_tx(bar(B_GFULL + g), VGRP);
 #pragma unroll
-              for (int bx = 0; bx < 4; ++bx)
-                tma_load_2d(dst + bx * VBOX, &p.vmap, 256 * nh + 64 * bx, row0 + 64 * kh, bar(B_GFULL + g));
+                for (int bx = 0; bx < 4; ++bx)
+                  tma_load_2d(dst + bx * VBOX, &p.vmap, 256 * nh + 64 * bx, row0 + 64 * kh, bar(B_GFULL + g));
+              }
               last = n;
             }
           }
@@ -521,7 +731,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       // ------------------------------------------------ MMA issuer: O += P . C
       if (lane == 0) {
-        constexpr uint32_t idesc = idesc_bf16(128, 256, 0, 1);
+        constexpr uint32_t idesc = F8 ? idesc_f16(128, 256, 0, 1) : idesc_bf16(128, 256, 0, 1);
         int j = 0, g = 0, n = 0;
         for (; ok && w.valid(); w.next(), ++g) {
           const int32_t send = w.seg_end();
@@ -539,7 +749,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t pmsg = sbase + V_OFF_PBUF + pb * PMSG;
             for (int s = 0; s < 4; ++s, ++n) {
               const int gi = n % V_RING;
-              if (!wait_bar(bar(B_GFULL + gi), (n / V_RING) & 1, lim)) { ok = false; break; }
+              if (!wait_bar(bar((F8 ? B_VCF : B_GFULL) + gi), (n / V_RING) & 1, lim)) { ok = false; break; }
               tc_fence_after();
               const int nh = s & 1, kh = s >> 1;
               const uint64_t adesc = sw128_desc(pmsg + 16384 * kh, 0, 1024);
@@ -559,6 +769,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
       }
+    } else if (F8 && (warp == 2 || warp == 3)) {
+      // ------------------------------------------------ FP8 code converters (64 threads)
+      // Thread rr converts row rr of both code boxes of every group into f16 (zeros for cache rows past
+      // the last sequence, which may hold anything).
+      const int rr = threadIdx.x - 64;
+      const int64_t total_rows = p.cu[p.B];
+      int n = 0;
+      for (; ok && w.valid(); w.next()) {
+        const int32_t ts_b = p.tile_start[w.b];
+        const int64_t row_base = p.cu[w.b];
+        const int32_t send = w.seg_end();
+        for (int32_t xt = w.x; ok && xt < send; ++xt) {
+          const int64_t row0 = row_base + (int64_t)(xt - ts_b) * NK;
+          for (int s = 0; s < 4; ++s, ++n) {
+            const int gi = n % V_RING, kh = s >> 1;
+            if (!wait_bar(bar(B_GFULL + gi), (n / V_RING) & 1, lim)) { ok = false; break; }
+            uint8_t* grp = smem + V_OFF_RING + gi * VGRP;
+            const bool past = row0 + 64 * kh + rr >= total_rows;
+            convert_code_row(grp + VBOX, grp, rr, past);
+            convert_code_row(grp + 3 * VBOX, grp + 2 * VBOX, rr, past);
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_VCF + gi));
+          }
+        }
+      }
+      if (!ok) flag_error(p.err, DEVERR_TIMEOUT);
     } else if (warp >= 4) {
       // ------------------------------------------------ rescale + piece epilogue (thread = head = TMEM lane)
       // Warps 4-7 rescale O when the running max moved and zero cache rows past the last sequence
@@ -625,7 +861,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // cache rows past the last sequence may hold anything (even NaN): zero them in this tile's
           // groups before P.V reads them (their P is zero, but 0 * NaN is not)
           const int64_t row0 = row_base + (int64_t)(xt - ts_b) * NK;
-          if (row0 + NK > total_rows) {
+          if (!F8 && row0 + NK > total_rows) {   // (FP8: the converters write those rows as zeros)
             const int nrows = (int)max((int64_t)0, total_rows - row0);
             for (int s2 = 0; s2 < 4; ++s2) {
               const int gi = (n + s2) % V_RING;
@@ -914,16 +1150,17 @@ CoreScratch carve(void* scratch, int64_t B, int32_t tq) {
   return c;
 }
 
+template <bool F8>
 cudaError_t launch_core(const CoreParams& p, dim3 grid, cudaStream_t st) {
   static bool configured = false;
+  constexpr uint32_t smem = F8 ? SMEM_BYTES8 : SMEM_BYTES;
   if (!configured) {
-    cudaError_t e =
-        cudaFuncSetAttribute(latent_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(latent_core_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   timer_begin(TIMED_LATENT_CORE, st);
-  latent_core_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p);
+  latent_core_kernel<F8><<<grid, kThreads, smem, st>>>(p);
   timer_end(TIMED_LATENT_CORE, st);
   note_launch();
   return cudaGetLastError();
@@ -963,8 +1200,8 @@ cudaError_t tc_core_prepare(const int64_t* cu, int64_t B, int32_t tq, int64_t ca
 }
 
 cudaError_t tc_core_run(const void* q_abs, const void* q_rope, int64_t B, int32_t tq, const int64_t* cu,
-                        const void* cache, int64_t capacity, void* o_lat, bool o_f32, float* lse, void* scratch,
-                        int num_sms, uint32_t* err, cudaStream_t st) {
+                        const void* cache, int64_t capacity, bool cache_fp8, void* o_lat, bool o_f32, float* lse,
+                        void* scratch, int num_sms, uint32_t* err, cudaStream_t st) {
   if (B <= 0) return cudaSuccess;
   if (B > (int64_t)1 << 20 || tq < 1 || tq > kMaxPairs || capacity > INT32_MAX || B * tq * H > INT32_MAX)
     return cudaErrorInvalidValue;
@@ -974,8 +1211,14 @@ cudaError_t tc_core_run(const void* q_abs, const void* q_rope, int64_t B, int32_
   cudaError_t e;
   CoreParams p;
   memset(&p, 0, sizeof(p));
-  if ((e = make_tmap_bf16(&p.kmap, cache, ROW, capacity, ROW, 64, NK)) != cudaSuccess) return e;
-  if ((e = make_tmap_bf16(&p.vmap, cache, ROW, capacity, ROW, 64, 64)) != cudaSuccess) return e;
+  if (cache_fp8) {
+    if ((e = make_tmap_u8(&p.kmap, cache, kFp8RowBytes, capacity, kFp8RowBytes, 128, NK)) != cudaSuccess) return e;
+    if ((e = make_tmap_u8(&p.vmap, cache, kFp8RowBytes, capacity, kFp8RowBytes, 128, 64)) != cudaSuccess) return e;
+    p.cache8 = reinterpret_cast<const uint8_t*>(cache);
+  } else {
+    if ((e = make_tmap_bf16(&p.kmap, cache, ROW, capacity, ROW, 64, NK)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&p.vmap, cache, ROW, capacity, ROW, 64, 64)) != cudaSuccess) return e;
+  }
   if ((e = make_tmap_bf16(&p.qmap, q_abs, DC, T * H, DC, 64, H)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&p.qrmap, q_rope, DR, T * H, DR, 64, H)) != cudaSuccess) return e;
   p.cu = cu;
@@ -998,7 +1241,7 @@ cudaError_t tc_core_run(const void* q_abs, const void* q_rope, int64_t B, int32_
   }
   p.err = err;
   dim3 grid((unsigned)(2 * pairs), (unsigned)tq);
-  e = launch_core(p, grid, st);
+  e = cache_fp8 ? launch_core<true>(p, grid, st) : launch_core<false>(p, grid, st);
   if (e != cudaSuccess) return e;
   dim3 cg((unsigned)T, (unsigned)(H / kCombHeads), (unsigned)(DC / kCombCols));
   if (o_f32) combine_kernel<true><<<cg, 256, 0, st>>>(c.sb, tq, c.s_max, c.part_o, c.part_lse, c.part_m, o_lat, lse);

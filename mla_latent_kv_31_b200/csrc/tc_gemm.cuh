@@ -69,6 +69,11 @@ size_t tc_gemm_partial_bytes(int64_t T, int64_t f_tiles, int64_t f_total, int64_
 cudaError_t make_tmap_bf16(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, int64_t ld, int box_inner,
                            int box_outer, int swizzle_bytes = 128);
 
+// 2-D byte TMA map over a row-major [outer, inner] byte matrix (row stride ld bytes, a multiple of
+// 16), box {box_inner <= 128, box_outer}, 128-byte swizzle, zero fill out of bounds.
+cudaError_t make_tmap_u8(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, int64_t ld, int box_inner,
+                         int box_outer);
+
 cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st);
 
 }  // namespace mla

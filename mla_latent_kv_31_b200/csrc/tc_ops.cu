@@ -161,7 +161,8 @@ cudaError_t tc_decode(const mla_dims_t& d, const mla_weights_t& w, const LayerOp
     a.batch = d.n_h; a.w_row_z = d.d_h; a.x_col_z = d.d_h;
     if ((e = tc_gemm(a, st)) != cudaSuccess) return e;
   }
-  e = tc_core_run(qabs, qr, B, tq, cu, cache, capacity, olat, false, lse, core_scratch, num_sms, err, st);
+  e = tc_core_run(qabs, qr, B, tq, cu, cache, capacity, lo.cache_fp8 != 0, olat, false, lse, core_scratch, num_sms,
+                  err, st);
   if (e != cudaSuccess) return e;
   // o_i = W_i^UV o^lat_i for every head i, in the same token chunks.
   for (int64_t t0 = 0; t0 < T; t0 += kSwapMaxTokens) {

@@ -6,7 +6,7 @@ f16 k^R / s [512, 640), fp32 s [640, 644), zero [644, 656)."""
 import numpy as np
 import pytest
 
-from mla_testlib import dev, dev_i64, host, make_module, mla, orc, synth
+from mla_testlib import TOL, dev, dev_i64, host, make_module, mla, orc, rel, synth
 
 pytestmark = pytest.mark.gpu
 
@@ -120,3 +120,136 @@ def test_cache_append_writes_fp8_rows(v3, T, cap):
     q = m.quantize_fp8(cache16[dev_i64(slots)].contiguous())
     torch.cuda.synchronize()
     assert np.array_equal(q.cpu().numpy(), raw[slots])
+
+
+# ---------------------------------------------------------------------------
+# Decode over an FP8 cache: the rows the oracle quantized, packed into the 656-byte layout, against
+# the oracle's attention over the rows they stand for (codes * s | (k^R / s) * s)
+# ---------------------------------------------------------------------------
+def encode_rows(codes, kr, s) -> np.ndarray:
+    """FP8 rows [n, 656] from the oracle's (e4m3 values, f16 k^R / s, s)."""
+    codes = np.asarray(codes, dtype=np.float64)
+    mag = np.abs(codes)
+    idx = np.searchsorted(E4M3, mag)
+    assert np.all(E4M3[np.minimum(idx, len(E4M3) - 1)] == mag), "not an e4m3 value"
+    byte = idx.astype(np.uint8) | np.where(np.signbit(codes), 0x80, 0).astype(np.uint8)
+    n = codes.shape[0]
+    out = np.zeros((n, mla.FP8_ROW_BYTES), dtype=np.uint8)
+    out[:, :512] = byte
+    out[:, 512:640] = np.ascontiguousarray(np.asarray(kr, dtype=np.float16)).view(np.uint8)
+    out[:, 640:644] = np.ascontiguousarray(np.asarray(s, dtype=np.float32)[:, None]).view(np.uint8)
+    return out
+
+
+def fp8_cache(rows_bf16):
+    """(FP8 bytes, the float64 rows they stand for) of bf16 cache rows, by the oracle's quantizer."""
+    codes, kr, s = orc.quantize_cache_rows_fp8(rows_bf16, V3)
+    return encode_rows(codes, kr, s), orc.dequantize_cache_rows_fp8(codes, kr, s)
+
+
+def test_encode_rows_round_trips_through_decode_rows():
+    rows = stress_rows(50, seed=70)
+    raw, deq = fp8_cache(rows)
+    vals, kr, s, pad = decode_rows(raw)
+    assert np.array_equal(orc.dequantize_cache_rows_fp8(vals, kr, s), deq) and not pad.any()
+
+
+def _core(m, q_abs, q_rope, B, tq, cu, raw):
+    import torch
+    m.set_cache_format(mla.CACHE_FP8)
+    try:
+        cache = torch.from_numpy(raw).to("cuda:0")
+        o_lat, lse = m.attn_decode_latent(dev(q_abs, "bf16"), dev(q_rope, "bf16"), B, tq, dev_i64(cu), cache)
+        assert m.sync_status() == 0, hex(mla.mla_device_error_bits(m.handle))
+    finally:
+        m.set_cache_format(mla.CACHE_BF16)
+    return host(o_lat), host(lse)
+
+
+@pytest.mark.parametrize("tq,lens", [(1, [1, 63, 64, 65, 129, 1000, 4097]), (2, [2, 63, 64, 65, 129, 1000, 4097]),
+                                     (1, [1, 40, 100]), (2, [33, 2, 97])])
+def test_fp8_attn_core_ragged(v3, tq, lens):
+    m, _ = v3
+    lens = np.array(lens)
+    cu = synth.cu_seqlens(lens)
+    B, T = len(lens), len(lens) * tq
+    raw, deq = fp8_cache(synth.latent_cache(V3, int(cu[-1]), seed=71 + tq, dtype="bf16"))
+    q_abs = synth.normal(72, 20, (T, V3.n_h, V3.d_c), std=0.5, dtype="bf16")
+    q_rope = synth.normal(72, 21, (T, V3.n_h, V3.d_r), std=1.0, dtype="bf16")
+    lat_ref, lse_ref = orc.attn_decode_latent(q_abs, q_rope, deq, cu, tq, V3)
+    o_lat, lse = _core(m, q_abs, q_rope, B, tq, cu, raw)
+    assert rel(o_lat, lat_ref) <= TOL["bf16"]
+    assert rel(lse, lse_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("tq", [1, 2])
+def test_fp8_attn_core_scales_far_apart_and_rows_past_the_end(v3, tq):
+    # cache rows whose scales span 2^-20 .. 2^4, so that the weights p_j s_j of the P'.C product span
+    # 2^24 and more while the softmax weights p_j stay within a few units (the queries are small);
+    # heads whose q~ and q^R magnitudes span 1e-2 .. 1e2 (the per-head f16 scaling of the queries:
+    # near-uniform softmax on the first heads, peaked on the last); garbage (0xFF: NaN codes and a
+    # NaN scale) in every row after the last sequence, which the last key tile reaches into. The
+    # scores stay within a few hundred, where fp32 holds the merge's m and lse to 2^-15.
+    m, _ = v3
+    lens = np.array([300, 77, 129])
+    cu = synth.cu_seqlens(lens)
+    B, T = len(lens), len(lens) * tq
+    total = int(cu[-1])
+    rows = synth.latent_cache(V3, total, seed=73, dtype="bf16")
+    rows *= np.exp2(np.random.default_rng(5).integers(-20, 5, size=total))[:, None]
+    raw, deq = fp8_cache(rows)
+    padded = np.full((total + 200, mla.FP8_ROW_BYTES), 0xFF, dtype=np.uint8)
+    padded[:total] = raw
+    head_scale = (10.0 ** np.linspace(-2, 2, V3.n_h))[None, :, None] * 2.0 ** -4
+    q_abs = bf16(synth.normal(74, 20, (T, V3.n_h, V3.d_c), std=0.5, dtype="bf16") * head_scale)
+    q_rope = bf16(synth.normal(74, 21, (T, V3.n_h, V3.d_r), std=1.0, dtype="bf16") * head_scale)
+    lat_ref, lse_ref = orc.attn_decode_latent(q_abs, q_rope, deq, cu, tq, V3)
+    assert np.abs(lse_ref).max() < 512
+    o_lat, lse = _core(m, q_abs, q_rope, B, tq, cu, padded)
+    for i in range(V3.n_h):
+        assert rel(o_lat[:, i], lat_ref[:, i]) <= TOL["bf16"], i
+    assert rel(lse, lse_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("tq", [1, 2])
+def test_fp8_decode_step(v3, tq):
+    import torch
+    m, W = v3
+    lens = np.array([1000, 4097, 65])
+    cu = synth.cu_seqlens(lens)
+    raw, deq = fp8_cache(synth.latent_cache(V3, int(cu[-1]), seed=75, dtype="bf16"))
+    h_q = synth.hidden(V3, len(lens) * tq, seed=76, dtype="bf16")
+    ref = orc.mla_decode_absorbed(h_q, deq, cu, tq, W, V3)
+    m.set_cache_format(mla.CACHE_FP8)
+    try:
+        u = m.decode(dev(h_q, "bf16"), len(lens), tq, dev_i64(cu), torch.from_numpy(raw).to("cuda:0"))
+        assert m.sync_status() == 0
+    finally:
+        m.set_cache_format(mla.CACHE_BF16)
+    assert rel(host(u), ref["u"]) <= TOL["bf16"]
+
+
+def test_fp8_append_then_decode(v3):
+    # the cache rows come from the FP8 append, which quantizes the projection's rows as the bf16
+    # format stores them (rounded to bf16); the reference quantizes the oracle's rows rounded the same
+    # way (without that rounding the scales, and with them every code, move by up to 2^-9 and the
+    # outputs by about 2 %)
+    import torch
+    m, W = v3
+    lens = np.array([150, 333])
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    h = synth.hidden(V3, T, seed=77, dtype="bf16")
+    pos = np.concatenate([np.arange(n) for n in lens])
+    _, deq = fp8_cache(bf16(orc.cache_append(h, pos, W, V3)))
+    rows = np.concatenate([np.arange(cu[b + 1] - 1, cu[b + 1]) for b in range(2)])
+    ref = orc.mla_decode_absorbed(h[rows], deq, cu, 1, W, V3)
+    m.set_cache_format(mla.CACHE_FP8)
+    try:
+        cache = torch.zeros(T, mla.FP8_ROW_BYTES, dtype=torch.uint8, device="cuda:0")
+        m.cache_append(dev(h, "bf16"), dev_i64(pos), dev_i64(np.arange(T)), cache)
+        u = m.decode(dev(h[rows], "bf16"), 2, 1, dev_i64(cu), cache)
+        assert m.sync_status() == 0
+    finally:
+        m.set_cache_format(mla.CACHE_BF16)
+    assert rel(host(u), ref["u"]) <= TOL["bf16"]
