@@ -46,6 +46,7 @@ WORKLOAD = synth.WORKLOADS["decode_b16_l4096"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CORE_FLOP_PER_ROW = 128 * 2 * (576 + 512)   # per cached row and query token: n_h * 2 * (d_c + d_R + d_c)
 ROW_BYTES = 576 * 2
+FP8_ROW_BYTES = 656     # FP8 cache row: 512 e4m3 codes, 64 f16 of k^R / s, fp32 s, 12 zero bytes
 PREFILL = synth.WORKLOADS["prefill_l32768"]
 
 
@@ -61,6 +62,9 @@ def parse():
                     help="prefill sequence length (default: the 32K-token workload; smaller for profiling)")
     ap.add_argument("--no-configs", dest="configs", action="store_false",
                     help="skip the other decode workloads and the tiny FP32 prefill")
+    ap.add_argument("--profile-core", choices=["bf16", "fp8"], default=None,
+                    help="only run the latent core on decode_b16_l4096 three times (a small case for ncu "
+                         "captures: -k regex:latent_core -s 2 -c 1); prints no bench line")
     return ap.parse_args()
 
 
@@ -482,7 +486,8 @@ def next_rows_leg(args, W, dev, rank, world, flush, timed, peaks, peak_src):
     - chunked prefill, unabsorbed form: one sequence, a 4096-token chunk after a 28672-row cached
       prefix (the 32K prefill shape taken in chunks);
     - chunked prefill, absorbed form: 16 sequences, 4-token chunks after 4092 cached rows each;
-    - the decode_b16_l4096 step with RMSNorm and YaRN (s = 40) on, next to the same step without."""
+    - the decode_b16_l4096 step with RMSNorm and YaRN (s = 40) on, next to the same step without;
+    - the decode_b16_l4096 and decode_long_b4_l131072 steps over an FP8 latent cache."""
     import torch
     from mla_latent_kv_31_b200 import mla
     dims = synth.V3
@@ -585,6 +590,71 @@ def next_rows_leg(args, W, dev, rank, world, flush, timed, peaks, peak_src):
         "gpu_launches_per_step": res["rmsnorm_yarn"][1], "gpu_launches_per_step_without": res["plain"][1],
         "note": "YaRN changes only the RoPE table and factor in the projection epilogues; RMSNorm adds one row-norm "
                 "kernel after W^DQ and one after the cache append"}
+
+    # decode over an FP8 latent cache (656-byte rows: e4m3 codes, f16 k^R / s, fp32 s), the whole
+    # step and the latent core alone, at the headline size and at the long-context size
+    for name in ("decode_b16_l4096", "decode_long_b4_l131072"):
+        wl = synth.WORKLOADS[name]
+        lens, cu_np, rows, cache16, h_np, pos_np, slots_np = decode_inputs(wl, rank, dev, on_device=True)
+        B, T = len(lens), len(lens) * wl.tq
+        m8 = mla.MLA(dims, W, mla.MLA_BF16, device=dev.index)
+        m8.set_cache_format(mla.CACHE_FP8)
+        h8 = m8.handle
+        cache = m8.quantize_fp8(cache16)
+        del cache16
+        h_dev = torch.from_numpy(h_np).to(dev, torch.bfloat16)
+        cu_dev, pos_dev, slots_dev = (torch.from_numpy(x).to(dev) for x in (cu_np, pos_np, slots_np))
+        u_dev = torch.empty(T, dims.d, dtype=torch.bfloat16, device=dev)
+        n_app = mla.mla_workspace_size(h8, mla.OP_CACHE_APPEND, 0, 1, T)
+        n_dec = mla.mla_workspace_size(h8, mla.OP_DECODE, B, wl.tq, 0)
+        n_core = mla.mla_workspace_size(h8, mla.OP_ATTN_DECODE_LATENT, B, wl.tq, 0)
+        ws_app = torch.empty(max(n_app, 1024), dtype=torch.uint8, device=dev)
+        ws_dec = torch.empty(n_dec, dtype=torch.uint8, device=dev)
+        ws_core = torch.empty(n_core, dtype=torch.uint8, device=dev)
+
+        def step8():
+            mla.mla_cache_append(h8, h_dev, pos_dev, slots_dev, T, cache, rows, ws_app, n_app, device=dev.index)
+            mla.mla_decode(h8, h_dev, B, wl.tq, cu_dev, cache, rows, u_dev, ws_dec, n_dec, device=dev.index)
+
+        off_qabs = mla.mla_workspace_offset(h8, mla.OP_DECODE, mla.BUF_QABS, B, wl.tq, 0)
+        off_qr = mla.mla_workspace_offset(h8, mla.OP_DECODE, mla.BUF_QR, B, wl.tq, 0)
+        o_lat = torch.empty(T, dims.n_h, dims.d_c, dtype=torch.float32, device=dev)
+        lse = torch.empty(T, dims.n_h, dtype=torch.float32, device=dev)
+
+        def core8():
+            mla.mla_attn_decode_latent(h8, ws_dec.data_ptr() + off_qabs, ws_dec.data_ptr() + off_qr, B, wl.tq, cu_dev,
+                                       cache, rows, o_lat, lse, ws_core, n_core, device=dev.index)
+
+        l0 = mla.mla_kernel_launches()
+        step8()
+        launches = mla.mla_kernel_launches() - l0
+        torch.cuda.synchronize()
+        if mla.mla_sync_status(h8, device=dev.index) != 0:
+            raise RuntimeError(f"device check failed in the FP8 {name} step")
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            step8()
+        iters = max(5, min(args.steps, 200))
+        ms_step = max_over_ranks([timed(g.replay, iters, 3)], dev)[0]
+        del g
+        ms_kernel = kernel_only_ms(core8, mla.TIMED_LATENT_CORE, iters, 2, flush, world)
+        cbytes = rows * FP8_ROW_BYTES
+        k_gbs = cbytes / (ms_kernel * 1e-3) / 1e9
+        k_tf = core_flops(lens, wl.tq) / (ms_kernel * 1e-3) / 1e12
+        out[name + "_fp8"] = {
+            "workload": name + " over an FP8 cache", "cache_rows": rows, "cache_bytes": cbytes,
+            "step": "mla_cache_append (FP8 rows) + mla_decode, CUDA-graph replay, L2 flushed",
+            "ms_per_step": round(ms_step, 5), "gpu_launches_per_step": int(launches),
+            "tokens_per_s": round(whole_job_rate(world, T, ms_step * 1e-3), 1),
+            "latent_core": {"kernel": "latent_core_kernel<FP8>", "kernel_ms": round(ms_kernel, 5),
+                            "algorithmic_bytes": cbytes, "gbs": round(k_gbs, 1), "tflops": round(k_tf, 1),
+                            "roofline": {"bound": "hbm", "achieved": round(k_gbs, 1), "peak": hbm, "unit": "GB/s",
+                                         "frac": round(k_gbs / hbm, 4), "peak_source": peak_src,
+                                         "traffic": (recorded_traffic("latent_core_kernel_fp8")
+                                                     if name == "decode_b16_l4096" else None)}},
+            "note": f"{FP8_ROW_BYTES} B per cached row against {ROW_BYTES} B in bf16"}
+        m8.close()
+        del cache
     return out
 
 
@@ -757,6 +827,39 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     return out
 
 
+def profile_core(fmt: str) -> int:
+    """The latent core alone on the decode_b16_l4096 shapes (cache, q~, q^R seeded as in the parity
+    tests), three launches, over a bf16 or an FP8 cache. The core needs no weights."""
+    import torch
+    from mla_latent_kv_31_b200 import mla
+    dev = torch.device("cuda", 0)
+    dims, wl = synth.V3, WORKLOAD
+    lens = wl.lengths(0)
+    cu_np = synth.cu_seqlens(lens)
+    rows, B, T = int(cu_np[-1]), len(lens), len(lens) * wl.tq
+    h = mla.mla_create(dims, mla.MLA_BF16, 0)
+    cache = synth.latent_cache_torch(dims, rows, seed=0, device=dev)
+    if fmt == "fp8":
+        mla.mla_set_cache_format(h, mla.CACHE_FP8)
+        c8 = torch.empty(rows, FP8_ROW_BYTES, dtype=torch.uint8, device=dev)
+        mla.mla_cache_quantize_fp8(h, cache, rows, c8)
+        cache = c8
+    q = synth.normal_torch(1, 20, (T, dims.n_h, dims.d_c), std=0.5, device=dev)
+    qr = synth.normal_torch(1, 21, (T, dims.n_h, dims.d_r), device=dev)
+    cu = torch.from_numpy(cu_np).to(dev)
+    o_lat = torch.empty(T, dims.n_h, dims.d_c, dtype=torch.float32, device=dev)
+    lse = torch.empty(T, dims.n_h, dtype=torch.float32, device=dev)
+    n = mla.mla_workspace_size(h, mla.OP_ATTN_DECODE_LATENT, B, wl.tq, 0)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        mla.mla_attn_decode_latent(h, q, qr, B, wl.tq, cu, cache, rows, o_lat, lse, ws, n)
+    torch.cuda.synchronize()
+    st = mla.mla_sync_status(h)
+    mla.mla_destroy(h)
+    print(f"profile-core {fmt}: status {mla.mla_status_string(st)}")
+    return 0 if st == 0 else 1
+
+
 def relaunch(args) -> int:
     """--gpus N outside torchrun: start N ranks on this node (one process per GPU) and return their
     exit status; rank 0 prints the line."""
@@ -787,6 +890,8 @@ def main():
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
+    if args.profile_core:
+        return profile_core(args.profile_core)
     if "WORLD_SIZE" not in os.environ and args.gpus > 1:
         return relaunch(args)
     if world != args.gpus:
