@@ -262,15 +262,56 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
             continue;
           }
         }
+        if constexpr (SWAP) {
+          // weight-streaming orientation: this thread holds feature f0 + r for CH consecutive tokens.
+          // The segment's fields are copied into registers once per tile: read in the loop through
+          // the parameter reference, they were reloaded for every element (they may alias the
+          // stores) and made this epilogue take microseconds per tile.
+          const TcEpiSeg S = d.s ? p.seg[1] : p.seg[0];
+          const int64_t f = f0 + r, T = p.T;
+          const bool fok = f < S.f_rows;
+          if (p.splits > 1) {
+            float* dst = p.partial + ((int64_t)d.split * T + t0 + c) * p.f_total + S.f_base + f;
+            const int64_t step = p.f_total;
+#pragma unroll
+            for (int j = 0; j < CH; ++j)
+              if (fok && t0 + c + j < T) dst[j * step] = __uint_as_float(v[j]);
+            continue;
+          }
+          const int64_t base = (int64_t)d.z * S.so_z + f * S.so_f;
+#pragma unroll
+          for (int j = 0; j < CH; ++j) {
+            const int64_t t = t0 + c + j;
+            float y = __uint_as_float(v[j]);
+            if (S.rope) {
+              const float partner = __shfl_xor_sync(0xffffffffu, y, 1);
+              if (!fok || t >= T) continue;
+              const int64_t ps = p.pos[t];
+              if (ps < 0) {
+                flag_error(p.err, DEVERR_POSITION);
+                continue;
+              }
+              y = rope_one(f, ps, y, partner, p.d_r, p.theta, p.rope_mul);
+            }
+            if (!fok || t >= T) continue;
+            int64_t row = t;
+            if (S.rowmap) {
+              row = S.rowmap[t];
+              if (row < 0 || row >= S.rowmap_limit) {
+                flag_error(p.err, DEVERR_SLOT);
+                continue;
+              }
+            }
+            const int64_t idx = base + row * S.so_t;
+            if (S.out_f32) reinterpret_cast<float*>(S.out)[idx] = y;
+            else reinterpret_cast<__nv_bfloat16*>(S.out)[idx] = __float2bfloat16_rn(y);
+          }
+        } else {
 #pragma unroll
         for (int j = 0; j < CH; ++j) {
           const float x = __uint_as_float(v[j]);
-          int64_t f, t;
-          if (SWAP) { f = f0 + r; t = t0 + c + j; }
-          else { f = f0 + c + j; t = t0 + r; }
-          float partner;
-          if (SWAP) partner = __shfl_xor_sync(0xffffffffu, x, 1);
-          else partner = __uint_as_float(v[j ^ 1]);
+          const int64_t f = f0 + c + j, t = t0 + r;
+          const float partner = __uint_as_float(v[j ^ 1]);
           if (f >= E.f_rows || t >= p.T) continue;
           if (p.splits > 1) {
             p.partial[((int64_t)d.split * p.T + t) * p.f_total + E.f_base + f] = x;
@@ -286,6 +327,7 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
             y = rope_one(f, ps, x, partner, p.d_r, p.theta, p.rope_mul);
           }
           store_out(E, p.err, d.z, f, t, y);
+        }
         }
       }
       tc_fence_before();
