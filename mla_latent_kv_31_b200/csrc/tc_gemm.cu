@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
     bool ok = true;
     for (int idx = blockIdx.x; ok && idx < p.tiles; idx += gridDim.x, ++n) {
       const Tile d = decode_tile(idx);
-      const TcEpiSeg& E = p.seg[d.s];
+      const TcEpiSeg E = d.s ? p.seg[1] : p.seg[0];   // in registers (see the swap path below)
       const int acc = n & 1;
       if (!mbar_wait(bar(B_ACCF + acc), (n >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
           // The segment's fields are copied into registers once per tile: read in the loop through
           // the parameter reference, they were reloaded for every element (they may alias the
           // stores) and made this epilogue take microseconds per tile.
-          const TcEpiSeg S = d.s ? p.seg[1] : p.seg[0];
+          const TcEpiSeg& S = E;
           const int64_t f = f0 + r, T = p.T;
           const bool fok = f < S.f_rows;
           if (p.splits > 1) {
@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constan
   }
   if (!active || l != 0) return;
   const int s = (p.nseg > 1 && f >= p.seg[1].f_base) ? 1 : 0;
-  const TcEpiSeg& E = p.seg[s];
+  const TcEpiSeg E = s ? p.seg[1] : p.seg[0];   // in registers, not read through the parameters
   const int64_t fl = f - E.f_base;
   if (E.rope) {
     const int64_t ps = p.pos[t];
