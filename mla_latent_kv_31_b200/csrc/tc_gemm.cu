@@ -355,33 +355,31 @@ struct ReduceParams {
   uint32_t* err;
 };
 
-// Sums the split-K partials of feature pairs (f, f+1), then applies the epilogue. One group of L lanes
-// (L a power of two >= splits, at most 32) per (token, feature pair): lane l adds partials l, l + L, ...
-// in order, then the group adds its lanes by a fixed xor tree, so the result does not depend on timing.
-template <int L>
+// Sums the split-K partials of feature pairs (f, f+1), then applies the epilogue. One thread per
+// (token, feature pair): it issues the loads of up to 8 splits at once and adds them in split order,
+// so the result does not depend on timing. (Groups of lanes per pair, one split each, needed thousands
+// of blocks for a few MB of L2-resident partials and were bound by the waves of blocks.)
+constexpr int kReduceBatch = 8;
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constant__ ReduceParams p) {
   const int64_t npairs = p.f_total / 2;
-  const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / L;
-  const int l = threadIdx.x & (L - 1);
-  const bool active = gid < npairs * p.T;
-  const int64_t t = active ? gid / npairs : 0;
-  const int64_t f = active ? 2 * (gid % npairs) : 0;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= npairs * p.T) return;
+  const int64_t t = gid / npairs, f = 2 * (gid % npairs);
+  const float* src = p.partial + t * p.f_total + f;
+  const int64_t kstride = p.T * p.f_total;
   float a = 0.f, b = 0.f;
-  if (active) {
-    const float* src = p.partial + t * p.f_total + f;
-    const int64_t kstride = p.T * p.f_total;
-    for (int k = l; k < p.splits; k += L) {
-      const float2 v = *reinterpret_cast<const float2*>(src + (int64_t)k * kstride);
-      a += v.x;
-      b += v.y;
+  for (int k0 = 0; k0 < p.splits; k0 += kReduceBatch) {
+    float2 v[kReduceBatch];
+#pragma unroll
+    for (int u = 0; u < kReduceBatch; ++u)
+      v[u] = k0 + u < p.splits ? *reinterpret_cast<const float2*>(src + (int64_t)(k0 + u) * kstride)
+                               : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kReduceBatch; ++u) {
+      a += v[u].x;
+      b += v[u].y;
     }
   }
-#pragma unroll
-  for (int o = L / 2; o > 0; o >>= 1) {
-    a += __shfl_xor_sync(0xffffffffu, a, o);
-    b += __shfl_xor_sync(0xffffffffu, b, o);
-  }
-  if (!active || l != 0) return;
   const int s = (p.nseg > 1 && f >= p.seg[1].f_base) ? 1 : 0;
   const TcEpiSeg E = s ? p.seg[1] : p.seg[0];   // in registers, not read through the parameters
   const int64_t fl = f - E.f_base;
@@ -607,17 +605,8 @@ cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st) {
   memcpy(r.theta, p.theta, sizeof(r.theta));
   r.rope_mul = p.rope_mul;
   r.err = g.err;
-  int L = 2;
-  while (L < p.splits && L < 32) L <<= 1;
-  const int64_t threads = (f_total / 2) * g.T * L;
-  const unsigned rg = (unsigned)((threads + 255) / 256);
-  switch (L) {
-    case 2: splitk_reduce_kernel<2><<<rg, 256, 0, st>>>(r); break;
-    case 4: splitk_reduce_kernel<4><<<rg, 256, 0, st>>>(r); break;
-    case 8: splitk_reduce_kernel<8><<<rg, 256, 0, st>>>(r); break;
-    case 16: splitk_reduce_kernel<16><<<rg, 256, 0, st>>>(r); break;
-    default: splitk_reduce_kernel<32><<<rg, 256, 0, st>>>(r); break;
-  }
+  const int64_t threads = (f_total / 2) * g.T;
+  splitk_reduce_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(r);
   note_launch();
   return cudaGetLastError();
 }
