@@ -69,6 +69,14 @@ __device__ __forceinline__ float rope_one(int64_t f, int64_t pos, float own, flo
   return ((f & 1) ? (partner * s + own * c) : (own * c - partner * s)) * mul;
 }
 
+// Weight-streaming launches with room for it stage each epilogue warp's [tokens x 32 features] block
+// in shared memory and store it as 16-byte vectors (per-element stores were issue-bound, about 150 to
+// 300 ns each once the store queue filled).
+template <int BN, bool SWAP>
+__host__ __device__ constexpr uint32_t epi_stage_bytes() {
+  return (SWAP && (BN == 16 || BN == 128)) ? 4u * (BN < 32 ? BN : 32) * 32u * 4u : 0u;
+}
+
 template <int BN, bool SWAP, bool W_MN, int STAGES>
 __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr uint32_t A_BYTES = 128 * 128;
@@ -87,6 +95,8 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
   // barriers: full[S], empty[S], acc_full[2], acc_empty[2]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  constexpr uint32_t EPI_STAGE = epi_stage_bytes<BN, SWAP>();
+  float* epi_stage = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256);   // [4 warps][CH][32]
   auto bar = [&](int i) { return smem_addr(&bars[i]); };
   const int B_FULL = 0, B_EMPTY = STAGES, B_ACCF = 2 * STAGES, B_ACCE = 2 * STAGES + 2;
 
@@ -264,26 +274,79 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
         }
         if constexpr (SWAP) {
           // weight-streaming orientation: this thread holds feature f0 + r for CH consecutive tokens.
-          // The segment's fields are copied into registers once per tile: read in the loop through
-          // the parameter reference, they were reloaded for every element (they may alias the
-          // stores) and made this epilogue take microseconds per tile.
-          const TcEpiSeg& S = E;
+          // The segment's fields are plain scalars read once per tile at fixed parameter offsets:
+          // read through a reference (or a struct copy the stores may alias), they were reloaded for
+          // every element, from L2 (the large shared-memory carve-out leaves little L1), and made
+          // this epilogue take microseconds per tile.
+          const bool s1 = d.s != 0;
+          char* const out = reinterpret_cast<char*>(s1 ? p.seg[1].out : p.seg[0].out);
+          const int64_t so_t = s1 ? p.seg[1].so_t : p.seg[0].so_t;
+          const int64_t so_f = s1 ? p.seg[1].so_f : p.seg[0].so_f;
+          const int64_t so_z = s1 ? p.seg[1].so_z : p.seg[0].so_z;
+          const bool out_f32 = (s1 ? p.seg[1].out_f32 : p.seg[0].out_f32) != 0;
+          const bool rope = (s1 ? p.seg[1].rope : p.seg[0].rope) != 0;
+          const int64_t* const rowmap = s1 ? p.seg[1].rowmap : p.seg[0].rowmap;
+          const int64_t rowmap_limit = s1 ? p.seg[1].rowmap_limit : p.seg[0].rowmap_limit;
+          const int64_t f_rows = s1 ? p.seg[1].f_rows : p.seg[0].f_rows;
+          const int64_t f_base = s1 ? p.seg[1].f_base : p.seg[0].f_base;
           const int64_t f = f0 + r, T = p.T;
-          const bool fok = f < S.f_rows;
+          const bool fok = f < f_rows;
+          if constexpr (EPI_STAGE > 0) {
+            // this warp's features fw .. fw + 31 for the CH tokens of this chunk, through shared memory
+            const int64_t fw = f0 + 32 * q;
+            const bool part = p.splits > 1;
+            const bool vec = (f_rows & (part ? 3 : 7)) == 0 &&   // a vector is all valid or all past f_rows
+                             (part ? ((p.f_total & 3) == 0 && (f_base & 3) == 0)
+                                   : (!rope && !rowmap && !out_f32 && so_f == 1 && (so_t & 7) == 0 &&
+                                      (((int64_t)d.z * so_z + fw) & 7) == 0 &&
+                                      (reinterpret_cast<uintptr_t>(out) & 15) == 0));
+            if (vec) {
+              float* stg = epi_stage + q * (CH * 32);
+              __syncwarp();
+#pragma unroll
+              for (int j = 0; j < CH; ++j) stg[j * 32 + lane] = __uint_as_float(v[j]);
+              __syncwarp();
+              if (part) {
+                // rows of 32 fp32 = 8 vectors of 4; CH rows over the 32 lanes
+#pragma unroll
+                for (int i = 0; i < CH / 4; ++i) {
+                  const int cid = i * 32 + lane, j = cid >> 3, c4 = cid & 7;
+                  const int64_t t = t0 + c + j, fe = fw + 4 * c4;
+                  if (t < T && fe < f_rows)
+                    *reinterpret_cast<float4*>(p.partial + ((int64_t)d.split * T + t) * p.f_total + f_base + fe) =
+                        *reinterpret_cast<const float4*>(stg + j * 32 + 4 * c4);
+                }
+              } else {
+                // rows of 32 bf16 = 4 vectors of 8; CH rows over the 32 lanes
+#pragma unroll
+                for (int i = 0; i < CH / 8; ++i) {
+                  const int cid = i * 32 + lane, j = cid >> 2, c8 = cid & 3;
+                  const int64_t t = t0 + c + j, fe = fw + 8 * c8;
+                  if (t < T && fe < f_rows) {
+                    const float* x = stg + j * 32 + 8 * c8;
+                    *reinterpret_cast<uint4*>(out + 2 * ((int64_t)d.z * so_z + fe + t * so_t)) =
+                        make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                                   pack_bf16(x[6], x[7]));
+                  }
+                }
+              }
+              continue;
+            }
+          }
           if (p.splits > 1) {
-            float* dst = p.partial + ((int64_t)d.split * T + t0 + c) * p.f_total + S.f_base + f;
+            float* dst = p.partial + ((int64_t)d.split * T + t0 + c) * p.f_total + f_base + f;
             const int64_t step = p.f_total;
 #pragma unroll
             for (int j = 0; j < CH; ++j)
               if (fok && t0 + c + j < T) dst[j * step] = __uint_as_float(v[j]);
             continue;
           }
-          const int64_t base = (int64_t)d.z * S.so_z + f * S.so_f;
+          const int64_t base = (int64_t)d.z * so_z + f * so_f;
 #pragma unroll
           for (int j = 0; j < CH; ++j) {
             const int64_t t = t0 + c + j;
             float y = __uint_as_float(v[j]);
-            if (S.rope) {
+            if (rope) {
               const float partner = __shfl_xor_sync(0xffffffffu, y, 1);
               if (!fok || t >= T) continue;
               const int64_t ps = p.pos[t];
@@ -295,16 +358,16 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
             }
             if (!fok || t >= T) continue;
             int64_t row = t;
-            if (S.rowmap) {
-              row = S.rowmap[t];
-              if (row < 0 || row >= S.rowmap_limit) {
+            if (rowmap) {
+              row = rowmap[t];
+              if (row < 0 || row >= rowmap_limit) {
                 flag_error(p.err, DEVERR_SLOT);
                 continue;
               }
             }
-            const int64_t idx = base + row * S.so_t;
-            if (S.out_f32) reinterpret_cast<float*>(S.out)[idx] = y;
-            else reinterpret_cast<__nv_bfloat16*>(S.out)[idx] = __float2bfloat16_rn(y);
+            const int64_t idx = base + row * so_t;
+            if (out_f32) reinterpret_cast<float*>(out)[idx] = y;
+            else reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(y);
           }
         } else {
 #pragma unroll
@@ -464,7 +527,7 @@ int num_sms() {
 
 template <int BN, bool SWAP, bool W_MN, int STAGES>
 cudaError_t launch_gemm(const GemmParams& p, int ctas_per_sm, cudaStream_t st) {
-  constexpr size_t smem = (size_t)STAGES * (128 * 128 + BN * 128) + 1024 + 256;
+  constexpr size_t smem = (size_t)STAGES * (128 * 128 + BN * 128) + 1024 + 256 + epi_stage_bytes<BN, SWAP>();
   static bool configured = false;
   auto kern = gemm_kernel<BN, SWAP, W_MN, STAGES>;
   if (!configured) {
