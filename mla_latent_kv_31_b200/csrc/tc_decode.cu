@@ -32,8 +32,8 @@
 // into its own shared-memory tile.
 //
 // Outputs. Every piece writes a partial: O = sum_j 2^((s_j - m) c) c_j unnormalised, its reference
-// m in natural units and its lse, O in a head-interleaved layout [token k][slot][column/4][head][4]
-// bf16 (fp32 accumulation, one rounding before the merge), so that the 32 heads of a warp store 256
+// m in natural units and its lse, O in a head-interleaved layout [token k][slot][column/8][head][8]
+// bf16 (fp32 accumulation, one rounding before the merge), so that the 32 heads of a warp store 512
 // contiguous bytes per instruction. The merge pass
 // weights each partial by e^{m_s - lse} with lse = log sum_s e^{lse_s} and writes o^lat [T][H][DC]
 // and lse [T][H] (a one-piece sequence is a weighted copy).
@@ -138,7 +138,7 @@ struct CoreParams {
   const int32_t* slot_base;     // [B+1]: first partial slot of each sequence
   const int4* pinfo;            // [pairs]: tile range [x, y), first sequence z, its partial slot w
   int32_t B, tq, pairs, s_max;
-  uint2* part_o;      // [tq][s_max][DC/4][H] x 4 bf16, unnormalised
+  uint4* part_o;      // [tq][s_max][DC/8][H] x 8 bf16, unnormalised
   float* part_lse;    // [tq][s_max][H]
   float* part_m;      // [tq][s_max][H], the reference of part_o in natural units
   float scale_log2;   // log2(e) / sqrt(d_h + d_h^R)
@@ -810,16 +810,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       auto dump = [&](int b, int g) -> bool {
         if (!wait_u(bar(B_ODONE), g & 1)) return false;
         tc_fence_after();
-        uint2* po = p.part_o + ((int64_t)k * p.s_max + piece_slot(b)) * (DC / 4) * H + i;
+        // 16-byte stores: the 32 heads of a warp write 512 contiguous bytes per instruction
+        uint4* po = p.part_o + ((int64_t)k * p.s_max + piece_slot(b)) * (DC / 8) * H + i;
 #pragma unroll 1
         for (int c = 256 * ehalf; c < 256 * ehalf + 256; c += 32) {
           uint32_t v[32];
           tmem_ld32(trow + c, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            po[(c / 4 + e) * H] = make_uint2(pack_bf16(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1])),
-                                             pack_bf16(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
+          for (int e = 0; e < 4; ++e)
+            po[(c / 8 + e) * H] = make_uint4(pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                                             pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                                             pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                                             pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
         }
         tc_fence_before();
         mbar_arrive(bar(B_OFREE));
@@ -1034,7 +1037,7 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
 // Exact merge of a sequence's pieces: lse = log sum_s e^{lse_s}, o = sum_s e^{m_s - lse} O_s from the
 // unnormalised head-interleaved bf16 partials O_s (O_s / l_s is the piece's own softmax average and
 // e^{lse_s} = e^{m_s} l_s, so the weight e^{lse_s - lse} / l_s is e^{m_s - lse}). One block per (token,
-// group of 32 heads, group of 128 columns): the reads of a (piece, 4-column group) are 256 contiguous
+// group of 32 heads, group of 128 columns): the reads of a (piece, 8-column group) are 512 contiguous
 // bytes over the 32 heads; the block's [32 heads x 128 columns] result goes through shared memory so
 // that each head's row is written as contiguous runs. The kernel is latency-bound (a few MB of L2-hot
 // partials), so the partials of up to kCombBatch pieces are in flight at once, the first batch issued
@@ -1042,7 +1045,7 @@ __global__ void __launch_bounds__(256) plan_kernel(const int64_t* cu, int32_t B,
 constexpr int kCombHeads = 32, kCombCols = 128, kCombBatch = 8;
 template <bool OUT_F32>
 __global__ void __launch_bounds__(256) combine_kernel(const int32_t* sb, int32_t tq, int32_t s_max,
-                                                      const uint2* part_o, const float* part_lse,
+                                                      const uint4* part_o, const float* part_lse,
                                                       const float* part_m, void* o_lat, float* lse) {
   __shared__ float s_lse[kMaxPairs][kCombHeads];
   __shared__ float s_m[kMaxPairs][kCombHeads];
@@ -1053,16 +1056,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* sb, int32_t
   const int32_t s0 = sb[b], ns = min(sb[b + 1] - s0, kMaxPairs);
   const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
   const int64_t slot0 = (int64_t)k * s_max + s0;
-  // thread (lane = head, grp): 4-column groups c4 = c0/4 + 4 grp + q, q = 0..3
-  const uint2* src = part_o + (slot0 * (DC / 4) + c0 / 4 + 4 * grp) * H + h0 + lane;
-  uint2 v[kCombBatch][4];
+  // thread (lane = head, grp): 8-column groups c8 = c0/8 + 2 grp + q, q = 0, 1 (16 columns)
+  const uint4* src = part_o + (slot0 * (DC / 8) + c0 / 8 + 2 * grp) * H + h0 + lane;
+  uint4 v[kCombBatch][2];
   auto load_batch = [&](int sl0) {
 #pragma unroll
     for (int j = 0; j < kCombBatch; ++j)
       if (sl0 + j < ns) {
-        const uint2* ps = src + (int64_t)(sl0 + j) * (DC / 4) * H;
+        const uint4* ps = src + (int64_t)(sl0 + j) * (DC / 8) * H;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v[j][q] = ps[q * H];
+        for (int q = 0; q < 2; ++q) v[j][q] = ps[q * H];
       }
   };
   load_batch(0);
@@ -1089,10 +1092,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* sb, int32_t
         const float ms = s_m[sl0 + j][lane];
         const float wgt = (tot > -INFINITY && ms > -INFINITY) ? __expf(ms - tot) : 0.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint2 u = v[j][q];
-          acc[q].x += wgt * bf16_lo(u.x); acc[q].y += wgt * bf16_hi(u.x);
-          acc[q].z += wgt * bf16_lo(u.y); acc[q].w += wgt * bf16_hi(u.y);
+        for (int q = 0; q < 2; ++q) {
+          const uint4 u = v[j][q];
+          acc[2 * q].x += wgt * bf16_lo(u.x); acc[2 * q].y += wgt * bf16_hi(u.x);
+          acc[2 * q].z += wgt * bf16_lo(u.y); acc[2 * q].w += wgt * bf16_hi(u.y);
+          acc[2 * q + 1].x += wgt * bf16_lo(u.z); acc[2 * q + 1].y += wgt * bf16_hi(u.z);
+          acc[2 * q + 1].z += wgt * bf16_lo(u.w); acc[2 * q + 1].w += wgt * bf16_hi(u.w);
         }
       }
   }
@@ -1128,7 +1133,7 @@ struct CoreScratch {
   int4* pinfo;
   float* part_lse;
   float* part_m;
-  uint2* part_o;
+  uint4* part_o;
   int32_t s_max;
 };
 
@@ -1146,7 +1151,7 @@ CoreScratch carve(void* scratch, int64_t B, int32_t tq) {
   ptr += align1k((size_t)tq * c.s_max * H * 4);
   c.part_m = (float*)ptr;
   ptr += align1k((size_t)tq * c.s_max * H * 4);
-  c.part_o = (uint2*)ptr;
+  c.part_o = (uint4*)ptr;
   return c;
 }
 

@@ -457,6 +457,21 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constan
     a = a2;
     b = b2;
   }
+  if (E.so_f == 1 && fl + 1 < E.f_rows && ((E.so_t | fl) & 1) == 0 && (reinterpret_cast<uintptr_t>(E.out) & 7) == 0) {
+    // the pair is contiguous: one 4-byte (bf16) or 8-byte (fp32) store
+    int64_t row = t;
+    if (E.rowmap) {
+      row = E.rowmap[t];
+      if (row < 0 || row >= E.rowmap_limit) {
+        flag_error(p.err, DEVERR_SLOT);
+        return;
+      }
+    }
+    const int64_t idx = row * E.so_t + fl;
+    if (E.out_f32) *reinterpret_cast<float2*>(reinterpret_cast<float*>(E.out) + idx) = make_float2(a, b);
+    else *reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(E.out) + idx) = pack_bf16(a, b);
+    return;
+  }
   store_out(E, p.err, 0, fl, t, a);
   if (fl + 1 < E.f_rows) store_out(E, p.err, 0, fl + 1, t, b);
 }
