@@ -235,6 +235,13 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
       tc_fence_after();
       const uint32_t trow = tmem + acc * ACC_COLS + ((uint32_t)(q * 32) << 16);
       const int64_t f0 = (int64_t)d.wt * W_TILE, t0 = (int64_t)d.tt * X_TILE;
+      // tile orientation: this thread's token row, through the row map (cache slots) when there is one
+      int64_t row_r = t0 + r;
+      bool row_ok = !SWAP && t0 + r < p.T;
+      if (!SWAP && row_ok && E.rowmap) {
+        row_r = E.rowmap[t0 + r];
+        row_ok = row_r >= 0 && row_r < E.rowmap_limit;
+      }
 #pragma unroll 1
       for (int c = 0; c < BN; c += CH) {
         uint32_t v[32];
@@ -244,8 +251,12 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
         if (!SWAP && CH == 32) {
           // a token row's 32 consecutive features: bf16, 16-byte stores, when the layout allows
           const int64_t t = t0 + r, f = f0 + c;
-          if (p.splits == 1 && !E.rowmap && !E.out_f32 && E.so_f == 1 && d.z == 0 && f + 32 <= E.f_rows &&
-              t < p.T && ((t * E.so_t + f) & 7) == 0 && (reinterpret_cast<uintptr_t>(E.out) & 15) == 0) {
+          if (p.splits == 1 && !E.out_f32 && E.so_f == 1 && d.z == 0 && f + 32 <= E.f_rows && t < p.T &&
+              ((row_r * E.so_t + f) & 7) == 0 && (reinterpret_cast<uintptr_t>(E.out) & 15) == 0) {
+            if (!row_ok) {
+              flag_error(p.err, DEVERR_SLOT);
+              continue;
+            }
             int64_t ps = 0;
             if (E.rope) {
               ps = p.pos[t];
@@ -266,7 +277,7 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
               }
               pk[j / 2] = pack_bf16(a, b2);
             }
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(E.out) + t * E.so_t + f);
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(E.out) + row_r * E.so_t + f);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
             continue;
