@@ -429,31 +429,43 @@ struct ReduceParams {
   uint32_t* err;
 };
 
-// Sums the split-K partials of feature pairs (f, f+1), then applies the epilogue. One thread per
-// (token, feature pair): it issues the loads of up to 8 splits at once and adds them in split order,
-// so the result does not depend on timing. (Groups of lanes per pair, one split each, needed thousands
-// of blocks for a few MB of L2-resident partials and were bound by the waves of blocks.)
+// Sums the split-K partials of feature pairs (f, f+1), then applies the epilogue. L lanes per (token,
+// feature pair), L = 1, 2 or 4 so that each lane has at most 8 splits: lane l issues the loads of splits
+// l, l + L, ... at once and adds them in order, then the group adds its lanes by a fixed xor tree, so
+// the result does not depend on timing. (One lane per split needed thousands of blocks for a few MB of
+// L2-resident partials and was bound by the waves of blocks; one thread per pair serialised up to four
+// rounds of loads when there are 28 splits.)
 constexpr int kReduceBatch = 8;
+template <int L>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const __grid_constant__ ReduceParams p) {
   const int64_t npairs = p.f_total / 2;
-  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (gid >= npairs * p.T) return;
-  const int64_t t = gid / npairs, f = 2 * (gid % npairs);
+  const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / L;
+  const int l = threadIdx.x & (L - 1);
+  const bool active = gid < npairs * p.T;
+  const int64_t t = active ? gid / npairs : 0, f = active ? 2 * (gid % npairs) : 0;
   const float* src = p.partial + t * p.f_total + f;
   const int64_t kstride = p.T * p.f_total;
   float a = 0.f, b = 0.f;
-  for (int k0 = 0; k0 < p.splits; k0 += kReduceBatch) {
-    float2 v[kReduceBatch];
+  if (active) {
+    for (int k0 = l; k0 < p.splits; k0 += kReduceBatch * L) {
+      float2 v[kReduceBatch];
 #pragma unroll
-    for (int u = 0; u < kReduceBatch; ++u)
-      v[u] = k0 + u < p.splits ? *reinterpret_cast<const float2*>(src + (int64_t)(k0 + u) * kstride)
-                               : make_float2(0.f, 0.f);
+      for (int u = 0; u < kReduceBatch; ++u)
+        v[u] = k0 + u * L < p.splits ? *reinterpret_cast<const float2*>(src + (int64_t)(k0 + u * L) * kstride)
+                                     : make_float2(0.f, 0.f);
 #pragma unroll
-    for (int u = 0; u < kReduceBatch; ++u) {
-      a += v[u].x;
-      b += v[u].y;
+      for (int u = 0; u < kReduceBatch; ++u) {
+        a += v[u].x;
+        b += v[u].y;
+      }
     }
   }
+#pragma unroll
+  for (int o = L / 2; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  if (!active || l != 0) return;
   const int s = (p.nseg > 1 && f >= p.seg[1].f_base) ? 1 : 0;
   const TcEpiSeg E = s ? p.seg[1] : p.seg[0];   // in registers, not read through the parameters
   const int64_t fl = f - E.f_base;
@@ -694,8 +706,11 @@ cudaError_t tc_gemm(const TcGemmDesc& g, cudaStream_t st) {
   memcpy(r.theta, p.theta, sizeof(r.theta));
   r.rope_mul = p.rope_mul;
   r.err = g.err;
-  const int64_t threads = (f_total / 2) * g.T;
-  splitk_reduce_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(r);
+  const int L = p.splits <= kReduceBatch ? 1 : p.splits <= 2 * kReduceBatch ? 2 : 4;
+  const unsigned rg = (unsigned)(((f_total / 2) * g.T * L + 255) / 256);
+  if (L == 1) splitk_reduce_kernel<1><<<rg, 256, 0, st>>>(r);
+  else if (L == 2) splitk_reduce_kernel<2><<<rg, 256, 0, st>>>(r);
+  else splitk_reduce_kernel<4><<<rg, 256, 0, st>>>(r);
   note_launch();
   return cudaGetLastError();
 }
