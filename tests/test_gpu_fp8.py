@@ -253,3 +253,24 @@ def test_fp8_append_then_decode(v3):
     finally:
         m.set_cache_format(mla.CACHE_BF16)
     assert rel(host(u), ref["u"]) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("tq", [1, 2])
+def test_fp8_attn_core_many_short_sequences(v3, tq):
+    # more sequences than clusters: each cluster walks many sequence pieces, so the converters' and
+    # the scale buffers' hand-offs cross piece boundaries (q~ loads between tiles) again and again
+    m, _ = v3
+    lens = synth.ragged_lengths(300, tq, 70, seed=10 + tq)
+    lens[:3] = tq
+    cu = synth.cu_seqlens(lens)
+    B, T = len(lens), len(lens) * tq
+    raw, deq = fp8_cache(synth.latent_cache(V3, int(cu[-1]), seed=78 + tq, dtype="bf16"))
+    q_abs = synth.normal(79, 20, (T, V3.n_h, V3.d_c), std=0.5, dtype="bf16")
+    q_rope = synth.normal(79, 21, (T, V3.n_h, V3.d_r), std=1.0, dtype="bf16")
+    seqs = [0, 1, 2, 57, 150, 299]
+    lat_ref, lse_ref = orc.attn_decode_latent(q_abs, q_rope, deq, cu, tq, V3, seqs=seqs)
+    o_lat, lse = _core(m, q_abs, q_rope, B, tq, cu, raw)
+    rows = np.concatenate([np.arange(b * tq, (b + 1) * tq) for b in seqs])
+    assert rel(o_lat[rows], lat_ref) <= TOL["bf16"]
+    assert rel(lse[rows], lse_ref) <= TOL["bf16"]
+    assert np.all(np.isfinite(o_lat))
