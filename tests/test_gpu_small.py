@@ -185,6 +185,28 @@ def test_v3_decode_bf16_steps(v3_module, v3_weights, tq):
     assert rel(host(u)[un["rows"]], un["u"]) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("B,tq", [(12, 2), (20, 2), (33, 1)])
+def test_v3_decode_bf16_token_counts_of_the_wider_tiles(v3_module, v3_weights, B, tq):
+    # 24, 40 and 33 query tokens: the projections' weight-streaming tiles are 32 and 64 tokens wide
+    # there (16 and 128 elsewhere in these tests), whose epilogue stores element by element
+    dims = synth.V3
+    lens = synth.ragged_lengths(B, tq, 600, seed=B)
+    cu = synth.cu_seqlens(lens)
+    T = B * tq
+    cache = synth.latent_cache(dims, int(cu[-1]), seed=25 + B, dtype="bf16")
+    h_q = synth.hidden(dims, T, seed=26 + B, dtype="bf16")
+    ref = orc.mla_decode_absorbed(h_q, cache, cu, tq, v3_weights, dims)
+    u = v3_module.decode(dev(h_q, "bf16"), B, tq, dev_i64(cu), dev(cache, "bf16"))
+    _status_ok(v3_module)
+    bf = v3_module.torch.bfloat16
+    reg = lambda which, shape, dt=bf: host(v3_module.region(mla.OP_DECODE, which, shape, dt, B, tq))  # noqa: E731
+    assert rel(reg(mla.BUF_QC, (T, dims.n_h, dims.d_h)), ref["q_c"]) <= TOL["bf16"]
+    assert rel(reg(mla.BUF_QR, (T, dims.n_h, dims.d_r)), ref["q_r"]) <= TOL["bf16"]
+    assert rel(reg(mla.BUF_QABS, (T, dims.n_h, dims.d_c)), ref["q_abs"]) <= TOL["bf16"]
+    assert rel(reg(mla.BUF_O, (T, dims.n_h, dims.d_h)), ref["o"]) <= TOL["bf16"]
+    assert rel(host(u), ref["u"]) <= TOL["bf16"]
+
+
 def test_v3_cache_append_bf16(v3_module, v3_weights):
     dims = synth.V3
     T, cap = 45, 300
