@@ -69,12 +69,13 @@ __device__ __forceinline__ float rope_one(int64_t f, int64_t pos, float own, flo
   return ((f & 1) ? (partner * s + own * c) : (own * c - partner * s)) * mul;
 }
 
-// Weight-streaming launches with room for it stage each epilogue warp's [tokens x 32 features] block
-// in shared memory and store it as 16-byte vectors (per-element stores were issue-bound, about 150 to
-// 300 ns each once the store queue filled).
+// Weight-streaming launches stage each epilogue warp's [16 tokens x 32 features] blocks in shared
+// memory (8 KB per CTA) and store them as 16-byte vectors (per-element stores were issue-bound, about
+// 150 to 300 ns each once the store queue filled).
+constexpr int kEpiRows = 16;
 template <int BN, bool SWAP>
 __host__ __device__ constexpr uint32_t epi_stage_bytes() {
-  return (SWAP && (BN == 16 || BN == 128)) ? 4u * (BN < 32 ? BN : 32) * 32u * 4u : 0u;
+  return SWAP ? 4u * kEpiRows * 32u * 4u : 0u;
 }
 
 template <int BN, bool SWAP, bool W_MN, int STAGES>
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
   constexpr uint32_t EPI_STAGE = epi_stage_bytes<BN, SWAP>();
-  float* epi_stage = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256);   // [4 warps][CH][32]
+  float* epi_stage = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256);   // [4 warps][16][32]
   auto bar = [&](int i) { return smem_addr(&bars[i]); };
   const int B_FULL = 0, B_EMPTY = STAGES, B_ACCF = 2 * STAGES, B_ACCE = 2 * STAGES + 2;
 
@@ -312,32 +313,36 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
                                       (((int64_t)d.z * so_z + fw) & 7) == 0 &&
                                       (reinterpret_cast<uintptr_t>(out) & 15) == 0));
             if (vec) {
-              float* stg = epi_stage + q * (CH * 32);
-              __syncwarp();
+              float* stg = epi_stage + q * (kEpiRows * 32);
 #pragma unroll
-              for (int j = 0; j < CH; ++j) stg[j * 32 + lane] = __uint_as_float(v[j]);
-              __syncwarp();
-              if (part) {
-                // rows of 32 fp32 = 8 vectors of 4; CH rows over the 32 lanes
+              for (int h = 0; h < CH / kEpiRows; ++h) {   // 16 tokens at a time
+                const int64_t tb = t0 + c + kEpiRows * h;
+                __syncwarp();
 #pragma unroll
-                for (int i = 0; i < CH / 4; ++i) {
-                  const int cid = i * 32 + lane, j = cid >> 3, c4 = cid & 7;
-                  const int64_t t = t0 + c + j, fe = fw + 4 * c4;
-                  if (t < T && fe < f_rows)
-                    *reinterpret_cast<float4*>(p.partial + ((int64_t)d.split * T + t) * p.f_total + f_base + fe) =
-                        *reinterpret_cast<const float4*>(stg + j * 32 + 4 * c4);
-                }
-              } else {
-                // rows of 32 bf16 = 4 vectors of 8; CH rows over the 32 lanes
+                for (int j = 0; j < kEpiRows; ++j) stg[j * 32 + lane] = __uint_as_float(v[kEpiRows * h + j]);
+                __syncwarp();
+                if (part) {
+                  // rows of 32 fp32 = 8 vectors of 4; 16 rows over the 32 lanes
 #pragma unroll
-                for (int i = 0; i < CH / 8; ++i) {
-                  const int cid = i * 32 + lane, j = cid >> 2, c8 = cid & 3;
-                  const int64_t t = t0 + c + j, fe = fw + 8 * c8;
-                  if (t < T && fe < f_rows) {
-                    const float* x = stg + j * 32 + 8 * c8;
-                    *reinterpret_cast<uint4*>(out + 2 * ((int64_t)d.z * so_z + fe + t * so_t)) =
-                        make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                                   pack_bf16(x[6], x[7]));
+                  for (int i = 0; i < kEpiRows / 4; ++i) {
+                    const int cid = i * 32 + lane, j = cid >> 3, c4 = cid & 7;
+                    const int64_t t = tb + j, fe = fw + 4 * c4;
+                    if (t < T && fe < f_rows)
+                      *reinterpret_cast<float4*>(p.partial + ((int64_t)d.split * T + t) * p.f_total + f_base + fe) =
+                          *reinterpret_cast<const float4*>(stg + j * 32 + 4 * c4);
+                  }
+                } else {
+                  // rows of 32 bf16 = 4 vectors of 8; 16 rows over the 32 lanes
+#pragma unroll
+                  for (int i = 0; i < kEpiRows / 8; ++i) {
+                    const int cid = i * 32 + lane, j = cid >> 2, c8 = cid & 3;
+                    const int64_t t = tb + j, fe = fw + 8 * c8;
+                    if (t < T && fe < f_rows) {
+                      const float* x = stg + j * 32 + 8 * c8;
+                      *reinterpret_cast<uint4*>(out + 2 * ((int64_t)d.z * so_z + fe + t * so_t)) =
+                          make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                                     pack_bf16(x[6], x[7]));
+                    }
                   }
                 }
               }
