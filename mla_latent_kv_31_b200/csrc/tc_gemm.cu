@@ -286,10 +286,8 @@ __global__ void __launch_bounds__(kThreads) gemm_kernel(const __grid_constant__ 
         }
         if constexpr (SWAP) {
           // weight-streaming orientation: this thread holds feature f0 + r for CH consecutive tokens.
-          // The segment's fields are plain scalars read once per tile at fixed parameter offsets:
-          // read through a reference (or a struct copy the stores may alias), they were reloaded for
-          // every element, from L2 (the large shared-memory carve-out leaves little L1), and made
-          // this epilogue take microseconds per tile.
+          // The segment's fields are plain scalars read once per tile at fixed parameter offsets, and
+          // the stores go through shared memory as 16-byte vectors where the layout allows (below).
           const bool s1 = d.s != 0;
           char* const out = reinterpret_cast<char*>(s1 ? p.seg[1].out : p.seg[0].out);
           const int64_t so_t = s1 ? p.seg[1].so_t : p.seg[0].so_t;
