@@ -6,31 +6,12 @@ f16 k^R / s [512, 640), fp32 s [640, 644), zero [644, 656)."""
 import numpy as np
 import pytest
 
-from mla_testlib import TOL, dev, dev_i64, host, make_module, mla, orc, rel, synth
+from mla_testlib import (E4M3, TOL, dev, dev_i64, fp8_cache, fp8_decode_rows, fp8_row_bound, host, make_module,
+                         mla, orc, rel, round_bf16, synth)
 
 pytestmark = pytest.mark.gpu
 
 V3 = synth.V3
-E4M3 = orc.e4m3_positive_values()
-
-
-def decode_rows(raw: np.ndarray):
-    """(codes as values [n, 512], k^R' [n, 64], s [n], padding bytes [n, 12]) of FP8 rows [n, 656]."""
-    raw = np.ascontiguousarray(raw, dtype=np.uint8)
-    codes = raw[:, :512]
-    assert not np.any((codes & 0x7F) == 0x7F), "NaN code"
-    vals = np.where(codes & 0x80, -1.0, 1.0) * E4M3[codes & 0x7F]
-    kr = raw[:, 512:640].copy().view(np.float16).astype(np.float64)
-    s = raw[:, 640:644].copy().view(np.float32)[:, 0].astype(np.float64)
-    return vals, kr, s, raw[:, 644:656]
-
-
-def bf16(x):
-    """x rounded to bf16 (round to nearest even), as float64."""
-    import torch
-    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
-
-
 def stress_rows(n: int, seed: int) -> np.ndarray:
     """bf16 cache rows [n, 576] that reach every branch of the format: N(0, 1) rows at scales from
     1e-30 to 1e30, an all-zero row, rows whose k^R sets the scale (so k^R / s is at the f16 range's
@@ -51,7 +32,7 @@ def stress_rows(n: int, seed: int) -> np.ndarray:
         rows[r, 1:512] = np.where(rng.random(511) < 0.5, -1.0, 1.0) * mid[pick]
         rows[r, 0] = 448.0
         rows[r, 512:] = rng.standard_normal(64)
-    return bf16(rows)
+    return round_bf16(rows)
 
 
 @pytest.fixture(scope="module")
@@ -67,27 +48,17 @@ def test_quantizer_matches_the_oracle_exactly(v3, n):
     import torch
     m, _ = v3
     rows = stress_rows(n, seed=61 + n)
-    assert np.all(bf16(rows) == rows)
+    assert np.all(round_bf16(rows) == rows)
     mid = (E4M3[1:] + E4M3[:-1]) / 2
-    assert np.all(bf16(mid) == mid)
+    assert np.all(round_bf16(mid) == mid)
     got = m.quantize_fp8(dev(rows, "bf16"))
     torch.cuda.synchronize()
-    vals, kr, s, pad = decode_rows(got.cpu().numpy())
+    vals, kr, s, pad = fp8_decode_rows(got.cpu().numpy())
     codes_ref, kr_ref, s_ref = orc.quantize_cache_rows_fp8(rows, V3)
     assert np.array_equal(s, s_ref)
     assert np.array_equal(vals, codes_ref)
     assert np.array_equal(kr, kr_ref)
     assert not pad.any()
-
-
-def _fp8_bound(ref, s):
-    """Per-element bound of |dequantized - ref| for rows that went fp64 -> bf16 -> FP8: bf16 rounding
-    (2^-8 relative) then e4m3 rounding (2^-4 relative; s 2^-10 absolute in the subnormals) of the
-    c^KV part, f16 rounding (2^-11 relative) of the k^R part, and the projection's fp32 accumulation."""
-    b = np.empty_like(ref)
-    b[:, :512] = (2.0 ** -4 + 2.0 ** -7) * np.abs(ref[:, :512]) + s[:, None] * 2.0 ** -9
-    b[:, 512:] = 2.0 ** -7 * np.abs(ref[:, 512:]) + s[:, None] * 2.0 ** -20
-    return b + 1e-5 * np.abs(ref).max(axis=1, keepdims=True)
 
 
 @pytest.mark.parametrize("T,cap", [(45, 64), (700, 1024)])
@@ -108,11 +79,11 @@ def test_cache_append_writes_fp8_rows(v3, T, cap):
     raw = cache8.cpu().numpy()
     untouched = np.setdiff1d(np.arange(cap), slots)
     assert not raw[untouched].any()
-    vals, kr, s, pad = decode_rows(raw[slots])
+    vals, kr, s, pad = fp8_decode_rows(raw[slots])
     assert not pad.any()
     deq = orc.dequantize_cache_rows_fp8(vals, kr, s)
     err = np.abs(deq - ref)
-    assert np.all(err <= _fp8_bound(ref, s)), float((err / _fp8_bound(ref, s)).max())
+    assert np.all(err <= fp8_row_bound(ref, s)), float((err / fp8_row_bound(ref, s)).max())
     # the rows the bf16 format writes for the same call, put through the library's own quantizer,
     # are the same bytes (the FP8 append quantizes the very rows the bf16 append would store)
     cache16 = torch.zeros(cap, 576, dtype=torch.bfloat16, device="cuda:0")
@@ -126,31 +97,10 @@ def test_cache_append_writes_fp8_rows(v3, T, cap):
 # Decode over an FP8 cache: the rows the oracle quantized, packed into the 656-byte layout, against
 # the oracle's attention over the rows they stand for (codes * s | (k^R / s) * s)
 # ---------------------------------------------------------------------------
-def encode_rows(codes, kr, s) -> np.ndarray:
-    """FP8 rows [n, 656] from the oracle's (e4m3 values, f16 k^R / s, s)."""
-    codes = np.asarray(codes, dtype=np.float64)
-    mag = np.abs(codes)
-    idx = np.searchsorted(E4M3, mag)
-    assert np.all(E4M3[np.minimum(idx, len(E4M3) - 1)] == mag), "not an e4m3 value"
-    byte = idx.astype(np.uint8) | np.where(np.signbit(codes), 0x80, 0).astype(np.uint8)
-    n = codes.shape[0]
-    out = np.zeros((n, mla.FP8_ROW_BYTES), dtype=np.uint8)
-    out[:, :512] = byte
-    out[:, 512:640] = np.ascontiguousarray(np.asarray(kr, dtype=np.float16)).view(np.uint8)
-    out[:, 640:644] = np.ascontiguousarray(np.asarray(s, dtype=np.float32)[:, None]).view(np.uint8)
-    return out
-
-
-def fp8_cache(rows_bf16):
-    """(FP8 bytes, the float64 rows they stand for) of bf16 cache rows, by the oracle's quantizer."""
-    codes, kr, s = orc.quantize_cache_rows_fp8(rows_bf16, V3)
-    return encode_rows(codes, kr, s), orc.dequantize_cache_rows_fp8(codes, kr, s)
-
-
 def test_encode_rows_round_trips_through_decode_rows():
     rows = stress_rows(50, seed=70)
     raw, deq = fp8_cache(rows)
-    vals, kr, s, pad = decode_rows(raw)
+    vals, kr, s, pad = fp8_decode_rows(raw)
     assert np.array_equal(orc.dequantize_cache_rows_fp8(vals, kr, s), deq) and not pad.any()
 
 
@@ -201,8 +151,8 @@ def test_fp8_attn_core_scales_far_apart_and_rows_past_the_end(v3, tq):
     padded = np.full((total + 200, mla.FP8_ROW_BYTES), 0xFF, dtype=np.uint8)
     padded[:total] = raw
     head_scale = (10.0 ** np.linspace(-2, 2, V3.n_h))[None, :, None] * 2.0 ** -4
-    q_abs = bf16(synth.normal(74, 20, (T, V3.n_h, V3.d_c), std=0.5, dtype="bf16") * head_scale)
-    q_rope = bf16(synth.normal(74, 21, (T, V3.n_h, V3.d_r), std=1.0, dtype="bf16") * head_scale)
+    q_abs = round_bf16(synth.normal(74, 20, (T, V3.n_h, V3.d_c), std=0.5, dtype="bf16") * head_scale)
+    q_rope = round_bf16(synth.normal(74, 21, (T, V3.n_h, V3.d_r), std=1.0, dtype="bf16") * head_scale)
     lat_ref, lse_ref = orc.attn_decode_latent(q_abs, q_rope, deq, cu, tq, V3)
     assert np.abs(lse_ref).max() < 512
     o_lat, lse = _core(m, q_abs, q_rope, B, tq, cu, padded)
@@ -241,7 +191,7 @@ def test_fp8_append_then_decode(v3):
     T = int(cu[-1])
     h = synth.hidden(V3, T, seed=77, dtype="bf16")
     pos = np.concatenate([np.arange(n) for n in lens])
-    _, deq = fp8_cache(bf16(orc.cache_append(h, pos, W, V3)))
+    _, deq = fp8_cache(round_bf16(orc.cache_append(h, pos, W, V3)))
     rows = np.concatenate([np.arange(cu[b + 1] - 1, cu[b + 1]) for b in range(2)])
     ref = orc.mla_decode_absorbed(h[rows], deq, cu, 1, W, V3)
     m.set_cache_format(mla.CACHE_FP8)

@@ -10,7 +10,8 @@ O(n_h d_h d_c), which is what makes 32K- and 128K-row sequences checkable on the
 import numpy as np
 import pytest
 
-from mla_testlib import TOL, dev, dev_i64, host, make_module, mla, orc, rel, synth
+from mla_testlib import (TOL, dev, dev_i64, fp8_cache, fp8_decode_rows, fp8_row_bound, host, make_module, mla, orc,
+                         rel, round_bf16, synth)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -80,6 +81,60 @@ def test_decode_mtp_b64_ragged_full(mod, w0):
 
 def test_decode_long_b4_l131072_full(mod, w0):
     _decode_step(mod, w0, "decode_long_b4_l131072", [0, 3])
+
+
+def _decode_step_fp8(mod, W, name, sample):
+    """The same step over an FP8 latent cache (656-byte rows): the seeded bf16 cache put through the
+    oracle's quantizer, the query tokens' rows appended by the library as FP8 rows, then the decode.
+    Every appended row is checked against the oracle's float64 append within the format's rounding
+    bound; u, o^lat and lse of the sampled sequences against the oracle's absorbed decode over the
+    rows the FP8 cache stands for (the appended ones quantized by the oracle from its own rows
+    rounded to bf16, as the bf16 format would store them)."""
+    wl = synth.WORKLOADS[name]
+    dims, tq = wl.dims, wl.tq
+    lens = wl.lengths(0)
+    cu = synth.cu_seqlens(lens)
+    B, T = len(lens), len(lens) * tq
+    raw, deq = fp8_cache(synth.latent_cache(dims, int(cu[-1]), seed=0), dims)
+    h_q = synth.hidden(dims, T, seed=0)
+    pos = np.concatenate([np.arange(L - tq, L) for L in lens]).astype(np.int64)
+    slots = np.repeat(cu[:-1], tq) + pos
+    new_rows = orc.cache_append(h_q, pos, W, dims)
+    _, deq[slots] = fp8_cache(round_bf16(new_rows), dims)
+    ref = orc.mla_decode_absorbed(h_q, deq, cu, tq, W, dims, seqs=sample)
+    torch = mod.torch
+    d_cache = torch.from_numpy(raw).to("cuda:0")
+    del raw
+    mod.set_cache_format(mla.CACHE_FP8)
+    try:
+        d_h = dev(h_q, "bf16")
+        mod.cache_append(d_h, dev_i64(pos), dev_i64(slots), d_cache)
+        u = mod.decode(d_h, B, tq, dev_i64(cu), d_cache)
+        _status_ok(mod)
+        rows = torch.from_numpy(ref["rows"]).to("cuda:0")
+        olat = mod.region(mla.OP_DECODE, mla.BUF_OLAT, (T, dims.n_h, dims.d_c), torch.bfloat16, B, tq)
+        lse = mod.region(mla.OP_DECODE, mla.BUF_LSE, (T, dims.n_h), torch.float32, B, tq)
+        olat_h, lse_h = host(olat[rows]), host(lse[rows])
+    finally:
+        mod.set_cache_format(mla.CACHE_BF16)
+    vals, kr, s, pad = fp8_decode_rows(d_cache[dev_i64(slots)].cpu().numpy())
+    assert not pad.any()
+    err = np.abs(orc.dequantize_cache_rows_fp8(vals, kr, s) - new_rows)
+    bound = fp8_row_bound(new_rows, s)
+    assert np.all(err <= bound), float((err / bound).max())
+    u_h = host(u)
+    assert np.all(np.isfinite(u_h))
+    assert rel(u_h[ref["rows"]], ref["u"]) <= TOL["bf16"]
+    assert rel(olat_h, ref["o_lat"]) <= TOL["bf16"]
+    assert rel(lse_h, ref["lse"]) <= TOL["bf16"]
+
+
+def test_decode_b16_l4096_fp8_full(mod, w0):
+    _decode_step_fp8(mod, w0, "decode_b16_l4096", [0, 7, 15])
+
+
+def test_decode_long_b4_l131072_fp8_full(mod, w0):
+    _decode_step_fp8(mod, w0, "decode_long_b4_l131072", [0, 3])
 
 
 def test_prefill_l32768_full(mod, w0):
