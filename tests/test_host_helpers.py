@@ -49,3 +49,30 @@ def test_torch_draws_equal_numpy_draws():
         assert np.array_equal(a, b)
     c = synth.latent_cache_torch(synth.TINY, 50, seed=2).float().numpy()
     assert np.array_equal(c, synth.latent_cache(synth.TINY, 50, seed=2))
+
+
+def test_fp8_row_packing_of_the_parity_tests():
+    """The 656-byte rows the FP8 parity tests build from the oracle's quantizer: the code bytes are
+    torch's own float8_e4m3fn encoding of the code values, k^R / s and s are their f16 / fp32 bytes,
+    the padding is zero, unpacking gives the values back, and quantizing in blocks changes nothing."""
+    import torch
+    from mla_testlib import fp8_cache, fp8_decode_rows, fp8_encode_rows, orc, round_bf16
+    rng = np.random.default_rng(11)
+    rows = rng.standard_normal((300, 576)) * 10.0 ** rng.integers(-6, 7, size=300)[:, None]
+    rows[3] = 0.0
+    rows[5, 512:] *= 1e5                        # k^R sets the scale: c^KV / s in the e4m3 subnormals
+    rows = round_bf16(rows)
+    codes, kr, s = orc.quantize_cache_rows_fp8(rows, synth.V3)
+    raw = fp8_encode_rows(codes, kr, s)
+    assert raw.shape == (300, 656)
+    want = torch.from_numpy(codes.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    same_value = (raw[:, :512] == want) | ((raw[:, :512] & 0x7F) == 0) & ((want & 0x7F) == 0)
+    assert np.all(same_value)                   # +0 and -0 may differ in sign only
+    assert np.array_equal(raw[:, 512:640].view(np.float16).astype(np.float64), kr)
+    assert np.array_equal(raw[:, 640:644].view(np.float32)[:, 0].astype(np.float64), s)
+    assert not raw[:, 644:].any()
+    vals, kr2, s2, pad = fp8_decode_rows(raw)
+    assert np.array_equal(vals, codes) and np.array_equal(kr2, kr) and np.array_equal(s2, s) and not pad.any()
+    raw_b, deq_b = fp8_cache(rows, synth.V3, chunk=37)
+    assert np.array_equal(raw_b, raw)
+    assert np.array_equal(deq_b, orc.dequantize_cache_rows_fp8(codes, kr, s))
