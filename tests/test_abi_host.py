@@ -247,6 +247,16 @@ def test_cache_format_setter_and_fp8_guards():
         with pytest.raises(mla.MLAError) as e:
             mla.mla_attn_prefill(h, A, A, A, A, 1, A, 64, 64, A, 64, A, stream=0)
         assert e.value.status == 3
+        with pytest.raises(mla.MLAError) as e:
+            mla.mla_prefill_chunk(h, A, 1, A, 4, 4, A, 64, A, 64, mla.CHUNK_AUTO, A, A, 1 << 30, stream=0)
+        assert e.value.status == 3
+        # the FP8 append stages its T bf16 rows (576 columns) in the workspace before quantizing them
+        for T in (1, 45, 700):
+            ws8 = mla.mla_workspace_size(h, mla.OP_CACHE_APPEND, 0, 1, T)
+            mla.mla_set_cache_format(h, mla.CACHE_BF16)
+            ws16 = mla.mla_workspace_size(h, mla.OP_CACHE_APPEND, 0, 1, T)
+            mla.mla_set_cache_format(h, mla.CACHE_FP8)
+            assert ws8 >= ws16 + T * 576 * 2, (T, ws8, ws16)
         # the quantizer validates its arguments on the host
         with pytest.raises(mla.MLAError) as e:
             mla.mla_cache_quantize_fp8(h, A, 0, A, stream=0)
