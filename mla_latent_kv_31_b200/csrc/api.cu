@@ -333,7 +333,7 @@ mla_status_t mla_cache_quantize_fp8(mla_handle_t* h, const void* rows, int64_t n
   if (!g.ok) return MLA_ERR_CUDA;
   mla_status_t s = ensure_device(h);
   if (s != MLA_OK) return s;
-  return cuda_status(mla::fp8_quantize_rows(rows, n, nullptr, n, out, (cudaStream_t)stream));
+  return cuda_status(mla::fp8_quantize_rows(rows, n, nullptr, n, out, h->d_err, (cudaStream_t)stream));
 }
 
 mla_status_t mla_set_yarn(mla_handle_t* h, double s, double alpha, double beta, double original_len) {

@@ -27,14 +27,17 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 
 __global__ void __launch_bounds__(32 * kRowsPerBlock)
     quantize_rows_kernel(const __nv_bfloat16* rows, int64_t n, const int64_t* rowmap, int64_t limit,
-                         uint8_t* out) {
+                         uint8_t* out, uint32_t* err) {
   const int64_t r = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= n) return;
   int64_t dst = r;
   if (rowmap) {
     dst = rowmap[r];
-    if (dst < 0 || dst >= limit) return;   // the projection that made the row flagged it
+    if (dst < 0 || dst >= limit) {         // a slot outside the cache: reported, nothing written
+      if (lane == 0) flag_error(err, DEVERR_SLOT);
+      return;
+    }
   }
   const __nv_bfloat16* src = rows + r * kFp8RowLatent;
   // lane: c^KV columns 16 lane .. 16 lane + 15, k^R columns 2 lane, 2 lane + 1
@@ -75,11 +78,11 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
 }  // namespace
 
 cudaError_t fp8_quantize_rows(const void* rows, int64_t n, const int64_t* rowmap, int64_t limit, void* out,
-                              cudaStream_t st) {
+                              uint32_t* err, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)((n + kRowsPerBlock - 1) / kRowsPerBlock);
   quantize_rows_kernel<<<grid, 32 * kRowsPerBlock, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(rows), n, rowmap,
-                                                            limit, reinterpret_cast<uint8_t*>(out));
+                                                            limit, reinterpret_cast<uint8_t*>(out), err);
   note_launch();
   return cudaGetLastError();
 }

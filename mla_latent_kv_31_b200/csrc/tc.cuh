@@ -25,9 +25,9 @@ constexpr int kFp8RowLatent = 576;   // bf16 elements of the cache row it is mad
 constexpr int kFp8KrOffset = 512;    // byte offsets of k^R / s and of s in the row
 constexpr int kFp8ScaleOffset = 640;
 // bf16 cache rows [n][576] -> FP8 rows at out + row(r) * 656, row(r) = rowmap ? rowmap[r] : r (rows
-// mapped outside [0, limit) are skipped).
+// mapped outside [0, limit) are not written and set DEVERR_SLOT in *err).
 cudaError_t fp8_quantize_rows(const void* rows, int64_t n, const int64_t* rowmap, int64_t limit, void* out,
-                              cudaStream_t st);
+                              uint32_t* err, cudaStream_t st);
 // Scratch bytes of the bf16 rows an FP8 append stages before quantizing them.
 inline size_t fp8_staging_bytes(int64_t T) { return (size_t)(T > 0 ? T : 1) * kFp8RowLatent * 2; }
 

@@ -71,7 +71,8 @@ cudaError_t cache_rows(const mla_dims_t& d, const mla_weights_t& w, const LayerO
   cudaError_t e = tc_gemm(g, st);
   if (e != cudaSuccess) return e;
   if (o.g_kv && (e = rmsnorm_rows(dst, true, R, map, limit, T, d.d_c, o.g_kv, o.eps, st)) != cudaSuccess) return e;
-  return fp8 ? fp8_quantize_rows(staging, T, rowmap, capacity, cache, st) : cudaSuccess;
+  // the projection wrote the staged rows without the slots, so the quantizer checks them
+  return fp8 ? fp8_quantize_rows(staging, T, rowmap, capacity, cache, err, st) : cudaSuccess;
 }
 
 // Steps (1)-(3): c^Q = W^DQ h (then the optional RMSNorm); q^C = W^UQ c^Q; q^R = RoPE(W^QR c^Q).

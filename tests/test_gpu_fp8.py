@@ -93,6 +93,33 @@ def test_cache_append_writes_fp8_rows(v3, T, cap):
     assert np.array_equal(q.cpu().numpy(), raw[slots])
 
 
+def test_fp8_append_flags_slots_outside_the_cache(v3):
+    # the projection writes the staged bf16 rows without the slots, so the quantizer is the step that
+    # must report a slot outside [0, capacity) (and write nothing for it), as the bf16 append does
+    import torch
+    m, W = v3
+    h = synth.hidden(V3, 3, seed=63, dtype="bf16")
+    pos = np.array([0, 1, 2])
+    ref = orc.cache_append(h, pos, W, V3)
+    m.set_cache_format(mla.CACHE_FP8)
+    try:
+        cache8 = torch.zeros(65, mla.FP8_ROW_BYTES, dtype=torch.uint8, device="cuda:0")
+        m.cache_append(dev(h, "bf16"), dev_i64(pos), dev_i64([3, 64, -1]), cache8[:64])
+        assert mla.STATUS_NAMES[m.sync_status()] == "MLA_ERR_DEVICE_CHECK"
+        assert mla.mla_device_error_bits(m.handle) & 4
+        assert m.sync_status() == 0
+        m.cache_append(dev(h[:1], "bf16"), dev_i64(pos[:1]), dev_i64([5]), cache8[:64])
+        assert m.sync_status() == 0
+    finally:
+        m.set_cache_format(mla.CACHE_BF16)
+    raw = cache8.cpu().numpy()
+    assert not raw[np.setdiff1d(np.arange(65), [3, 5])].any()    # row 64 lies past the cache given
+    for slot, t in ((3, 0), (5, 0)):
+        vals, kr, s, pad = fp8_decode_rows(raw[slot:slot + 1])
+        err = np.abs(orc.dequantize_cache_rows_fp8(vals, kr, s) - ref[t:t + 1])
+        assert np.all(err <= fp8_row_bound(ref[t:t + 1], s)) and not pad.any()
+
+
 # ---------------------------------------------------------------------------
 # Decode over an FP8 cache: the rows the oracle quantized, packed into the 656-byte layout, against
 # the oracle's attention over the rows they stand for (codes * s | (k^R / s) * s)
