@@ -28,7 +28,8 @@
  *     Host-side validation (null pointers, sizes, alignment, workspace) runs before any launch:
  *     on failure nothing is launched and nothing is written. Device-side checks (cu_seqlens
  *     order, lengths, slots, positions) set a sticky error word in the handle and skip the
- *     offending rows; mla_sync_status() reports it.
+ *     offending rows or elements; mla_sync_status() reports it. Outputs that depend on a flagged
+ *     input are not valid (see each call for what is written).
  *   - Device pointers must be 16-byte aligned (MLA_ERR_ALIGNMENT otherwise).
  *   - Calls make the handle's device current while they run and restore the calling thread's
  *     current device before they return.
@@ -165,7 +166,9 @@ mla_status_t mla_workspace_offset(const mla_handle_t *h, mla_op_t op, int64_t nu
 /* Steps (5), (7) and the cache write of section 一(一)3: for each of the T tokens,
  * c^KV = W^DKV h_t and k^R = RoPE_pos(W^KR h_t), stored as one row at cache[slots[t]].
  *   h          [T, d]            handle dtype
- *   positions  [T] device int64  position of each token within its sequence (>= 0)
+ *   positions  [T] device int64  position of each token within its sequence (>= 0; a negative
+ *                                one is flagged and that token's cache row is not valid after the
+ *                                call: its k^R is not computed, while c^KV may be written)
  *   slots      [T] device int64  destination row, 0 <= slot < capacity (else skipped + flagged)
  *   cache      [capacity, d_c + d_r]
  * ws: mla_workspace_size(MLA_OP_CACHE_APPEND, total_tokens = T) bytes (split-K partials of the
