@@ -76,3 +76,31 @@ def test_fp8_row_packing_of_the_parity_tests():
     raw_b, deq_b = fp8_cache(rows, synth.V3, chunk=37)
     assert np.array_equal(raw_b, raw)
     assert np.array_equal(deq_b, orc.dequantize_cache_rows_fp8(codes, kr, s))
+
+
+def test_algorithmic_costs_the_rooflines_divide_by():
+    """The per-unit costs behind every roofline fraction of the bench line, against their closed forms
+    at the DeepSeek-V3 sizes: a cached row is 576 bf16 (1152 B) or one 656-byte FP8 row; the latent
+    core spends n_h * 2 * (576 + 512) flops per (query token, visible row); the unabsorbed prefill
+    attention 2 * (192 + 128) flops per causal pair and head (43.98 TFLOP at 32768 tokens) and its
+    five projection GEMMs 2 flops per MAC (12.26 TFLOP at 32768 tokens)."""
+    d = synth.V3
+    assert bench.ROW_BYTES == (d.d_c + d.d_r) * 2 == 1152
+    assert bench.FP8_ROW_BYTES == d.d_c + 2 * d.d_r + 4 + 12 == 656
+    assert bench.CORE_FLOP_PER_ROW == d.n_h * 2 * ((d.d_c + d.d_r) + d.d_c) == 278528
+    # decode_b16_l4096: one query token per sequence sees all 4096 rows
+    assert bench.core_flops([4096] * 16, 1) == 16 * 4096 * 278528 == 18_253_611_008
+    # two query tokens: the first sees L - 1 rows, the second all L
+    lens = [5, 2, 33]
+    assert bench.core_flops(lens, 2) == sum((L - 1) + L for L in lens) * 278528
+    attn, proj = bench.prefill_flops(d, [32768])
+    assert attn == 32768 * 32769 // 2 * d.n_h * 2 * (2 * d.d_h + d.d_r)
+    assert abs(attn / 1e12 - 43.98) < 0.005
+    hd = d.n_h * d.d_h
+    macs_per_token = (d.d * (d.d_c + d.d_r) + d.d * d.d_cq + d.d_cq * (hd + d.n_h * d.d_r) + 2 * d.d_c * hd
+                      + hd * d.d)
+    assert proj == 2 * 32768 * macs_per_token
+    assert abs(proj / 1e12 - 12.26) < 0.005
+    # two sequences: pairs add per sequence, projections per token
+    a2, p2 = bench.prefill_flops(d, [3, 4])
+    assert a2 == (6 + 10) * d.n_h * 2 * (2 * d.d_h + d.d_r) and p2 == 2 * 7 * macs_per_token
