@@ -133,9 +133,12 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def oracle_sample(seconds: float):
+def oracle_sample(seconds: float, steps: int = 0, warmup: int = 0):
     """The oracle as it stands on all host cores this process may use: BLAS threads = the affinity
-    mask's size, which is the `cores` reported."""
+    mask's size, which is the `cores` reported. A step is the decode of one sequence of the workload
+    (all heads, u included), the sequences taken in turn. Up to one untimed warm-up step (`warmup` > 0),
+    then timed steps until `steps` of them (0: all sequences) have run or `seconds` have passed, at
+    least one."""
     from threadpoolctl import threadpool_limits
 
     from oracle import mla_oracle as orc
@@ -146,19 +149,24 @@ def oracle_sample(seconds: float):
     cache = synth.latent_cache(dims, int(cu[-1]), seed=0, dtype="bf16")
     h_q = synth.hidden(dims, n_seq * tq, seed=0, dtype="bf16")
     cores = len(os.sched_getaffinity(0))
+    limit = steps if steps > 0 else n_seq
+    warm = min(warmup, 1)
     done = 0
     with threadpool_limits(limits=cores):
+        for i in range(warm):
+            orc.mla_decode(h_q, cache, cu, tq, W, dims, seqs=[i % n_seq])
         t0 = time.perf_counter()
-        while done < n_seq:
-            orc.mla_decode(h_q, cache, cu, tq, W, dims, seqs=[done])
+        while done < limit:
+            orc.mla_decode(h_q, cache, cu, tq, W, dims, seqs=[(warm + done) % n_seq])
             done += 1
             if time.perf_counter() - t0 >= seconds:
                 break
         dt = time.perf_counter() - t0
     gbs = done * L * ROW_BYTES / dt / 1e9
     return {"value": gbs, "unit": "GB/s", "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
-            "sample": f"{done} of {n_seq} sequences (all {dims.n_h} heads, u included), float64 unabsorbed "
-                      f"definition, {dt:.1f} s", "tokens_per_s": done * tq / dt, "seconds": dt}
+            "sample": f"{done} sequence decodes of {n_seq} sequences x {L} rows (all {dims.n_h} heads, u "
+                      f"included), float64 unabsorbed definition, {dt:.1f} s", "tokens_per_s": done * tq / dt,
+            "seconds": dt, "steps": done, "warmup": warm}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -883,9 +891,13 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cpu = oracle_sample(args.oracle_seconds)
+        # a step is one sequence's decode through the oracle: the steps that fit in the time budget run
+        # (at most --steps), after at most one warm-up step; the line reports the counts that ran
+        cpu = oracle_sample(args.oracle_seconds, args.steps, args.warmup)
         line = {"impl": "reference", "metric": METRIC, "value": round(cpu["value"], 4), "unit": "GB/s",
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                "n_gpus": args.gpus, "steps": cpu["steps"], "warmup": cpu["warmup"],
+                "steps_requested": args.steps, "warmup_requested": args.warmup,
+                "ms_per_step": round(cpu["seconds"] / cpu["steps"] * 1e3, 1), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": dict(workload_config(), parallelism="cpu"),
                 "cpu_baseline": cpu,
