@@ -22,7 +22,7 @@ Decode semantics (cache the keys/values of past tokens, compute only the new
 query, attend over every cached position) follow the explainer at
 mlqm.cn/news/135256, paragraph "KV Cache的核心原理".
 
-Readings where the pages leave a step open (each is also listed in the design doc):
+Readings where the pages leave a step open:
   R1 RoPE pairs are the interleaved pairs (2m, 2m+1) of the block-diagonal
      form, rotated by [[cos, -sin], [sin, cos]] with angle pos * base^(-2m/d_R).
   R2 Positions are 0-based within a sequence; packing does not shift them.
