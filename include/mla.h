@@ -54,7 +54,7 @@ typedef enum {
   MLA_OK = 0,
   MLA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, Tq outside {1, 2}, bad op        */
   MLA_ERR_ALIGNMENT = 2,     /* a device pointer is not 16-byte aligned                         */
-  MLA_ERR_UNSUPPORTED = 3,   /* dims/dtype combination this build has no kernel for              */
+  MLA_ERR_UNSUPPORTED = 3,   /* dims/dtype combination the library has no kernel for            */
   MLA_ERR_WORKSPACE = 4,     /* ws_bytes below mla_workspace_size()                              */
   MLA_ERR_CUDA = 5,          /* a CUDA runtime call failed (the CUDA error is not cleared)       */
   MLA_ERR_TIMEOUT = 6,       /* a device-side bounded wait gave up (kernel returned early)       */

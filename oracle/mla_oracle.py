@@ -475,7 +475,7 @@ def mla_cache_elements_per_token(dims, layers: int) -> int:
 
 # ---------------------------------------------------------------------------
 # FP8 (e4m3) latent cache (opt-in; reading R15). The notes' FP8 section scales 1 x 128 tiles for
-# training GEMMs; for the cache this build takes one fp32 scale per cached row.
+# training GEMMs; the cache takes one fp32 scale per cached row.
 # ---------------------------------------------------------------------------
 E4M3_MAX = 448.0
 KR_F16_RANGE = 32768.0
