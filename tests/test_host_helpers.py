@@ -104,3 +104,30 @@ def test_algorithmic_costs_the_rooflines_divide_by():
     # two sequences: pairs add per sequence, projections per token
     a2, p2 = bench.prefill_flops(d, [3, 4])
     assert a2 == (6 + 10) * d.n_h * 2 * (2 * d.d_h + d.d_r) and p2 == 2 * 7 * macs_per_token
+
+
+def test_clock_sampler_reads_the_nvidia_smi_fallback(tmp_path):
+    """Without NVML the sampler reads nvidia-smi's CSV: the median SM clock under load, the maximum,
+    and the union of the clock-event reasons it names (0x40 | 0x4: thermal slowdown and power cap);
+    malformed lines are skipped."""
+    import threading
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.device, s.samples, s.smax, s.nvml, s.thread = 0, [], None, None, None
+    s.stop_ev = threading.Event()
+    path = tmp_path / "clocks.csv"
+    path.write_text("1965, 1965, 0x0000000000000000\n1800, 1965, 0x0000000000000004\nnot a sample\n"
+                    "1327, 1965, 0x0000000000000044\n")
+
+    class Proc:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    s.proc, s.path = Proc(), str(path)
+    out = s.stop()
+    assert out["samples"] == 3 and out["sm_mhz"] == 1800.0 and out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert out["source"] == "nvidia-smi 200 ms"
+    assert not path.exists()
