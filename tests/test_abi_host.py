@@ -267,3 +267,21 @@ def test_cache_format_setter_and_fp8_guards():
         mla.mla_set_cache_format(h, mla.CACHE_BF16)
     finally:
         mla.mla_destroy(h)
+
+
+def test_a_plain_c_caller_compiles_links_and_runs(tmp_path):
+    """include/mla.h as C99 (-Wall -Werror) and libmla.so linked like any C library: a C program makes
+    the host-side calls (handle, workspace arithmetic, validation before any launch, the FP8 format's
+    guards, status strings) and checks every status."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(mla._LIB_PATH)
+    exe = tmp_path / "abi_c_client"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "abi_c_client.c"), "-o", str(exe), mla._LIB_PATH,
+                    f"-Wl,-rpath,{libdir}"], check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
